@@ -1,0 +1,420 @@
+"""Benchmark of the fused DyT forward + backward on B200.
+
+One step = one forward and one backward (dx, dgamma, dbeta, dalpha) of the
+workload over one batch of synthetic input. Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): each rank runs the whole workload
+on its own batch of rows (weak scaling); the parameter gradients are summed
+across ranks with one NCCL all-reduce of 2N+1 values per step, the exchange
+that row sharding of the column sums requires.
+
+Device timing: CUDA events around a CUDA graph of K steps on the launching
+stream, barrier + synchronize on both sides, max over ranks. The steps cycle
+through enough buffer sets that the data touched between two uses of a set
+is more than twice the L2 size, so no step reads another's data from L2.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DyT fwd+bwd achieved HBM GB/s (and % of B200 peak), rows/s per shape"
+FALLBACK_HBM_GBS = 6650.0
+PROFILES = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = [os.path.join(ROOT, "elementwise_reduction_b200", "csrc", f)
+                  for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_api.cu")]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=None)
+    p.add_argument("--e2e-steps", type=int, default=None)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args()
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str, kernel: str):
+    """dram read+write bytes per launch from a committed ncu summary, or None when the
+    kernel sources changed since it was taken."""
+    path = os.path.join(PROFILES, "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---- clocks sampled during the timed region ---------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, enabled: bool = True):
+        self.index, self.enabled, self.rows, self.proc = index, enabled, [], None
+
+    def __enter__(self):
+        if self.enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.thread = threading.Thread(target=self._read, daemon=True)
+                self.thread.start()
+            except Exception:
+                self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return None
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ---- CPU baseline: the oracle on a bounded sample ---------------------------------------------
+
+def oracle_sample_rows(w, seconds_budget: float) -> int:
+    # about 40 ns per element for forward + backward in binary64 with libm tanh/cosh
+    rows = int(seconds_budget / (40e-9 * max(1, w.N)))
+    return max(1, min(w.M, rows))
+
+
+def run_oracle_sample(w, rows: int):
+    """Oracle forward + backward on the first `rows` rows of the workload; returns
+    (seconds, algorithmic bytes of the sample)."""
+    import oracle
+    from synth import workloads
+
+    ws = workloads.Workload(w.name, rows, w.N, w.x_dtype, w.p_dtype, w.alpha, w.x_std, w.dy_std,
+                            w.gamma_mean, w.gamma_std, w.beta_mean, w.beta_std, w.nonzero, w.seed)
+    inp = workloads.make_inputs(ws)
+    t0 = time.perf_counter()
+    oracle.forward(inp["x"], inp["alpha"], inp["gamma"], inp["beta"], rows, w.N, w.x_dtype, w.p_dtype)
+    oracle.backward(inp["x"], inp["dy"], inp["alpha"], inp["gamma"], rows, w.N, w.x_dtype, w.p_dtype)
+    dt = time.perf_counter() - t0
+    return dt, ws.fwd_bytes() + ws.bwd_bytes()
+
+
+def cpu_baseline(w, seconds_budget=12.0):
+    rows = oracle_sample_rows(w, seconds_budget)
+    dt, nbytes = run_oracle_sample(w, rows)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of {w.M} rows (x {w.N} columns), one forward + backward, "
+                      f"single-threaded binary64 C oracle, {dt:.2f} s",
+            "rows_per_s": rows / dt}
+
+
+# ---- the reference arm: the oracle as it stands ------------------------------------------------
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step_budget = min(10.0, 120.0 / max(1, args.steps + args.warmup))
+    rows = oracle_sample_rows(w, per_step_budget)
+    for _ in range(args.warmup):
+        run_oracle_sample(w, max(1, rows // 8))
+    times, nbytes = [], 0
+    for _ in range(args.steps):
+        dt, nbytes = run_oracle_sample(w, rows)
+        times.append(dt)
+    total = sum(times)
+    value = nbytes * args.steps / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {rows} of {w.M} rows per step, forward + backward, "
+                                   "single-threaded binary64 C oracle"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "M": w.M, "N": w.N, "x_dtype": w.x_dtype, "param_dtype": w.p_dtype,
+            "alpha": w.alpha, "x_std": w.x_std, "dy_std": w.dy_std, "gamma": f"N({w.gamma_mean},{w.gamma_std})",
+            "beta": f"N({w.beta_mean},{w.beta_std})", "seed": w.seed}
+
+
+# ---- our arm ------------------------------------------------------------------------------------
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import elementwise_reduction_b200 as dyt
+    from synth import workloads
+
+    def to_torch(a, dtype, device):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dtype == "bf16" else torch.from_numpy(a)
+        return t if str(device) == "cpu" else t.to(device)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    M, N = w.M, w.N
+    inp = workloads.make_inputs(w)
+    L2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    set_bytes = 4 * M * N * workloads.ITEMSIZE[w.x_dtype]  # x, dy, y, dx
+    nsets = int(min(64, max(1, -(-3 * L2 // set_bytes))))
+    x0 = to_torch(inp["x"], w.x_dtype, dev).view(M, N)
+    dy0 = to_torch(inp["dy"], w.x_dtype, dev).view(M, N)
+    alpha = to_torch(inp["alpha"], w.p_dtype, dev)
+    gamma = to_torch(inp["gamma"], w.p_dtype, dev)
+    beta = to_torch(inp["beta"], w.p_dtype, dev)
+    sets = []
+    for i in range(nsets):
+        x = x0 if i == 0 else x0.clone()
+        d = dy0 if i == 0 else dy0.clone()
+        sets.append({"x": x, "dy": d, "y": torch.empty_like(x), "dx": torch.empty_like(x),
+                     "dg": torch.empty_like(gamma), "db": torch.empty_like(gamma),
+                     "da": torch.empty(1, dtype=gamma.dtype, device=dev)})
+    ws = dyt.workspace(x0, gamma)
+    grads = torch.empty(2 * N + 1, dtype=torch.float32, device=dev)
+
+    def allreduce_grads(s):
+        grads[:N].copy_(s["dg"])
+        grads[N:2 * N].copy_(s["db"])
+        grads[2 * N:].copy_(s["da"])
+        dist.all_reduce(grads)
+        s["dg"].copy_(grads[:N])
+        s["db"].copy_(grads[N:2 * N])
+        s["da"].copy_(grads[2 * N:])
+
+    def fwd(s):
+        dyt.forward(s["x"], alpha, gamma, beta, out=s["y"])
+
+    def bwd(s):
+        dyt.backward(s["x"], s["dy"], alpha, gamma, dx=s["dx"], dgamma=s["dg"], dbeta=s["db"],
+                     dalpha=s["da"], ws=ws)
+
+    def step(i):
+        s = sets[i % nsets]
+        fwd(s)
+        bwd(s)
+        if world > 1:
+            allreduce_grads(s)
+
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize(dev)
+        launch_info_fwd = None
+
+        def capture(fn, n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    fn(i)
+            return g
+
+        g_step = capture(step, args.steps)
+        g_fwd = capture(lambda i: fwd(sets[i % nsets]), args.steps)
+        launch_info_fwd = dyt.dyt_last_launch_info()
+        g_bwd = capture(lambda i: bwd(sets[i % nsets]), args.steps)
+        launch_info_bwd = dyt.dyt_last_launch_info()
+        for g in (g_step, g_fwd, g_bwd):  # untimed replay: first-launch costs
+            g.replay()
+        torch.cuda.synchronize(dev)
+
+        def timed(g):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if world > 1:
+                dist.barrier()
+            ms = e0.elapsed_time(e1)
+            if world > 1:
+                t = torch.tensor([ms], device=dev)
+                dist.all_reduce(t, op=dist.ReduceOp.MAX)
+                ms = float(t.item())
+            return ms
+
+        with ClockSampler(local, enabled=not args.no_clocks) as clk:
+            ms_step = timed(g_step)
+            ms_fwd = timed(g_fwd)
+            ms_bwd = timed(g_bwd)
+        clocks = clk.summary()
+        del g_step, g_fwd, g_bwd  # graphs that may hold NCCL calls go before the process group
+
+    # ---- end to end through the public API: pinned host buffers in, results out ----
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, int(2e9 // max(1, set_bytes)) or 3))
+    hx = to_torch(inp["x"], w.x_dtype, "cpu").view(M, N).pin_memory()
+    hdy = to_torch(inp["dy"], w.x_dtype, "cpu").view(M, N).pin_memory()
+    hy, hdx = torch.empty_like(hx).pin_memory(), torch.empty_like(hx).pin_memory()
+    hdg = torch.empty(N, dtype=gamma.dtype).pin_memory()
+    hdb, hda = torch.empty_like(hdg).pin_memory(), torch.empty(1, dtype=gamma.dtype).pin_memory()
+    s0 = sets[0]
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            s0["x"].copy_(hx, non_blocking=True)
+            s0["dy"].copy_(hdy, non_blocking=True)
+            fwd(s0)
+            bwd(s0)
+            if world > 1:
+                allreduce_grads(s0)
+            hy.copy_(s0["y"], non_blocking=True)
+            hdx.copy_(s0["dx"], non_blocking=True)
+            hdg.copy_(s0["dg"], non_blocking=True)
+            hdb.copy_(s0["db"], non_blocking=True)
+            hda.copy_(s0["da"], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+    sx = workloads.ITEMSIZE[w.x_dtype]
+    sp = workloads.ITEMSIZE[w.p_dtype]
+    h2d = 2 * M * N * sx
+    d2h = 2 * M * N * sx + (2 * N + 1) * sp
+
+    # ---- numbers ----
+    fb, bb = w.fwd_bytes(), w.bwd_bytes()
+    step_bytes = (fb + bb) * world
+    ms_per_step = ms_step / args.steps
+    value = step_bytes / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    t_fwd, t_bwd = ms_fwd / args.steps * 1e-3, ms_bwd / args.steps * 1e-3
+    bw_fwd, bw_bwd = fb / t_fwd / 1e9, bb / t_bwd / 1e9
+    dominant = "bwd" if t_bwd >= t_fwd else "fwd"
+    traffic = committed_traffic(w.name, "dyt_bwd_kernel" if dominant == "bwd" else "dyt_fwd_kernel")
+    roofline = {
+        "bound": "hbm", "kernel": "dyt_backward (stage-1 + finalize)" if dominant == "bwd" else "dyt_forward",
+        "achieved": bw_bwd if dominant == "bwd" else bw_fwd, "peak": peak, "unit": "GB/s",
+        "frac": (bw_bwd if dominant == "bwd" else bw_fwd) / peak, "peak_kind": peak_kind,
+        "traffic": traffic,
+        "algorithmic_bytes_per_launch": bb if dominant == "bwd" else fb,
+    }
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(w), io_dtype=w.x_dtype, parallelism=f"rows{world}",
+                       l2=f"{nsets} rotating buffer sets, {nsets * set_bytes / 2**20:.0f} MiB touched per "
+                          f"cycle vs L2 {L2 / 2**20:.0f} MiB"),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "rows_per_s": M * world / (ms_per_step * 1e-3),
+        "fwd": {"us": t_fwd * 1e6, "GB_s": bw_fwd, "frac": bw_fwd / peak, "rows_per_s": M / t_fwd,
+                "launch": launch_info_fwd},
+        "bwd": {"us": t_bwd * 1e6, "GB_s": bw_bwd, "frac": bw_bwd / peak, "rows_per_s": M / t_bwd,
+                "launch": launch_info_bwd},
+        "roofline": roofline,
+        "e2e": {"value": (fb + bb) * world * e2e_steps / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": ms_e2e / e2e_steps},
+        "gpu_launches": args.steps * (launch_info_fwd["kernels"] + launch_info_bwd["kernels"]),
+        "clocks": clocks,
+    }
+    if world > 1:
+        dist.destroy_process_group()
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from synth import workloads
+
+    name = args.workload or workloads.DEFAULT_BENCH
+    w = workloads.WORKLOADS[name]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,132 @@
+"""Fused Dynamic Tanh (DyT) forward/backward for NVIDIA B200 (sm_100a).
+
+The computation lives in hand-written CUDA kernels behind a C ABI
+(``include/dyt.h``, built into ``libdyt.so``). This package is a thin layer
+over it: ctypes marshalling (``_abi``), tensor helpers that take PyTorch
+tensors for their device memory and stream, and an autograd module. PyTorch
+allocates memory and provides streams; it computes nothing here.
+
+    y = gamma * tanh(alpha * x) + beta      (x: [..., N], alpha: [1], gamma/beta: [N])
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _abi
+from ._abi import (DYT_BF16, DYT_F16, DYT_F32, DytError, dyt_backward, dyt_backward_workspace_bytes,
+                   dyt_forward, dyt_last_launch_info, dyt_plan_query, dyt_status_string)
+
+__all__ = ["forward", "backward", "workspace", "DyT", "DyTFunction", "dyt_forward", "dyt_backward",
+           "dyt_backward_workspace_bytes", "dyt_status_string", "dyt_last_launch_info", "dyt_plan_query",
+           "DytError",
+           "DTYPE_CODE", "DYT_F32", "DYT_BF16", "DYT_F16"]
+
+DTYPE_CODE = {torch.float32: DYT_F32, torch.bfloat16: DYT_BF16, torch.float16: DYT_F16}
+
+
+def _code(t: torch.Tensor, what: str) -> int:
+    try:
+        return DTYPE_CODE[t.dtype]
+    except KeyError:
+        raise TypeError(f"{what}: dtype {t.dtype} is not supported (float32, bfloat16, float16)") from None
+
+
+def _cuda_contig(t: torch.Tensor, what: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+
+
+def _shape(x: torch.Tensor, gamma: torch.Tensor):
+    N = gamma.numel()
+    if x.dim() == 0 or x.shape[-1] != N:
+        raise ValueError(f"x's last dimension {tuple(x.shape)} must equal gamma's length {N}")
+    M = x.numel() // N if N else 0
+    return M, N
+
+
+def _stream(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def forward(x: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
+            out: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """y = gamma * tanh(alpha * x) + beta in x's dtype (one kernel launch)."""
+    for t, w in ((x, "x"), (alpha, "alpha"), (gamma, "gamma"), (beta, "beta")):
+        _cuda_contig(t, w)
+    M, N = _shape(x, gamma)
+    y = torch.empty_like(x) if out is None else out
+    _cuda_contig(y, "out")
+    with torch.cuda.device(x.device):
+        st = dyt_forward(x.data_ptr(), alpha.data_ptr(), gamma.data_ptr(), beta.data_ptr(), y.data_ptr(),
+                         M, N, _code(x, "x"), _code(gamma, "gamma"), _stream(x.device, stream))
+    _abi._check(st, "dyt_forward")
+    return y
+
+
+def workspace(x: torch.Tensor, gamma: torch.Tensor) -> torch.Tensor:
+    """A device workspace large enough for backward on x's shape and device."""
+    M, N = _shape(x, gamma)
+    with torch.cuda.device(x.device):
+        n = dyt_backward_workspace_bytes(M, N, _code(x, "x"), _code(gamma, "gamma"))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=x.device)
+
+
+def backward(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor,
+             dx: torch.Tensor | None = None, dgamma: torch.Tensor | None = None,
+             dbeta: torch.Tensor | None = None, dalpha: torch.Tensor | None = None,
+             ws: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
+    """(dx, dalpha, dgamma, dbeta): dx in x's dtype, the others in gamma's dtype."""
+    for t, w in ((x, "x"), (dy, "dy"), (alpha, "alpha"), (gamma, "gamma")):
+        _cuda_contig(t, w)
+    if dy.shape != x.shape or dy.dtype != x.dtype:
+        raise ValueError("dy must match x in shape and dtype")
+    M, N = _shape(x, gamma)
+    dx = torch.empty_like(x) if dx is None else dx
+    dgamma = torch.empty_like(gamma) if dgamma is None else dgamma
+    dbeta = torch.empty_like(gamma) if dbeta is None else dbeta
+    dalpha = torch.empty(1, dtype=gamma.dtype, device=gamma.device) if dalpha is None else dalpha
+    ws = workspace(x, gamma) if ws is None else ws
+    with torch.cuda.device(x.device):
+        st = dyt_backward(x.data_ptr(), dy.data_ptr(), alpha.data_ptr(), gamma.data_ptr(), dx.data_ptr(),
+                          dgamma.data_ptr(), dbeta.data_ptr(), dalpha.data_ptr(), M, N, _code(x, "x"),
+                          _code(gamma, "gamma"), ws.data_ptr(), ws.numel(), _stream(x.device, stream))
+    _abi._check(st, "dyt_backward")
+    return dx, dalpha, dgamma, dbeta
+
+
+class DyTFunction(torch.autograd.Function):
+    """Autograd wrapper: t is recomputed in the backward, only x is saved."""
+
+    @staticmethod
+    def forward(ctx, x, alpha, gamma, beta):
+        x, alpha, gamma, beta = (t.contiguous() for t in (x, alpha, gamma, beta))
+        ctx.save_for_backward(x, alpha, gamma)
+        return forward(x, alpha, gamma, beta)
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, alpha, gamma = ctx.saved_tensors
+        dx, dalpha, dgamma, dbeta = backward(x, dy.contiguous(), alpha, gamma)
+        return dx, dalpha.reshape(alpha.shape), dgamma, dbeta
+
+
+class DyT(torch.nn.Module):
+    """DyT(x) = gamma * tanh(alpha * x) + beta over the last dimension.
+
+    alpha is one scalar parameter; gamma and beta have one entry per channel.
+    Parameters live in ``param_dtype``; gradients come back in it.
+    """
+
+    def __init__(self, num_features: int, alpha_init: float = 0.5, param_dtype=torch.float32,
+                 device=None):
+        super().__init__()
+        self.alpha = torch.nn.Parameter(torch.full((1,), alpha_init, dtype=param_dtype, device=device))
+        self.gamma = torch.nn.Parameter(torch.ones(num_features, dtype=param_dtype, device=device))
+        self.beta = torch.nn.Parameter(torch.zeros(num_features, dtype=param_dtype, device=device))
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        return DyTFunction.apply(x, self.alpha, self.gamma, self.beta)

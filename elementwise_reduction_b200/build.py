@@ -1,0 +1,49 @@
+"""Build libdyt.so (the C-ABI library) in-tree with nvcc for sm_100a.
+
+Run as ``python elementwise_reduction_b200/build.py`` (by path: importing the package
+loads the library this script builds).
+No GPU is needed to build.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libdyt.so")
+SOURCES = [os.path.join(CSRC, "dyt_api.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("dyt_kernels.cuh", "dyt_math.cuh")] + [
+    os.path.join(INCLUDE, "dyt.h")]
+
+NVCC_FLAGS = [
+    "-std=c++17", "-O3", "-lineinfo",
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-Xcompiler", "-fPIC", "-shared",
+    "-I", INCLUDE, "-I", CSRC,
+]
+
+
+def nvcc() -> str:
+    cand = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    return cand if os.path.exists(cand) else "nvcc"
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libdyt.so if any source is newer than it. Returns its path."""
+    if not force and os.path.exists(LIB):
+        built = os.path.getmtime(LIB)
+        if all(os.path.getmtime(d) <= built for d in DEPS):
+            return LIB
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", LIB + ".tmp", *SOURCES,
+           "-lcudart"]
+    subprocess.check_call(cmd)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force=True, verbose="-v" in sys.argv))

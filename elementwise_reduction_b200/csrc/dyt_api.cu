@@ -1,0 +1,390 @@
+// C ABI of the fused DyT layer (declared in include/dyt.h): argument checks,
+// launch planning and kernel dispatch. All device work is in dyt_kernels.cuh.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include "dyt.h"
+#include "dyt_kernels.cuh"
+
+namespace {
+
+using dyt::Geom;
+
+thread_local dyt_launch_info t_info = {};
+thread_local int t_cuda_err = 0;
+
+constexpr int kBlock = 1024;          // threads per CTA of the main kernels
+constexpr int kMaxRowsPerLane = 96;   // sequential binary32 adds per thread per group
+constexpr int kUnrollVec = 2;         // rows in flight per thread, 16-byte access
+constexpr int kUnrollScalar = 8;      // rows in flight per thread, scalar access
+
+dyt_status cuda_fail(cudaError_t e) {
+  t_cuda_err = (int)e;
+  return DYT_ERR_CUDA;
+}
+
+size_t dsize(dyt_dtype d) { return d == DYT_F32 ? 4 : 2; }
+bool valid_dtype(int d) { return d == DYT_F32 || d == DYT_BF16 || d == DYT_F16; }
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---- per-device facts and per-kernel occupancy (cached, thread-safe) -------
+
+std::mutex g_mu;
+std::unordered_map<int, int> g_sms;                   // device -> SM count
+std::unordered_map<uint64_t, int> g_occ;              // (device, kernel) -> CTAs per SM
+
+dyt_status current_sms(int *dev_out, int *sms_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_sms.find(dev);
+    if (it != g_sms.end()) {
+      *dev_out = dev;
+      *sms_out = it->second;
+      return DYT_OK;
+    }
+  }
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_sms[dev] = sms;
+  *dev_out = dev;
+  *sms_out = sms;
+  return DYT_OK;
+}
+
+dyt_status occupancy(int dev, const void *kernel, int block, int *ctas) {
+  const uint64_t key = ((uint64_t)(uint32_t)dev << 48) ^ (uint64_t)(uintptr_t)kernel;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_occ.find(key);
+    if (it != g_occ.end()) {
+      *ctas = it->second;
+      return DYT_OK;
+    }
+  }
+  int n = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, 0);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (n < 1) n = 1;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_occ[key] = n;
+  *ctas = n;
+  return DYT_OK;
+}
+
+// ---- launch plan ---------------------------------------------------------------
+
+struct Plan {
+  Geom g;
+  int vec;
+  int unroll;
+  int grid;
+  int path;
+  size_t ws_dg, ws_db, ws_da, ws_total;  // workspace byte offsets / sizes
+};
+
+size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
+
+// vec: elements per access (1 or 16 / element size). ctas_per_sm from the
+// kernel's occupancy. The plan depends only on (M, N, vec, SM count, occupancy).
+Plan make_plan(int64_t M, int64_t N, int vec, int sms, int ctas_per_sm) {
+  Plan p = {};
+  p.vec = vec;
+  p.unroll = vec > 1 ? kUnrollVec : kUnrollScalar;
+  const int64_t NV = N / vec;
+  Geom &g = p.g;
+  g.M = M;
+  g.N = N;
+  g.NV = (int)NV;
+  if (NV <= kBlock / 2) {
+    g.RL = kBlock / (int)NV;
+    g.ncc = 1;
+    p.path = 1;
+  } else {
+    g.RL = 1;
+    g.ncc = (int)ceil_div(NV, kBlock);
+    p.path = 2;
+  }
+  const int64_t target = (int64_t)sms * ctas_per_sm;
+  // One wave of items: `fill` row groups per column chunk, fill * ncc <= target
+  // (at least one group), but no group thinner than one row per lane.
+  int64_t fill = target / g.ncc;
+  if (fill < 1) fill = 1;
+  const int64_t rows_per_lane_min = ceil_div(M, (int64_t)g.RL);
+  if (fill > rows_per_lane_min) fill = rows_per_lane_min;
+  int64_t nrg = fill;
+  // Cap the rows a lane adds in one group; keep the group count a multiple of
+  // the fill so every CTA gets the same number of items.
+  const int64_t max_rows = (int64_t)g.RL * kMaxRowsPerLane;
+  if (ceil_div(M, nrg) > max_rows) nrg = ceil_div(ceil_div(M, max_rows), fill) * fill;
+  g.nrg = (int)nrg;
+  g.nitems = (int)(nrg * g.ncc);
+  int64_t grid = fill * g.ncc;
+  if (grid > target) grid = target;
+  if (grid > g.nitems) grid = g.nitems;
+  p.grid = (int)grid;
+  p.ws_dg = 0;
+  p.ws_db = align16((size_t)nrg * (size_t)N * sizeof(float));
+  p.ws_da = p.ws_db + align16((size_t)nrg * (size_t)N * sizeof(float));
+  p.ws_total = p.ws_da + align16((size_t)p.grid * sizeof(double));
+  return p;
+}
+
+// ---- kernel tables ---------------------------------------------------------------
+
+template <typename T>
+constexpr int vec_of() {
+  return 16 / (int)sizeof(T);
+}
+
+template <typename T, typename P>
+const void *fwd_kernel(int vec) {
+  if (vec > 1) return (const void *)dyt::dyt_fwd_kernel<T, P, vec_of<T>(), kUnrollVec, kBlock>;
+  return (const void *)dyt::dyt_fwd_kernel<T, P, 1, kUnrollScalar, kBlock>;
+}
+
+template <typename T, typename P>
+const void *bwd_kernel(int vec) {
+  if (vec > 1) return (const void *)dyt::dyt_bwd_kernel<T, P, vec_of<T>(), kUnrollVec, kBlock>;
+  return (const void *)dyt::dyt_bwd_kernel<T, P, 1, kUnrollScalar, kBlock>;
+}
+
+template <typename F>
+dyt_status with_types(dyt_dtype xd, dyt_dtype pd, F &&f) {
+  auto with_p = [&](auto tx) -> dyt_status {
+    using T = decltype(tx);
+    switch (pd) {
+      case DYT_F32: return f(T{}, float{});
+      case DYT_BF16: return f(T{}, __nv_bfloat16{});
+      case DYT_F16: return f(T{}, __half{});
+    }
+    return DYT_ERR_UNSUPPORTED_DTYPE;
+  };
+  switch (xd) {
+    case DYT_F32: return with_p(float{});
+    case DYT_BF16: return with_p(__nv_bfloat16{});
+    case DYT_F16: return with_p(__half{});
+  }
+  return DYT_ERR_UNSUPPORTED_DTYPE;
+}
+
+dyt_status check_shape(int64_t M, int64_t N, dyt_dtype xd, dyt_dtype pd) {
+  if (!valid_dtype(xd) || !valid_dtype(pd)) return DYT_ERR_UNSUPPORTED_DTYPE;
+  if (M < 0 || N < 0 || N > INT32_MAX) return DYT_ERR_INVALID_VALUE;
+  if (N > 0 && M > INT64_MAX / N / 8) return DYT_ERR_INVALID_VALUE;
+  // group and item counts are ints
+  if (M > ((int64_t)1 << 40)) return DYT_ERR_INVALID_VALUE;
+  return DYT_OK;
+}
+
+dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
+  dyt_launch_info i = {};
+  i.op = op;
+  i.kernels = kernels;
+  i.workspace_bytes = (int64_t)ws;
+  if (p) {
+    i.path = p->path;
+    i.vec = p->vec;
+    i.block = kBlock;
+    i.grid = p->grid;
+    i.row_lanes = p->g.RL;
+    i.rows_per_step = p->g.RL * p->unroll;
+    i.col_chunks = p->g.ncc;
+    i.row_groups = p->g.nrg;
+  }
+  return i;
+}
+
+void record(int op, const Plan *p, int kernels, size_t ws) { t_info = describe(op, p, kernels, ws); }
+
+// Plan for given pointers' alignment on the current device.
+template <typename T, typename P>
+dyt_status plan_for(int64_t M, int64_t N, bool vec_ok, bool backward, Plan *out) {
+  int dev = 0, sms = 0;
+  dyt_status st = current_sms(&dev, &sms);
+  if (st != DYT_OK) return st;
+  const int vec = (vec_ok && N % vec_of<T>() == 0) ? vec_of<T>() : 1;
+  const void *k = backward ? bwd_kernel<T, P>(vec) : fwd_kernel<T, P>(vec);
+  int occ = 1;
+  st = occupancy(dev, k, kBlock, &occ);
+  if (st != DYT_OK) return st;
+  *out = make_plan(M, N, vec, sms, occ);
+  return DYT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, const void *beta, void *y,
+                       int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
+                       dyt_stream_t stream) {
+  dyt_status st = check_shape(M, N, x_dtype, param_dtype);
+  if (st != DYT_OK) return st;
+  if (M == 0 || N == 0) {
+    record(1, nullptr, 0, 0);
+    return DYT_OK;
+  }
+  if (!x || !alpha || !gamma || !beta || !y) return DYT_ERR_INVALID_VALUE;
+  return with_types(x_dtype, param_dtype, [&](auto tx, auto tp) -> dyt_status {
+    using T = decltype(tx);
+    using P = decltype(tp);
+    constexpr int V = vec_of<T>();
+    Plan p;
+    dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y), false, &p);
+    if (s != DYT_OK) return s;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(kBlock);
+    cfg.stream = (cudaStream_t)stream;
+    cudaError_t e;
+    if (p.vec > 1)
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, V, kUnrollVec, kBlock>,
+                             (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y,
+                             p.g);
+    else
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, 1, kUnrollScalar, kBlock>, (const T *)x,
+                             (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
+    if (e != cudaSuccess) return cuda_fail(e);
+    record(1, &p, 1, 0);
+    return DYT_OK;
+  });
+}
+
+size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype) {
+  if (check_shape(M, N, x_dtype, param_dtype) != DYT_OK) return 0;
+  if (M == 0 || N == 0) return 0;
+  size_t need = 0;
+  dyt_status st = with_types(x_dtype, param_dtype, [&](auto tx, auto tp) -> dyt_status {
+    using T = decltype(tx);
+    using P = decltype(tp);
+    // The vectorised and the scalar plan may differ; cover both.
+    for (int v = 0; v < 2; ++v) {
+      Plan p;
+      dyt_status s = plan_for<T, P>(M, N, v == 1, true, &p);
+      if (s != DYT_OK) return s;
+      if (p.ws_total > need) need = p.ws_total;
+    }
+    return DYT_OK;
+  });
+  return st == DYT_OK ? need : 0;
+}
+
+dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const void *gamma, void *dx,
+                        void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
+                        dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace,
+                        size_t workspace_bytes, dyt_stream_t stream) {
+  dyt_status st = check_shape(M, N, x_dtype, param_dtype);
+  if (st != DYT_OK) return st;
+  if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return DYT_ERR_INVALID_VALUE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t ps = dsize(param_dtype);
+  if (M == 0 || N == 0) {
+    // Empty sums: every gradient is +0 (all-zero bits in each dtype).
+    cudaError_t e = cudaSuccess;
+    if (N > 0) {
+      e = cudaMemsetAsync(dgamma, 0, (size_t)N * ps, s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, (size_t)N * ps, s);
+    }
+    if (e == cudaSuccess) e = cudaMemsetAsync(dalpha, 0, ps, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    record(2, nullptr, 0, 0);
+    return DYT_OK;
+  }
+  if (!x || !dy || !alpha || !gamma || !dx || !workspace) return DYT_ERR_INVALID_VALUE;
+  if (!aligned16(workspace)) return DYT_ERR_INVALID_VALUE;
+  return with_types(x_dtype, param_dtype, [&](auto tx, auto tp) -> dyt_status {
+    using T = decltype(tx);
+    using P = decltype(tp);
+    constexpr int V = vec_of<T>();
+    Plan p;
+    dyt_status r = plan_for<T, P>(M, N, aligned16(x) && aligned16(dy) && aligned16(dx), true, &p);
+    if (r != DYT_OK) return r;
+    if (workspace_bytes < p.ws_total) return DYT_ERR_WORKSPACE_TOO_SMALL;
+    char *ws = (char *)workspace;
+    float *pdg = (float *)(ws + p.ws_dg);
+    float *pdb = (float *)(ws + p.ws_db);
+    double *pda = (double *)(ws + p.ws_da);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(kBlock);
+    cfg.stream = s;
+    cudaError_t e;
+    if (p.vec > 1)
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, V, kUnrollVec, kBlock>,
+                             (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx,
+                             pdg, pdb, pda, p.g);
+    else
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, 1, kUnrollScalar, kBlock>, (const T *)x,
+                             (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda,
+                             p.g);
+    if (e != cudaSuccess) return cuda_fail(e);
+
+    // Stage 2, as a programmatic dependent launch: it may start while stage 1
+    // drains and waits (griddepcontrol.wait) for stage 1's results.
+    const int CT = N >= (int64_t)32 * 148 ? 32 : 8;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t fcfg = {};
+    fcfg.gridDim = dim3((unsigned)ceil_div(N, CT));
+    fcfg.blockDim = dim3(dyt::kFinThreads);
+    fcfg.stream = s;
+    fcfg.attrs = attr;
+    fcfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&fcfg, dyt::dyt_finalize_kernel<P>, (const float *)pdg, (const float *)pdb,
+                           (const double *)pda, (P *)dgamma, (P *)dbeta, (P *)dalpha, (int64_t)N,
+                           p.g.nrg, p.grid, CT);
+    if (e != cudaSuccess) return cuda_fail(e);
+    record(2, &p, 2, p.ws_total);
+    return DYT_OK;
+  });
+}
+
+const char *dyt_status_string(dyt_status status) {
+  switch (status) {
+    case DYT_OK: return "DYT_OK";
+    case DYT_ERR_INVALID_VALUE: return "DYT_ERR_INVALID_VALUE: bad pointer, size or alignment";
+    case DYT_ERR_UNSUPPORTED_DTYPE: return "DYT_ERR_UNSUPPORTED_DTYPE";
+    case DYT_ERR_WORKSPACE_TOO_SMALL: return "DYT_ERR_WORKSPACE_TOO_SMALL";
+    case DYT_ERR_CUDA: return "DYT_ERR_CUDA: the CUDA runtime refused a query or a launch";
+  }
+  return "DYT_ERR_UNKNOWN";
+}
+
+int dyt_last_cuda_error(void) { return t_cuda_err; }
+
+dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype, int backward,
+                          int vectorized, int sm_count, int ctas_per_sm, dyt_launch_info *out) {
+  if (!out || sm_count < 1 || ctas_per_sm < 1) return DYT_ERR_INVALID_VALUE;
+  dyt_status st = check_shape(M, N, x_dtype, param_dtype);
+  if (st != DYT_OK) return st;
+  const int op = backward ? 2 : 1;
+  if (M == 0 || N == 0) {
+    *out = describe(op, nullptr, 0, 0);
+    return DYT_OK;
+  }
+  const int v = 16 / (int)dsize(x_dtype);
+  const int vec = (vectorized && N % v == 0) ? v : 1;
+  const Plan p = make_plan(M, N, vec, sm_count, ctas_per_sm);
+  *out = describe(op, &p, backward ? 2 : 1, backward ? p.ws_total : 0);
+  return DYT_OK;
+}
+
+dyt_status dyt_last_launch_info(dyt_launch_info *out) {
+  if (!out) return DYT_ERR_INVALID_VALUE;
+  *out = t_info;
+  return DYT_OK;
+}
+
+}  // extern "C"

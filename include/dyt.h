@@ -1,0 +1,172 @@
+/*
+ * dyt.h -- C ABI of the fused Dynamic Tanh (DyT) layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one of the Liger-Kernel pull request "fix(dyt): use a 1D
+ * grid and tile small-width rows" (Summary): a scalar alpha, per-column gamma
+ * and beta, a fused forward kernel and a fused backward kernel that returns
+ * dx and the parameter gradients dalpha, dgamma and dbeta. For an M x N
+ * row-major activation x:
+ *
+ *   forward   y[i,j]    = gamma[j] * tanh(alpha * x[i,j]) + beta[j]
+ *   backward  t[i,j]    = tanh(alpha * x[i,j])            (recomputed, not saved)
+ *             dx[i,j]   = alpha * gamma[j] * dy[i,j] * (1 - t[i,j]^2)
+ *             dgamma[j] = sum_i dy[i,j] * t[i,j]
+ *             dbeta[j]  = sum_i dy[i,j]
+ *             dalpha    = sum_{i,j} gamma[j] * dy[i,j] * (1 - t[i,j]^2) * x[i,j]
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers: every tensor pointer is a DEVICE pointer (or memory the device
+ *   can address, such as managed memory), alpha included, so no call reads
+ *   device memory on the host or synchronises. The caller owns every buffer,
+ *   the workspace included; the library allocates nothing and keeps no state
+ *   other than the calling thread's last-launch record.
+ * - Layout: x, dy, y and dx are contiguous row-major M x N arrays (row stride
+ *   N elements). gamma, beta, dgamma and dbeta hold N elements; alpha and
+ *   dalpha hold one. Any alignment is accepted; 16-byte aligned tensors take
+ *   the vectorised path.
+ * - Dtypes (the page's Summary, "Precision"): x, dy, y and dx share x_dtype;
+ *   alpha, gamma, beta and all three parameter gradients share param_dtype.
+ *   y and dx come back in x_dtype, the parameter gradients in param_dtype.
+ *   Arithmetic is binary32 with binary64 partial sums.
+ * - Outputs are overwritten, never accumulated into.
+ * - Aliasing: y may alias x, and dx may alias x or dy (each element is read
+ *   before the same thread writes it). Any other overlap is undefined.
+ * - Sizes: M, N >= 0 and M * N * element size must fit in int64. M is not
+ *   limited by the CUDA grid (the page's Summary, "Launch limit": more than
+ *   65,535 rows must launch): the grid is one-dimensional and persistent.
+ * - Asynchrony: calls only enqueue work on `stream` (0 = legacy default
+ *   stream) and return. DYT_ERR_CUDA reports a launch error; a fault in a
+ *   kernel surfaces at the caller's next synchronisation. No call aborts, and
+ *   no failure is reported as DYT_OK.
+ * - Results are deterministic: the same inputs on the same device give the
+ *   same bits (static schedule, fixed reduction order, no atomics in sums).
+ */
+#ifndef DYT_H_
+#define DYT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t. */
+typedef struct CUstream_st *dyt_stream_t;
+
+typedef enum dyt_dtype {
+  DYT_F32 = 0,  /* IEEE binary32 */
+  DYT_BF16 = 1, /* bfloat16 */
+  DYT_F16 = 2   /* IEEE binary16 */
+} dyt_dtype;
+
+typedef enum dyt_status {
+  DYT_OK = 0,
+  DYT_ERR_INVALID_VALUE = 1,       /* null pointer, negative size, size overflow, bad enum */
+  DYT_ERR_UNSUPPORTED_DTYPE = 2,   /* dtype enum outside dyt_dtype */
+  DYT_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < dyt_backward_workspace_bytes(...) */
+  DYT_ERR_CUDA = 4                 /* the CUDA runtime refused a query or a launch */
+} dyt_status;
+
+/*
+ * Forward: y = gamma * tanh(alpha * x) + beta, one kernel launch.
+ *   x      [M*N] x_dtype, read
+ *   alpha  [1]   param_dtype, read on the device
+ *   gamma  [N]   param_dtype, read
+ *   beta   [N]   param_dtype, read
+ *   y      [M*N] x_dtype, written (may alias x)
+ * Each y element is rounded once to x_dtype. For 16-bit x_dtype an element
+ * whose binary32 value of gamma*t + beta cancels (|y| < tau |gamma*t|, tau =
+ * 2^-12 for bf16 and 2^-9 for fp16) is recomputed in binary64, so every y is
+ * within one unit in the last place of the correctly rounded value.
+ * M * N == 0 launches nothing. Null pointers with M * N > 0 give
+ * DYT_ERR_INVALID_VALUE.
+ */
+dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, const void *beta,
+                       void *y, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
+                       dyt_stream_t stream);
+
+/*
+ * Bytes of device workspace dyt_backward needs for this shape on the CURRENT
+ * device (the grid, and with it the number of partial sums, depends on the
+ * device's SM count). Returns 0 for invalid arguments or when no workspace is
+ * needed (M * N == 0).
+ */
+size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype);
+
+/*
+ * Backward: recomputes t = tanh(alpha * x) and writes dx, dgamma, dbeta and
+ * dalpha. Two kernel launches on `stream`: the fused elementwise pass, which
+ * also writes partial sums to the workspace (binary32 per row group and
+ * column for dgamma and dbeta, binary64 per CTA for dalpha), and a finalize
+ * pass that adds the partials in binary64 in a fixed order and rounds them
+ * once to param_dtype.
+ *   x, dy     [M*N] x_dtype, read
+ *   alpha     [1]   param_dtype, read on the device
+ *   gamma     [N]   param_dtype, read
+ *   dx        [M*N] x_dtype, written (may alias x or dy)
+ *   dgamma    [N]   param_dtype, written
+ *   dbeta     [N]   param_dtype, written
+ *   dalpha    [1]   param_dtype, written
+ *   workspace device scratch of at least dyt_backward_workspace_bytes(M, N,
+ *             x_dtype, param_dtype) bytes, 16-byte aligned, owned by the
+ *             caller; its contents on entry do not matter and on exit are
+ *             unspecified. Two calls in flight at once need two workspaces.
+ * Contributions of lanes outside [0,M) x [0,N) are removed by a select after
+ * the arithmetic, never by multiplying with a mask (the page's Summary,
+ * "Padding"), so alpha = +inf cannot put NaN into the sums through them.
+ * With M * N == 0: dgamma and dbeta (when N > 0) and dalpha are set to zero,
+ * and no workspace is used.
+ */
+dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const void *gamma,
+                        void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
+                        dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace,
+                        size_t workspace_bytes, dyt_stream_t stream);
+
+/* Static, human-readable name of a status. Never NULL. */
+const char *dyt_status_string(dyt_status status);
+
+/* The cudaError_t value behind the calling thread's last DYT_ERR_CUDA (0 if none). */
+int dyt_last_cuda_error(void);
+
+/*
+ * Launch geometry of the calling thread's last successful dyt_forward or
+ * dyt_backward call, so tests can check which path ran.
+ */
+typedef struct dyt_launch_info {
+  int op;            /* 1 = forward, 2 = backward, 0 = none yet */
+  int path;          /* 0 = nothing launched, 1 = row-tiled (several rows per CTA step),
+                        2 = row-per-CTA (one row per CTA step, columns across threads) */
+  int vec;           /* elements per vector access (1 = scalar) */
+  int block;         /* threads per CTA */
+  int grid;          /* CTAs of the main kernel (1D) */
+  int row_lanes;     /* rows one CTA step covers side by side */
+  int rows_per_step; /* rows one CTA step covers in total */
+  int col_chunks;    /* column chunks the grid is split into */
+  int row_groups;    /* row groups (= partial sums per column) */
+  int kernels;       /* kernels this call launched */
+  int64_t workspace_bytes;
+} dyt_launch_info;
+
+dyt_status dyt_last_launch_info(dyt_launch_info *out);
+
+/*
+ * The launch plan dyt_forward (backward = 0) or dyt_backward (backward != 0)
+ * would use for this shape on a device with `sm_count` SMs running
+ * `ctas_per_sm` CTAs of the kernel each, with 16-byte aligned tensors
+ * (vectorized != 0) or not. Host arithmetic only: touches no device, so the
+ * planning is testable without a GPU. out->kernels is the number of kernels
+ * the call would launch and out->workspace_bytes the workspace it needs.
+ * Errors: as the shape checks of dyt_forward, or DYT_ERR_INVALID_VALUE for
+ * out == NULL or sm_count / ctas_per_sm < 1.
+ */
+dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
+                          int backward, int vectorized, int sm_count, int ctas_per_sm,
+                          dyt_launch_info *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DYT_H_ */

@@ -1,0 +1,107 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry point,
+validates arguments on the host, and plans launches (host arithmetic only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dyt.h")
+
+
+def _lib():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("dyt_build", os.path.join(ROOT, "elementwise_reduction_b200",
+                                                                            "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import elementwise_reduction_b200 as dyt
+    return dyt
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dyt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("dyt_forward", "dyt_backward", "dyt_backward_workspace_bytes", "dyt_status_string",
+              "dyt_last_launch_info", "dyt_plan_query"):
+        assert f in names
+
+
+def test_library_exports_every_declared_function():
+    dyt = _lib()
+    lib = ctypes.CDLL(dyt._abi.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/dyt.h but not exported"
+
+
+def test_host_validation_without_a_device():
+    dyt = _lib()
+    # negative sizes, bad dtypes and null pointers are rejected before any CUDA call
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, -1, 4, 0, 0, None) == 1
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, 4, -1, 0, 0, None) == 1
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, 4, 4, 7, 0, None) == 2
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, 4, 4, 0, 3, None) == 2
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, 4, 4, 0, 0, None) == 1          # null pointers
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, 4, 2**31, 0, 0, None) == 1      # N beyond int32
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, 2**62, 2**20, 0, 0, None) == 1  # M*N*size overflows
+    assert dyt.dyt_forward(0, 0, 0, 0, 0, 0, 5, 0, 0, None) == 0          # empty: nothing to do
+    assert dyt.dyt_last_launch_info()["kernels"] == 0
+    assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 0, 3, 3, 0, 0, 0, 0, None) == 1  # null dalpha
+    assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 1, 3, 3, 1, 0, 0, 0, None) == 1  # null dgamma/dbeta
+    assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 0, -3, 3, 0, 0, 0, 0, None) == 1
+    assert dyt.dyt_backward_workspace_bytes(-1, 3, 0, 0) == 0
+    assert dyt.dyt_backward_workspace_bytes(0, 3, 0, 0) == 0
+    for s in range(5):
+        assert dyt.dyt_status_string(s).startswith("DYT_")
+    assert dyt.dyt_status_string(99) == "DYT_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("M,N,xd", [(1024, 64, 0), (65537, 32, 1), (100003, 17, 0), (100003, 100, 0),
+                                    (100003, 255, 0), (16384, 4096, 1), (32768, 8192, 1), (1, 1, 0),
+                                    (3, 70000, 2), (10**7, 8, 1), (5, 513, 0)])
+@pytest.mark.parametrize("vectorized", [0, 1])
+@pytest.mark.parametrize("sms,occ", [(148, 1), (148, 2), (7, 1)])
+def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
+    dyt = _lib()
+    p = dyt.dyt_plan_query(M, N, xd, 0, 1, vectorized, sms, occ)
+    size = 4 if xd == 0 else 2
+    vec = p["vec"]
+    assert vec in (1, 16 // size)
+    if vec > 1:
+        assert vectorized and N % vec == 0
+    nv = N // vec
+    assert p["block"] == 1024 and p["kernels"] == 2
+    assert 1 <= p["grid"] <= sms * occ            # persistent 1D grid: never beyond one wave
+    if p["path"] == 1:                             # row-tiled: several rows per CTA step
+        assert p["row_lanes"] == 1024 // nv >= 2 and p["col_chunks"] == 1
+    else:                                          # row-per-CTA: columns across the CTA
+        assert p["row_lanes"] == 1 and p["col_chunks"] == -(-nv // 1024)
+    items = p["row_groups"] * p["col_chunks"]
+    assert p["grid"] <= items
+    # every lane adds at most 96 rows per group (bounded binary32 error)
+    rows_per_group = -(-M // p["row_groups"])
+    assert -(-rows_per_group // p["row_lanes"]) <= 96
+    # every CTA gets the same number of work items, unless there are more
+    # column chunks than CTAs
+    if p["col_chunks"] <= sms * occ:
+        assert items % p["grid"] == 0
+        assert p["grid"] > (sms * occ) // 2 or p["grid"] == items
+    # workspace: binary32 dgamma and dbeta partials per group and column + binary64 dalpha per CTA
+    al = lambda v: (v + 15) // 16 * 16
+    assert p["workspace_bytes"] == 2 * al(p["row_groups"] * N * 4) + al(p["grid"] * 8)
+
+
+def test_page_narrow_widths_take_the_row_tiled_path():
+    dyt = _lib()
+    for N in (16, 17, 32, 64, 100, 128, 255, 256):
+        for xd in (0, 1, 2):
+            p = dyt.dyt_plan_query(65537, N, xd, 0, 1, 1, 148, 1)
+            assert p["path"] == 1 and p["rows_per_step"] > 1
+    assert dyt.dyt_plan_query(32768, 8192, 1, 0, 1, 1, 148, 1)["path"] == 2

@@ -1,0 +1,306 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on seeded synthetic inputs.
+
+Tolerances are those of tests/helpers.py. Shapes cover several tiles and a
+ragged tail, both launch paths, every dtype pair, the edge cases of the
+Liger-Kernel page ("fix(dyt): use a 1D grid and tile small-width rows":
+65,537 rows, small and ragged widths, infinite alpha with padded rows, bf16
+activations with fp32 parameters) and the full-size workloads on sampled rows.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import workloads
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    import elementwise_reduction_b200  # noqa: F401  (fails loudly if libdyt.so is missing)
+
+
+def make(M, N, x_dtype="f32", p_dtype="f32", alpha=0.7, x_std=1.0, dy_std=1.0, seed=0, nonzero=False,
+         gamma_std=0.1, beta_std=0.1):
+    w = workloads.Workload("case", M, N, x_dtype, p_dtype, alpha=alpha, x_std=x_std, dy_std=dy_std,
+                           gamma_std=gamma_std, beta_std=beta_std, nonzero=nonzero, seed=seed)
+    return workloads.make_inputs(w)
+
+
+def roundtrip(M, N, xd="f32", pd="f32", **kw):
+    inp = make(M, N, xd, pd, **kw)
+    out, info = H.run_cuda(inp, M, N, xd, pd)
+    stats = H.compare_all(inp, out, M, N, xd, pd)
+    return out, info, stats
+
+
+# ---- shape sweep: both paths, tile boundaries, ragged tails ----------------------------------
+
+NARROW = [1, 2, 3, 4, 7, 8, 9, 16, 17, 31, 32, 33, 63, 64, 100, 127, 128, 129, 255, 256]
+WIDE = [257, 511, 512, 513, 1000, 1024, 2048, 4096, 4104, 8192, 8200, 16392]
+
+
+@pytest.mark.parametrize("N", NARROW)
+@pytest.mark.parametrize("xd,pd", [("f32", "f32"), ("bf16", "f32")])
+def test_narrow_widths(N, xd, pd):
+    M = 3000 + 7  # several groups and a ragged last step
+    _, info, _ = roundtrip(M, N, xd, pd)
+    assert info["bwd"]["path"] == 1 and info["fwd"]["path"] == 1
+
+
+@pytest.mark.parametrize("N", WIDE)
+@pytest.mark.parametrize("xd,pd", [("f32", "f32"), ("bf16", "f32"), ("f16", "f32")])
+def test_wide_widths(N, xd, pd):
+    M = 97
+    roundtrip(M, N, xd, pd)
+
+
+@pytest.mark.parametrize("xd,pd", [("f32", "bf16"), ("f32", "f16"), ("bf16", "bf16"), ("f16", "f16"),
+                                   ("bf16", "f16"), ("f16", "bf16")])
+@pytest.mark.parametrize("M,N", [(513, 64), (257, 17), (33, 4096), (5, 9000)])
+def test_dtype_matrix(xd, pd, M, N):
+    roundtrip(M, N, xd, pd)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 255, 256, 257, 1023, 1025])
+def test_row_counts(M):
+    roundtrip(M, 64, "bf16", "f32")
+    roundtrip(M, 4096, "bf16", "f32")
+
+
+# ---- edge cases from the page and the method ---------------------------------------------------
+
+def test_page_row_count_crosses_grid_limit():
+    facts = json.load(open(os.path.join(GOLDEN, "liger_dyt_page_facts.json")))
+    M = facts["rows_case"]["value"]
+    assert M > facts["grid_dim_limit"]["value"]
+    for N, xd in ((32, "bf16"), (1, "f32"), (300, "f32")):
+        _, info, _ = roundtrip(M, N, xd, "f32")
+        assert info["bwd"]["grid"] <= 148 * 8  # 1D persistent grid
+
+
+@pytest.mark.parametrize("N", [17, 100, 255, 1, 7, 300, 4100])
+@pytest.mark.parametrize("xd", ["f32", "bf16"])
+def test_infinite_alpha_with_padded_rows(N, xd):
+    # Ragged row counts leave padded lanes in the last step; with alpha = +inf a
+    # padded zero would give tanh(inf * 0) = NaN unless masked after the arithmetic.
+    M = 1000 + 13
+    inp = make(M, N, xd, "f32", alpha=float("inf"), nonzero=True)
+    out, info = H.run_cuda(inp, M, N, xd, "f32")
+    H.compare_all(inp, out, M, N, xd, "f32")
+    dg = H.decode(out["dgamma"], "f32")
+    db = H.decode(out["dbeta"], "f32")
+    assert np.isfinite(dg).all() and np.isfinite(db).all()
+    assert out["dalpha"] == 0.0
+    assert np.isnan(H.decode(out["dx"], xd)).all()
+
+
+def test_alpha_zero_gives_beta_and_zero_gradients():
+    M, N = 777, 96
+    for xd in ("f32", "bf16"):
+        inp = make(M, N, xd, "f32", alpha=0.0)
+        out, _ = H.run_cuda(inp, M, N, xd, "f32")
+        y = H.decode(out["y"], xd).reshape(M, N)
+        want = H.decode(oracle.round_to(inp["beta"].astype(np.float64), xd), xd)
+        assert np.array_equal(y, np.broadcast_to(want, (M, N)))
+        assert np.all(H.decode(out["dx"], xd) == 0.0)
+        assert np.all(H.decode(out["dgamma"], "f32") == 0.0)
+        H.compare_all(inp, out, M, N, xd, "f32")
+
+
+def test_odd_symmetry_with_zero_beta():
+    M, N = 300, 130
+    inp = make(M, N, "f32", "f32", alpha=1.1)
+    inp["beta"] = np.zeros(N, np.float32)
+    out, _ = H.run_cuda(inp, M, N, "f32", "f32", bwd=False)
+    neg = dict(inp, x=(-inp["x"]).astype(np.float32))
+    outn, _ = H.run_cuda(neg, M, N, "f32", "f32", bwd=False)
+    assert np.array_equal(outn["y"], -out["y"])
+
+
+def test_dbeta_is_exact_for_integer_dy():
+    M, N = 5000, 40
+    inp = make(M, N, "f32", "f32")
+    inp["dy"] = np.round(synth.normal(M * N, "f32", 0.0, 8.0, 1, 2)).astype(np.float32)
+    out, _ = H.run_cuda(inp, M, N, "f32", "f32", fwd=False)
+    want = inp["dy"].astype(np.int64).reshape(M, N).sum(0)
+    assert np.array_equal(H.decode(out["dbeta"], "f32"), want.astype(np.float64))
+
+
+def test_cancelling_outputs_are_correctly_rounded():
+    # beta chosen so that gamma * tanh(alpha * x) + beta cancels for many x: each
+    # column's beta is minus the value at one of its own entries.
+    M, N = 4096, 64
+    for xd in ("bf16", "f16"):
+        inp = make(M, N, xd, "f32", alpha=0.9)
+        X = H.decode(inp["x"], xd).reshape(M, N)
+        g = inp["gamma"].astype(np.float64)
+        inp["beta"] = (-g * np.tanh(0.9 * X[17])).astype(np.float32)
+        out, _ = H.run_cuda(inp, M, N, xd, "f32", bwd=False)
+        st = H.compare_all(inp, out, M, N, xd, "f32")
+        assert st["y"]["max_ulp"] <= 1
+
+
+def test_extreme_arguments():
+    # Large |alpha x| (tanh saturates, 1 - t^2 underflows), tiny |alpha x|, and
+    # special values in x.
+    M, N = 64, 64
+    inp = make(M, N, "f32", "f32", alpha=3.0, x_std=20.0)
+    x = inp["x"]
+    x[:8] = [0.0, -0.0, 1e-30, -1e-38, 1e-45, np.inf, -np.inf, np.nan]
+    x[8:16] = [5.0, 10.0, 15.0, 20.0, 29.0, 30.0, 40.0, 50.0]
+    out, _ = H.run_cuda(inp, M, N, "f32", "f32")
+    H.compare_all(inp, out, M, N, "f32", "f32")
+
+
+def test_empty_shapes():
+    import elementwise_reduction_b200 as dyt
+    x = torch.empty(0, 7, device="cuda")
+    g = torch.ones(7, device="cuda")
+    a = torch.tensor([0.5], device="cuda")
+    y = dyt.forward(x, a, g, g)
+    assert y.shape == (0, 7)
+    dg = torch.full((7,), 3.0, device="cuda")
+    db = torch.full((7,), 3.0, device="cuda")
+    da = torch.full((1,), 3.0, device="cuda")
+    dyt.backward(x, x, a, g, dgamma=dg, dbeta=db, dalpha=da)
+    torch.cuda.synchronize()
+    assert (dg == 0).all() and (db == 0).all() and (da == 0).all()
+
+
+# ---- layout: unaligned pointers, in-place, determinism ------------------------------------------
+
+def test_unaligned_pointers_take_the_scalar_path():
+    import elementwise_reduction_b200 as dyt
+    M, N = 300, 64
+    inp = make(M, N, "bf16", "f32")
+    t = H.gpu_inputs(inp, "bf16", "f32")
+    buf = torch.empty(M * N + 1, dtype=torch.bfloat16, device="cuda")
+    buf[1:] = t["x"]
+    x = buf[1:].view(M, N)  # 2-byte offset: not 16-byte aligned
+    y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"])
+    assert dyt.dyt_last_launch_info()["vec"] == 1
+    dx, da, dg, db = dyt.backward(x, t["dy"].view(M, N), t["alpha"], t["gamma"])
+    assert dyt.dyt_last_launch_info()["vec"] == 1
+    out = {"y": H.to_numpy(y, "bf16"), "dx": H.to_numpy(dx, "bf16"), "dgamma": H.to_numpy(dg, "f32"),
+           "dbeta": H.to_numpy(db, "f32"), "dalpha": float(da.item())}
+    H.compare_all(inp, out, M, N, "bf16", "f32")
+
+
+def test_in_place_aliasing():
+    import elementwise_reduction_b200 as dyt
+    M, N = 1000, 256
+    inp = make(M, N, "bf16", "f32")
+    ref, _ = H.run_cuda(inp, M, N, "bf16", "f32")
+    t = H.gpu_inputs(inp, "bf16", "f32")
+    x = t["x"].view(M, N).clone()
+    dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=x)  # y over x
+    assert np.array_equal(H.to_numpy(x, "bf16"), ref["y"])
+    x = t["x"].view(M, N)
+    dy = t["dy"].view(M, N).clone()
+    dyt.backward(x, dy, t["alpha"], t["gamma"], dx=dy)  # dx over dy
+    assert np.array_equal(H.to_numpy(dy, "bf16"), ref["dx"])
+    x2 = t["x"].view(M, N).clone()
+    dyt.backward(x2, t["dy"].view(M, N), t["alpha"], t["gamma"], dx=x2)  # dx over x
+    assert np.array_equal(H.to_numpy(x2, "bf16"), ref["dx"])
+
+
+@pytest.mark.parametrize("M,N,xd", [(65537, 32, "bf16"), (3001, 4096, "bf16"), (20000, 255, "f32")])
+def test_backward_is_bitwise_deterministic(M, N, xd):
+    inp = make(M, N, xd, "f32")
+    a, _ = H.run_cuda(inp, M, N, xd, "f32", fwd=False)
+    b, _ = H.run_cuda(inp, M, N, xd, "f32", fwd=False)
+    for k in ("dx", "dgamma", "dbeta"):
+        assert np.array_equal(a[k], b[k])
+    assert a["dalpha"] == b["dalpha"] or (np.isnan(a["dalpha"]) and np.isnan(b["dalpha"]))
+
+
+def test_workspace_errors():
+    import elementwise_reduction_b200 as dyt
+    M, N = 100, 64
+    x = torch.randn(M, N, device="cuda")
+    g = torch.ones(N, device="cuda")
+    a = torch.tensor([0.5], device="cuda")
+    ws = dyt.workspace(x, g)
+    with pytest.raises(dyt.DytError) as e:
+        dyt.backward(x, x, a, g, ws=ws[: ws.numel() - 16])
+    assert e.value.status == 3
+    with pytest.raises(dyt.DytError) as e:
+        dyt.backward(x, x, a, g, ws=ws[8:])
+    assert e.value.status == 1
+
+
+def test_autograd_module_matches_oracle():
+    import elementwise_reduction_b200 as dyt
+    M, N = 512, 384
+    inp = make(M, N, "bf16", "f32", alpha=0.6)
+    t = H.gpu_inputs(inp, "bf16", "f32")
+    mod = dyt.DyT(N, device="cuda")
+    with torch.no_grad():
+        mod.alpha.copy_(t["alpha"])
+        mod.gamma.copy_(t["gamma"])
+        mod.beta.copy_(t["beta"])
+    x = t["x"].view(M, N).clone().requires_grad_(True)
+    y = mod(x)
+    y.backward(t["dy"].view(M, N))
+    out = {"y": H.to_numpy(y, "bf16"), "dx": H.to_numpy(x.grad, "bf16"),
+           "dgamma": H.to_numpy(mod.gamma.grad, "f32"), "dbeta": H.to_numpy(mod.beta.grad, "f32"),
+           "dalpha": float(mod.alpha.grad.item())}
+    H.compare_all(inp, out, M, N, "bf16", "f32")
+
+
+# ---- tanh accuracy over a dense sweep of binary32 inputs -----------------------------------------
+
+def test_tanh_and_sech2_accuracy_sweep():
+    import elementwise_reduction_b200 as dyt
+    # every 97th positive binary32 pattern from 2^-30 to 64, plus their negatives
+    lo, hi = np.float32(2.0 ** -30).view(np.uint32), np.float32(64.0).view(np.uint32)
+    bits = np.arange(lo, hi, 97, dtype=np.uint32)
+    xs = np.concatenate([bits.view(np.float32), -bits.view(np.float32)])
+    n = xs.size
+    one = torch.ones(n, device="cuda")
+    x = torch.from_numpy(xs).cuda().view(1, n)
+    a = torch.tensor([1.0], device="cuda")
+    t = dyt.forward(x, a, one, torch.zeros(n, device="cuda")).cpu().numpy().ravel().astype(np.float64)
+    dx, _, _, _ = dyt.backward(x, one.view(1, n), a, one)
+    s = dx.cpu().numpy().ravel().astype(np.float64)
+    X = xs.astype(np.float64)
+    rel_t = np.abs(t - np.tanh(X)) / np.abs(np.tanh(X))
+    s_ref = 1.0 / np.cosh(X) ** 2
+    ok = s_ref > 1e-37  # binary32 normal range
+    rel_s = np.abs(s[ok] - s_ref[ok]) / s_ref[ok]
+    # bounds the kernel's error analysis uses: |t| within 2^-21 relative, 1 - t^2 within 2^-19
+    assert rel_t.max() <= 2.0 ** -21, rel_t.max()
+    assert rel_s.max() <= 2.0 ** -19, rel_s.max()
+
+
+# ---- the workloads at full size -----------------------------------------------------------------
+
+def _sample_rows(M, rng):
+    rows = set(range(0, min(M, 4))) | set(range(max(0, M - 4), M))
+    rows |= set(rng.integers(0, M, 24).tolist())
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_workload_full_size(name):
+    w = workloads.WORKLOADS[name]
+    inp = workloads.make_inputs(w)
+    out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype)
+    rows = None if w.M * w.N <= 30_000_000 else _sample_rows(w.M, np.random.default_rng(0))
+    stats = H.compare_all(inp, out, w.M, w.N, w.x_dtype, w.p_dtype, rows=rows)
+    print(name, info, stats)
+    if w.N <= 256:
+        assert info["bwd"]["path"] == 1

@@ -14,11 +14,12 @@ import torch
 
 from . import _abi
 from ._abi import (DYT_BF16, DYT_F16, DYT_F32, DytError, dyt_backward, dyt_backward_workspace_bytes,
-                   dyt_forward, dyt_last_launch_info, dyt_plan_query, dyt_status_string)
+                   dyt_device_error, dyt_forward, dyt_last_launch_info, dyt_plan_query,
+                   dyt_selftest_wait_timeout, dyt_status_string)
 
 __all__ = ["forward", "backward", "workspace", "DyT", "DyTFunction", "dyt_forward", "dyt_backward",
            "dyt_backward_workspace_bytes", "dyt_status_string", "dyt_last_launch_info", "dyt_plan_query",
-           "DytError",
+           "dyt_device_error", "dyt_selftest_wait_timeout", "DytError",
            "DTYPE_CODE", "DYT_F32", "DYT_BF16", "DYT_F16"]
 
 DTYPE_CODE = {torch.float32: DYT_F32, torch.bfloat16: DYT_BF16, torch.float16: DYT_F16}

@@ -29,7 +29,8 @@ _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_s
 class LaunchInfo(ctypes.Structure):
     _fields_ = [("op", _i32), ("path", _i32), ("vec", _i32), ("block", _i32), ("grid", _i32),
                 ("row_lanes", _i32), ("rows_per_step", _i32), ("col_chunks", _i32),
-                ("row_groups", _i32), ("kernels", _i32), ("workspace_bytes", _i64)]
+                ("row_groups", _i32), ("kernels", _i32), ("tma_stages", _i32), ("async_stages", _i32),
+                ("workspace_bytes", _i64)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -50,6 +51,10 @@ lib.dyt_last_launch_info.argtypes = [ctypes.POINTER(LaunchInfo)]
 lib.dyt_last_launch_info.restype = _i32
 lib.dyt_plan_query.argtypes = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(LaunchInfo)]
 lib.dyt_plan_query.restype = _i32
+lib.dyt_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
+lib.dyt_device_error.restype = _i32
+lib.dyt_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp, _vp]
+lib.dyt_selftest_wait_timeout.restype = _i32
 
 
 class DytError(RuntimeError):
@@ -92,6 +97,17 @@ def dyt_plan_query(M, N, x_dtype, param_dtype, backward, vectorized, sm_count, c
     _check(lib.dyt_plan_query(M, N, x_dtype, param_dtype, int(backward), int(vectorized), sm_count,
                               ctas_per_sm, ctypes.byref(info)), "dyt_plan_query")
     return info.as_dict()
+
+
+def dyt_device_error(clear: bool = False) -> int:
+    """The sticky device error word of the current device (synchronises)."""
+    w = ctypes.c_uint(0)
+    _check(lib.dyt_device_error(ctypes.byref(w), int(clear)), "dyt_device_error")
+    return int(w.value)
+
+
+def dyt_selftest_wait_timeout(spin_limit: int, gave_up_ptr: int, stream) -> int:
+    return lib.dyt_selftest_wait_timeout(spin_limit, gave_up_ptr, stream)
 
 
 def dyt_last_launch_info() -> dict:

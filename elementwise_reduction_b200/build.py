@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdyt.so")
 SOURCES = [os.path.join(CSRC, "dyt_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("dyt_kernels.cuh", "dyt_math.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_tma.cuh", "dyt_async.cuh")] + [
     os.path.join(INCLUDE, "dyt.h")]
 
 NVCC_FLAGS = [
@@ -32,17 +32,21 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libdyt.so if any source is newer than it. Returns its path."""
-    if not force and os.path.exists(LIB):
-        built = os.path.getmtime(LIB)
+def build(force: bool = False, verbose: bool = False, defines=(), out: str | None = None) -> str:
+    """Compile libdyt.so if any source is newer than it. Returns its path.
+
+    defines: extra -D tuning overrides; out: another output path (for sweeps).
+    """
+    out = out or LIB
+    if not force and not defines and os.path.exists(out):
+        built = os.path.getmtime(out)
         if all(os.path.getmtime(d) <= built for d in DEPS):
-            return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", LIB + ".tmp", *SOURCES,
-           "-lcudart"]
+            return out
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), *[f"-D{d}" for d in defines],
+           "-o", out + ".tmp", *SOURCES, "-lcudart"]
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":

@@ -9,6 +9,8 @@
 
 #include "dyt.h"
 #include "dyt_kernels.cuh"
+#include "dyt_tma.cuh"
+#include "dyt_async.cuh"
 
 namespace {
 
@@ -17,10 +19,51 @@ using dyt::Geom;
 thread_local dyt_launch_info t_info = {};
 thread_local int t_cuda_err = 0;
 
+// Tuning constants (compile-time; -D overrides them for sweeps).
+#ifndef DYT_FWD_UNROLL_VEC
+#define DYT_FWD_UNROLL_VEC 2
+#endif
+#ifndef DYT_BWD_UNROLL_VEC
+#define DYT_BWD_UNROLL_VEC 2
+#endif
+#ifndef DYT_FWD_UNROLL_SCALAR
+#define DYT_FWD_UNROLL_SCALAR 8
+#endif
+#ifndef DYT_BWD_UNROLL_SCALAR
+#define DYT_BWD_UNROLL_SCALAR 8
+#endif
+// Pipeline of the 16-byte aligned path: 0 = loads into registers, 1 = CTA-wide
+// bulk-copy (TMA) ring, 2 = per-thread asynchronous-copy ring.
+#ifndef DYT_PIPE
+#define DYT_PIPE 2
+#endif
+#define DYT_USE_TMA (DYT_PIPE == 1)
+#ifndef DYT_ASYNC_STAGES_FWD
+#define DYT_ASYNC_STAGES_FWD 8
+#endif
+#ifndef DYT_ASYNC_STAGES_BWD
+#define DYT_ASYNC_STAGES_BWD 6
+#endif
+#ifndef DYT_TILE_BYTES
+#define DYT_TILE_BYTES 32768
+#endif
+#ifndef DYT_MAX_STAGES
+#define DYT_MAX_STAGES 8
+#endif
 constexpr int kBlock = 1024;          // threads per CTA of the main kernels
+constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits (iterations)
+constexpr int kMaxDynSmem = 227 * 1024;
+#ifndef DYT_ASYNC_BLOCK
+#define DYT_ASYNC_BLOCK 512
+#endif
+constexpr int kAsyncBlock = DYT_ASYNC_BLOCK;  // one CTA per SM: up to 128 registers a thread
+constexpr int kAsyncStagesFwd = DYT_ASYNC_STAGES_FWD;
+constexpr int kAsyncStagesBwd = DYT_ASYNC_STAGES_BWD;
 constexpr int kMaxRowsPerLane = 96;   // sequential binary32 adds per thread per group
-constexpr int kUnrollVec = 2;         // rows in flight per thread, 16-byte access
-constexpr int kUnrollScalar = 8;      // rows in flight per thread, scalar access
+constexpr int kFwdUnrollVec = DYT_FWD_UNROLL_VEC;        // rows in flight per thread, 16-byte access
+constexpr int kBwdUnrollVec = DYT_BWD_UNROLL_VEC;
+constexpr int kFwdUnrollScalar = DYT_FWD_UNROLL_SCALAR;  // rows in flight per thread, scalar access
+constexpr int kBwdUnrollScalar = DYT_BWD_UNROLL_SCALAR;
 
 dyt_status cuda_fail(cudaError_t e) {
   t_cuda_err = (int)e;
@@ -85,10 +128,15 @@ dyt_status occupancy(int dev, const void *kernel, int block, int *ctas) {
 
 struct Plan {
   Geom g;
+  int block;  // threads per CTA of the main kernel
   int vec;
   int unroll;
   int grid;
   int path;
+  bool tma;
+  bool async;
+  dyt::TmaGeom tg;
+  size_t smem;  // dynamic shared memory of the pipelined kernel
   size_t ws_dg, ws_db, ws_da, ws_total;  // workspace byte offsets / sizes
 };
 
@@ -96,22 +144,24 @@ size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
 // vec: elements per access (1 or 16 / element size). ctas_per_sm from the
 // kernel's occupancy. The plan depends only on (M, N, vec, SM count, occupancy).
-Plan make_plan(int64_t M, int64_t N, int vec, int sms, int ctas_per_sm) {
+Plan make_plan(int64_t M, int64_t N, int vec, bool backward, int sms, int ctas_per_sm, int block = kBlock) {
   Plan p = {};
+  p.block = block;
   p.vec = vec;
-  p.unroll = vec > 1 ? kUnrollVec : kUnrollScalar;
+  p.unroll = backward ? (vec > 1 ? kBwdUnrollVec : kBwdUnrollScalar)
+                      : (vec > 1 ? kFwdUnrollVec : kFwdUnrollScalar);
   const int64_t NV = N / vec;
   Geom &g = p.g;
   g.M = M;
   g.N = N;
   g.NV = (int)NV;
-  if (NV <= kBlock / 2) {
-    g.RL = kBlock / (int)NV;
+  if (NV <= block / 2) {
+    g.RL = block / (int)NV;
     g.ncc = 1;
     p.path = 1;
   } else {
     g.RL = 1;
-    g.ncc = (int)ceil_div(NV, kBlock);
+    g.ncc = (int)ceil_div(NV, block);
     p.path = 2;
   }
   const int64_t target = (int64_t)sms * ctas_per_sm;
@@ -139,6 +189,33 @@ Plan make_plan(int64_t M, int64_t N, int vec, int sms, int ctas_per_sm) {
   return p;
 }
 
+// Tiles of the pipelined kernels: about DYT_TILE_BYTES per stage, as many
+// stages as fit next to the kernel's static shared memory.
+void plan_tma(Plan &p, size_t elem, bool backward, int static_smem) {
+  const dyt::Geom &g = p.g;
+  const int64_t chunk_cols = g.ncc == 1 ? g.N : (int64_t)kBlock * p.vec;
+  dyt::TmaGeom &tg = p.tg;
+  tg.pitch = (int)(chunk_cols * (int64_t)elem);
+  const int ntensors = backward ? 2 : 1;
+  const int64_t per_u = (int64_t)g.RL * tg.pitch * ntensors;  // bytes per row per lane
+  int64_t U = DYT_TILE_BYTES / per_u;
+  if (U < 1) U = 1;
+  const int64_t rows_per_group = ceil_div(g.M, g.nrg);
+  const int64_t u_cap = ceil_div(rows_per_group, g.RL);
+  if (U > u_cap) U = u_cap;
+  if (U > kMaxRowsPerLane) U = kMaxRowsPerLane;
+  tg.U = (int)U;
+  tg.SR = g.RL * tg.U;
+  const int64_t stage = (int64_t)tg.SR * tg.pitch * ntensors;
+  int64_t S = (kMaxDynSmem - static_smem - 16 * DYT_MAX_STAGES - 64) / stage;
+  if (S > DYT_MAX_STAGES) S = DYT_MAX_STAGES;
+  tg.stages = (int)S;
+  tg.spin = kSpinLimit;
+  p.smem = (size_t)S * stage + 16 * S + 16;
+  p.tma = S >= 2;
+  p.unroll = tg.U;
+}
+
 // ---- kernel tables ---------------------------------------------------------------
 
 template <typename T>
@@ -148,14 +225,14 @@ constexpr int vec_of() {
 
 template <typename T, typename P>
 const void *fwd_kernel(int vec) {
-  if (vec > 1) return (const void *)dyt::dyt_fwd_kernel<T, P, vec_of<T>(), kUnrollVec, kBlock>;
-  return (const void *)dyt::dyt_fwd_kernel<T, P, 1, kUnrollScalar, kBlock>;
+  if (vec > 1) return (const void *)dyt::dyt_fwd_kernel<T, P, vec_of<T>(), kFwdUnrollVec, kBlock>;
+  return (const void *)dyt::dyt_fwd_kernel<T, P, 1, kFwdUnrollScalar, kBlock>;
 }
 
 template <typename T, typename P>
 const void *bwd_kernel(int vec) {
-  if (vec > 1) return (const void *)dyt::dyt_bwd_kernel<T, P, vec_of<T>(), kUnrollVec, kBlock>;
-  return (const void *)dyt::dyt_bwd_kernel<T, P, 1, kUnrollScalar, kBlock>;
+  if (vec > 1) return (const void *)dyt::dyt_bwd_kernel<T, P, vec_of<T>(), kBwdUnrollVec, kBlock>;
+  return (const void *)dyt::dyt_bwd_kernel<T, P, 1, kBwdUnrollScalar, kBlock>;
 }
 
 template <typename F>
@@ -194,17 +271,61 @@ dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
   if (p) {
     i.path = p->path;
     i.vec = p->vec;
-    i.block = kBlock;
+    i.block = p->block;
     i.grid = p->grid;
     i.row_lanes = p->g.RL;
     i.rows_per_step = p->g.RL * p->unroll;
     i.col_chunks = p->g.ncc;
     i.row_groups = p->g.nrg;
+    i.tma_stages = p->tma ? p->tg.stages : 0;
+    i.async_stages = p->async ? (op == 2 ? kAsyncStagesBwd : kAsyncStagesFwd) : 0;
   }
   return i;
 }
 
 void record(int op, const Plan *p, int kernels, size_t ws) { t_info = describe(op, p, kernels, ws); }
+
+// Columns per thread in the pipelined kernels (their shared-memory reads are
+// 4 elements wide; the bulk copies move whole rows regardless).
+constexpr int kTmaVec = 4;
+
+template <typename T, typename P>
+const void *tma_kernel(bool backward) {
+  return backward ? (const void *)dyt::dyt_bwd_tma_kernel<T, P, kTmaVec, kBlock>
+                  : (const void *)dyt::dyt_fwd_tma_kernel<T, P, kTmaVec, kBlock>;
+}
+
+template <typename T, typename P>
+const void *async_kernel(bool backward) {
+  return backward ? (const void *)dyt::dyt_bwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesBwd>
+                  : (const void *)dyt::dyt_fwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesFwd>;
+}
+
+// Static shared memory of a kernel and, once, the opt-in to the largest
+// dynamic shared memory (cached per device and kernel).
+std::unordered_map<uint64_t, int> g_static_smem;
+
+dyt_status prepare_tma_kernel(int dev, const void *kernel, int *static_smem) {
+  const uint64_t key = ((uint64_t)(uint32_t)dev << 48) ^ (uint64_t)(uintptr_t)kernel;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_static_smem.find(key);
+    if (it != g_static_smem.end()) {
+      *static_smem = it->second;
+      return DYT_OK;
+    }
+  }
+  cudaFuncAttributes a;
+  cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int dyn = kMaxDynSmem - (int)a.sharedSizeBytes;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_static_smem[key] = (int)a.sharedSizeBytes;
+  *static_smem = (int)a.sharedSizeBytes;
+  return DYT_OK;
+}
 
 // Plan for given pointers' alignment on the current device.
 template <typename T, typename P>
@@ -213,11 +334,29 @@ dyt_status plan_for(int64_t M, int64_t N, bool vec_ok, bool backward, Plan *out)
   dyt_status st = current_sms(&dev, &sms);
   if (st != DYT_OK) return st;
   const int vec = (vec_ok && N % vec_of<T>() == 0) ? vec_of<T>() : 1;
-  const void *k = backward ? bwd_kernel<T, P>(vec) : fwd_kernel<T, P>(vec);
+  const bool use_tma = DYT_USE_TMA && vec > 1;
+  const bool use_async = DYT_PIPE == 2 && vec > 1;
+  const void *k = use_tma     ? tma_kernel<T, P>(backward)
+                  : use_async ? async_kernel<T, P>(backward)
+                  : backward  ? bwd_kernel<T, P>(vec)
+                              : fwd_kernel<T, P>(vec);
   int occ = 1;
-  st = occupancy(dev, k, kBlock, &occ);
-  if (st != DYT_OK) return st;
-  *out = make_plan(M, N, vec, sms, occ);
+  int static_smem = 0;
+  if (use_tma || use_async) {
+    st = prepare_tma_kernel(dev, k, &static_smem);
+    if (st != DYT_OK) return st;
+  } else {
+    st = occupancy(dev, k, kBlock, &occ);
+    if (st != DYT_OK) return st;
+  }
+  *out = make_plan(M, N, use_tma ? kTmaVec : vec, backward, sms, occ, use_async ? kAsyncBlock : kBlock);
+  out->tma = false;
+  out->async = use_async;
+  if (use_tma) plan_tma(*out, sizeof(T), backward, static_smem);
+  if (use_async) {
+    out->smem = backward ? (size_t)kAsyncStagesBwd * 2 * kAsyncBlock * 16 : (size_t)kAsyncStagesFwd * kAsyncBlock * 16;
+    out->unroll = 1;
+  }
   return DYT_OK;
 }
 
@@ -244,15 +383,23 @@ dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, cons
     if (s != DYT_OK) return s;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(kBlock);
+    cfg.blockDim = dim3(p.block);
     cfg.stream = (cudaStream_t)stream;
     cudaError_t e;
-    if (p.vec > 1)
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, V, kUnrollVec, kBlock>,
+    if (p.tma) {
+      cfg.dynamicSmemBytes = p.smem;
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_tma_kernel<T, P, kTmaVec, kBlock>, (const T *)x, (const P *)alpha,
+                             (const P *)gamma, (const P *)beta, (T *)y, p.g, p.tg);
+    } else if (p.async) {
+      cfg.dynamicSmemBytes = p.smem;
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd>, (const T *)x,
+                             (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
+    } else if (p.vec > 1)
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, V, kFwdUnrollVec, kBlock>,
                              (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y,
                              p.g);
     else
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, 1, kUnrollScalar, kBlock>, (const T *)x,
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, 1, kFwdUnrollScalar, kBlock>, (const T *)x,
                              (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
     if (e != cudaSuccess) return cuda_fail(e);
     record(1, &p, 1, 0);
@@ -317,22 +464,33 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(kBlock);
+    cfg.blockDim = dim3(p.block);
     cfg.stream = s;
     cudaError_t e;
-    if (p.vec > 1)
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, V, kUnrollVec, kBlock>,
+    if (p.tma) {
+      cfg.dynamicSmemBytes = p.smem;
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_tma_kernel<T, P, kTmaVec, kBlock>, (const T *)x, (const T *)dy,
+                             (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda, p.g, p.tg);
+    } else if (p.async) {
+      cfg.dynamicSmemBytes = p.smem;
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd>, (const T *)x,
+                             (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda, p.g);
+    } else if (p.vec > 1)
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, V, kBwdUnrollVec, kBlock>,
                              (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx,
                              pdg, pdb, pda, p.g);
     else
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, 1, kUnrollScalar, kBlock>, (const T *)x,
+      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, 1, kBwdUnrollScalar, kBlock>, (const T *)x,
                              (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda,
                              p.g);
     if (e != cudaSuccess) return cuda_fail(e);
 
     // Stage 2, as a programmatic dependent launch: it may start while stage 1
     // drains and waits (griddepcontrol.wait) for stage 1's results.
-    const int CT = N >= (int64_t)32 * 148 ? 32 : 8;
+    // Lanes per column: enough that each lane reads at most four partials.
+    int L = 1;
+    while (L < dyt::kFinThreads && (int64_t)L * 4 < p.g.nrg) L <<= 1;
+    const int CT = dyt::kFinThreads / L;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -364,6 +522,26 @@ const char *dyt_status_string(dyt_status status) {
 
 int dyt_last_cuda_error(void) { return t_cuda_err; }
 
+dyt_status dyt_device_error(unsigned int *word, int clear) {
+  if (!word) return DYT_ERR_INVALID_VALUE;
+  cudaError_t e = cudaMemcpyFromSymbol(word, dyt::g_dyt_device_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(dyt::g_dyt_device_error, &zero, sizeof(unsigned int));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return DYT_OK;
+}
+
+dyt_status dyt_selftest_wait_timeout(unsigned int spin_limit, int *gave_up, dyt_stream_t stream) {
+  if (!gave_up || spin_limit == 0) return DYT_ERR_INVALID_VALUE;
+  dyt::dyt_wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(spin_limit, gave_up);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DYT_OK;
+}
+
 dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype, int backward,
                           int vectorized, int sm_count, int ctas_per_sm, dyt_launch_info *out) {
   if (!out || sm_count < 1 || ctas_per_sm < 1) return DYT_ERR_INVALID_VALUE;
@@ -376,7 +554,14 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
   }
   const int v = 16 / (int)dsize(x_dtype);
   const int vec = (vectorized && N % v == 0) ? v : 1;
-  const Plan p = make_plan(M, N, vec, sm_count, ctas_per_sm);
+  const bool use_tma = DYT_USE_TMA && vec > 1;
+  const bool use_async = DYT_PIPE == 2 && vec > 1;
+  Plan p = make_plan(M, N, use_tma ? kTmaVec : vec, backward != 0, sm_count, ctas_per_sm,
+                     use_async ? kAsyncBlock : kBlock);
+  p.tma = false;
+  p.async = use_async;
+  if (p.async) p.unroll = 1;
+  if (use_tma) plan_tma(p, dsize(x_dtype), backward != 0, backward ? 17 * 1024 : 256);
   *out = describe(op, &p, backward ? 2 : 1, backward ? p.ws_total : 0);
   return DYT_OK;
 }

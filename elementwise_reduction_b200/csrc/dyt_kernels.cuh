@@ -76,6 +76,7 @@ struct VecIO;
 template <typename T>
 struct VecIO<T, 1> {
   using Raw = T;
+  static constexpr int kPairs = 0;
   static __device__ __forceinline__ Raw load(const T *p) { return ld_scalar(p); }
   static __device__ __forceinline__ Raw zero() { return from_f32<T>(0.0f); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[1]) { f[0] = to_f32<T>(r); }
@@ -88,6 +89,15 @@ struct VecIO<T, 1> {
 template <>
 struct VecIO<float, 4> {
   using Raw = uint4;
+  static constexpr int kPairs = 2;
+  static __device__ __forceinline__ void unpack2(const Raw &r, float2 (&f)[2]) {
+    f[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
+    f[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
+  }
+  static __device__ __forceinline__ Raw pack2(const float2 (&f)[2]) {
+    return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y), __float_as_uint(f[1].x),
+                      __float_as_uint(f[1].y));
+  }
   static __device__ __forceinline__ Raw load(const float *p) { return ld_stream16(p); }
   static __device__ __forceinline__ Raw zero() { return make_uint4(0, 0, 0, 0); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[4]) {
@@ -124,6 +134,24 @@ __device__ __forceinline__ void set_word(uint4 &r, int w, uint32_t v) {
 template <>
 struct VecIO<__nv_bfloat16, 8> {
   using Raw = uint4;
+  static constexpr int kPairs = 4;
+  static __device__ __forceinline__ void unpack2(const Raw &r, float2 (&f)[4]) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t u = word_of(r, w);
+      f[w] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
+  }
+  static __device__ __forceinline__ Raw pack2(const float2 (&f)[4]) {
+    Raw r;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t u;
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f[w].y), "f"(f[w].x));
+      set_word(r, w, u);
+    }
+    return r;
+  }
   static __device__ __forceinline__ Raw load(const __nv_bfloat16 *p) { return ld_stream16(p); }
   static __device__ __forceinline__ Raw zero() { return make_uint4(0, 0, 0, 0); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[8]) {
@@ -155,6 +183,24 @@ struct VecIO<__nv_bfloat16, 8> {
 template <>
 struct VecIO<__half, 8> {
   using Raw = uint4;
+  static constexpr int kPairs = 4;
+  static __device__ __forceinline__ void unpack2(const Raw &r, float2 (&f)[4]) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t u = word_of(r, w);
+      f[w] = __half22float2(*reinterpret_cast<const __half2 *>(&u));
+    }
+  }
+  static __device__ __forceinline__ Raw pack2(const float2 (&f)[4]) {
+    Raw r;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t u;
+      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f[w].y), "f"(f[w].x));
+      set_word(r, w, u);
+    }
+    return r;
+  }
   static __device__ __forceinline__ Raw load(const __half *p) { return ld_stream16(p); }
   static __device__ __forceinline__ Raw zero() { return make_uint4(0, 0, 0, 0); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[8]) {
@@ -182,6 +228,66 @@ struct VecIO<__half, 8> {
   }
   static __device__ __forceinline__ void store_raw(__half *p, const Raw &r) { st16(p, r); }
 };
+
+// Four 16-bit elements (8 bytes): the unit the pipelined kernels read from
+// shared memory and store to global memory.
+template <typename T>
+struct VecIO16x4 {
+  using Raw = uint2;
+  static constexpr int kPairs = 2;
+  static __device__ __forceinline__ float2 lo_hi(uint32_t u);
+  static __device__ __forceinline__ uint32_t pack_pair(float2 f);
+  static __device__ __forceinline__ Raw zero() { return make_uint2(0, 0); }
+  static __device__ __forceinline__ void unpack2(const Raw &r, float2 (&f)[2]) {
+    f[0] = lo_hi(r.x);
+    f[1] = lo_hi(r.y);
+  }
+  static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[4]) {
+    const float2 a = lo_hi(r.x), b = lo_hi(r.y);
+    f[0] = a.x;
+    f[1] = a.y;
+    f[2] = b.x;
+    f[3] = b.y;
+  }
+  static __device__ __forceinline__ Raw pack2(const float2 (&f)[2]) {
+    return make_uint2(pack_pair(f[0]), pack_pair(f[1]));
+  }
+  static __device__ __forceinline__ Raw pack(const float (&f)[4]) {
+    return make_uint2(pack_pair(make_float2(f[0], f[1])), pack_pair(make_float2(f[2], f[3])));
+  }
+  static __device__ __forceinline__ void set(Raw &r, int e, T v) {
+    const uint32_t b = (uint32_t)(*reinterpret_cast<const unsigned short *>(&v));
+    uint32_t &w = (e >> 1) ? r.y : r.x;
+    w = (e & 1) ? ((w & 0x0000FFFFu) | (b << 16)) : ((w & 0xFFFF0000u) | b);
+  }
+  static __device__ __forceinline__ void store_raw(T *p, const Raw &r) {
+    asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(r.x), "r"(r.y) : "memory");
+  }
+};
+template <>
+__device__ __forceinline__ float2 VecIO16x4<__nv_bfloat16>::lo_hi(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ uint32_t VecIO16x4<__nv_bfloat16>::pack_pair(float2 f) {
+  uint32_t u;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f.y), "f"(f.x));
+  return u;
+}
+template <>
+__device__ __forceinline__ float2 VecIO16x4<__half>::lo_hi(uint32_t u) {
+  return __half22float2(*reinterpret_cast<const __half2 *>(&u));
+}
+template <>
+__device__ __forceinline__ uint32_t VecIO16x4<__half>::pack_pair(float2 f) {
+  uint32_t u;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f.y), "f"(f.x));
+  return u;
+}
+template <>
+struct VecIO<__nv_bfloat16, 4> : VecIO16x4<__nv_bfloat16> {};
+template <>
+struct VecIO<__half, 4> : VecIO16x4<__half> {};
 
 template <typename P>
 __device__ __forceinline__ float param(const P *p, int64_t i) {
@@ -211,6 +317,64 @@ __device__ __forceinline__ Lane lane_of(const Geom &g, int tid) {
 
 // ---- forward -----------------------------------------------------------------
 
+// y for one vector of VEC elements (one row, VEC consecutive columns).
+// bth[e] = tau |beta[e]|: below it the binary32 value may have cancelled.
+template <typename T, int VEC>
+__device__ __forceinline__ typename VecIO<T, VEC>::Raw fwd_vector(const typename VecIO<T, VEC>::Raw &rx,
+                                                                 float alpha, const float (&gam)[VEC],
+                                                                 const float (&bet)[VEC],
+                                                                 const float (&bth)[VEC]) {
+  using IO = VecIO<T, VEC>;
+  typename IO::Raw out;
+  bool cancel_any = false;
+  if constexpr (IO::kPairs > 0) {
+    constexpr int H = IO::kPairs;
+    float2 x2[H], y2[H];
+    IO::unpack2(rx, x2);
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const float2 t = dyt_tanh2(mul2(f2(alpha), x2[h]));
+      y2[h] = fma2(make_float2(gam[2 * h], gam[2 * h + 1]), t, make_float2(bet[2 * h], bet[2 * h + 1]));
+      if (CancelGuard<T>::kOn)
+        cancel_any |= (fabsf(y2[h].x) < bth[2 * h]) | (fabsf(y2[h].y) < bth[2 * h + 1]);
+    }
+    out = IO::pack2(y2);
+  } else {
+    float xf[VEC], yf[VEC];
+    IO::unpack(rx, xf);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      yf[e] = fmaf(gam[e], dyt_tanh(alpha * xf[e]), bet[e]);
+      if (CancelGuard<T>::kOn) cancel_any |= fabsf(yf[e]) < bth[e];
+    }
+    out = IO::pack(yf);
+  }
+  if (CancelGuard<T>::kOn && cancel_any) {
+    // Rare: redo the test per element (the scalar formulas round exactly as the
+    // pair ones) and replace the cancelling elements with the binary64 value.
+    float xf[VEC];
+    IO::unpack(rx, xf);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const float y = fmaf(gam[e], dyt_tanh(alpha * xf[e]), bet[e]);
+      if (fabsf(y) < bth[e]) IO::set(out, e, dyt_y_refined<T>(alpha, xf[e], gam[e], bet[e]));
+    }
+  }
+  return out;
+}
+
+// gamma, beta and the cancellation thresholds of VEC columns.
+template <typename T, typename P, int VEC>
+__device__ __forceinline__ void fwd_params(const P *gamma, const P *beta, int64_t c0, bool ok, float (&gam)[VEC],
+                                           float (&bet)[VEC], float (&bth)[VEC]) {
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    gam[e] = ok ? param(gamma, c0 + e) : 0.0f;
+    bet[e] = ok ? param(beta, c0 + e) : 0.0f;
+    bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
+  }
+}
+
 template <typename T, typename P, int VEC, int U, int B>
 __global__ void __launch_bounds__(B, 1)
     dyt_fwd_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma,
@@ -226,12 +390,8 @@ __global__ void __launch_bounds__(B, 1)
     const bool col_ok = ln.live && cv < g.NV;
     if (!col_ok) continue;
     const int64_t c0 = (int64_t)cv * VEC;
-    float gam[VEC], bet[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      gam[e] = param(gamma, c0 + e);
-      bet[e] = param(beta, c0 + e);
-    }
+    float gam[VEC], bet[VEC], bth[VEC];
+    fwd_params<T, P, VEC>(gamma, beta, c0, true, gam, bet, bth);
     const int64_t step = (int64_t)g.RL * U;
     for (int64_t r0 = rb + ln.rl; r0 < re; r0 += step) {
       typename IO::Raw raw[U];
@@ -243,25 +403,7 @@ __global__ void __launch_bounds__(B, 1)
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t row = r0 + (int64_t)u * g.RL;
-        if (row >= re) continue;
-        float xf[VEC], yf[VEC];
-        IO::unpack(raw[u], xf);
-        bool cancel_any = false;
-        bool cancel[VEC];
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const float t = dyt_tanh(alpha * xf[e]);
-          yf[e] = fmaf(gam[e], t, bet[e]);
-          cancel[e] = CancelGuard<T>::kOn && fabsf(yf[e]) < fabsf(gam[e] * t) * CancelGuard<T>::kTau;
-          cancel_any |= cancel[e];
-        }
-        typename IO::Raw out = IO::pack(yf);
-        if (CancelGuard<T>::kOn && cancel_any) {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e)
-            if (cancel[e]) IO::set(out, e, dyt_y_refined<T>(alpha, xf[e], gam[e], bet[e]));
-        }
-        IO::store_raw(y + row * g.N + c0, out);
+        if (row < re) IO::store_raw(y + row * g.N + c0, fwd_vector<T, VEC>(raw[u], alpha, gam, bet, bth));
       }
     }
   }
@@ -270,19 +412,87 @@ __global__ void __launch_bounds__(B, 1)
 // ---- backward, stage 1 ---------------------------------------------------------
 
 // Fixed-order tree over the RL row lanes of a CTA: lane rl absorbs lane rl + h,
-// h = ceil(n / 2), until one lane is left. red[] holds B * VEC floats laid out
-// by thread; afterwards lane 0's entries hold the CTA sums.
+// h = ceil(n / 2), until one lane is left. red[] holds VEC * B floats,
+// element-major (red[e * B + thread]) so that a warp touches 32 consecutive
+// banks; afterwards lane 0's entries hold the CTA sums.
 template <int VEC, int B>
 __device__ __forceinline__ void lane_tree(float *red, const Geom &g, const Lane &ln) {
   for (int n = g.RL; n > 1;) {
     const int h = (n + 1) >> 1;
     if (ln.live && ln.rl < n - h) {
-      const int src = (threadIdx.x + h * g.NV) * VEC;
+      const int src = threadIdx.x + h * g.NV;
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) red[threadIdx.x * VEC + e] += red[src + e];
+      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] += red[e * B + src];
     }
     __syncthreads();
     n = h;
+  }
+}
+
+// Per-thread backward state for VEC columns.
+template <int VEC>
+struct BwdAcc {
+  float g[VEC];  // sum of dy * t over this group's rows
+  float b[VEC];  // sum of dy
+};
+
+// One vector (one row, VEC columns): dx out, sums in. MASKED: the row may be
+// padding; its results are computed like any other and dropped afterwards.
+template <typename T, int VEC, bool MASKED>
+__device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename VecIO<T, VEC>::Raw &rx,
+                                                                 const typename VecIO<T, VEC>::Raw &rdy,
+                                                                 float alpha, const float (&gam)[VEC],
+                                                                 BwdAcc<VEC> &acc, float2 &ca, bool ok) {
+  using IO = VecIO<T, VEC>;
+  if constexpr (IO::kPairs > 0) {
+    constexpr int H = IO::kPairs;
+    float2 x2[H], dy2[H], dx2[H];
+    IO::unpack2(rx, x2);
+    IO::unpack2(rdy, dy2);
+    bool huge = false;
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      float2 t, s;
+      const float2 z = mul2(f2(alpha), x2[h]);
+      if (dyt_tanh_sech2_2(z, t, s)) {  // rare: 40 < |z| < 53
+        huge = true;
+        if (huge_arg(z.x)) s.x = sech2_huge(z.x);
+        if (huge_arg(z.y)) s.y = sech2_huge(z.y);
+      }
+      const float2 gdys = mul2(mul2(make_float2(gam[2 * h], gam[2 * h + 1]), dy2[h]), s);
+      dx2[h] = mul2(f2(alpha), gdys);
+      const float2 ag = make_float2(acc.g[2 * h], acc.g[2 * h + 1]);
+      const float2 ab = make_float2(acc.b[2 * h], acc.b[2 * h + 1]);
+      float2 ng = fma2(dy2[h], t, ag), nb = add2(ab, dy2[h]), nca = fma2(gdys, x2[h], ca);
+      if (MASKED) {  // drop a padded row's results, after the arithmetic
+        ng = ok ? ng : ag;
+        nb = ok ? nb : ab;
+        nca = ok ? nca : ca;
+      }
+      acc.g[2 * h] = ng.x;
+      acc.g[2 * h + 1] = ng.y;
+      acc.b[2 * h] = nb.x;
+      acc.b[2 * h + 1] = nb.y;
+      ca = nca;
+    }
+    (void)huge;
+    return IO::pack2(dx2);
+  } else {
+    float xf[VEC], dyf[VEC], dxf[VEC];
+    IO::unpack(rx, xf);
+    IO::unpack(rdy, dyf);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      float t, s;
+      dyt_tanh_sech2(alpha * xf[e], t, s);
+      const float gdys = (gam[e] * dyf[e]) * s;
+      dxf[e] = alpha * gdys;
+      const float ng = fmaf(dyf[e], t, acc.g[e]), nb = acc.b[e] + dyf[e], nca = fmaf(gdys, xf[e], ca.x);
+      acc.g[e] = (MASKED && !ok) ? acc.g[e] : ng;
+      acc.b[e] = (MASKED && !ok) ? acc.b[e] : nb;
+      ca.x = (MASKED && !ok) ? ca.x : nca;
+    }
+    return IO::pack(dxf);
   }
 }
 
@@ -292,7 +502,7 @@ __global__ void __launch_bounds__(B, 1)
                    const P *__restrict__ gamma, T *dx, float *__restrict__ part_dg,
                    float *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
   using IO = VecIO<T, VEC>;
-  __shared__ float red[B * VEC];
+  __shared__ float red[VEC * B];
   __shared__ double red_a[B / 32];
   // Let the finalize kernel, launched as a programmatic dependent, get
   // scheduled early; it still waits for this grid to finish before reading.
@@ -308,46 +518,43 @@ __global__ void __launch_bounds__(B, 1)
     const int cv = cc * B + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
     const int64_t c0 = (int64_t)cv * VEC;
-    float gam[VEC], acc_g[VEC], acc_b[VEC];
+    float gam[VEC];
+    BwdAcc<VEC> acc;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       gam[e] = col_ok ? param(gamma, c0 + e) : 0.0f;
-      acc_g[e] = 0.0f;
-      acc_b[e] = 0.0f;
+      acc.g[e] = 0.0f;
+      acc.b[e] = 0.0f;
     }
     if (col_ok) {
       const int64_t step = (int64_t)g.RL * U;
       for (int64_t r0 = rb + ln.rl; r0 < re; r0 += step) {
         typename IO::Raw rx[U], rdy[U];
-        bool rok[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int64_t row = r0 + (int64_t)u * g.RL;
-          rok[u] = row < re;
-          rx[u] = rok[u] ? IO::load(x + row * g.N + c0) : IO::zero();
-          rdy[u] = rok[u] ? IO::load(dy + row * g.N + c0) : IO::zero();
+          const bool ok = row < re;
+          rx[u] = ok ? IO::load(x + row * g.N + c0) : IO::zero();
+          rdy[u] = ok ? IO::load(dy + row * g.N + c0) : IO::zero();
         }
-        float ca = 0.0f;
+        float2 ca = make_float2(0.0f, 0.0f);
+        if (r0 + (int64_t)(U - 1) * g.RL < re) {  // every row of the step is real
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          float xf[VEC], dyf[VEC], dxf[VEC];
-          IO::unpack(rx[u], xf);
-          IO::unpack(rdy[u], dyf);
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) {
-            float t, s;
-            dyt_tanh_sech2(alpha * xf[e], t, s);
-            const float gdys = (gam[e] * dyf[e]) * s;  // gamma * dy * (1 - t^2)
-            dxf[e] = alpha * gdys;
-            // Padded rows were loaded as zeros and went through the arithmetic
-            // above; their results are dropped here, after it.
-            acc_g[e] = rok[u] ? fmaf(dyf[e], t, acc_g[e]) : acc_g[e];
-            acc_b[e] = rok[u] ? acc_b[e] + dyf[e] : acc_b[e];
-            ca = rok[u] ? fmaf(gdys, xf[e], ca) : ca;
+          for (int u = 0; u < U; ++u) {
+            const int64_t row = r0 + (int64_t)u * g.RL;
+            IO::store_raw(dx + row * g.N + c0, bwd_vector<T, VEC, false>(rx[u], rdy[u], alpha, gam, acc, ca, true));
           }
-          if (rok[u]) IO::store_raw(dx + (r0 + (int64_t)u * g.RL) * g.N + c0, IO::pack(dxf));
+        } else {  // ragged last step of the group
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int64_t row = r0 + (int64_t)u * g.RL;
+            const bool ok = row < re;
+            const typename IO::Raw d = bwd_vector<T, VEC, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok);
+            if (ok) IO::store_raw(dx + row * g.N + c0, d);
+          }
         }
-        acc_a += (double)ca;
+        acc_a += (double)ca.x;
+        acc_a += (double)ca.y;
       }
     }
     // Per-(group, column) partials.
@@ -357,27 +564,27 @@ __global__ void __launch_bounds__(B, 1)
       if (col_ok) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          pg[c0 + e] = acc_g[e];
-          pb[c0 + e] = acc_b[e];
+          pg[c0 + e] = acc.g[e];
+          pb[c0 + e] = acc.b[e];
         }
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) red[threadIdx.x * VEC + e] = acc_g[e];
+      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.g[e];
       __syncthreads();
       lane_tree<VEC, B>(red, g, ln);
       if (col_ok && ln.rl == 0) {
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) pg[c0 + e] = red[threadIdx.x * VEC + e];
+        for (int e = 0; e < VEC; ++e) pg[c0 + e] = red[e * B + threadIdx.x];
       }
       __syncthreads();
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) red[threadIdx.x * VEC + e] = acc_b[e];
+      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.b[e];
       __syncthreads();
       lane_tree<VEC, B>(red, g, ln);
       if (col_ok && ln.rl == 0) {
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) pb[c0 + e] = red[threadIdx.x * VEC + e];
+        for (int e = 0; e < VEC; ++e) pb[c0 + e] = red[e * B + threadIdx.x];
       }
       __syncthreads();
     }
@@ -396,9 +603,10 @@ __global__ void __launch_bounds__(B, 1)
 
 // ---- backward, stage 2 -------------------------------------------------------
 
-// Block of 256 threads = CT columns x (256 / CT) lanes. Lane l adds partials
-// l, l + L, ... of its column in binary64, then a fixed-order tree adds the
-// lanes; the sum is rounded once to P. Block 0 also reduces dalpha.
+// Block of 256 threads = CT columns x L lanes (L = 256 / CT, chosen on the host
+// so that a lane reads at most a few partials). Lane l adds partials l, l + L,
+// ... of its column in binary64, a fixed-order tree adds the lanes, and the
+// sum is rounded once to P. Block 0 also reduces dalpha.
 constexpr int kFinThreads = 256;
 
 template <typename P>
@@ -415,7 +623,22 @@ __global__ void __launch_bounds__(kFinThreads)
   const int64_t col = (int64_t)blockIdx.x * CT + c;
   double a = 0.0, b = 0.0;
   if (col < N) {
-    for (int r = lane; r < nrg; r += L) {
+    int r = lane;
+    for (; r + 3 * L < nrg; r += 4 * L) {  // four independent loads in flight
+      const float a0 = part_dg[(int64_t)r * N + col], a1 = part_dg[(int64_t)(r + L) * N + col];
+      const float a2 = part_dg[(int64_t)(r + 2 * L) * N + col], a3 = part_dg[(int64_t)(r + 3 * L) * N + col];
+      const float b0 = part_db[(int64_t)r * N + col], b1 = part_db[(int64_t)(r + L) * N + col];
+      const float b2 = part_db[(int64_t)(r + 2 * L) * N + col], b3 = part_db[(int64_t)(r + 3 * L) * N + col];
+      a += (double)a0;
+      a += (double)a1;
+      a += (double)a2;
+      a += (double)a3;
+      b += (double)b0;
+      b += (double)b1;
+      b += (double)b2;
+      b += (double)b3;
+    }
+    for (; r < nrg; r += L) {
       a += (double)part_dg[(int64_t)r * N + col];
       b += (double)part_db[(int64_t)r * N + col];
     }

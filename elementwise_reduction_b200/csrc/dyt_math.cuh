@@ -11,14 +11,16 @@ namespace dyt {
 
 // ---- hardware approximations (special-function unit) ---------------------
 
-// 2^w. Subnormal results are kept, so exp(-2|z|) decays smoothly to zero.
+// 2^w for w >= 0 (the only range it is used on: results are >= 1, so flushing
+// subnormals changes nothing).
 __device__ __forceinline__ float ex2_approx(float w) {
   float r;
-  asm("ex2.approx.f32 %0, %1;" : "=f"(r) : "f"(w));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(w));
   return r;
 }
 
-// 1/v for v in [1, 2] (the only range it is used on).
+// 1/v for v >= 2 (results <= 1/2; results below 2^-126, for |z| > 43.6, flush to
+// zero and are handled by the binary64 path below).
 __device__ __forceinline__ float rcp_approx(float v) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
@@ -28,54 +30,123 @@ __device__ __forceinline__ float rcp_approx(float v) {
 // ---- tanh(z) and 1 - tanh(z)^2 in binary32 --------------------------------
 //
 // a = |z|.
-//   a <  0.5: tanh a = a + a^3 Q(a^2), Q a degree-4 polynomial fitted to
+//   a <  0.5: tanh z = z + z^3 Q(z^2), Q a degree-4 polynomial fitted to
 //             minimise the relative error on [0, 0.5] (fit_tanh_poly.py next to
 //             this file; fitted error 3.6e-10, 0.67 ulp after binary32
-//             evaluation). 1 - t^2 = fma(-t, t, 1) has no cancellation there
-//             (t <= 0.47).
-//   a >= 0.5: with e = exp(-2a) = 2^(-2a log2 e) in (0, 0.37],
-//             tanh a = (1 - e) / (1 + e) and 1 - tanh^2 a = 4e / (1 + e)^2,
-//             both free of cancellation; e is one ex2 and 1/(1+e) one rcp.
-// tanh is odd: the sign of z is copied onto tanh(a), so t(-z) = -t(z)
-// exactly. a = +inf gives t = +-1 and 1 - t^2 = 0; NaN gives NaN in both.
+//             evaluation); odd in z, so the sign needs no handling. 1 - t^2 =
+//             fma(-t, t, 1) has no cancellation there (|t| <= 0.47).
+//   a >= 0.5: with E = exp(2a) = 2^(2a log2 e) >= e and r = 1 / (1 + E) <= 0.27,
+//             tanh a = 1 - 2r and 1 - tanh^2 a = 4r(1 - r), both free of
+//             cancellation; E is one ex2 and r one rcp. The sign of z is copied
+//             onto t.
+//   40 < a < 53: r < 2^-115 and 4r(1 - r) would lose precision, then flush to
+//             zero (a > 43.6) although 1 - t^2 = 4 exp(-2a) is still a binary32
+//             subnormal; it is recomputed in binary64 (a rare branch). From
+//             a = 52.7 on, 1 - t^2 rounds to 0 in binary32 and 4r(1 - r) = 0 is
+//             exact, infinities included.
+// t(-z) = -t(z) exactly. z = +-inf gives t = +-1, 1 - t^2 = 0; NaN gives NaN.
 constexpr float kTanhSplit = 0.5f;
-constexpr float kMinus2Log2e = -2.88539008177792681f;  // -2 / ln 2
+constexpr float kHugeArg = 40.0f;
+constexpr float kHugeArgEnd = 53.0f;
+
+__device__ __forceinline__ bool huge_arg(float z) {
+  const float a = fabsf(z);
+  return a > kHugeArg && a < kHugeArgEnd;
+}
+constexpr float k2Log2e = 2.88539008177792681f;  // 2 / ln 2
 constexpr float kQ0 = -0.333333283662796f;
 constexpr float kQ1 = 0.13332964479923248f;
 constexpr float kQ2 = -0.053899213671684265f;
 constexpr float kQ3 = 0.02129811979830265f;
 constexpr float kQ4 = -0.00664772093296051f;
 
-__device__ __forceinline__ float tanh_small(float a) {
-  const float u = a * a;
+__device__ __forceinline__ float tanh_small(float z) {
+  const float u = z * z;
   float q = fmaf(kQ4, u, kQ3);
   q = fmaf(q, u, kQ2);
   q = fmaf(q, u, kQ1);
   q = fmaf(q, u, kQ0);
-  return fmaf(a * u, q, a);
+  return fmaf(z * u, q, z);
+}
+
+__device__ __forceinline__ float tanh_r(float z) {  // r = 1 / (1 + exp(2|z|))
+  const float E = ex2_approx(fabsf(z * k2Log2e));
+  return rcp_approx(1.0f + E);
 }
 
 __device__ __forceinline__ float dyt_tanh(float z) {
-  const float a = fabsf(z);
-  const float e = ex2_approx(a * kMinus2Log2e);
-  const float r = rcp_approx(1.0f + e);
-  const float t_large = (1.0f - e) * r;
-  const float t_small = tanh_small(a);
-  return copysignf(a < kTanhSplit ? t_small : t_large, z);
+  const float r = tanh_r(z);
+  const float t_large = copysignf(fmaf(r, -2.0f, 1.0f), z);
+  const float t_small = tanh_small(z);
+  return fabsf(z) < kTanhSplit ? t_small : t_large;
+}
+
+// 1 - tanh(z)^2 for 40 < |z| < 53, from binary64: 4e / (1 + e)^2, e = exp(-2|z|).
+__device__ __noinline__ float sech2_huge(float z) {
+  const double e = exp(-2.0 * fabs((double)z));
+  const double d = 1.0 + e;
+  return (float)(4.0 * e / (d * d));
 }
 
 // t = tanh(z) and s = 1 - tanh(z)^2 from one evaluation.
 __device__ __forceinline__ void dyt_tanh_sech2(float z, float &t, float &s) {
-  const float a = fabsf(z);
-  const float e = ex2_approx(a * kMinus2Log2e);
-  const float r = rcp_approx(1.0f + e);
-  const float t_large = (1.0f - e) * r;
-  const float s_large = (4.0f * e) * (r * r);
-  const float t_small = tanh_small(a);
+  const float r = tanh_r(z);
+  const float t_large = copysignf(fmaf(r, -2.0f, 1.0f), z);
+  const float s_large = (4.0f * r) * fmaf(r, -1.0f, 1.0f);
+  const float t_small = tanh_small(z);
   const float s_small = fmaf(-t_small, t_small, 1.0f);
-  const bool small = a < kTanhSplit;
-  t = copysignf(small ? t_small : t_large, z);
+  const bool small = fabsf(z) < kTanhSplit;
+  t = small ? t_small : t_large;
   s = small ? s_small : s_large;
+  if (huge_arg(z)) s = sech2_huge(z);
+}
+
+// ---- the same on element pairs (packed f32x2 arithmetic of sm_100) ---------
+//
+// Identical formulas; the multiplies and adds run as two-lane f32x2
+// instructions, halving their issue cost. Every lane is rounded exactly as
+// its scalar counterpart (round to nearest even, no fused differences), so a
+// pair result equals two scalar results bit for bit.
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+__device__ __forceinline__ float2 tanh_small2(float2 z) {
+  const float2 u = mul2(z, z);
+  float2 q = fma2(f2(kQ4), u, f2(kQ3));
+  q = fma2(q, u, f2(kQ2));
+  q = fma2(q, u, f2(kQ1));
+  q = fma2(q, u, f2(kQ0));
+  return fma2(mul2(z, u), q, z);
+}
+
+__device__ __forceinline__ float2 tanh_r2(float2 z) {
+  const float2 w = mul2(z, f2(k2Log2e));
+  const float2 ope = add2(make_float2(ex2_approx(fabsf(w.x)), ex2_approx(fabsf(w.y))), f2(1.0f));
+  return make_float2(rcp_approx(ope.x), rcp_approx(ope.y));
+}
+
+__device__ __forceinline__ float2 dyt_tanh2(float2 z) {
+  const float2 r = tanh_r2(z);
+  const float2 tl = fma2(r, f2(-2.0f), f2(1.0f));
+  const float2 ts = tanh_small2(z);
+  return make_float2(fabsf(z.x) < kTanhSplit ? ts.x : copysignf(tl.x, z.x),
+                     fabsf(z.y) < kTanhSplit ? ts.y : copysignf(tl.y, z.y));
+}
+
+// t, s = 1 - t^2 for a pair; returns true when an element has 40 < |z| < 53
+// (its s must then be replaced by sech2_huge).
+__device__ __forceinline__ bool dyt_tanh_sech2_2(float2 z, float2 &t, float2 &s) {
+  const float2 r = tanh_r2(z);
+  const float2 tl = fma2(r, f2(-2.0f), f2(1.0f));
+  const float2 sl = mul2(mul2(r, f2(4.0f)), fma2(r, f2(-1.0f), f2(1.0f)));
+  const float2 ts = tanh_small2(z);
+  const float2 ss = make_float2(fmaf(-ts.x, ts.x, 1.0f), fmaf(-ts.y, ts.y, 1.0f));
+  const bool sx = fabsf(z.x) < kTanhSplit, sy = fabsf(z.y) < kTanhSplit;
+  t = make_float2(sx ? ts.x : copysignf(tl.x, z.x), sy ? ts.y : copysignf(tl.y, z.y));
+  s = make_float2(sx ? ss.x : sl.x, sy ? ss.y : sl.y);
+  return huge_arg(z.x) || huge_arg(z.y);
 }
 
 // ---- storage conversions ---------------------------------------------------
@@ -119,14 +190,15 @@ __device__ __forceinline__ __half from_f64<__half>(double v) {
 // ---- forward output with cancellation refinement ---------------------------
 //
 // y = gamma * t + beta. The binary32 value carries an error of at most
-// eps |gamma t| + 2^-24 |y|, with eps <= 2^-21 covering the error of t and of
-// z = alpha * x. A 16-bit output keeps p = 8 (bf16) or 11 (fp16) significant
-// bits, so one unit in its last place is at least 2^-p |y|; the binary32 value
-// is therefore within one unit whenever |y| >= tau |gamma t| with
-// tau = 2^-12 (bf16) or 2^-9 (fp16), with a factor-two margin. Elements below
-// that (cancellation, about 1e-3 of unit-scale data) are recomputed in
-// binary64 with the CUDA math library's tanh and rounded once, so every
-// 16-bit y is within one unit of the correctly rounded value.
+// eps |gamma t| + 2^-24 |y|, with eps <= 2^-20.5 covering the error of t and of
+// z = alpha * x. Since |gamma t| = |y - beta| <= |y| + |beta|, the error is at
+// most (eps (1 + 1/tau) + 2^-24) |y| whenever |y| >= tau |beta|. A 16-bit
+// output keeps p = 8 (bf16) or 11 (fp16) significant bits, so one unit in its
+// last place is at least 2^-p |y|; with tau = 2^-12 (bf16) or 2^-9 (fp16) the
+// binary32 value is within that, and the rounded result within one unit of the
+// correctly rounded one. Elements with |y| < tau |beta| (cancellation, about
+// 1e-3 of unit-scale data) are recomputed in binary64 with the CUDA math
+// library's tanh and rounded once.
 template <typename T>
 struct CancelGuard;
 template <>
@@ -149,16 +221,6 @@ template <typename T>
 __device__ __noinline__ T dyt_y_refined(float alpha, float x, float gamma, float beta) {
   const double t = tanh((double)alpha * (double)x);  // the product is exact in binary64
   return from_f64<T>(fma((double)gamma, t, (double)beta));
-}
-
-template <typename T>
-__device__ __forceinline__ T dyt_y(float alpha, float x, float gamma, float beta) {
-  const float t = dyt_tanh(alpha * x);
-  const float y = fmaf(gamma, t, beta);
-  if (CancelGuard<T>::kOn && fabsf(y) < fabsf(gamma * t) * CancelGuard<T>::kTau) {
-    return dyt_y_refined<T>(alpha, x, gamma, beta);
-  }
-  return from_f32<T>(y);
 }
 
 }  // namespace dyt

@@ -146,6 +146,8 @@ typedef struct dyt_launch_info {
   int col_chunks;    /* column chunks the grid is split into */
   int row_groups;    /* row groups (= partial sums per column) */
   int kernels;       /* kernels this call launched */
+  int tma_stages;    /* shared-memory stages of the CTA-wide bulk-copy pipeline (0 = unused) */
+  int async_stages;  /* per-thread asynchronous-copy ring slots (0 = unused) */
   int64_t workspace_bytes;
 } dyt_launch_info;
 
@@ -164,6 +166,22 @@ dyt_status dyt_last_launch_info(dyt_launch_info *out);
 dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
                           int backward, int vectorized, int sm_count, int ctas_per_sm,
                           dyt_launch_info *out);
+
+/*
+ * The device error word of the current device, a sticky bit set: bit 0 means a
+ * bounded wait inside a pipelined kernel gave up (its results are not valid).
+ * Synchronises with the device. clear != 0 resets the word to 0 afterwards.
+ */
+dyt_status dyt_device_error(unsigned int *word, int clear);
+
+/*
+ * Self-test of the bounded wait used by the pipelined kernels: enqueues on
+ * `stream` one kernel that waits on a barrier phase nothing will complete,
+ * giving up after `spin_limit` polls. It writes 1 to *gave_up (a DEVICE int)
+ * when the wait gave up and sets bit 0 of the device error word. The kernel
+ * always returns; nothing faults or hangs.
+ */
+dyt_status dyt_selftest_wait_timeout(unsigned int spin_limit, int *gave_up, dyt_stream_t stream);
 
 #ifdef __cplusplus
 }

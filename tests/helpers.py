@@ -160,6 +160,7 @@ def run_cuda(inp: dict, M: int, N: int, x_dtype: str, p_dtype: str, fwd: bool = 
         out.update(dx=to_numpy(dx, x_dtype), dgamma=to_numpy(dg, p_dtype), dbeta=to_numpy(db, p_dtype),
                    dalpha=float(decode(to_numpy(da, p_dtype), p_dtype)[0]))
     torch.cuda.synchronize()
+    assert dyt.dyt_device_error() == 0, "a pipelined kernel reported a wait that gave up"
     return out, info
 
 

@@ -73,16 +73,24 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
     p = dyt.dyt_plan_query(M, N, xd, 0, 1, vectorized, sms, occ)
     size = 4 if xd == 0 else 2
     vec = p["vec"]
-    assert vec in (1, 16 // size)
-    if vec > 1:
-        assert vectorized and N % vec == 0
+    assert not (p["tma_stages"] and p["async_stages"])
+    if p["async_stages"]:    # per-thread copy ring: 16-byte rows, one 16-byte vector per thread
+        assert vectorized and vec == 16 // size and N % vec == 0
+    if p["tma_stages"]:      # bulk-copy pipeline: 16-byte rows, 4 columns per thread
+        assert vectorized and (N * size) % 16 == 0 and vec == 4
+        assert 2 <= p["tma_stages"] <= 8
+    else:
+        assert vec in (1, 16 // size)
+        if vec > 1:
+            assert vectorized and N % vec == 0
     nv = N // vec
-    assert p["block"] == 1024 and p["kernels"] == 2
+    B = p["block"]
+    assert B in (512, 1024) and p["kernels"] == 2
     assert 1 <= p["grid"] <= sms * occ            # persistent 1D grid: never beyond one wave
     if p["path"] == 1:                             # row-tiled: several rows per CTA step
-        assert p["row_lanes"] == 1024 // nv >= 2 and p["col_chunks"] == 1
+        assert p["row_lanes"] == B // nv >= 2 and p["col_chunks"] == 1
     else:                                          # row-per-CTA: columns across the CTA
-        assert p["row_lanes"] == 1 and p["col_chunks"] == -(-nv // 1024)
+        assert p["row_lanes"] == 1 and p["col_chunks"] == -(-nv // B)
     items = p["row_groups"] * p["col_chunks"]
     assert p["grid"] <= items
     # every lane adds at most 96 rows per group (bounded binary32 error)

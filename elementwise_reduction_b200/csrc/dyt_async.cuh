@@ -161,24 +161,29 @@ __global__ void __launch_bounds__(B, 1)
       }
     } else {
       __syncthreads();  // every thread's ring is drained: reuse it for the reduction
+      if ((32 % g.NV) == 0) {
+        // the chunk's columns start at 0 on the row-tiled path (one chunk)
+        lane_reduce_warps<VEC, B>(acc.g, acc.b, red, g, ln, 0, pg, pb);
+      } else {
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.g[e];
-      __syncthreads();
-      lane_tree<VEC, B>(red, g, ln);
-      if (col_ok && ln.rl == 0) {
+        for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.g[e];
+        __syncthreads();
+        lane_tree<VEC, B>(red, g, ln);
+        if (col_ok && ln.rl == 0) {
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) pg[c0 + e] = red[e * B + threadIdx.x];
+          for (int e = 0; e < VEC; ++e) pg[c0 + e] = red[e * B + threadIdx.x];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.b[e];
+        __syncthreads();
+        lane_tree<VEC, B>(red, g, ln);
+        if (col_ok && ln.rl == 0) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) pb[c0 + e] = red[e * B + threadIdx.x];
+        }
+        __syncthreads();
       }
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.b[e];
-      __syncthreads();
-      lane_tree<VEC, B>(red, g, ln);
-      if (col_ok && ln.rl == 0) {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) pb[c0 + e] = red[e * B + threadIdx.x];
-      }
-      __syncthreads();
     }
   }
 #pragma unroll

@@ -429,6 +429,49 @@ __device__ __forceinline__ void lane_tree(float *red, const Geom &g, const Lane 
   }
 }
 
+// CTA sums of the row lanes when NV divides 32: every warp then holds 32 / NV
+// whole row lanes of the same NV vector-columns, so a butterfly over lane
+// offsets NV, 2 NV, ... 16 adds them in registers (both partners of an
+// exchange compute the same sum, so every lane ends with identical bits), and
+// one pass over the warps in order adds the warp sums. red[] holds
+// (B / 32) x NV x VEC floats. Results go to out_g / out_b (row of the group's
+// partials) at the thread's columns.
+template <int VEC, int B>
+__device__ __forceinline__ void lane_reduce_warps(const float (&vg)[VEC], const float (&vb)[VEC], float *red,
+                                                  const Geom &g, const Lane &ln, int64_t c0_chunk,
+                                                  float *out_g, float *out_b) {
+  float ag[VEC], ab[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    ag[e] = vg[e];
+    ab[e] = vb[e];
+  }
+  for (int off = g.NV; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      ag[e] += __shfl_xor_sync(0xFFFFFFFFu, ag[e], off);
+      ab[e] += __shfl_xor_sync(0xFFFFFFFFu, ab[e], off);
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int width = g.NV * VEC;  // floats per warp and sum
+  if (lane < g.NV) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      red[(2 * warp) * width + lane * VEC + e] = ag[e];
+      red[(2 * warp + 1) * width + lane * VEC + e] = ab[e];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 2 * width) {
+    const int which = threadIdx.x / width, k = threadIdx.x - which * width;
+    float sum = 0.0f;
+    for (int w = 0; w < B / 32; ++w) sum += red[(2 * w + which) * width + k];
+    (which ? out_b : out_g)[c0_chunk + k] = sum;
+  }
+  __syncthreads();
+}
+
 // Per-thread backward state for VEC columns.
 template <int VEC>
 struct BwdAcc {
@@ -449,16 +492,10 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
     float2 x2[H], dy2[H], dx2[H];
     IO::unpack2(rx, x2);
     IO::unpack2(rdy, dy2);
-    bool huge = false;
 #pragma unroll
     for (int h = 0; h < H; ++h) {
       float2 t, s;
-      const float2 z = mul2(f2(alpha), x2[h]);
-      if (dyt_tanh_sech2_2(z, t, s)) {  // rare: 40 < |z| < 53
-        huge = true;
-        if (huge_arg(z.x)) s.x = sech2_huge(z.x);
-        if (huge_arg(z.y)) s.y = sech2_huge(z.y);
-      }
+      dyt_tanh_sech2_2(mul2(f2(alpha), x2[h]), t, s);
       const float2 gdys = mul2(mul2(make_float2(gam[2 * h], gam[2 * h + 1]), dy2[h]), s);
       dx2[h] = mul2(f2(alpha), gdys);
       const float2 ag = make_float2(acc.g[2 * h], acc.g[2 * h + 1]);
@@ -475,7 +512,6 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       acc.b[2 * h + 1] = nb.y;
       ca = nca;
     }
-    (void)huge;
     return IO::pack2(dx2);
   } else {
     float xf[VEC], dyf[VEC], dxf[VEC];

@@ -11,16 +11,21 @@ namespace dyt {
 
 // ---- hardware approximations (special-function unit) ---------------------
 
-// 2^w for w >= 0 (the only range it is used on: results are >= 1, so flushing
-// subnormals changes nothing).
+// 2^w for w >= 0 (results >= 1, so flushing subnormals changes nothing).
 __device__ __forceinline__ float ex2_approx(float w) {
   float r;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(w));
   return r;
 }
 
-// 1/v for v >= 2 (results <= 1/2; results below 2^-126, for |z| > 43.6, flush to
-// zero and are handled by the binary64 path below).
+// 2^w for w <= 0, subnormal results kept (exp(-2|z|) decays smoothly to 0).
+__device__ __forceinline__ float ex2_approx_sub(float w) {
+  float r;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(r) : "f"(w));
+  return r;
+}
+
+// 1/v for v >= 1 (normal results only).
 __device__ __forceinline__ float rcp_approx(float v) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
@@ -30,75 +35,54 @@ __device__ __forceinline__ float rcp_approx(float v) {
 // ---- tanh(z) and 1 - tanh(z)^2 in binary32 --------------------------------
 //
 // a = |z|.
-//   a <  0.5: tanh z = z + z^3 Q(z^2), Q a degree-4 polynomial fitted to
+//   a <  0.5: tanh z = z + z^3 Q(z^2), Q a degree-3 polynomial fitted to
 //             minimise the relative error on [0, 0.5] (fit_tanh_poly.py next to
-//             this file; fitted error 3.6e-10, 0.67 ulp after binary32
+//             this file; fitted error 1.5e-8, 0.84 ulp after binary32
 //             evaluation); odd in z, so the sign needs no handling. 1 - t^2 =
 //             fma(-t, t, 1) has no cancellation there (|t| <= 0.47).
-//   a >= 0.5: with E = exp(2a) = 2^(2a log2 e) >= e and r = 1 / (1 + E) <= 0.27,
-//             tanh a = 1 - 2r and 1 - tanh^2 a = 4r(1 - r), both free of
-//             cancellation; E is one ex2 and r one rcp. The sign of z is copied
-//             onto t.
-//   40 < a < 53: r < 2^-115 and 4r(1 - r) would lose precision, then flush to
-//             zero (a > 43.6) although 1 - t^2 = 4 exp(-2a) is still a binary32
-//             subnormal; it is recomputed in binary64 (a rare branch). From
-//             a = 52.7 on, 1 - t^2 rounds to 0 in binary32 and 4r(1 - r) = 0 is
-//             exact, infinities included.
+//   a >= 0.5, forward (t only): with E = exp(2a) = 2^(2a log2 e) >= e and
+//             r = 1 / (1 + E) <= 0.27, tanh a = 1 - 2r (no cancellation).
+//   a >= 0.5, backward (t and 1 - t^2): with e = exp(-2a) <= 0.37 (subnormal
+//             values kept) and rc = 1 / (1 + e) in [0.73, 1],
+//             tanh a = (1 - e) rc and 1 - tanh^2 a = 4 e rc^2; both stay
+//             accurate, relative to binary32's own precision, down to the
+//             subnormal range and reach 0 when 1 - t^2 does.
+//   The sign of z is copied onto t in both forms.
 // t(-z) = -t(z) exactly. z = +-inf gives t = +-1, 1 - t^2 = 0; NaN gives NaN.
 constexpr float kTanhSplit = 0.5f;
-constexpr float kHugeArg = 40.0f;
-constexpr float kHugeArgEnd = 53.0f;
-
-__device__ __forceinline__ bool huge_arg(float z) {
-  const float a = fabsf(z);
-  return a > kHugeArg && a < kHugeArgEnd;
-}
 constexpr float k2Log2e = 2.88539008177792681f;  // 2 / ln 2
-constexpr float kQ0 = -0.333333283662796f;
-constexpr float kQ1 = 0.13332964479923248f;
-constexpr float kQ2 = -0.053899213671684265f;
-constexpr float kQ3 = 0.02129811979830265f;
-constexpr float kQ4 = -0.00664772093296051f;
+constexpr float kQ0 = -0.333331435918808f;
+constexpr float kQ1 = 0.13325883448123932f;
+constexpr float kQ2 = -0.053045812994241714f;
+constexpr float kQ3 = 0.017242243513464928f;
 
 __device__ __forceinline__ float tanh_small(float z) {
   const float u = z * z;
-  float q = fmaf(kQ4, u, kQ3);
-  q = fmaf(q, u, kQ2);
+  float q = fmaf(kQ3, u, kQ2);
   q = fmaf(q, u, kQ1);
   q = fmaf(q, u, kQ0);
   return fmaf(z * u, q, z);
 }
 
-__device__ __forceinline__ float tanh_r(float z) {  // r = 1 / (1 + exp(2|z|))
-  const float E = ex2_approx(fabsf(z * k2Log2e));
-  return rcp_approx(1.0f + E);
-}
-
 __device__ __forceinline__ float dyt_tanh(float z) {
-  const float r = tanh_r(z);
+  const float E = ex2_approx(fabsf(z * k2Log2e));
+  const float r = rcp_approx(1.0f + E);
   const float t_large = copysignf(fmaf(r, -2.0f, 1.0f), z);
   const float t_small = tanh_small(z);
   return fabsf(z) < kTanhSplit ? t_small : t_large;
 }
 
-// 1 - tanh(z)^2 for 40 < |z| < 53, from binary64: 4e / (1 + e)^2, e = exp(-2|z|).
-__device__ __noinline__ float sech2_huge(float z) {
-  const double e = exp(-2.0 * fabs((double)z));
-  const double d = 1.0 + e;
-  return (float)(4.0 * e / (d * d));
-}
-
 // t = tanh(z) and s = 1 - tanh(z)^2 from one evaluation.
 __device__ __forceinline__ void dyt_tanh_sech2(float z, float &t, float &s) {
-  const float r = tanh_r(z);
-  const float t_large = copysignf(fmaf(r, -2.0f, 1.0f), z);
-  const float s_large = (4.0f * r) * fmaf(r, -1.0f, 1.0f);
+  const float e = ex2_approx_sub(-fabsf(z * k2Log2e));
+  const float rc = rcp_approx(1.0f + e);
+  const float t_large = copysignf(fmaf(e, -1.0f, 1.0f) * rc, z);
+  const float s_large = (4.0f * e) * (rc * rc);
   const float t_small = tanh_small(z);
   const float s_small = fmaf(-t_small, t_small, 1.0f);
   const bool small = fabsf(z) < kTanhSplit;
   t = small ? t_small : t_large;
   s = small ? s_small : s_large;
-  if (huge_arg(z)) s = sech2_huge(z);
 }
 
 // ---- the same on element pairs (packed f32x2 arithmetic of sm_100) ---------
@@ -114,39 +98,34 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 
 __device__ __forceinline__ float2 tanh_small2(float2 z) {
   const float2 u = mul2(z, z);
-  float2 q = fma2(f2(kQ4), u, f2(kQ3));
-  q = fma2(q, u, f2(kQ2));
+  float2 q = fma2(f2(kQ3), u, f2(kQ2));
   q = fma2(q, u, f2(kQ1));
   q = fma2(q, u, f2(kQ0));
   return fma2(mul2(z, u), q, z);
 }
 
-__device__ __forceinline__ float2 tanh_r2(float2 z) {
+__device__ __forceinline__ float2 dyt_tanh2(float2 z) {
   const float2 w = mul2(z, f2(k2Log2e));
   const float2 ope = add2(make_float2(ex2_approx(fabsf(w.x)), ex2_approx(fabsf(w.y))), f2(1.0f));
-  return make_float2(rcp_approx(ope.x), rcp_approx(ope.y));
-}
-
-__device__ __forceinline__ float2 dyt_tanh2(float2 z) {
-  const float2 r = tanh_r2(z);
+  const float2 r = make_float2(rcp_approx(ope.x), rcp_approx(ope.y));
   const float2 tl = fma2(r, f2(-2.0f), f2(1.0f));
   const float2 ts = tanh_small2(z);
   return make_float2(fabsf(z.x) < kTanhSplit ? ts.x : copysignf(tl.x, z.x),
                      fabsf(z.y) < kTanhSplit ? ts.y : copysignf(tl.y, z.y));
 }
 
-// t, s = 1 - t^2 for a pair; returns true when an element has 40 < |z| < 53
-// (its s must then be replaced by sech2_huge).
-__device__ __forceinline__ bool dyt_tanh_sech2_2(float2 z, float2 &t, float2 &s) {
-  const float2 r = tanh_r2(z);
-  const float2 tl = fma2(r, f2(-2.0f), f2(1.0f));
-  const float2 sl = mul2(mul2(r, f2(4.0f)), fma2(r, f2(-1.0f), f2(1.0f)));
+__device__ __forceinline__ void dyt_tanh_sech2_2(float2 z, float2 &t, float2 &s) {
+  const float2 w = mul2(z, f2(k2Log2e));
+  const float2 e = make_float2(ex2_approx_sub(-fabsf(w.x)), ex2_approx_sub(-fabsf(w.y)));
+  const float2 ope = add2(e, f2(1.0f));
+  const float2 rc = make_float2(rcp_approx(ope.x), rcp_approx(ope.y));
+  const float2 tl = mul2(fma2(e, f2(-1.0f), f2(1.0f)), rc);
+  const float2 sl = mul2(mul2(f2(4.0f), e), mul2(rc, rc));
   const float2 ts = tanh_small2(z);
   const float2 ss = make_float2(fmaf(-ts.x, ts.x, 1.0f), fmaf(-ts.y, ts.y, 1.0f));
   const bool sx = fabsf(z.x) < kTanhSplit, sy = fabsf(z.y) < kTanhSplit;
   t = make_float2(sx ? ts.x : copysignf(tl.x, z.x), sy ? ts.y : copysignf(tl.y, z.y));
   s = make_float2(sx ? ss.x : sl.x, sy ? ss.y : sl.y);
-  return huge_arg(z.x) || huge_arg(z.y);
 }
 
 // ---- storage conversions ---------------------------------------------------

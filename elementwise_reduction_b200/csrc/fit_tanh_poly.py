@@ -7,7 +7,7 @@ binary32 coefficients and the error after binary32 evaluation.
 import numpy as np
 
 T = 0.5
-deg = 4
+deg = 3
 def tanh_hi(a):  # binary64 is plenty for a fit target at the 1e-10 level
     return np.tanh(a)
 u = np.linspace(1e-8, T*T, 20001)

@@ -51,6 +51,9 @@ lib.dyt_last_launch_info.argtypes = [ctypes.POINTER(LaunchInfo)]
 lib.dyt_last_launch_info.restype = _i32
 lib.dyt_plan_query.argtypes = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(LaunchInfo)]
 lib.dyt_plan_query.restype = _i32
+lib.dyt_backward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp]
+lib.dyt_backward_noalloc.restype = _i32
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # DYT_NOALLOC_SCRATCH_BYTES in include/dyt.h
 lib.dyt_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
 lib.dyt_device_error.restype = _i32
 lib.dyt_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp, _vp]
@@ -85,6 +88,14 @@ def dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, 
     """Raw C-ABI call: pointers as ints. Returns the status code."""
     return lib.dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
                             workspace, workspace_bytes, stream)
+
+
+def dyt_backward_noalloc(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
+                         stream) -> int:
+    """Raw C-ABI call of the backward that uses the library's built-in scratch
+    instead of a workspace (for callers that cannot allocate). Returns the status."""
+    return lib.dyt_backward_noalloc(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
+                                    stream)
 
 
 def dyt_status_string(status: int) -> str:

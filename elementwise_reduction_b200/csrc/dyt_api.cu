@@ -573,3 +573,52 @@ dyt_status dyt_last_launch_info(dyt_launch_info *out) {
 }
 
 }  // extern "C"
+
+// ---- backward without a caller-provided workspace ---------------------------------
+//
+// For callers that cannot allocate device memory themselves (an embedding
+// application owning all device memory, or loops that cannot afford
+// cudaMalloc's implicit synchronisation): the scratch is a fixed file-scope
+// device array. Host code only ever sees a stand-in for its name, so the
+// device address is looked up with cudaGetSymbolAddress, once per device,
+// with that device current, and handed to the kernels.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_dyt_noalloc_scratch[DYT_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+std::unordered_map<int, void *> g_noalloc_ptr;  // device -> address of the array
+
+dyt_status noalloc_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  auto it = g_noalloc_ptr.find(dev);
+  if (it != g_noalloc_ptr.end()) {
+    *out = it->second;
+    return DYT_OK;
+  }
+  void *p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_dyt_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e);
+  g_noalloc_ptr[dev] = p;
+  *out = p;
+  return DYT_OK;
+}
+
+}  // namespace
+
+extern "C" dyt_status dyt_backward_noalloc(const void *x, const void *dy, const void *alpha, const void *gamma,
+                                           void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M,
+                                           int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
+                                           dyt_stream_t stream) {
+  void *scratch = nullptr;
+  const dyt_status st = noalloc_scratch(&scratch);
+  if (st != DYT_OK) return st;
+  // dyt_backward checks the arguments and rejects, before launching, a shape
+  // whose scratch need exceeds the array (DYT_ERR_WORKSPACE_TOO_SMALL).
+  return dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype, scratch,
+                      DYT_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -183,6 +183,35 @@ dyt_status dyt_device_error(unsigned int *word, int clear);
  */
 dyt_status dyt_selftest_wait_timeout(unsigned int spin_limit, int *gave_up, dyt_stream_t stream);
 
+/*
+ * Backward without a caller-provided workspace (no counterpart in the paper:
+ * it exists for callers that cannot allocate device memory themselves, such as
+ * code embedded in a host application that owns all device memory through its
+ * own pool, or latency-critical loops where cudaMalloc's implicit device
+ * synchronisation is not acceptable).
+ *
+ * Same arguments, results and errors as dyt_backward, minus the workspace: the
+ * scratch comes from a fixed array of DYT_NOALLOC_SCRATCH_BYTES bytes that the
+ * library keeps in device memory (every device that loads the library holds it
+ * until the process exits). The call allocates nothing.
+ * - The first call on each device looks the array's device address up
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Shapes whose scratch need (dyt_backward_workspace_bytes) exceeds
+ *   DYT_NOALLOC_SCRATCH_BYTES are rejected with DYT_ERR_WORKSPACE_TOO_SMALL
+ *   before anything is launched.
+ * - Every call on a device shares the one array, which keeps the last call's
+ *   contents; nothing in it has to start at zero (each call rewrites every
+ *   partial sum before reading it). Calls that overlap on the GPU (on
+ *   different streams, or from different host threads without ordering) race
+ *   on the array and give undefined results: order them on one stream.
+ */
+#define DYT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+dyt_status dyt_backward_noalloc(const void *x, const void *dy, const void *alpha, const void *gamma,
+                                void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
+                                dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

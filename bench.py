@@ -49,6 +49,11 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-shapes", action="store_true", help="skip the per-shape table of the other workloads")
+    p.add_argument("--record-traffic", metavar="NCU_CSV", default=None,
+                   help="store DRAM bytes per launch from an ncu --csv capture of dram__bytes_read.sum and "
+                        "dram__bytes_write.sum into profiles/dram_traffic.json for --workload, then exit")
+    p.add_argument("--ncu-command", default="", help="the ncu command line that wrote --record-traffic's CSV")
     return p.parse_args()
 
 
@@ -83,6 +88,48 @@ def committed_traffic(workload: str, kernel: str):
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
     return e.get("bytes_per_launch")
+
+
+def record_traffic(csv_path: str, workload: str, command: str) -> None:
+    """DRAM bytes per launch of each DyT kernel from an ncu CSV, stored with the hash of
+    the kernel sources they were taken on."""
+    import csv
+    import re
+
+    per = {}
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(f) if len(r) > 5]
+    hdr = rows[0]
+    ki, mi, vi, ui = (hdr.index(k) for k in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit"))
+    idi = hdr.index("ID")
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    launches = {}
+    for r in rows[1:]:
+        m = re.search(r"(dyt_\w+)", r[ki])
+        if not m or not r[mi].startswith("dram__bytes_"):
+            continue
+        kernel = "dyt_bwd_kernel" if "bwd" in m.group(1) else "dyt_fwd_kernel" if "fwd" in m.group(1) \
+            else "dyt_finalize_kernel"
+        per.setdefault(kernel, 0.0)
+        per[kernel] += float(r[vi].replace(",", "")) * scale.get(r[ui], 1)
+        launches.setdefault(kernel, set()).add(r[idi])
+    path = os.path.join(PROFILES, "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        d = {}
+    entry = {k: {"bytes_per_launch": v / len(launches[k]), "launches": len(launches[k]),
+                 "source_hash": kernel_source_hash(), "command": command} for k, v in per.items()}
+    if "dyt_bwd_kernel" in entry and "dyt_finalize_kernel" in entry:
+        entry["dyt_backward"] = {
+            "bytes_per_launch": entry["dyt_bwd_kernel"]["bytes_per_launch"]
+            + entry["dyt_finalize_kernel"]["bytes_per_launch"],
+            "source_hash": kernel_source_hash(), "command": command}
+    d[workload] = entry
+    with open(path, "w") as f:
+        json.dump(d, f, indent=1, sort_keys=True)
+    print(json.dumps(entry, indent=1))
 
 
 # ---- clocks sampled during the timed region ---------------------------------------------------
@@ -308,9 +355,19 @@ def run_ours(args, w):
             return ms
 
         with ClockSampler(local, enabled=not args.no_clocks) as clk:
+            # Keep the GPU under the same load for ~0.3 s around the timed replays so
+            # that the sampled clocks (every 100 ms) describe the timed region.
+            t_end = time.perf_counter() + 0.3
+            while time.perf_counter() < t_end:
+                g_step.replay()
+                torch.cuda.synchronize(dev)
             ms_step = timed(g_step)
             ms_fwd = timed(g_fwd)
             ms_bwd = timed(g_bwd)
+            t_end = time.perf_counter() + 0.15
+            while time.perf_counter() < t_end:
+                g_step.replay()
+                torch.cuda.synchronize(dev)
         clocks = clk.summary()
         del g_step, g_fwd, g_bwd  # graphs that may hold NCCL calls go before the process group
 
@@ -365,7 +422,7 @@ def run_ours(args, w):
     t_fwd, t_bwd = ms_fwd / args.steps * 1e-3, ms_bwd / args.steps * 1e-3
     bw_fwd, bw_bwd = fb / t_fwd / 1e9, bb / t_bwd / 1e9
     dominant = "bwd" if t_bwd >= t_fwd else "fwd"
-    traffic = committed_traffic(w.name, "dyt_bwd_kernel" if dominant == "bwd" else "dyt_fwd_kernel")
+    traffic = committed_traffic(w.name, "dyt_backward" if dominant == "bwd" else "dyt_fwd_kernel")
     roofline = {
         "bound": "hbm", "kernel": "dyt_backward (stage-1 + finalize)" if dominant == "bwd" else "dyt_forward",
         "achieved": bw_bwd if dominant == "bwd" else bw_fwd, "peak": peak, "unit": "GB/s",
@@ -399,9 +456,78 @@ def run_ours(args, w):
     }
     if world > 1:
         dist.destroy_process_group()
+    if world == 1 and not args.no_shapes:
+        line["shapes"] = other_shapes(w, args, dev)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
+
+
+def other_shapes(w0, args, dev):
+    """Forward and backward throughput of the other workloads (the metric is quoted per
+    shape), each timed like the main one: a CUDA graph of K calls over rotating buffer
+    sets that exceed L2."""
+    import torch
+
+    import elementwise_reduction_b200 as dyt
+    from synth import workloads
+
+    out = {}
+    peak, _ = hbm_peak()
+    L2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    for name, w in workloads.WORKLOADS.items():
+        if name == w0.name:
+            continue
+        inp = workloads.make_inputs(w)
+        M, N = w.M, w.N
+
+        def dev_t(a, dt):
+            a = np.ascontiguousarray(a)
+            t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dt == "bf16" else torch.from_numpy(a)
+            return t.to(dev)
+
+        x0, dy0 = dev_t(inp["x"], w.x_dtype).view(M, N), dev_t(inp["dy"], w.x_dtype).view(M, N)
+        a, g, b = (dev_t(inp[k], w.p_dtype) for k in ("alpha", "gamma", "beta"))
+        set_bytes = 4 * M * N * workloads.ITEMSIZE[w.x_dtype]
+        nsets = int(min(64, max(1, -(-3 * L2 // set_bytes))))
+        sets = [{"x": x0.clone(), "dy": dy0.clone(), "y": torch.empty_like(x0), "dx": torch.empty_like(x0),
+                 "dg": torch.empty_like(g), "db": torch.empty_like(g),
+                 "da": torch.empty(1, dtype=g.dtype, device=dev)} for _ in range(nsets)]
+        ws = dyt.workspace(x0, g)
+        stream = torch.cuda.Stream(dev)
+        K = args.steps
+        res = {}
+        with torch.cuda.stream(stream):
+            for op in ("fwd", "bwd"):
+                def call(i, op=op):
+                    s = sets[i % nsets]
+                    if op == "fwd":
+                        dyt.forward(s["x"], a, g, b, out=s["y"])
+                    else:
+                        dyt.backward(s["x"], s["dy"], a, g, dx=s["dx"], dgamma=s["dg"], dbeta=s["db"],
+                                     dalpha=s["da"], ws=ws)
+                for i in range(3):
+                    call(i)
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=stream):
+                    for i in range(K):
+                        call(i)
+                graph.replay()
+                torch.cuda.synchronize(dev)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                t = e0.elapsed_time(e1) / K * 1e-3
+                nbytes = w.fwd_bytes() if op == "fwd" else w.bwd_bytes()
+                res[op] = {"us": t * 1e6, "GB_s": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
+                           "rows_per_s": M / t}
+                del graph
+        out[name] = res
+        del sets, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -410,6 +536,9 @@ def main():
 
     name = args.workload or workloads.DEFAULT_BENCH
     w = workloads.WORKLOADS[name]
+    if args.record_traffic:
+        record_traffic(args.record_traffic, w.name, args.ncu_command)
+        return
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(B, 1)
     BwdAcc<VEC> acc;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      gam[e] = col_ok ? param(gamma, c0 + e) : 0.0f;
+      gam[e] = col_ok ? 4.0f * param(gamma, c0 + e) : 0.0f;  // 4 gamma (see bwd_vector)
       acc.g[e] = 0.0f;
       acc.b[e] = 0.0f;
     }

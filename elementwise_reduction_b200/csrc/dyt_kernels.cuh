@@ -479,12 +479,14 @@ struct BwdAcc {
   float b[VEC];  // sum of dy
 };
 
-// One vector (one row, VEC columns): dx out, sums in. MASKED: the row may be
-// padding; its results are computed like any other and dropped afterwards.
+// One vector (one row, VEC columns): dx out, sums in. g4[e] = 4 gamma[e]
+// (with q = (1 - t^2) / 4, g4 * dy * q rounds exactly as gamma * dy * (1 - t^2)).
+// MASKED: the row may be padding; its results are computed like any other and
+// dropped afterwards.
 template <typename T, int VEC, bool MASKED>
 __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename VecIO<T, VEC>::Raw &rx,
                                                                  const typename VecIO<T, VEC>::Raw &rdy,
-                                                                 float alpha, const float (&gam)[VEC],
+                                                                 float alpha, const float (&g4)[VEC],
                                                                  BwdAcc<VEC> &acc, float2 &ca, bool ok) {
   using IO = VecIO<T, VEC>;
   if constexpr (IO::kPairs > 0) {
@@ -494,9 +496,9 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
     IO::unpack2(rdy, dy2);
 #pragma unroll
     for (int h = 0; h < H; ++h) {
-      float2 t, s;
-      dyt_tanh_sech2_2(mul2(f2(alpha), x2[h]), t, s);
-      const float2 gdys = mul2(mul2(make_float2(gam[2 * h], gam[2 * h + 1]), dy2[h]), s);
+      float2 t, q;
+      dyt_tanh_qsech2_2(mul2(f2(alpha), x2[h]), t, q);
+      const float2 gdys = mul2(mul2(make_float2(g4[2 * h], g4[2 * h + 1]), dy2[h]), q);  // gamma dy (1-t^2)
       dx2[h] = mul2(f2(alpha), gdys);
       const float2 ag = make_float2(acc.g[2 * h], acc.g[2 * h + 1]);
       const float2 ab = make_float2(acc.b[2 * h], acc.b[2 * h + 1]);
@@ -519,9 +521,9 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
     IO::unpack(rdy, dyf);
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      float t, s;
-      dyt_tanh_sech2(alpha * xf[e], t, s);
-      const float gdys = (gam[e] * dyf[e]) * s;
+      float t, q;
+      dyt_tanh_qsech2(alpha * xf[e], t, q);
+      const float gdys = (g4[e] * dyf[e]) * q;
       dxf[e] = alpha * gdys;
       const float ng = fmaf(dyf[e], t, acc.g[e]), nb = acc.b[e] + dyf[e], nca = fmaf(gdys, xf[e], ca.x);
       acc.g[e] = (MASKED && !ok) ? acc.g[e] : ng;
@@ -558,7 +560,7 @@ __global__ void __launch_bounds__(B, 1)
     BwdAcc<VEC> acc;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      gam[e] = col_ok ? param(gamma, c0 + e) : 0.0f;
+      gam[e] = col_ok ? 4.0f * param(gamma, c0 + e) : 0.0f;  // 4 gamma (see bwd_vector)
       acc.g[e] = 0.0f;
       acc.b[e] = 0.0f;
     }

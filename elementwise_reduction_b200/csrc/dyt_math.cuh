@@ -42,11 +42,14 @@ __device__ __forceinline__ float rcp_approx(float v) {
 //             fma(-t, t, 1) has no cancellation there (|t| <= 0.47).
 //   a >= 0.5, forward (t only): with E = exp(2a) = 2^(2a log2 e) >= e and
 //             r = 1 / (1 + E) <= 0.27, tanh a = 1 - 2r (no cancellation).
-//   a >= 0.5, backward (t and 1 - t^2): with e = exp(-2a) <= 0.37 (subnormal
-//             values kept) and rc = 1 / (1 + e) in [0.73, 1],
-//             tanh a = (1 - e) rc and 1 - tanh^2 a = 4 e rc^2; both stay
-//             accurate, relative to binary32's own precision, down to the
-//             subnormal range and reach 0 when 1 - t^2 does.
+//   a >= 0.5, backward t: with e = exp(-2a) <= 0.37 (subnormal values kept)
+//             and rc = 1 / (1 + e), tanh a = (1 - e) rc (no cancellation).
+//   backward 1 - t^2, every a: 1 - tanh^2 a = 4 e rc^2 with e = exp(-2a) in
+//             (0, 1] and rc in [1/2, 1]: no cancellation anywhere, accurate to
+//             about 2^-21 relative down to the subnormal range, 0 exactly when
+//             1 - t^2 rounds to 0, and exactly 1 at z = 0. The kernels carry
+//             q = (1 - t^2) / 4 = e rc^2 and multiply it by 4 gamma, which
+//             rounds exactly as gamma (1 - t^2) would (scaling by 4 is exact).
 //   The sign of z is copied onto t in both forms.
 // t(-z) = -t(z) exactly. z = +-inf gives t = +-1, 1 - t^2 = 0; NaN gives NaN.
 constexpr float kTanhSplit = 0.5f;
@@ -72,17 +75,13 @@ __device__ __forceinline__ float dyt_tanh(float z) {
   return fabsf(z) < kTanhSplit ? t_small : t_large;
 }
 
-// t = tanh(z) and s = 1 - tanh(z)^2 from one evaluation.
-__device__ __forceinline__ void dyt_tanh_sech2(float z, float &t, float &s) {
+// t = tanh(z) and q = (1 - tanh(z)^2) / 4 from one evaluation.
+__device__ __forceinline__ void dyt_tanh_qsech2(float z, float &t, float &q) {
   const float e = ex2_approx_sub(-fabsf(z * k2Log2e));
   const float rc = rcp_approx(1.0f + e);
   const float t_large = copysignf(fmaf(e, -1.0f, 1.0f) * rc, z);
-  const float s_large = (4.0f * e) * (rc * rc);
-  const float t_small = tanh_small(z);
-  const float s_small = fmaf(-t_small, t_small, 1.0f);
-  const bool small = fabsf(z) < kTanhSplit;
-  t = small ? t_small : t_large;
-  s = small ? s_small : s_large;
+  q = (e * rc) * rc;
+  t = fabsf(z) < kTanhSplit ? tanh_small(z) : t_large;
 }
 
 // ---- the same on element pairs (packed f32x2 arithmetic of sm_100) ---------
@@ -114,18 +113,16 @@ __device__ __forceinline__ float2 dyt_tanh2(float2 z) {
                      fabsf(z.y) < kTanhSplit ? ts.y : copysignf(tl.y, z.y));
 }
 
-__device__ __forceinline__ void dyt_tanh_sech2_2(float2 z, float2 &t, float2 &s) {
+__device__ __forceinline__ void dyt_tanh_qsech2_2(float2 z, float2 &t, float2 &q) {
   const float2 w = mul2(z, f2(k2Log2e));
   const float2 e = make_float2(ex2_approx_sub(-fabsf(w.x)), ex2_approx_sub(-fabsf(w.y)));
   const float2 ope = add2(e, f2(1.0f));
   const float2 rc = make_float2(rcp_approx(ope.x), rcp_approx(ope.y));
   const float2 tl = mul2(fma2(e, f2(-1.0f), f2(1.0f)), rc);
-  const float2 sl = mul2(mul2(f2(4.0f), e), mul2(rc, rc));
+  q = mul2(mul2(e, rc), rc);
   const float2 ts = tanh_small2(z);
-  const float2 ss = make_float2(fmaf(-ts.x, ts.x, 1.0f), fmaf(-ts.y, ts.y, 1.0f));
-  const bool sx = fabsf(z.x) < kTanhSplit, sy = fabsf(z.y) < kTanhSplit;
-  t = make_float2(sx ? ts.x : copysignf(tl.x, z.x), sy ? ts.y : copysignf(tl.y, z.y));
-  s = make_float2(sx ? ss.x : sl.x, sy ? ss.y : sl.y);
+  t = make_float2(fabsf(z.x) < kTanhSplit ? ts.x : copysignf(tl.x, z.x),
+                  fabsf(z.y) < kTanhSplit ? ts.y : copysignf(tl.y, z.y));
 }
 
 // ---- storage conversions ---------------------------------------------------

@@ -59,7 +59,7 @@ constexpr int kMaxDynSmem = 227 * 1024;
 constexpr int kAsyncBlock = DYT_ASYNC_BLOCK;  // one CTA per SM: up to 128 registers a thread
 constexpr int kAsyncStagesFwd = DYT_ASYNC_STAGES_FWD;
 constexpr int kAsyncStagesBwd = DYT_ASYNC_STAGES_BWD;
-constexpr int kMaxRowsPerLane = 96;   // sequential binary32 adds per thread per group
+constexpr int kMaxRowsPerLane = 128;  // sequential binary32 adds per thread per group
 constexpr int kFwdUnrollVec = DYT_FWD_UNROLL_VEC;        // rows in flight per thread, 16-byte access
 constexpr int kBwdUnrollVec = DYT_BWD_UNROLL_VEC;
 constexpr int kFwdUnrollScalar = DYT_FWD_UNROLL_SCALAR;  // rows in flight per thread, scalar access
@@ -381,10 +381,18 @@ dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, cons
     Plan p;
     dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y), false, &p);
     if (s != DYT_OK) return s;
+    // Programmatic dependent launch: the kernel may be scheduled while its
+    // predecessor in the stream drains; its first instruction waits
+    // (griddepcontrol.wait) for that predecessor, so stream order holds.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
     cfg.blockDim = dim3(p.block);
     cfg.stream = (cudaStream_t)stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
     cudaError_t e;
     if (p.tma) {
       cfg.dynamicSmemBytes = p.smem;
@@ -462,10 +470,15 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
     float *pdb = (float *)(ws + p.ws_db);
     double *pda = (double *)(ws + p.ws_da);
 
+    cudaLaunchAttribute pdl[1];  // see dyt_forward
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
     cfg.blockDim = dim3(p.block);
     cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
     cudaError_t e;
     if (p.tma) {
       cfg.dynamicSmemBytes = p.smem;

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(B, 1)
   using IO = VecIO<T, VEC>;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
   extern __shared__ uint4 ring[];  // [S][B]
+  pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
   uint4 *slot0 = ring + threadIdx.x;
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(B, 1)
   // its first VEC * B floats serve the row-lane reduction.
   extern __shared__ uint4 ring[];
   __shared__ double red_a[B / 32];
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
   float *red = reinterpret_cast<float *>(ring);

@@ -294,6 +294,15 @@ __device__ __forceinline__ float param(const P *p, int64_t i) {
   return to_f32<P>(ld_scalar(p + i));
 }
 
+// First statement of every main kernel: wait until the preceding grid in the
+// stream has completed and its memory is visible (a no-op without a
+// programmatic predecessor), then let the next grid get scheduled. The kernels
+// touch no global memory before this, so programmatic launch keeps stream order.
+__device__ __forceinline__ void pdl_prologue() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Thread -> (row lane, vector-column) of the CTA.
 struct Lane {
   int rl;     // row lane
@@ -380,6 +389,7 @@ __global__ void __launch_bounds__(B, 1)
     dyt_fwd_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma,
                    const P *__restrict__ beta, T *y, Geom g) {
   using IO = VecIO<T, VEC>;
+  pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
@@ -544,7 +554,7 @@ __global__ void __launch_bounds__(B, 1)
   __shared__ double red_a[B / 32];
   // Let the finalize kernel, launched as a programmatic dependent, get
   // scheduled early; it still waits for this grid to finish before reading.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_prologue();
 
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);

@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(B, 1)
   using IO = VecIO<T, VEC>;
   extern __shared__ __align__(128) char smem[];
   __shared__ Producer prod;
+  pdl_prologue();
   const int stage_bytes = tg.SR * tg.pitch;
   volatile int *abort_flag = pipeline_setup<B>(smem, tg, stage_bytes);
   const Lane ln = lane_of(g, threadIdx.x);
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(B, 1)
   __shared__ float red[VEC * B];
   __shared__ double red_a[B / 32];
   __shared__ Producer prod;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_prologue();
   const int stage_bytes = 2 * tg.SR * tg.pitch;
   volatile int *abort_flag = pipeline_setup<B>(smem, tg, stage_bytes);
   const Lane ln = lane_of(g, threadIdx.x);

@@ -93,9 +93,9 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
         assert p["row_lanes"] == 1 and p["col_chunks"] == -(-nv // B)
     items = p["row_groups"] * p["col_chunks"]
     assert p["grid"] <= items
-    # every lane adds at most 96 rows per group (bounded binary32 error)
+    # every lane adds at most 128 rows per group (bounded binary32 error)
     rows_per_group = -(-M // p["row_groups"])
-    assert -(-rows_per_group // p["row_lanes"]) <= 96
+    assert -(-rows_per_group // p["row_lanes"]) <= 128
     # every CTA gets the same number of work items, unless there are more
     # column chunks than CTAs
     if p["col_chunks"] <= sms * occ:

@@ -288,15 +288,10 @@ def run_ours(args, w):
                      "da": torch.empty(1, dtype=gamma.dtype, device=dev)})
     ws = dyt.workspace(x0, gamma)
     grads = torch.empty(2 * N + 1, dtype=torch.float32, device=dev)
+    from elementwise_reduction_b200.dist import allreduce_param_grads
 
     def allreduce_grads(s):
-        grads[:N].copy_(s["dg"])
-        grads[N:2 * N].copy_(s["db"])
-        grads[2 * N:].copy_(s["da"])
-        dist.all_reduce(grads)
-        s["dg"].copy_(grads[:N])
-        s["db"].copy_(grads[N:2 * N])
-        s["da"].copy_(grads[2 * N:])
+        allreduce_param_grads(s["dg"], s["db"], s["da"], buf=grads)
 
     def fwd(s):
         dyt.forward(s["x"], alpha, gamma, beta, out=s["y"])

@@ -60,6 +60,7 @@ constexpr int kAsyncBlock = DYT_ASYNC_BLOCK;  // one CTA per SM: up to 128 regis
 constexpr int kAsyncStagesFwd = DYT_ASYNC_STAGES_FWD;
 constexpr int kAsyncStagesBwd = DYT_ASYNC_STAGES_BWD;
 constexpr int kMaxRowsPerLane = 128;  // sequential binary32 adds per thread per group
+
 constexpr int kFwdUnrollVec = DYT_FWD_UNROLL_VEC;        // rows in flight per thread, 16-byte access
 constexpr int kBwdUnrollVec = DYT_BWD_UNROLL_VEC;
 constexpr int kFwdUnrollScalar = DYT_FWD_UNROLL_SCALAR;  // rows in flight per thread, scalar access
@@ -178,6 +179,9 @@ Plan make_plan(int64_t M, int64_t N, int vec, bool backward, int sms, int ctas_p
   if (ceil_div(M, nrg) > max_rows) nrg = ceil_div(ceil_div(M, max_rows), fill) * fill;
   g.nrg = (int)nrg;
   g.nitems = (int)(nrg * g.ncc);
+  g.gq = M / nrg;
+  g.grem = M % nrg;
+  g.nv_magic = NV >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)NV - 1) / (uint64_t)NV) : 0u;
   int64_t grid = fill * g.ncc;
   if (grid > target) grid = target;
   if (grid > g.nitems) grid = g.nitems;

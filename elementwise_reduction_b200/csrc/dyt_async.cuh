@@ -47,24 +47,26 @@ __global__ void __launch_bounds__(B, 1)
   const float alpha = param(alpha_p, 0);
   uint4 *slot0 = ring + threadIdx.x;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
-    const int cc = item % g.ncc, rg = item / g.ncc;
+    int cc, rg;
+    item_split(g, item, cc, rg);
     int64_t rb, re;
-    group_rows(g.M, g.nrg, rg, rb, re);
+    group_rows(g, rg, rb, re);
     const int cv = cc * B + ln.cv;
     if (!(ln.live && cv < g.NV)) continue;
     const int64_t c0 = (int64_t)cv * VEC;
-    float gam[VEC], bet[VEC], bth[VEC];
-    fwd_params<T, P, VEC>(gamma, beta, c0, true, gam, bet, bth);
     int64_t first;
     const int64_t n = thread_rows(rb, re, ln.rl, g.RL, first);
     const int64_t stride = (int64_t)g.RL * g.N;
     const T *px = x + first * g.N + c0;
     T *py = y + first * g.N + c0;
+    // Rows first, parameters second: the parameter loads overlap the copies.
 #pragma unroll
     for (int k = 0; k < S - 1; ++k) {
       if (k < n) cp_async16(slot0 + k * B, px + k * stride);
       cp_async_commit();
     }
+    float gam[VEC], bet[VEC], bth[VEC];
+    fwd_params<T, P, VEC>(gamma, beta, c0, true, gam, bet, bth);
     int s_rd = 0, s_wr = S - 1;
     for (int64_t k = 0; k < n; ++k) {
       if (k + S - 1 < n) cp_async16(slot0 + s_wr * B, px + (k + S - 1) * stride);
@@ -100,9 +102,10 @@ __global__ void __launch_bounds__(B, 1)
   uint4 *slot0 = ring + threadIdx.x;
   double acc_a = 0.0;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
-    const int cc = item % g.ncc, rg = item / g.ncc;
+    int cc, rg;
+    item_split(g, item, cc, rg);
     int64_t rb, re;
-    group_rows(g.M, g.nrg, rg, rb, re);
+    group_rows(g, rg, rb, re);
     const int cv = cc * B + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
     const int64_t c0 = (int64_t)cv * VEC;
@@ -110,7 +113,6 @@ __global__ void __launch_bounds__(B, 1)
     BwdAcc<VEC> acc;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      gam[e] = col_ok ? 4.0f * param(gamma, c0 + e) : 0.0f;  // 4 gamma (see bwd_vector)
       acc.g[e] = 0.0f;
       acc.b[e] = 0.0f;
     }
@@ -121,6 +123,7 @@ __global__ void __launch_bounds__(B, 1)
       const T *px = x + first * g.N + c0;
       const T *pd = dy + first * g.N + c0;
       T *pdx = dx + first * g.N + c0;
+      // Rows first, parameters second: the gamma loads overlap the copies.
 #pragma unroll
       for (int k = 0; k < S - 1; ++k) {
         if (k < n) {
@@ -129,6 +132,8 @@ __global__ void __launch_bounds__(B, 1)
         }
         cp_async_commit();
       }
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) gam[e] = 4.0f * param(gamma, c0 + e);  // 4 gamma (see bwd_vector)
       int s_rd = 0, s_wr = S - 1;
       for (int64_t k = 0; k < n; ++k) {
         if (k + S - 1 < n) {

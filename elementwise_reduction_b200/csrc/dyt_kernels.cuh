@@ -31,20 +31,33 @@
 namespace dyt {
 
 struct Geom {
-  int64_t M;   // rows
-  int64_t N;   // columns
-  int NV;      // vector-columns per row (N / VEC)
-  int RL;      // row lanes per CTA step (1 on the row-per-CTA path)
-  int ncc;     // column chunks (of B vector-columns)
-  int nrg;     // row groups
-  int nitems;  // ncc * nrg
+  int64_t M;      // rows
+  int64_t N;      // columns
+  int NV;         // vector-columns per row (N / VEC)
+  int RL;         // row lanes per CTA step (1 on the row-per-CTA path)
+  int ncc;        // column chunks (of B vector-columns)
+  int nrg;        // row groups
+  int nitems;     // ncc * nrg
+  int64_t gq;     // M / nrg     (computed on the host: the kernels divide nothing)
+  int64_t grem;   // M % nrg
+  uint32_t nv_magic;  // ceil(2^32 / NV) for NV >= 2: tid / NV = umulhi(tid, nv_magic), tid < 1024
 };
 
 // Rows [begin, end) of group rg when [0, M) is cut into nrg balanced groups.
-__device__ __forceinline__ void group_rows(int64_t M, int nrg, int rg, int64_t &begin, int64_t &end) {
-  const int64_t q = M / nrg, rem = M % nrg;
-  begin = (int64_t)rg * q + (rg < rem ? rg : rem);
-  end = begin + q + (rg < rem ? 1 : 0);
+__device__ __forceinline__ void group_rows(const Geom &g, int rg, int64_t &begin, int64_t &end) {
+  begin = (int64_t)rg * g.gq + (rg < g.grem ? rg : g.grem);
+  end = begin + g.gq + (rg < g.grem ? 1 : 0);
+}
+
+// Work item -> (column chunk, row group); a single chunk needs no division.
+__device__ __forceinline__ void item_split(const Geom &g, int item, int &cc, int &rg) {
+  if (g.ncc == 1) {
+    cc = 0;
+    rg = item;
+  } else {
+    cc = item % g.ncc;
+    rg = item / g.ncc;
+  }
 }
 
 // ---- global memory access --------------------------------------------------
@@ -313,7 +326,7 @@ struct Lane {
 __device__ __forceinline__ Lane lane_of(const Geom &g, int tid) {
   Lane l;
   if (g.RL > 1) {
-    l.rl = tid / g.NV;
+    l.rl = g.NV == 1 ? tid : (int)__umulhi((unsigned)tid, g.nv_magic);
     l.cv = tid - l.rl * g.NV;
     l.live = l.rl < g.RL;
   } else {
@@ -393,9 +406,10 @@ __global__ void __launch_bounds__(B, 1)
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
-    const int cc = item % g.ncc, rg = item / g.ncc;
+    int cc, rg;
+    item_split(g, item, cc, rg);
     int64_t rb, re;
-    group_rows(g.M, g.nrg, rg, rb, re);
+    group_rows(g, rg, rb, re);
     const int cv = cc * B + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
     if (!col_ok) continue;
@@ -560,9 +574,10 @@ __global__ void __launch_bounds__(B, 1)
   const float alpha = param(alpha_p, 0);
   double acc_a = 0.0;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
-    const int cc = item % g.ncc, rg = item / g.ncc;
+    int cc, rg;
+    item_split(g, item, cc, rg);
     int64_t rb, re;
-    group_rows(g.M, g.nrg, rg, rb, re);
+    group_rows(g, rg, rb, re);
     const int cv = cc * B + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
     const int64_t c0 = (int64_t)cv * VEC;

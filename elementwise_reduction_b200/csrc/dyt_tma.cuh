@@ -91,7 +91,7 @@ __device__ __forceinline__ int item_rg(const Geom &g, int item) { return item / 
 __device__ __forceinline__ bool cursor_begin(TileCursor &c, const Geom &g, int item) {
   for (; item < g.nitems; item += gridDim.x) {
     int64_t rb, re;
-    group_rows(g.M, g.nrg, item_rg(g, item), rb, re);
+    group_rows(g, item_rg(g, item), rb, re);
     c.item = item;
     c.r = rb;
     c.re = re;

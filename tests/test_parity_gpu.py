@@ -244,6 +244,44 @@ def test_backward_is_bitwise_deterministic(M, N, xd):
     assert a["dalpha"] == b["dalpha"] or (np.isnan(a["dalpha"]) and np.isnan(b["dalpha"]))
 
 
+@pytest.mark.parametrize("M,N,xd", [(65537, 32, "bf16"), (1024, 64, "f32"), (20000, 17, "f32"),
+                                    (4096, 4096, "bf16")])
+def test_backward_in_cuda_graph_replays_and_with_garbage_workspace(M, N, xd):
+    # A fresh workspace holds arbitrary bytes, and a captured graph replays the
+    # same launches: both must give the eager bits.
+    import elementwise_reduction_b200 as dyt
+    inp = make(M, N, xd, "f32")
+    t = H.gpu_inputs(inp, xd, "f32")
+    x, dy = t["x"].view(M, N), t["dy"].view(M, N)
+    ref = [u.clone() for u in dyt.backward(x, dy, t["alpha"], t["gamma"])]
+    info = dyt.dyt_last_launch_info()
+    ws = dyt.workspace(x, t["gamma"])
+    ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda"))
+    outs = [torch.empty_like(u) for u in ref]
+    dyt.backward(x, dy, t["alpha"], t["gamma"], dx=outs[0], dalpha=outs[1], dgamma=outs[2], dbeta=outs[3],
+                 ws=ws)
+    torch.cuda.synchronize()
+    for a, b in zip(outs, ref):
+        assert torch.equal(a, b)
+    stream = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        dyt.backward(x, dy, t["alpha"], t["gamma"], dx=outs[0], dalpha=outs[1], dgamma=outs[2], dbeta=outs[3],
+                     ws=ws)  # warm-up on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            dyt.backward(x, dy, t["alpha"], t["gamma"], dx=outs[0], dalpha=outs[1], dgamma=outs[2],
+                         dbeta=outs[3], ws=ws)
+    for _ in range(4):
+        for u in outs:
+            u.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for a, b in zip(outs, ref):
+            assert torch.equal(a, b)
+    assert info["kernels"] == 2
+
+
 def test_workspace_errors():
     import elementwise_reduction_b200 as dyt
     M, N = 100, 64

@@ -30,7 +30,7 @@ class LaunchInfo(ctypes.Structure):
     _fields_ = [("op", _i32), ("path", _i32), ("vec", _i32), ("block", _i32), ("grid", _i32),
                 ("row_lanes", _i32), ("rows_per_step", _i32), ("col_chunks", _i32),
                 ("row_groups", _i32), ("kernels", _i32), ("tma_stages", _i32), ("async_stages", _i32),
-                ("workspace_bytes", _i64)]
+                ("pack_rows", _i32), ("workspace_bytes", _i64)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}

@@ -50,6 +50,11 @@ thread_local int t_cuda_err = 0;
 #ifndef DYT_MAX_STAGES
 #define DYT_MAX_STAGES 8
 #endif
+// Inputs read by one launch below which the L2 prefetch of the first rows is
+// skipped (bytes).
+#ifndef DYT_PREFETCH_MIN_BYTES
+#define DYT_PREFETCH_MIN_BYTES (1 << 20)
+#endif
 constexpr int kBlock = 1024;          // threads per CTA of the main kernels
 constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits (iterations)
 constexpr int kMaxDynSmem = 227 * 1024;
@@ -60,6 +65,7 @@ constexpr int kAsyncBlock = DYT_ASYNC_BLOCK;  // one CTA per SM: up to 128 regis
 constexpr int kAsyncStagesFwd = DYT_ASYNC_STAGES_FWD;
 constexpr int kAsyncStagesBwd = DYT_ASYNC_STAGES_BWD;
 constexpr int kMaxRowsPerLane = 128;  // sequential binary32 adds per thread per group
+constexpr int64_t kPrefetchMinBytes = DYT_PREFETCH_MIN_BYTES;
 
 constexpr int kFwdUnrollVec = DYT_FWD_UNROLL_VEC;        // rows in flight per thread, 16-byte access
 constexpr int kBwdUnrollVec = DYT_BWD_UNROLL_VEC;
@@ -136,6 +142,7 @@ struct Plan {
   int path;
   bool tma;
   bool async;
+  bool packed;  // ragged N on 16-byte aligned rows: packs of vec rows (see dyt_kernels.cuh)
   dyt::TmaGeom tg;
   size_t smem;  // dynamic shared memory of the pipelined kernel
   size_t ws_dg, ws_db, ws_da, ws_total;  // workspace byte offsets / sizes
@@ -144,17 +151,25 @@ struct Plan {
 size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
 // vec: elements per access (1 or 16 / element size). ctas_per_sm from the
-// kernel's occupancy. The plan depends only on (M, N, vec, SM count, occupancy).
-Plan make_plan(int64_t M, int64_t N, int vec, bool backward, int sms, int ctas_per_sm, int block = kBlock) {
+// kernel's occupancy. packed: N is not a multiple of vec, and the matrix is
+// laid out as ceil(M / vec) packs of vec rows, each of pitch vec * N. The
+// plan depends only on (M, N, vec, packed, SM count, occupancy).
+Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, int sms, int ctas_per_sm,
+               int block = kBlock, bool packed = false, int64_t elem_bytes = 4) {
   Plan p = {};
   p.block = block;
   p.vec = vec;
+  p.packed = packed;
+  const int64_t M = packed ? ceil_div(M_rows, (int64_t)vec) : M_rows;
+  const int64_t N = packed ? (int64_t)vec * N_cols : N_cols;
   p.unroll = backward ? (vec > 1 ? kBwdUnrollVec : kBwdUnrollScalar)
                       : (vec > 1 ? kFwdUnrollVec : kFwdUnrollScalar);
   const int64_t NV = N / vec;
   Geom &g = p.g;
   g.M = M;
   g.N = N;
+  g.Nc = N_cols;
+  g.total = M_rows * N_cols;
   g.NV = (int)NV;
   if (NV <= block / 2) {
     g.RL = block / (int)NV;
@@ -182,6 +197,11 @@ Plan make_plan(int64_t M, int64_t N, int vec, bool backward, int sms, int ctas_p
   g.gq = M / nrg;
   g.grem = M % nrg;
   g.nv_magic = NV >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)NV - 1) / (uint64_t)NV) : 0u;
+  // L2 prefetch of the first rows (pipelined kernels): worth its issue cost
+  // only when the launch reads enough that its inputs are unlikely to be
+  // resident in L2 already and each CTA's first rows take a DRAM round trip
+  // or more; below kPrefetchMinBytes it is skipped.
+  g.l2_prefetch = (int64_t)(backward ? 2 : 1) * M_rows * N_cols * elem_bytes >= kPrefetchMinBytes;
   int64_t grid = fill * g.ncc;
   if (grid > target) grid = target;
   if (grid > g.nitems) grid = g.nitems;
@@ -278,7 +298,8 @@ dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
     i.block = p->block;
     i.grid = p->grid;
     i.row_lanes = p->g.RL;
-    i.rows_per_step = p->g.RL * p->unroll;
+    i.pack_rows = p->packed ? p->vec : 1;
+    i.rows_per_step = p->g.RL * p->unroll * i.pack_rows;
     i.col_chunks = p->g.ncc;
     i.row_groups = p->g.nrg;
     i.tma_stages = p->tma ? p->tg.stages : 0;
@@ -299,10 +320,10 @@ const void *tma_kernel(bool backward) {
                   : (const void *)dyt::dyt_fwd_tma_kernel<T, P, kTmaVec, kBlock>;
 }
 
-template <typename T, typename P>
+template <typename T, typename P, bool PK>
 const void *async_kernel(bool backward) {
-  return backward ? (const void *)dyt::dyt_bwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesBwd>
-                  : (const void *)dyt::dyt_fwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesFwd>;
+  return backward ? (const void *)dyt::dyt_bwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesBwd, PK>
+                  : (const void *)dyt::dyt_fwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesFwd, PK>;
 }
 
 // Static shared memory of a kernel and, once, the opt-in to the largest
@@ -337,11 +358,14 @@ dyt_status plan_for(int64_t M, int64_t N, bool vec_ok, bool backward, Plan *out)
   int dev = 0, sms = 0;
   dyt_status st = current_sms(&dev, &sms);
   if (st != DYT_OK) return st;
-  const int vec = (vec_ok && N % vec_of<T>() == 0) ? vec_of<T>() : 1;
+  // Ragged rows of an aligned matrix go through the asynchronous-copy
+  // kernels as packs; unaligned matrices take the scalar kernels.
+  const bool packed = DYT_PIPE == 2 && vec_ok && N % vec_of<T>() != 0;
+  const int vec = (vec_ok && (packed || N % vec_of<T>() == 0)) ? vec_of<T>() : 1;
   const bool use_tma = DYT_USE_TMA && vec > 1;
   const bool use_async = DYT_PIPE == 2 && vec > 1;
   const void *k = use_tma     ? tma_kernel<T, P>(backward)
-                  : use_async ? async_kernel<T, P>(backward)
+                  : use_async ? (packed ? async_kernel<T, P, true>(backward) : async_kernel<T, P, false>(backward))
                   : backward  ? bwd_kernel<T, P>(vec)
                               : fwd_kernel<T, P>(vec);
   int occ = 1;
@@ -353,7 +377,8 @@ dyt_status plan_for(int64_t M, int64_t N, bool vec_ok, bool backward, Plan *out)
     st = occupancy(dev, k, kBlock, &occ);
     if (st != DYT_OK) return st;
   }
-  *out = make_plan(M, N, use_tma ? kTmaVec : vec, backward, sms, occ, use_async ? kAsyncBlock : kBlock);
+  *out = make_plan(M, N, use_tma ? kTmaVec : vec, backward, sms, occ, use_async ? kAsyncBlock : kBlock, packed,
+                   (int64_t)sizeof(T));
   out->tma = false;
   out->async = use_async;
   if (use_tma) plan_tma(*out, sizeof(T), backward, static_smem);
@@ -404,8 +429,12 @@ dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, cons
                              (const P *)gamma, (const P *)beta, (T *)y, p.g, p.tg);
     } else if (p.async) {
       cfg.dynamicSmemBytes = p.smem;
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd>, (const T *)x,
-                             (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
+      if (p.packed)
+        e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, true>,
+                               (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
+      else
+        e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, false>,
+                               (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
     } else if (p.vec > 1)
       e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, V, kFwdUnrollVec, kBlock>,
                              (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y,
@@ -490,8 +519,14 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
                              (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda, p.g, p.tg);
     } else if (p.async) {
       cfg.dynamicSmemBytes = p.smem;
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd>, (const T *)x,
-                             (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda, p.g);
+      if (p.packed)
+        e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, true>,
+                               (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb,
+                               pda, p.g);
+      else
+        e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, false>,
+                               (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb,
+                               pda, p.g);
     } else if (p.vec > 1)
       e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, V, kBwdUnrollVec, kBlock>,
                              (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx,
@@ -504,9 +539,12 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
 
     // Stage 2, as a programmatic dependent launch: it may start while stage 1
     // drains and waits (griddepcontrol.wait) for stage 1's results.
+    // The partials form (nrg x pack rows) rows of N columns: a packed row group
+    // holds vec partial rows, one per row of the pack, in pack order.
+    const int nparts = p.g.nrg * (p.packed ? p.vec : 1);
     // Lanes per column: enough that each lane reads at most four partials.
     int L = 1;
-    while (L < dyt::kFinThreads && (int64_t)L * 4 < p.g.nrg) L <<= 1;
+    while (L < dyt::kFinThreads && (int64_t)L * 4 < nparts) L <<= 1;
     const int CT = dyt::kFinThreads / L;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -519,7 +557,7 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
     fcfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&fcfg, dyt::dyt_finalize_kernel<P>, (const float *)pdg, (const float *)pdb,
                            (const double *)pda, (P *)dgamma, (P *)dbeta, (P *)dalpha, (int64_t)N,
-                           p.g.nrg, p.grid, CT);
+                           nparts, p.grid, CT);
     if (e != cudaSuccess) return cuda_fail(e);
     record(2, &p, 2, p.ws_total);
     return DYT_OK;
@@ -570,11 +608,12 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
     return DYT_OK;
   }
   const int v = 16 / (int)dsize(x_dtype);
-  const int vec = (vectorized && N % v == 0) ? v : 1;
+  const bool packed = DYT_PIPE == 2 && vectorized && N % v != 0;
+  const int vec = (vectorized && (packed || N % v == 0)) ? v : 1;
   const bool use_tma = DYT_USE_TMA && vec > 1;
   const bool use_async = DYT_PIPE == 2 && vec > 1;
   Plan p = make_plan(M, N, use_tma ? kTmaVec : vec, backward != 0, sm_count, ctas_per_sm,
-                     use_async ? kAsyncBlock : kBlock);
+                     use_async ? kAsyncBlock : kBlock, packed, (int64_t)dsize(x_dtype));
   p.tma = false;
   p.async = use_async;
   if (p.async) p.unroll = 1;

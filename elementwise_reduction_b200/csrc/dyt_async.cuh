@@ -21,10 +21,86 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
   const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
 }
+// The same copy reading only the first src_bytes (0..16) of the source and
+// zero-filling the rest of the slot: nothing past src + src_bytes is read.
+__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, uint32_t src_bytes) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem_src), "r"(src_bytes) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Matrix columns of the VEC elements of the vector at offset c0 of a row:
+// c0 + e, or on the packed path (c0 + e) mod Nc, where c0 < VEC * Nc.
+template <int VEC, bool PK>
+__device__ __forceinline__ void vector_columns(int64_t c0, int64_t Nc, int64_t (&col)[VEC]) {
+  if constexpr (PK) {
+    int64_t c = c0;
+    while (c >= Nc) c -= Nc;  // at most VEC - 1 times
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      col[e] = c;
+      c = c + 1 == Nc ? 0 : c + 1;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) col[e] = c0 + e;
+  }
+}
+
+// The first n (< VEC) elements of a 16-byte vector, one by one: the vector
+// that straddles the end of a packed matrix.
+template <typename T, int VEC>
+__device__ __forceinline__ void store_first(T *p, const uint4 &r, int n) {
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    if (e < n) {
+      if constexpr (sizeof(T) == 4) {
+        *reinterpret_cast<uint32_t *>(p + e) = word_of(r, e);
+      } else {
+        const uint32_t u = word_of(r, e >> 1);
+        *reinterpret_cast<unsigned short *>(p + e) = (unsigned short)((e & 1) ? (u >> 16) : (u & 0xFFFFu));
+      }
+    }
+  }
+}
+
+// Start pulling into L2 the rows this CTA copies first: those of its first
+// work item, at most as many as the rings hold (S - 1 steps). This runs before
+// griddepcontrol.wait, while the preceding grid may still be writing. That is
+// safe: a prefetch changes no memory state, and the ring copies after the wait
+// read L2 (cp.async.cg), so a line written later is read in its final state.
+// Rows are 16-byte aligned on this path, so every range below is too.
+template <typename T, int VEC, int B, int S>
+__device__ __forceinline__ void prefetch_first_rows_l2(const T *p, const Geom &g) {
+  if (!g.l2_prefetch || (int)blockIdx.x >= g.nitems) return;
+  int cc, rg;
+  item_split(g, blockIdx.x, cc, rg);
+  int64_t rb, re;
+  group_rows(g, rg, rb, re);
+  const int64_t rows = min(re - rb, (int64_t)(S - 1) * g.RL);
+  if (rows <= 0) return;
+  constexpr uint32_t kPiece = 16384;
+  // Ranges end at the matrix's last element (a packed matrix's last row may
+  // be short) and are rounded down to whole 16-byte units.
+  if (g.ncc == 1) {  // whole rows: one contiguous range, cut into pieces
+    const int64_t bytes = (min(rows * g.N, g.total - rb * g.N) * (int64_t)sizeof(T)) & ~(int64_t)15;
+    const int64_t k = threadIdx.x;
+    if (k * kPiece < bytes) {
+      const uint32_t n = (uint32_t)min((int64_t)kPiece, bytes - k * kPiece);
+      const char *a = reinterpret_cast<const char *>(p + rb * g.N) + k * kPiece;
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
+    }
+  } else if (threadIdx.x < rows) {  // one column chunk of each row
+    const int64_t c0 = (int64_t)cc * B * VEC;
+    const int64_t at = (rb + threadIdx.x) * g.N + c0;
+    const int64_t n = (min(min((int64_t)B * VEC, g.N - c0), g.total - at) * (int64_t)sizeof(T)) & ~(int64_t)15;
+    if (n > 0)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + at), "r"((uint32_t)n) : "memory");
+  }
 }
 
 // Rows of the current item owned by this thread: first row and count.
@@ -35,13 +111,34 @@ __device__ __forceinline__ int64_t thread_rows(int64_t rb, int64_t re, int rl, i
 
 // ---- forward ------------------------------------------------------------------
 
-template <typename T, typename P, int VEC, int B, int S>
+// Real elements of the vector at offset c0 of (packed) row `row`: VEC, except
+// in the vector that straddles the end of a packed matrix; 0 past it.
+__device__ __forceinline__ int64_t vector_real(const Geom &g, int64_t row, int64_t c0) {
+  return g.total - (row * g.N + c0);
+}
+
+// Trims a thread's row count on the packed path: drops a last vector that
+// lies wholly past the matrix and returns the real elements of the last one
+// (VEC when it is whole).
+template <int VEC, bool PK>
+__device__ __forceinline__ int last_vector_real(const Geom &g, int64_t first, int64_t c0, int64_t &n) {
+  if (!PK || n <= 0) return VEC;
+  const int64_t r = vector_real(g, first + (n - 1) * g.RL, c0);
+  if (r <= 0) {
+    --n;  // only the matrix's last pack is short, so the one before is whole
+    return VEC;
+  }
+  return r < VEC ? (int)r : VEC;
+}
+
+template <typename T, typename P, int VEC, int B, int S, bool PK>
 __global__ void __launch_bounds__(B, 1)
     dyt_fwd_async_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma,
                          const P *__restrict__ beta, T *y, Geom g) {
   using IO = VecIO<T, VEC>;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
   extern __shared__ uint4 ring[];  // [S][B]
+  prefetch_first_rows_l2<T, VEC, B, S>(x, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
@@ -55,25 +152,38 @@ __global__ void __launch_bounds__(B, 1)
     if (!(ln.live && cv < g.NV)) continue;
     const int64_t c0 = (int64_t)cv * VEC;
     int64_t first;
-    const int64_t n = thread_rows(rb, re, ln.rl, g.RL, first);
+    int64_t n = thread_rows(rb, re, ln.rl, g.RL, first);
+    const int nl = last_vector_real<VEC, PK>(g, first, c0, n);
+    const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
     const int64_t stride = (int64_t)g.RL * g.N;
     const T *px = x + first * g.N + c0;
     T *py = y + first * g.N + c0;
     // Rows first, parameters second: the parameter loads overlap the copies.
 #pragma unroll
     for (int k = 0; k < S - 1; ++k) {
-      if (k < n) cp_async16(slot0 + k * B, px + k * stride);
+      if (k < n) {
+        if (PK) cp_async16_zfill(slot0 + k * B, px + k * stride, k == n - 1 ? last_bytes : 16u);
+        else cp_async16(slot0 + k * B, px + k * stride);
+      }
       cp_async_commit();
     }
+    int64_t col[VEC];
+    vector_columns<VEC, PK>(c0, g.Nc, col);
     float gam[VEC], bet[VEC], bth[VEC];
-    fwd_params<T, P, VEC>(gamma, beta, c0, true, gam, bet, bth);
+    fwd_params_at<T, P, VEC>(gamma, beta, col, gam, bet, bth);
     int s_rd = 0, s_wr = S - 1;
     for (int64_t k = 0; k < n; ++k) {
-      if (k + S - 1 < n) cp_async16(slot0 + s_wr * B, px + (k + S - 1) * stride);
+      const int64_t kn = k + S - 1;
+      if (kn < n) {
+        if (PK) cp_async16_zfill(slot0 + s_wr * B, px + kn * stride, kn == n - 1 ? last_bytes : 16u);
+        else cp_async16(slot0 + s_wr * B, px + kn * stride);
+      }
       cp_async_commit();
       cp_async_wait<S - 1>();
       const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + s_rd * B);
-      IO::store_raw(py, fwd_vector<T, VEC>(rx, alpha, gam, bet, bth));
+      const typename IO::Raw ry = fwd_vector<T, VEC>(rx, alpha, gam, bet, bth);
+      if (PK && k == n - 1 && nl < VEC) store_first<T, VEC>(py, ry, nl);  // zero-filled tail: not stored
+      else IO::store_raw(py, ry);
       py += stride;
       s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
       s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
@@ -84,17 +194,20 @@ __global__ void __launch_bounds__(B, 1)
 
 // ---- backward, stage 1 ----------------------------------------------------------
 
-template <typename T, typename P, int VEC, int B, int S>
+template <typename T, typename P, int VEC, int B, int S, bool PK>
 __global__ void __launch_bounds__(B, 1)
     dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
                          const P *__restrict__ gamma, T *dx, float *__restrict__ part_dg,
                          float *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
   using IO = VecIO<T, VEC>;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
+  static_assert(2 * VEC * sizeof(float) <= 2 * S * 16, "the reduction fits in the drained ring");
   // [S][2][B] 16-byte slots; after an item's last row the ring is empty and
-  // its first VEC * B floats serve the row-lane reduction.
+  // its first 2 VEC * B floats (at most 32 KB) serve the row-lane reduction.
   extern __shared__ uint4 ring[];
   __shared__ double red_a[B / 32];
+  prefetch_first_rows_l2<T, VEC, B, S>(x, g);
+  prefetch_first_rows_l2<T, VEC, B, S>(dy, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
@@ -118,7 +231,9 @@ __global__ void __launch_bounds__(B, 1)
     }
     if (col_ok) {
       int64_t first;
-      const int64_t n = thread_rows(rb, re, ln.rl, g.RL, first);
+      int64_t n = thread_rows(rb, re, ln.rl, g.RL, first);
+      const int nl = last_vector_real<VEC, PK>(g, first, c0, n);
+      const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
       const int64_t stride = (int64_t)g.RL * g.N;
       const T *px = x + first * g.N + c0;
       const T *pd = dy + first * g.N + c0;
@@ -127,25 +242,44 @@ __global__ void __launch_bounds__(B, 1)
 #pragma unroll
       for (int k = 0; k < S - 1; ++k) {
         if (k < n) {
-          cp_async16(slot0 + (2 * k) * B, px + k * stride);
-          cp_async16(slot0 + (2 * k + 1) * B, pd + k * stride);
+          if (PK) {
+            const uint32_t b = k == n - 1 ? last_bytes : 16u;
+            cp_async16_zfill(slot0 + (2 * k) * B, px + k * stride, b);
+            cp_async16_zfill(slot0 + (2 * k + 1) * B, pd + k * stride, b);
+          } else {
+            cp_async16(slot0 + (2 * k) * B, px + k * stride);
+            cp_async16(slot0 + (2 * k + 1) * B, pd + k * stride);
+          }
         }
         cp_async_commit();
       }
+      int64_t col[VEC];
+      vector_columns<VEC, PK>(c0, g.Nc, col);
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) gam[e] = 4.0f * param(gamma, c0 + e);  // 4 gamma (see bwd_vector)
+      for (int e = 0; e < VEC; ++e) gam[e] = 4.0f * param(gamma, col[e]);  // 4 gamma (see bwd_vector)
       int s_rd = 0, s_wr = S - 1;
       for (int64_t k = 0; k < n; ++k) {
-        if (k + S - 1 < n) {
-          cp_async16(slot0 + (2 * s_wr) * B, px + (k + S - 1) * stride);
-          cp_async16(slot0 + (2 * s_wr + 1) * B, pd + (k + S - 1) * stride);
+        const int64_t kn = k + S - 1;
+        if (kn < n) {
+          if (PK) {
+            const uint32_t b = kn == n - 1 ? last_bytes : 16u;
+            cp_async16_zfill(slot0 + (2 * s_wr) * B, px + kn * stride, b);
+            cp_async16_zfill(slot0 + (2 * s_wr + 1) * B, pd + kn * stride, b);
+          } else {
+            cp_async16(slot0 + (2 * s_wr) * B, px + kn * stride);
+            cp_async16(slot0 + (2 * s_wr + 1) * B, pd + kn * stride);
+          }
         }
         cp_async_commit();
         cp_async_wait<S - 1>();
         const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + (2 * s_rd) * B);
         const typename IO::Raw rd = *(const typename IO::Raw *)(slot0 + (2 * s_rd + 1) * B);
         float2 ca = make_float2(0.0f, 0.0f);
-        IO::store_raw(pdx, bwd_vector<T, VEC, false>(rx, rd, alpha, gam, acc, ca, true));
+        if (PK && k == n - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
+          store_first<T, VEC>(pdx, bwd_vector<T, VEC, true>(rx, rd, alpha, gam, acc, ca, nl), nl);
+        } else {
+          IO::store_raw(pdx, bwd_vector<T, VEC, false>(rx, rd, alpha, gam, acc, ca, VEC));
+        }
         acc_a += (double)ca.x;
         acc_a += (double)ca.y;
         pdx += stride;
@@ -170,23 +304,20 @@ __global__ void __launch_bounds__(B, 1)
       if ((32 % g.NV) == 0) {
         // the chunk's columns start at 0 on the row-tiled path (one chunk)
         lane_reduce_warps<VEC, B>(acc.g, acc.b, red, g, ln, 0, pg, pb);
-      } else {
+      } else {  // dgamma and dbeta sums in one tree: 2 VEC floats per thread
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.g[e];
-        __syncthreads();
-        lane_tree<VEC, B>(red, g, ln);
-        if (col_ok && ln.rl == 0) {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) pg[c0 + e] = red[e * B + threadIdx.x];
+        for (int e = 0; e < VEC; ++e) {
+          red[e * B + threadIdx.x] = acc.g[e];
+          red[(VEC + e) * B + threadIdx.x] = acc.b[e];
         }
         __syncthreads();
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.b[e];
-        __syncthreads();
-        lane_tree<VEC, B>(red, g, ln);
+        lane_tree<2 * VEC, B>(red, g, ln);
         if (col_ok && ln.rl == 0) {
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) pb[c0 + e] = red[e * B + threadIdx.x];
+          for (int e = 0; e < VEC; ++e) {
+            pg[c0 + e] = red[e * B + threadIdx.x];
+            pb[c0 + e] = red[(VEC + e) * B + threadIdx.x];
+          }
         }
         __syncthreads();
       }

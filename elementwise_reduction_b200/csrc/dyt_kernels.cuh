@@ -3,8 +3,15 @@
 // Work decomposition (one 1D persistent grid, the page's Summary "Launch
 // limit": rows never sit on grid dimension 1, so M is unbounded):
 //   - a thread owns one vector-column cv (VEC consecutive columns; VEC = 16
-//     bytes / element size, or 1 for unaligned or ragged rows) and keeps its
+//     bytes / element size, or 1 for unaligned rows) and keeps its
 //     gamma/beta in registers;
+//   - packed rows (16-byte aligned matrix, N not a multiple of VEC): VEC
+//     consecutive rows always span exactly N 16-byte vectors, so such a pack
+//     is treated as one row of pitch VEC * N with NV = N vector-columns; the
+//     element e of vector-column cv then lies in matrix column
+//     (cv * VEC + e) mod N, fixed for the thread. The last pack may hold
+//     fewer than VEC rows: its vectors past the matrix are not read, and the
+//     one vector that straddles the end is zero-filled and masked;
 //   - row-tiled path (NV = N / VEC <= B / 2, the page's narrow rows): RL =
 //     B / NV row lanes share a CTA step, so one step covers RL * U whole rows
 //     (the page's Summary "Small widths": several rows per tile);
@@ -15,7 +22,7 @@
 //     (column chunk, row group) and CTA b takes items b, b + grid, ... (a
 //     static schedule: the same inputs always give the same bits).
 // Backward sums: each thread accumulates its columns in binary32 over at most
-// 96 rows per group (the host sizes the groups so), the
+// 128 rows per group (the host sizes the groups so), the
 // row lanes of a CTA are added by a fixed-order tree in shared memory, and
 // each (group, column) partial goes to the workspace; dalpha is carried in
 // binary64 per thread, reduced per CTA in a fixed order. The finalize kernel
@@ -31,8 +38,10 @@
 namespace dyt {
 
 struct Geom {
-  int64_t M;      // rows
-  int64_t N;      // columns
+  int64_t M;      // rows (packs of VEC rows on the packed path)
+  int64_t N;      // columns: the row pitch in elements (VEC x Nc on the packed path)
+  int64_t Nc;     // columns of the matrix (= N unless packed)
+  int64_t total;  // elements of the matrix (its rows x Nc): later ones are padding
   int NV;         // vector-columns per row (N / VEC)
   int RL;         // row lanes per CTA step (1 on the row-per-CTA path)
   int ncc;        // column chunks (of B vector-columns)
@@ -41,6 +50,7 @@ struct Geom {
   int64_t gq;     // M / nrg     (computed on the host: the kernels divide nothing)
   int64_t grem;   // M % nrg
   uint32_t nv_magic;  // ceil(2^32 / NV) for NV >= 2: tid / NV = umulhi(tid, nv_magic), tid < 1024
+  int l2_prefetch;    // the pipelined kernels prefetch their first rows into L2 (large inputs only)
 };
 
 // Rows [begin, end) of group rg when [0, M) is cut into nrg balanced groups.
@@ -361,6 +371,21 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw fwd_vector(const typename
         cancel_any |= (fabsf(y2[h].x) < bth[2 * h]) | (fabsf(y2[h].y) < bth[2 * h + 1]);
     }
     out = IO::pack2(y2);
+    if (CancelGuard<T>::kOn && cancel_any) {
+      // Rare: find the cancelling elements again from the rounded outputs.
+      // Rounding moves |y| by at most max(2^-8 |y|, kTiny / 2) (relative
+      // above the subnormal range, half a subnormal step within it), so
+      // |y| < bth implies |round(y)| < bth (1 + 2^-7) + kTiny: the test below
+      // flags every element the binary32 test flagged (and at most a few
+      // more, whose binary64 value is as good). Those get the binary64 value.
+      float yr[VEC], xf[VEC];
+      IO::unpack(out, yr);
+      IO::unpack(rx, xf);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e)
+        if (fabsf(yr[e]) < fmaf(bth[e], 1.0f + 0x1p-7f, CancelGuard<T>::kTiny))
+          IO::set(out, e, dyt_y_refined<T>(alpha, xf[e], gam[e], bet[e]));
+    }
   } else {
     float xf[VEC], yf[VEC];
     IO::unpack(rx, xf);
@@ -370,16 +395,10 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw fwd_vector(const typename
       if (CancelGuard<T>::kOn) cancel_any |= fabsf(yf[e]) < bth[e];
     }
     out = IO::pack(yf);
-  }
-  if (CancelGuard<T>::kOn && cancel_any) {
-    // Rare: redo the test per element (the scalar formulas round exactly as the
-    // pair ones) and replace the cancelling elements with the binary64 value.
-    float xf[VEC];
-    IO::unpack(rx, xf);
+    if (CancelGuard<T>::kOn && cancel_any) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const float y = fmaf(gam[e], dyt_tanh(alpha * xf[e]), bet[e]);
-      if (fabsf(y) < bth[e]) IO::set(out, e, dyt_y_refined<T>(alpha, xf[e], gam[e], bet[e]));
+      for (int e = 0; e < VEC; ++e)
+        if (fabsf(yf[e]) < bth[e]) IO::set(out, e, dyt_y_refined<T>(alpha, xf[e], gam[e], bet[e]));
     }
   }
   return out;
@@ -393,6 +412,18 @@ __device__ __forceinline__ void fwd_params(const P *gamma, const P *beta, int64_
   for (int e = 0; e < VEC; ++e) {
     gam[e] = ok ? param(gamma, c0 + e) : 0.0f;
     bet[e] = ok ? param(beta, c0 + e) : 0.0f;
+    bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
+  }
+}
+
+// The same for the VEC columns col[e] (not necessarily consecutive).
+template <typename T, typename P, int VEC>
+__device__ __forceinline__ void fwd_params_at(const P *gamma, const P *beta, const int64_t (&col)[VEC],
+                                              float (&gam)[VEC], float (&bet)[VEC], float (&bth)[VEC]) {
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    gam[e] = param(gamma, col[e]);
+    bet[e] = param(beta, col[e]);
     bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
   }
 }
@@ -454,36 +485,62 @@ __device__ __forceinline__ void lane_tree(float *red, const Geom &g, const Lane 
 }
 
 // CTA sums of the row lanes when NV divides 32: every warp then holds 32 / NV
-// whole row lanes of the same NV vector-columns, so a butterfly over lane
-// offsets NV, 2 NV, ... 16 adds them in registers (both partners of an
-// exchange compute the same sum, so every lane ends with identical bits), and
-// one pass over the warps in order adds the warp sums. red[] holds
-// (B / 32) x NV x VEC floats. Results go to out_g / out_b (row of the group's
-// partials) at the thread's columns.
+// whole row lanes of the same NV vector-columns, so their sums are formed in
+// registers by a reduce-scatter over lane offsets NV, 2 NV, ... 16. The 2 VEC
+// values of a thread (VEC dgamma sums, then VEC dbeta sums) are halved at each
+// level: the partner with the offset bit clear keeps the lower half, the
+// other the upper half, and each adds the half the partner sent, so one
+// exchange moves half of what a full butterfly would. When one value is left
+// before the offsets run out, the remaining levels are a butterfly (both
+// partners form the same sum). The order of every sum is fixed. Each warp
+// then holds each of its 2 NV VEC sums once; one pass over the warps in order
+// adds them. red[] holds (B / 32) x 2 NV VEC floats. Results go to out_g /
+// out_b (row of the group's partials) at the thread's columns.
 template <int VEC, int B>
 __device__ __forceinline__ void lane_reduce_warps(const float (&vg)[VEC], const float (&vb)[VEC], float *red,
                                                   const Geom &g, const Lane &ln, int64_t c0_chunk,
                                                   float *out_g, float *out_b) {
-  float ag[VEC], ab[VEC];
+  constexpr int V2 = 2 * VEC;
+  float v[V2];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
-    ag[e] = vg[e];
-    ab[e] = vb[e];
+    v[e] = vg[e];
+    v[VEC + e] = vb[e];
   }
-  for (int off = g.NV; off < 32; off <<= 1) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int start = 0;     // index (in 0 .. 2 VEC - 1) of this thread's first kept value
+  int m = V2;        // values kept
+  bool dup = false;  // a butterfly level ran: lanes with its bit set hold copies
+  int off = g.NV;
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      ag[e] += __shfl_xor_sync(0xFFFFFFFFu, ag[e], off);
-      ab[e] += __shfl_xor_sync(0xFFFFFFFFu, ab[e], off);
+  for (int i = 0; i < 5; ++i) {
+    const int h = V2 >> (i + 1);  // a constant once unrolled
+    if (off < 32) {
+      const bool up = (lane & off) != 0;
+      if (h >= 1) {
+#pragma unroll
+        for (int j = 0; j < h; ++j) {
+          const float send = up ? v[j] : v[j + h];
+          const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, off);
+          v[j] = (up ? v[j + h] : v[j]) + recv;
+        }
+        start += up ? h : 0;
+        m = h;
+      } else {
+        v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], off);
+        dup = dup || up;
+      }
+      off <<= 1;
     }
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int width = g.NV * VEC;  // floats per warp and sum
-  if (lane < g.NV) {
+  if (!dup) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      red[(2 * warp) * width + lane * VEC + e] = ag[e];
-      red[(2 * warp + 1) * width + lane * VEC + e] = ab[e];
+    for (int j = 0; j < V2; ++j) {
+      if (j < m) {
+        const int idx = start + j, which = idx >= VEC, e = idx - which * VEC;
+        red[(2 * warp + which) * width + ln.cv * VEC + e] = v[j];
+      }
     }
   }
   __syncthreads();
@@ -505,13 +562,14 @@ struct BwdAcc {
 
 // One vector (one row, VEC columns): dx out, sums in. g4[e] = 4 gamma[e]
 // (with q = (1 - t^2) / 4, g4 * dy * q rounds exactly as gamma * dy * (1 - t^2)).
-// MASKED: the row may be padding; its results are computed like any other and
-// dropped afterwards.
+// MASKED: only the first nvalid elements are real (0 for a padded row, fewer
+// than VEC for the vector that straddles the end of a packed matrix); the
+// others are computed like any other and their results dropped afterwards.
 template <typename T, int VEC, bool MASKED>
 __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename VecIO<T, VEC>::Raw &rx,
                                                                  const typename VecIO<T, VEC>::Raw &rdy,
                                                                  float alpha, const float (&g4)[VEC],
-                                                                 BwdAcc<VEC> &acc, float2 &ca, bool ok) {
+                                                                 BwdAcc<VEC> &acc, float2 &ca, int nvalid) {
   using IO = VecIO<T, VEC>;
   if constexpr (IO::kPairs > 0) {
     constexpr int H = IO::kPairs;
@@ -527,10 +585,11 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       const float2 ag = make_float2(acc.g[2 * h], acc.g[2 * h + 1]);
       const float2 ab = make_float2(acc.b[2 * h], acc.b[2 * h + 1]);
       float2 ng = fma2(dy2[h], t, ag), nb = add2(ab, dy2[h]), nca = fma2(gdys, x2[h], ca);
-      if (MASKED) {  // drop a padded row's results, after the arithmetic
-        ng = ok ? ng : ag;
-        nb = ok ? nb : ab;
-        nca = ok ? nca : ca;
+      if (MASKED) {  // drop padded elements' results, after the arithmetic
+        const bool okx = 2 * h < nvalid, oky = 2 * h + 1 < nvalid;
+        ng = make_float2(okx ? ng.x : ag.x, oky ? ng.y : ag.y);
+        nb = make_float2(okx ? nb.x : ab.x, oky ? nb.y : ab.y);
+        nca = make_float2(okx ? nca.x : ca.x, oky ? nca.y : ca.y);
       }
       acc.g[2 * h] = ng.x;
       acc.g[2 * h + 1] = ng.y;
@@ -550,6 +609,7 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       const float gdys = (g4[e] * dyf[e]) * q;
       dxf[e] = alpha * gdys;
       const float ng = fmaf(dyf[e], t, acc.g[e]), nb = acc.b[e] + dyf[e], nca = fmaf(gdys, xf[e], ca.x);
+      const bool ok = e < nvalid;
       acc.g[e] = (MASKED && !ok) ? acc.g[e] : ng;
       acc.b[e] = (MASKED && !ok) ? acc.b[e] : nb;
       ca.x = (MASKED && !ok) ? ca.x : nca;
@@ -605,14 +665,16 @@ __global__ void __launch_bounds__(B, 1)
 #pragma unroll
           for (int u = 0; u < U; ++u) {
             const int64_t row = r0 + (int64_t)u * g.RL;
-            IO::store_raw(dx + row * g.N + c0, bwd_vector<T, VEC, false>(rx[u], rdy[u], alpha, gam, acc, ca, true));
+            IO::store_raw(dx + row * g.N + c0,
+                          bwd_vector<T, VEC, false>(rx[u], rdy[u], alpha, gam, acc, ca, VEC));
           }
         } else {  // ragged last step of the group
 #pragma unroll
           for (int u = 0; u < U; ++u) {
             const int64_t row = r0 + (int64_t)u * g.RL;
             const bool ok = row < re;
-            const typename IO::Raw d = bwd_vector<T, VEC, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok);
+            const typename IO::Raw d =
+                bwd_vector<T, VEC, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok ? VEC : 0);
             if (ok) IO::store_raw(dx + row * g.N + c0, d);
           }
         }
@@ -667,9 +729,14 @@ __global__ void __launch_bounds__(B, 1)
 // ---- backward, stage 2 -------------------------------------------------------
 
 // Block of 256 threads = CT columns x L lanes (L = 256 / CT, chosen on the host
-// so that a lane reads at most a few partials). Lane l adds partials l, l + L,
-// ... of its column in binary64, a fixed-order tree adds the lanes, and the
-// sum is rounded once to P. Block 0 also reduces dalpha.
+// so that a lane reads at most a few partials), thread = lane * CT + column.
+// Lane l adds partials l, l + L, ... of its column in binary64, in that order;
+// each batch of four is loaded before any is added, so a lane waits for one
+// round trip per batch. The lanes of a column are then added by a fixed-order
+// warp butterfly (lanes CT apart share a warp when CT < 32) and the warps'
+// results by one thread per column, in warp order; the sum is rounded once
+// to P. The last block also reduces dalpha, with its loads issued together
+// with the column loads.
 constexpr int kFinThreads = 256;
 
 template <typename P>
@@ -677,62 +744,66 @@ __global__ void __launch_bounds__(kFinThreads)
     dyt_finalize_kernel(const float *__restrict__ part_dg, const float *__restrict__ part_db,
                         const double *__restrict__ part_da, P *dgamma, P *dbeta, P *dalpha,
                         int64_t N, int nrg, int nda, int CT) {
-  __shared__ double sg[kFinThreads], sb[kFinThreads];
+  __shared__ double sg[kFinThreads], sb[kFinThreads], sa[kFinThreads / 32];
   // Wait until the stage-1 grid has finished and its writes are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x;
   const int L = kFinThreads / CT;
   const int lane = tid / CT, c = tid - lane * CT;
   const int64_t col = (int64_t)blockIdx.x * CT + c;
+  const bool da_block = blockIdx.x == gridDim.x - 1;
+  // dalpha partials: thread i adds i, i + 256, ...; the first is loaded here
+  // and added only after the column loads below are under way.
+  const double da0 = da_block && tid < nda ? part_da[tid] : 0.0;
   double a = 0.0, b = 0.0;
   if (col < N) {
-    int r = lane;
-    for (; r + 3 * L < nrg; r += 4 * L) {  // four independent loads in flight
-      const float a0 = part_dg[(int64_t)r * N + col], a1 = part_dg[(int64_t)(r + L) * N + col];
-      const float a2 = part_dg[(int64_t)(r + 2 * L) * N + col], a3 = part_dg[(int64_t)(r + 3 * L) * N + col];
-      const float b0 = part_db[(int64_t)r * N + col], b1 = part_db[(int64_t)(r + L) * N + col];
-      const float b2 = part_db[(int64_t)(r + 2 * L) * N + col], b3 = part_db[(int64_t)(r + 3 * L) * N + col];
-      a += (double)a0;
-      a += (double)a1;
-      a += (double)a2;
-      a += (double)a3;
-      b += (double)b0;
-      b += (double)b1;
-      b += (double)b2;
-      b += (double)b3;
+    for (int r = lane; r < nrg; r += 4 * L) {
+      float va[4], vb[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int rk = r + k * L;
+        va[k] = rk < nrg ? part_dg[(int64_t)rk * N + col] : 0.0f;  // + 0 leaves a sum unchanged
+        vb[k] = rk < nrg ? part_db[(int64_t)rk * N + col] : 0.0f;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        a += (double)va[k];
+        b += (double)vb[k];
+      }
     }
-    for (; r < nrg; r += L) {
-      a += (double)part_dg[(int64_t)r * N + col];
-      b += (double)part_db[(int64_t)r * N + col];
-    }
+  }
+  // Lanes of a column within a warp: a butterfly (both partners of an
+  // exchange form the same sum, so every lane ends with identical bits).
+  for (int off = CT; off < 32; off <<= 1) {
+    a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
+    b += __shfl_xor_sync(0xFFFFFFFFu, b, off);
   }
   sg[tid] = a;
   sb[tid] = b;
+  if (da_block) {
+    double da = 0.0 + da0;
+    for (int i = tid + kFinThreads; i < nda; i += kFinThreads) da += part_da[i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) da += __shfl_xor_sync(0xFFFFFFFFu, da, off);
+    if ((tid & 31) == 0) sa[tid >> 5] = da;
+  }
   __syncthreads();
-  for (int n = L; n > 1;) {
-    const int h = (n + 1) >> 1;
-    if (lane < n - h) {
-      sg[tid] += sg[tid + h * CT];
-      sb[tid] += sb[tid + h * CT];
+  // One value per warp and column when CT < 32 (stride 32), else one per lane
+  // (stride CT): kFinThreads / stride of them, added in order.
+  const int stride = CT < 32 ? 32 : CT;
+  if (tid < CT && col < N) {
+    double sgc = 0.0, sbc = 0.0;
+    for (int k = 0; k < kFinThreads / stride; ++k) {
+      sgc += sg[k * stride + tid];
+      sbc += sb[k * stride + tid];
     }
-    __syncthreads();
-    n = h;
+    dgamma[col] = from_f64<P>(sgc);
+    dbeta[col] = from_f64<P>(sbc);
   }
-  if (lane == 0 && col < N) {
-    dgamma[col] = from_f64<P>(sg[tid]);
-    dbeta[col] = from_f64<P>(sb[tid]);
-  }
-  if (blockIdx.x == 0) {
-    __syncthreads();
+  if (da_block && tid == 0) {
     double s = 0.0;
-    for (int i = tid; i < nda; i += kFinThreads) s += part_da[i];
-    sg[tid] = s;
-    __syncthreads();
-    for (int n = kFinThreads; n > 1; n >>= 1) {
-      if (tid < n / 2) sg[tid] += sg[tid + n / 2];
-      __syncthreads();
-    }
-    if (tid == 0) dalpha[0] = from_f64<P>(sg[0]);
+    for (int w = 0; w < kFinThreads / 32; ++w) s += sa[w];
+    dalpha[0] = from_f64<P>(s);
   }
 }
 

@@ -325,10 +325,10 @@ __global__ void __launch_bounds__(B, 1)
           const typename IO::Raw rx = *(const typename IO::Raw *)(st + (size_t)ri * tg.pitch);
           const typename IO::Raw rd = *(const typename IO::Raw *)(sd + (size_t)ri * tg.pitch);
           if (full_tile) {
-            IO::store_raw(dx + row * g.N + c0, bwd_vector<T, VEC, false>(rx, rd, alpha, gam, acc, ca, true));
+            IO::store_raw(dx + row * g.N + c0, bwd_vector<T, VEC, false>(rx, rd, alpha, gam, acc, ca, VEC));
           } else {  // the item's last, ragged tile: padded rows are dropped after the arithmetic
             const bool ok = row < cons.re;
-            const typename IO::Raw o = bwd_vector<T, VEC, true>(rx, rd, alpha, gam, acc, ca, ok);
+            const typename IO::Raw o = bwd_vector<T, VEC, true>(rx, rd, alpha, gam, acc, ca, ok ? VEC : 0);
             if (ok) IO::store_raw(dx + row * g.N + c0, o);
           }
         }

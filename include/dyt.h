@@ -24,7 +24,8 @@
  * - Layout: x, dy, y and dx are contiguous row-major M x N arrays (row stride
  *   N elements). gamma, beta, dgamma and dbeta hold N elements; alpha and
  *   dalpha hold one. Any alignment is accepted; 16-byte aligned tensors take
- *   the vectorised path.
+ *   the vectorised path, for any N (a ragged N is streamed in packs of
+ *   16 / element-size rows, which always span whole 16-byte vectors).
  * - Dtypes (the page's Summary, "Precision"): x, dy, y and dx share x_dtype;
  *   alpha, gamma, beta and all three parameter gradients share param_dtype.
  *   y and dx come back in x_dtype, the parameter gradients in param_dtype.
@@ -141,13 +142,16 @@ typedef struct dyt_launch_info {
   int vec;           /* elements per vector access (1 = scalar) */
   int block;         /* threads per CTA */
   int grid;          /* CTAs of the main kernel (1D) */
-  int row_lanes;     /* rows one CTA step covers side by side */
-  int rows_per_step; /* rows one CTA step covers in total */
+  int row_lanes;     /* rows (packs of pack_rows rows) one CTA step covers side by side */
+  int rows_per_step; /* matrix rows one CTA step covers in total */
   int col_chunks;    /* column chunks the grid is split into */
   int row_groups;    /* row groups (= partial sums per column) */
   int kernels;       /* kernels this call launched */
   int tma_stages;    /* shared-memory stages of the CTA-wide bulk-copy pipeline (0 = unused) */
   int async_stages;  /* per-thread asynchronous-copy ring slots (0 = unused) */
+  int pack_rows;     /* 1, or vec on the packed path: a 16-byte aligned matrix whose N is not a
+                        multiple of vec is streamed as packs of vec rows (vec x N elements,
+                        exactly N 16-byte vectors) */
   int64_t workspace_bytes;
 } dyt_launch_info;
 

@@ -65,7 +65,8 @@ def test_host_validation_without_a_device():
 
 @pytest.mark.parametrize("M,N,xd", [(1024, 64, 0), (65537, 32, 1), (100003, 17, 0), (100003, 100, 0),
                                     (100003, 255, 0), (16384, 4096, 1), (32768, 8192, 1), (1, 1, 0),
-                                    (3, 70000, 2), (10**7, 8, 1), (5, 513, 0)])
+                                    (3, 70000, 2), (10**7, 8, 1), (5, 513, 0), (7, 3, 1), (1, 17, 0),
+                                    (100003, 4097, 1), (4099, 1001, 0)])
 @pytest.mark.parametrize("vectorized", [0, 1])
 @pytest.mark.parametrize("sms,occ", [(148, 1), (148, 2), (7, 1)])
 def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
@@ -73,17 +74,23 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
     p = dyt.dyt_plan_query(M, N, xd, 0, 1, vectorized, sms, occ)
     size = 4 if xd == 0 else 2
     vec = p["vec"]
+    pk = p["pack_rows"]
     assert not (p["tma_stages"] and p["async_stages"])
-    if p["async_stages"]:    # per-thread copy ring: 16-byte rows, one 16-byte vector per thread
-        assert vectorized and vec == 16 // size and N % vec == 0
+    if p["async_stages"]:    # per-thread copy ring: 16-byte vectors, one per thread
+        assert vectorized and vec == 16 // size
+        # a ragged N is streamed in packs of vec rows (exactly N vectors each)
+        assert pk == (vec if N % vec else 1)
+    else:
+        assert pk == 1
     if p["tma_stages"]:      # bulk-copy pipeline: 16-byte rows, 4 columns per thread
         assert vectorized and (N * size) % 16 == 0 and vec == 4
         assert 2 <= p["tma_stages"] <= 8
     else:
         assert vec in (1, 16 // size)
         if vec > 1:
-            assert vectorized and N % vec == 0
-    nv = N // vec
+            assert vectorized and (N % vec == 0 or pk == vec)
+    Mp, Np = -(-M // pk), pk * N                   # (packed) rows and their pitch
+    nv = Np // vec
     B = p["block"]
     assert B in (512, 1024) and p["kernels"] == 2
     assert 1 <= p["grid"] <= sms * occ            # persistent 1D grid: never beyond one wave
@@ -91,19 +98,22 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
         assert p["row_lanes"] == B // nv >= 2 and p["col_chunks"] == 1
     else:                                          # row-per-CTA: columns across the CTA
         assert p["row_lanes"] == 1 and p["col_chunks"] == -(-nv // B)
+    if p["async_stages"]:
+        assert p["rows_per_step"] == p["row_lanes"] * pk
     items = p["row_groups"] * p["col_chunks"]
     assert p["grid"] <= items
-    # every lane adds at most 128 rows per group (bounded binary32 error)
-    rows_per_group = -(-M // p["row_groups"])
+    # every lane adds at most 128 (packed) rows per group (bounded binary32 error)
+    rows_per_group = -(-Mp // p["row_groups"])
     assert -(-rows_per_group // p["row_lanes"]) <= 128
     # every CTA gets the same number of work items, unless there are more
     # column chunks than CTAs
     if p["col_chunks"] <= sms * occ:
         assert items % p["grid"] == 0
         assert p["grid"] > (sms * occ) // 2 or p["grid"] == items
-    # workspace: binary32 dgamma and dbeta partials per group and column + binary64 dalpha per CTA
+    # workspace: binary32 dgamma and dbeta partials per group and row position
+    # (pack_rows x N of them) + binary64 dalpha per CTA
     al = lambda v: (v + 15) // 16 * 16
-    assert p["workspace_bytes"] == 2 * al(p["row_groups"] * N * 4) + al(p["grid"] * 8)
+    assert p["workspace_bytes"] == 2 * al(p["row_groups"] * Np * 4) + al(p["grid"] * 8)
 
 
 def test_page_narrow_widths_take_the_row_tiled_path():

@@ -153,6 +153,25 @@ def test_cancelling_outputs_are_correctly_rounded():
         assert st["y"]["max_ulp"] <= 1
 
 
+def test_cancelling_outputs_in_the_f16_subnormal_range():
+    # x ~ N(0, 1e-3) and beta ~ -tanh(x) of one row: y = gamma t + beta lands
+    # around 1e-6, inside fp16's subnormal range (below 6.1e-5), where rounding
+    # errors are absolute, and the cancellation threshold tau |beta| ~ 2e-6 is
+    # itself subnormal.
+    M, N = 4096, 64
+    for pd in ("f32", "f16"):
+        inp = make(M, N, "f16", pd, alpha=1.0, x_std=1e-3)
+        X = H.decode(inp["x"], "f16").reshape(M, N)
+        g = H.decode(inp["gamma"], pd)
+        beta = -g * np.tanh(X[17])
+        inp["beta"] = beta.astype(np.float32) if pd == "f32" else beta.astype(np.float16)
+        out, _ = H.run_cuda(inp, M, N, "f16", pd, bwd=False)
+        Y = np.abs(H.decode(out["y"], "f16"))
+        assert ((Y > 0) & (Y < 6.1e-5)).sum() > 1000  # many subnormal outputs
+        st = H.compare_all(inp, out, M, N, "f16", pd)
+        assert st["y"]["max_ulp"] <= 1
+
+
 def test_extreme_arguments():
     # Large |alpha x| (tanh saturates, 1 - t^2 underflows), tiny |alpha x|, and
     # special values in x.
@@ -216,9 +235,52 @@ def test_unaligned_pointers_take_the_scalar_path():
     H.compare_all(inp, out, M, N, "bf16", "f32")
 
 
-def test_in_place_aliasing():
+# Ragged widths of aligned tensors are streamed in packs of 16 / size rows; the
+# last pack may be short, down to a single row, and its one straddling vector
+# is zero-filled and masked.
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 7, 8, 9, 13, 4099])
+@pytest.mark.parametrize("N,xd", [(17, "f32"), (3, "f32"), (255, "bf16"), (1001, "f16"), (17, "bf16"),
+                                  (4097, "f32")])
+def test_ragged_widths_take_the_packed_path(M, N, xd):
+    _, info, _ = roundtrip(M, N, xd, "f32")
+    vec = 4 if xd == "f32" else 8
+    for op in ("fwd", "bwd"):
+        assert info[op]["pack_rows"] == vec and info[op]["vec"] == vec and info[op]["async_stages"] > 0
+
+
+@pytest.mark.parametrize("N", [17, 1001])
+def test_infinite_alpha_in_the_straddling_vector(N):
+    # 4099 rows of 17 or 1001 fp32 columns end inside a 16-byte vector whose
+    # zero-filled tail would give tanh(inf * 0) = NaN if it entered a sum.
+    M = 4099
+    inp = make(M, N, "f32", "f32", alpha=float("inf"), nonzero=True)
+    out, info = H.run_cuda(inp, M, N, "f32", "f32")
+    assert info["bwd"]["pack_rows"] == 4
+    H.compare_all(inp, out, M, N, "f32", "f32")
+    assert np.isfinite(H.decode(out["dgamma"], "f32")).all()
+    assert np.isfinite(H.decode(out["dbeta"], "f32")).all()
+
+
+def test_unaligned_ragged_rows_take_the_scalar_path():
     import elementwise_reduction_b200 as dyt
-    M, N = 1000, 256
+    M, N = 301, 17
+    inp = make(M, N, "f32", "f32")
+    t = H.gpu_inputs(inp, "f32", "f32")
+    buf = torch.empty(M * N + 1, dtype=torch.float32, device="cuda")
+    buf[1:] = t["x"]
+    x = buf[1:].view(M, N)  # 4-byte offset: not 16-byte aligned
+    y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"])
+    info = dyt.dyt_last_launch_info()
+    assert info["vec"] == 1 and info["pack_rows"] == 1
+    dx, da, dg, db = dyt.backward(x, t["dy"].view(M, N), t["alpha"], t["gamma"])
+    out = {"y": H.to_numpy(y, "f32"), "dx": H.to_numpy(dx, "f32"), "dgamma": H.to_numpy(dg, "f32"),
+           "dbeta": H.to_numpy(db, "f32"), "dalpha": float(da.item())}
+    H.compare_all(inp, out, M, N, "f32", "f32")
+
+
+@pytest.mark.parametrize("M,N", [(1000, 256), (1001, 255)])
+def test_in_place_aliasing(M, N):
+    import elementwise_reduction_b200 as dyt
     inp = make(M, N, "bf16", "f32")
     ref, _ = H.run_cuda(inp, M, N, "bf16", "f32")
     t = H.gpu_inputs(inp, "bf16", "f32")

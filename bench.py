@@ -50,6 +50,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--no-shapes", action="store_true", help="skip the per-shape table of the other workloads")
+    p.add_argument("--no-latency", action="store_true", help="skip the per-call cold-L2 latency percentiles")
     p.add_argument("--record-traffic", metavar="NCU_CSV", default=None,
                    help="store DRAM bytes per launch from an ncu --csv capture of dram__bytes_read.sum and "
                         "dram__bytes_write.sum into profiles/dram_traffic.json for --workload, then exit")
@@ -476,9 +477,65 @@ def run_ours(args, w):
         dist.destroy_process_group()
     if world == 1 and not args.no_shapes:
         line["shapes"] = other_shapes(w, args, dev)
+    if world == 1 and not args.no_latency:
+        line["latency_us"] = call_latency(args, dev)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
+
+
+def call_latency(args, dev, calls=30):
+    """Per-call device time of one forward and one backward call (both backward
+    kernels), each with L2 flushed just before it, as p10 / p50 / p90 over
+    `calls` calls; forward and backward alternate, and the workloads are visited
+    in rotation. This is the latency of one isolated call, next to the graph
+    throughput figures."""
+    import torch
+
+    import elementwise_reduction_b200 as dyt
+    from synth import workloads
+
+    L2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * L2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    state = {}
+    for name, w in workloads.WORKLOADS.items():
+        inp = workloads.make_inputs(w)
+
+        def dev_t(a, dt):
+            a = np.ascontiguousarray(a)
+            t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dt == "bf16" else torch.from_numpy(a)
+            return t.to(dev)
+
+        x = dev_t(inp["x"], w.x_dtype).view(w.M, w.N)
+        st = {"x": x, "dy": dev_t(inp["dy"], w.x_dtype).view(w.M, w.N), "y": torch.empty_like(x),
+              "dx": torch.empty_like(x), "p": [dev_t(inp[k], w.p_dtype) for k in ("alpha", "gamma", "beta")],
+              "ws": None, "t": {"fwd": [], "bwd": []}}
+        st["ws"] = dyt.workspace(x, st["p"][1])
+        state[name] = st
+    with torch.cuda.stream(stream):
+        for i in range(calls + 2):  # the first two rounds are warm-up
+            for name, st in state.items():
+                a, g, b = st["p"]
+                for op in ("fwd", "bwd"):
+                    flush.fill_(i & 0xFF)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    if op == "fwd":
+                        dyt.forward(st["x"], a, g, b, out=st["y"])
+                    else:
+                        dyt.backward(st["x"], st["dy"], a, g, dx=st["dx"], ws=st["ws"])
+                    e1.record(stream)
+                    e1.synchronize()
+                    if i >= 2:
+                        st["t"][op].append(e0.elapsed_time(e1) * 1e3)
+    out = {}
+    for name, st in state.items():
+        out[name] = {op: {q: round(float(np.percentile(v, p)), 2) for q, p in (("p10", 10), ("p50", 50), ("p90", 90))}
+                     for op, v in st["t"].items()}
+    del state, flush
+    torch.cuda.empty_cache()
+    return out
 
 
 def other_shapes(w0, args, dev):

@@ -13,11 +13,12 @@ from __future__ import annotations
 import torch
 
 from . import _abi
-from ._abi import (DYT_BF16, DYT_F16, DYT_F32, DytError, dyt_backward, dyt_backward_workspace_bytes,
-                   dyt_device_error, dyt_forward, dyt_last_launch_info, dyt_plan_query,
-                   dyt_selftest_wait_timeout, dyt_status_string)
+from ._abi import (DYT_BF16, DYT_F16, DYT_F32, DytError, dyt_backward, dyt_backward_strided,
+                   dyt_backward_workspace_bytes, dyt_device_error, dyt_forward, dyt_forward_strided,
+                   dyt_last_launch_info, dyt_plan_query, dyt_selftest_wait_timeout, dyt_status_string)
 
 __all__ = ["forward", "backward", "workspace", "DyT", "DyTFunction", "dyt_forward", "dyt_backward",
+           "dyt_forward_strided", "dyt_backward_strided", "row_pitch",
            "dyt_backward_workspace_bytes", "dyt_status_string", "dyt_last_launch_info", "dyt_plan_query",
            "dyt_device_error", "dyt_selftest_wait_timeout", "DytError",
            "DTYPE_CODE", "DYT_F32", "DYT_BF16", "DYT_F16"]
@@ -39,6 +40,33 @@ def _cuda_contig(t: torch.Tensor, what: str) -> None:
         raise ValueError(f"{what} must be contiguous")
 
 
+def row_pitch(t: torch.Tensor) -> int | None:
+    """Elements between consecutive rows when t's leading dimensions collapse into
+    one row index with a uniform pitch and its last dimension is dense; else None."""
+    if t.dim() == 0:
+        return None
+    if t.dim() == 1:
+        return t.shape[0] if t.shape[0] <= 1 or t.stride(0) == 1 else None
+    if t.shape[-1] > 1 and t.stride(-1) != 1:
+        return None
+    ld = t.stride(-2)
+    for i in range(t.dim() - 2):  # dimension i must step over whole blocks of dimension i + 1
+        if t.shape[i] > 1 and t.stride(i) != t.shape[i + 1] * t.stride(i + 1):
+            return None
+    if t.numel() > t.shape[-1] and ld < t.shape[-1]:
+        return None
+    return max(ld, t.shape[-1])
+
+
+def _rows(t: torch.Tensor, what: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    ld = row_pitch(t)
+    if ld is None:
+        raise ValueError(f"{what}: rows must be dense and evenly spaced (stride 1 along the last dimension)")
+    return ld
+
+
 def _shape(x: torch.Tensor, gamma: torch.Tensor):
     N = gamma.numel()
     if x.dim() == 0 or x.shape[-1] != N:
@@ -55,15 +83,20 @@ def _stream(device, stream):
 
 def forward(x: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
             out: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
-    """y = gamma * tanh(alpha * x) + beta in x's dtype (one kernel launch)."""
-    for t, w in ((x, "x"), (alpha, "alpha"), (gamma, "gamma"), (beta, "beta")):
+    """y = gamma * tanh(alpha * x) + beta in x's dtype (one kernel launch). x and out
+    may be row-strided views (dense rows, evenly spaced): no copy is made."""
+    for t, w in ((alpha, "alpha"), (gamma, "gamma"), (beta, "beta")):
         _cuda_contig(t, w)
+    ldx = _rows(x, "x")
     M, N = _shape(x, gamma)
-    y = torch.empty_like(x) if out is None else out
-    _cuda_contig(y, "out")
+    y = torch.empty(x.shape, dtype=x.dtype, device=x.device) if out is None else out
+    if y.shape != x.shape or y.dtype != x.dtype:
+        raise ValueError("out must match x in shape and dtype")
+    ldy = _rows(y, "out")
     with torch.cuda.device(x.device):
-        st = dyt_forward(x.data_ptr(), alpha.data_ptr(), gamma.data_ptr(), beta.data_ptr(), y.data_ptr(),
-                         M, N, _code(x, "x"), _code(gamma, "gamma"), _stream(x.device, stream))
+        st = dyt_forward_strided(x.data_ptr(), ldx, alpha.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
+                                 y.data_ptr(), ldy, M, N, _code(x, "x"), _code(gamma, "gamma"),
+                                 _stream(x.device, stream))
     _abi._check(st, "dyt_forward")
     return y
 
@@ -80,21 +113,27 @@ def backward(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, gamma: torc
              dx: torch.Tensor | None = None, dgamma: torch.Tensor | None = None,
              dbeta: torch.Tensor | None = None, dalpha: torch.Tensor | None = None,
              ws: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
-    """(dx, dalpha, dgamma, dbeta): dx in x's dtype, the others in gamma's dtype."""
-    for t, w in ((x, "x"), (dy, "dy"), (alpha, "alpha"), (gamma, "gamma")):
+    """(dx, dalpha, dgamma, dbeta): dx in x's dtype, the others in gamma's dtype.
+    x, dy and dx may be row-strided views (dense rows, evenly spaced)."""
+    for t, w in ((alpha, "alpha"), (gamma, "gamma")):
         _cuda_contig(t, w)
     if dy.shape != x.shape or dy.dtype != x.dtype:
         raise ValueError("dy must match x in shape and dtype")
+    ldx, lddy = _rows(x, "x"), _rows(dy, "dy")
     M, N = _shape(x, gamma)
-    dx = torch.empty_like(x) if dx is None else dx
+    dx = torch.empty(x.shape, dtype=x.dtype, device=x.device) if dx is None else dx
+    if dx.shape != x.shape or dx.dtype != x.dtype:
+        raise ValueError("dx must match x in shape and dtype")
+    lddx = _rows(dx, "dx")
     dgamma = torch.empty_like(gamma) if dgamma is None else dgamma
     dbeta = torch.empty_like(gamma) if dbeta is None else dbeta
     dalpha = torch.empty(1, dtype=gamma.dtype, device=gamma.device) if dalpha is None else dalpha
     ws = workspace(x, gamma) if ws is None else ws
     with torch.cuda.device(x.device):
-        st = dyt_backward(x.data_ptr(), dy.data_ptr(), alpha.data_ptr(), gamma.data_ptr(), dx.data_ptr(),
-                          dgamma.data_ptr(), dbeta.data_ptr(), dalpha.data_ptr(), M, N, _code(x, "x"),
-                          _code(gamma, "gamma"), ws.data_ptr(), ws.numel(), _stream(x.device, stream))
+        st = dyt_backward_strided(x.data_ptr(), ldx, dy.data_ptr(), lddy, alpha.data_ptr(), gamma.data_ptr(),
+                                  dx.data_ptr(), lddx, dgamma.data_ptr(), dbeta.data_ptr(), dalpha.data_ptr(), M,
+                                  N, _code(x, "x"), _code(gamma, "gamma"), ws.data_ptr(), ws.numel(),
+                                  _stream(x.device, stream))
     _abi._check(st, "dyt_backward")
     return dx, dalpha, dgamma, dbeta
 
@@ -104,14 +143,16 @@ class DyTFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, x, alpha, gamma, beta):
-        x, alpha, gamma, beta = (t.contiguous() for t in (x, alpha, gamma, beta))
+        alpha, gamma, beta = (t.contiguous() for t in (alpha, gamma, beta))
+        x = x if row_pitch(x) is not None else x.contiguous()
         ctx.save_for_backward(x, alpha, gamma)
         return forward(x, alpha, gamma, beta)
 
     @staticmethod
     def backward(ctx, dy):
         x, alpha, gamma = ctx.saved_tensors
-        dx, dalpha, dgamma, dbeta = backward(x, dy.contiguous(), alpha, gamma)
+        dy = dy if row_pitch(dy) is not None else dy.contiguous()
+        dx, dalpha, dgamma, dbeta = backward(x, dy, alpha, gamma)
         return dx, dalpha.reshape(alpha.shape), dgamma, dbeta
 
 

@@ -43,6 +43,11 @@ lib.dyt_backward_workspace_bytes.restype = _sz
 lib.dyt_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _sz,
                              _vp]
 lib.dyt_backward.restype = _i32
+lib.dyt_forward_strided.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _vp]
+lib.dyt_forward_strided.restype = _i32
+lib.dyt_backward_strided.argtypes = [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i32,
+                                     _i32, _vp, _sz, _vp]
+lib.dyt_backward_strided.restype = _i32
 lib.dyt_status_string.argtypes = [_i32]
 lib.dyt_status_string.restype = ctypes.c_char_p
 lib.dyt_last_cuda_error.argtypes = []
@@ -88,6 +93,18 @@ def dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, 
     """Raw C-ABI call: pointers as ints. Returns the status code."""
     return lib.dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
                             workspace, workspace_bytes, stream)
+
+
+def dyt_forward_strided(x, ldx, alpha, gamma, beta, y, ldy, M, N, x_dtype, param_dtype, stream) -> int:
+    """Raw C-ABI call with row pitches (elements). Returns the status code."""
+    return lib.dyt_forward_strided(x, ldx, alpha, gamma, beta, y, ldy, M, N, x_dtype, param_dtype, stream)
+
+
+def dyt_backward_strided(x, ldx, dy, lddy, alpha, gamma, dx, lddx, dgamma, dbeta, dalpha, M, N, x_dtype,
+                         param_dtype, workspace, workspace_bytes, stream) -> int:
+    """Raw C-ABI call with row pitches (elements). Returns the status code."""
+    return lib.dyt_backward_strided(x, ldx, dy, lddy, alpha, gamma, dx, lddx, dgamma, dbeta, dalpha, M, N,
+                                    x_dtype, param_dtype, workspace, workspace_bytes, stream)
 
 
 def dyt_backward_noalloc(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,

@@ -170,6 +170,7 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, int sms, 
   g.N = N;
   g.Nc = N_cols;
   g.total = M_rows * N_cols;
+  g.ldx = g.ldd = g.ldo = N;  // adjacent rows; the strided entry points override this
   g.NV = (int)NV;
   if (NV <= block / 2) {
     g.RL = block / (int)NV;
@@ -197,6 +198,7 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, int sms, 
   g.gq = M / nrg;
   g.grem = M % nrg;
   g.nv_magic = NV >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)NV - 1) / (uint64_t)NV) : 0u;
+  g.rl_magic = g.RL >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)g.RL - 1) / (uint64_t)g.RL) : 0u;
   // L2 prefetch of the first rows (pipelined kernels): worth its issue cost
   // only when the launch reads enough that its inputs are unlikely to be
   // resident in L2 already and each CTA's first rows take a DRAM round trip
@@ -287,6 +289,16 @@ dyt_status check_shape(int64_t M, int64_t N, dyt_dtype xd, dyt_dtype pd) {
   return DYT_OK;
 }
 
+// Row pitches: at least N, and the last element of every tensor addressable.
+dyt_status check_pitch(int64_t M, int64_t N, int64_t ld) {
+  if (ld < N) return DYT_ERR_INVALID_VALUE;
+  if (M > 1 && ld > 0 && (M - 1) > (INT64_MAX / 8 - N) / ld) return DYT_ERR_INVALID_VALUE;
+  return DYT_OK;
+}
+
+// A row pitch of whole 16-byte vectors.
+bool vec_pitch(int64_t ld, size_t elem) { return ((uint64_t)ld * elem) % 16 == 0; }
+
 dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
   dyt_launch_info i = {};
   i.op = op;
@@ -353,17 +365,38 @@ dyt_status prepare_tma_kernel(int dev, const void *kernel, int *static_smem) {
 }
 
 // Plan for given pointers' alignment on the current device.
+// Which kernels a call takes. aligned: every tensor starts on a 16-byte
+// boundary; pitched: every row pitch is a whole number of 16-byte vectors;
+// adjacent: every pitch is N. v: elements per 16-byte vector.
+struct PathChoice {
+  bool packed;  // ragged N on adjacent rows: packs of v rows through the 16-byte kernels
+  int vec;      // elements per access: v, or 1 for the scalar kernels
+  bool tma;     // the CTA-wide bulk-copy pipeline (compile-time option)
+  bool async;   // the per-thread asynchronous-copy rings
+};
+
+PathChoice choose_path(int64_t N, int v, bool aligned, bool pitched, bool adjacent) {
+  PathChoice c;
+  // A pack of v adjacent rows is a whole number of vectors whatever N is.
+  c.packed = DYT_PIPE == 2 && aligned && adjacent && N % v != 0;
+  const bool vec_ok = aligned && (c.packed || (pitched && N % v == 0));
+  c.tma = DYT_USE_TMA && vec_ok && adjacent;
+  c.vec = vec_ok && (!DYT_USE_TMA || c.tma) ? v : 1;
+  c.async = DYT_PIPE == 2 && c.vec > 1;
+  return c;
+}
+
+// aligned, pitched, adjacent: as for choose_path.
 template <typename T, typename P>
-dyt_status plan_for(int64_t M, int64_t N, bool vec_ok, bool backward, Plan *out) {
+dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjacent, bool backward, Plan *out) {
   int dev = 0, sms = 0;
   dyt_status st = current_sms(&dev, &sms);
   if (st != DYT_OK) return st;
   // Ragged rows of an aligned matrix go through the asynchronous-copy
   // kernels as packs; unaligned matrices take the scalar kernels.
-  const bool packed = DYT_PIPE == 2 && vec_ok && N % vec_of<T>() != 0;
-  const int vec = (vec_ok && (packed || N % vec_of<T>() == 0)) ? vec_of<T>() : 1;
-  const bool use_tma = DYT_USE_TMA && vec > 1;
-  const bool use_async = DYT_PIPE == 2 && vec > 1;
+  const PathChoice pc = choose_path(N, vec_of<T>(), aligned, pitched, adjacent);
+  const bool packed = pc.packed, use_tma = pc.tma, use_async = pc.async;
+  const int vec = pc.vec;
   const void *k = use_tma     ? tma_kernel<T, P>(backward)
                   : use_async ? (packed ? async_kernel<T, P, true>(backward) : async_kernel<T, P, false>(backward))
                   : backward  ? bwd_kernel<T, P>(vec)
@@ -396,8 +429,15 @@ extern "C" {
 dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, const void *beta, void *y,
                        int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
                        dyt_stream_t stream) {
+  return dyt_forward_strided(x, N, alpha, gamma, beta, y, N, M, N, x_dtype, param_dtype, stream);
+}
+
+dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, const void *gamma,
+                               const void *beta, void *y, int64_t ldy, int64_t M, int64_t N,
+                               dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream) {
   dyt_status st = check_shape(M, N, x_dtype, param_dtype);
   if (st != DYT_OK) return st;
+  if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, ldy) != DYT_OK) return DYT_ERR_INVALID_VALUE;
   if (M == 0 || N == 0) {
     record(1, nullptr, 0, 0);
     return DYT_OK;
@@ -408,8 +448,14 @@ dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, cons
     using P = decltype(tp);
     constexpr int V = vec_of<T>();
     Plan p;
-    dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y), false, &p);
+    dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y),
+                                  vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)), ldx == N && ldy == N,
+                                  false, &p);
     if (s != DYT_OK) return s;
+    if (!p.packed) {
+      p.g.ldx = ldx;
+      p.g.ldo = ldy;
+    }
     // Programmatic dependent launch: the kernel may be scheduled while its
     // predecessor in the stream drains; its first instruction waits
     // (griddepcontrol.wait) for that predecessor, so stream order holds.
@@ -458,7 +504,7 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
     // The vectorised and the scalar plan may differ; cover both.
     for (int v = 0; v < 2; ++v) {
       Plan p;
-      dyt_status s = plan_for<T, P>(M, N, v == 1, true, &p);
+      dyt_status s = plan_for<T, P>(M, N, v == 1, v == 1, true, true, &p);
       if (s != DYT_OK) return s;
       if (p.ws_total > need) need = p.ws_total;
     }
@@ -471,8 +517,18 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
                         void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
                         dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace,
                         size_t workspace_bytes, dyt_stream_t stream) {
+  return dyt_backward_strided(x, N, dy, N, alpha, gamma, dx, N, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
+                              workspace, workspace_bytes, stream);
+}
+
+dyt_status dyt_backward_strided(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
+                                const void *gamma, void *dx, int64_t lddx, void *dgamma, void *dbeta,
+                                void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
+                                void *workspace, size_t workspace_bytes, dyt_stream_t stream) {
   dyt_status st = check_shape(M, N, x_dtype, param_dtype);
   if (st != DYT_OK) return st;
+  if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, lddy) != DYT_OK || check_pitch(M, N, lddx) != DYT_OK)
+    return DYT_ERR_INVALID_VALUE;
   if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return DYT_ERR_INVALID_VALUE;
   cudaStream_t s = (cudaStream_t)stream;
   const size_t ps = dsize(param_dtype);
@@ -495,8 +551,16 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
     using P = decltype(tp);
     constexpr int V = vec_of<T>();
     Plan p;
-    dyt_status r = plan_for<T, P>(M, N, aligned16(x) && aligned16(dy) && aligned16(dx), true, &p);
+    const size_t es = sizeof(T);
+    dyt_status r = plan_for<T, P>(M, N, aligned16(x) && aligned16(dy) && aligned16(dx),
+                                  vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es),
+                                  ldx == N && lddy == N && lddx == N, true, &p);
     if (r != DYT_OK) return r;
+    if (!p.packed) {
+      p.g.ldx = ldx;
+      p.g.ldd = lddy;
+      p.g.ldo = lddx;
+    }
     if (workspace_bytes < p.ws_total) return DYT_ERR_WORKSPACE_TOO_SMALL;
     char *ws = (char *)workspace;
     float *pdg = (float *)(ws + p.ws_dg);
@@ -608,10 +672,9 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
     return DYT_OK;
   }
   const int v = 16 / (int)dsize(x_dtype);
-  const bool packed = DYT_PIPE == 2 && vectorized && N % v != 0;
-  const int vec = (vectorized && (packed || N % v == 0)) ? v : 1;
-  const bool use_tma = DYT_USE_TMA && vec > 1;
-  const bool use_async = DYT_PIPE == 2 && vec > 1;
+  const PathChoice pc = choose_path(N, v, vectorized != 0, vectorized != 0, true);  // adjacent rows
+  const bool packed = pc.packed, use_tma = pc.tma, use_async = pc.async;
+  const int vec = pc.vec;
   Plan p = make_plan(M, N, use_tma ? kTmaVec : vec, backward != 0, sm_count, ctas_per_sm,
                      use_async ? kAsyncBlock : kBlock, packed, (int64_t)dsize(x_dtype));
   p.tma = false;

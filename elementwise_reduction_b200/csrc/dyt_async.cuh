@@ -73,10 +73,11 @@ __device__ __forceinline__ void store_first(T *p, const uint4 &r, int n) {
 // griddepcontrol.wait, while the preceding grid may still be writing. That is
 // safe: a prefetch changes no memory state, and the ring copies after the wait
 // read L2 (cp.async.cg), so a line written later is read in its final state.
-// Rows are 16-byte aligned on this path, so every range below is too.
-template <typename T, int VEC, int B, int S>
-__device__ __forceinline__ void prefetch_first_rows_l2(const T *p, const Geom &g) {
-  if (!g.l2_prefetch || (int)blockIdx.x >= g.nitems) return;
+// Rows are 16-byte aligned on this path, so every range below is too. ld: the
+// tensor's row pitch in elements.
+template <typename T, int VEC, int B, int S, bool PK>
+__device__ __forceinline__ void prefetch_first_rows_l2(const T *p, int64_t ld, const Geom &g) {
+  if (!g.l2_prefetch || threadIdx.x >= 32 || (int)blockIdx.x >= g.nitems) return;  // warp 0 issues them
   int cc, rg;
   item_split(g, blockIdx.x, cc, rg);
   int64_t rb, re;
@@ -86,7 +87,7 @@ __device__ __forceinline__ void prefetch_first_rows_l2(const T *p, const Geom &g
   constexpr uint32_t kPiece = 16384;
   // Ranges end at the matrix's last element (a packed matrix's last row may
   // be short) and are rounded down to whole 16-byte units.
-  if (g.ncc == 1) {  // whole rows: one contiguous range, cut into pieces
+  if (g.ncc == 1 && ld == g.N) {  // whole, adjacent rows: one range, cut into pieces
     const int64_t bytes = (min(rows * g.N, g.total - rb * g.N) * (int64_t)sizeof(T)) & ~(int64_t)15;
     const int64_t k = threadIdx.x;
     if (k * kPiece < bytes) {
@@ -96,17 +97,23 @@ __device__ __forceinline__ void prefetch_first_rows_l2(const T *p, const Geom &g
     }
   } else if (threadIdx.x < rows) {  // one column chunk of each row
     const int64_t c0 = (int64_t)cc * B * VEC;
-    const int64_t at = (rb + threadIdx.x) * g.N + c0;
-    const int64_t n = (min(min((int64_t)B * VEC, g.N - c0), g.total - at) * (int64_t)sizeof(T)) & ~(int64_t)15;
+    const int64_t at = (rb + threadIdx.x) * ld + c0;
+    int64_t n = min((int64_t)B * VEC, g.N - c0);
+    if (PK) n = min(n, g.total - at);  // packed rows are adjacent (ld = N)
+    n = (n * (int64_t)sizeof(T)) & ~(int64_t)15;
     if (n > 0)
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + at), "r"((uint32_t)n) : "memory");
   }
 }
 
-// Rows of the current item owned by this thread: first row and count.
-__device__ __forceinline__ int64_t thread_rows(int64_t rb, int64_t re, int rl, int RL, int64_t &first) {
+// Rows of the current item owned by this thread: first row and count. A group
+// has at most 128 RL rows (the host caps it), so the quotient is formed with
+// the host's multiply-high constant, exactly, instead of a 64-bit division.
+__device__ __forceinline__ int64_t thread_rows(const Geom &g, int64_t rb, int64_t re, int rl, int64_t &first) {
   first = rb + rl;
-  return first < re ? (re - first + RL - 1) / RL : 0;
+  if (first >= re) return 0;
+  const uint32_t n = (uint32_t)(re - first) + (uint32_t)(g.RL - 1);
+  return g.RL == 1 ? (int64_t)n : (int64_t)__umulhi(n, g.rl_magic);
 }
 
 // ---- forward ------------------------------------------------------------------
@@ -138,7 +145,7 @@ __global__ void __launch_bounds__(B, 1)
   using IO = VecIO<T, VEC>;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
   extern __shared__ uint4 ring[];  // [S][B]
-  prefetch_first_rows_l2<T, VEC, B, S>(x, g);
+  prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
@@ -152,18 +159,18 @@ __global__ void __launch_bounds__(B, 1)
     if (!(ln.live && cv < g.NV)) continue;
     const int64_t c0 = (int64_t)cv * VEC;
     int64_t first;
-    int64_t n = thread_rows(rb, re, ln.rl, g.RL, first);
+    int64_t n = thread_rows(g, rb, re, ln.rl, first);
     const int nl = last_vector_real<VEC, PK>(g, first, c0, n);
     const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
-    const int64_t stride = (int64_t)g.RL * g.N;
-    const T *px = x + first * g.N + c0;
-    T *py = y + first * g.N + c0;
+    const int64_t sx = (int64_t)g.RL * g.ldx, sy = (int64_t)g.RL * g.ldo;
+    const T *px = x + first * g.ldx + c0;
+    T *py = y + first * g.ldo + c0;
     // Rows first, parameters second: the parameter loads overlap the copies.
 #pragma unroll
     for (int k = 0; k < S - 1; ++k) {
       if (k < n) {
-        if (PK) cp_async16_zfill(slot0 + k * B, px + k * stride, k == n - 1 ? last_bytes : 16u);
-        else cp_async16(slot0 + k * B, px + k * stride);
+        if (PK) cp_async16_zfill(slot0 + k * B, px + k * sx, k == n - 1 ? last_bytes : 16u);
+        else cp_async16(slot0 + k * B, px + k * sx);
       }
       cp_async_commit();
     }
@@ -175,8 +182,8 @@ __global__ void __launch_bounds__(B, 1)
     for (int64_t k = 0; k < n; ++k) {
       const int64_t kn = k + S - 1;
       if (kn < n) {
-        if (PK) cp_async16_zfill(slot0 + s_wr * B, px + kn * stride, kn == n - 1 ? last_bytes : 16u);
-        else cp_async16(slot0 + s_wr * B, px + kn * stride);
+        if (PK) cp_async16_zfill(slot0 + s_wr * B, px + kn * sx, kn == n - 1 ? last_bytes : 16u);
+        else cp_async16(slot0 + s_wr * B, px + kn * sx);
       }
       cp_async_commit();
       cp_async_wait<S - 1>();
@@ -184,7 +191,7 @@ __global__ void __launch_bounds__(B, 1)
       const typename IO::Raw ry = fwd_vector<T, VEC>(rx, alpha, gam, bet, bth);
       if (PK && k == n - 1 && nl < VEC) store_first<T, VEC>(py, ry, nl);  // zero-filled tail: not stored
       else IO::store_raw(py, ry);
-      py += stride;
+      py += sy;
       s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
       s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
     }
@@ -206,8 +213,8 @@ __global__ void __launch_bounds__(B, 1)
   // its first 2 VEC * B floats (at most 32 KB) serve the row-lane reduction.
   extern __shared__ uint4 ring[];
   __shared__ double red_a[B / 32];
-  prefetch_first_rows_l2<T, VEC, B, S>(x, g);
-  prefetch_first_rows_l2<T, VEC, B, S>(dy, g);
+  prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
+  prefetch_first_rows_l2<T, VEC, B, S, PK>(dy, g.ldd, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = param(alpha_p, 0);
@@ -231,24 +238,24 @@ __global__ void __launch_bounds__(B, 1)
     }
     if (col_ok) {
       int64_t first;
-      int64_t n = thread_rows(rb, re, ln.rl, g.RL, first);
+      int64_t n = thread_rows(g, rb, re, ln.rl, first);
       const int nl = last_vector_real<VEC, PK>(g, first, c0, n);
       const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
-      const int64_t stride = (int64_t)g.RL * g.N;
-      const T *px = x + first * g.N + c0;
-      const T *pd = dy + first * g.N + c0;
-      T *pdx = dx + first * g.N + c0;
+      const int64_t sx = (int64_t)g.RL * g.ldx, sd = (int64_t)g.RL * g.ldd, so = (int64_t)g.RL * g.ldo;
+      const T *px = x + first * g.ldx + c0;
+      const T *pd = dy + first * g.ldd + c0;
+      T *pdx = dx + first * g.ldo + c0;
       // Rows first, parameters second: the gamma loads overlap the copies.
 #pragma unroll
       for (int k = 0; k < S - 1; ++k) {
         if (k < n) {
           if (PK) {
             const uint32_t b = k == n - 1 ? last_bytes : 16u;
-            cp_async16_zfill(slot0 + (2 * k) * B, px + k * stride, b);
-            cp_async16_zfill(slot0 + (2 * k + 1) * B, pd + k * stride, b);
+            cp_async16_zfill(slot0 + (2 * k) * B, px + k * sx, b);
+            cp_async16_zfill(slot0 + (2 * k + 1) * B, pd + k * sd, b);
           } else {
-            cp_async16(slot0 + (2 * k) * B, px + k * stride);
-            cp_async16(slot0 + (2 * k + 1) * B, pd + k * stride);
+            cp_async16(slot0 + (2 * k) * B, px + k * sx);
+            cp_async16(slot0 + (2 * k + 1) * B, pd + k * sd);
           }
         }
         cp_async_commit();
@@ -263,11 +270,11 @@ __global__ void __launch_bounds__(B, 1)
         if (kn < n) {
           if (PK) {
             const uint32_t b = kn == n - 1 ? last_bytes : 16u;
-            cp_async16_zfill(slot0 + (2 * s_wr) * B, px + kn * stride, b);
-            cp_async16_zfill(slot0 + (2 * s_wr + 1) * B, pd + kn * stride, b);
+            cp_async16_zfill(slot0 + (2 * s_wr) * B, px + kn * sx, b);
+            cp_async16_zfill(slot0 + (2 * s_wr + 1) * B, pd + kn * sd, b);
           } else {
-            cp_async16(slot0 + (2 * s_wr) * B, px + kn * stride);
-            cp_async16(slot0 + (2 * s_wr + 1) * B, pd + kn * stride);
+            cp_async16(slot0 + (2 * s_wr) * B, px + kn * sx);
+            cp_async16(slot0 + (2 * s_wr + 1) * B, pd + kn * sd);
           }
         }
         cp_async_commit();
@@ -282,7 +289,7 @@ __global__ void __launch_bounds__(B, 1)
         }
         acc_a += (double)ca.x;
         acc_a += (double)ca.y;
-        pdx += stride;
+        pdx += so;
         s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
         s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
       }

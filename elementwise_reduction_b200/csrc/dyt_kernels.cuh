@@ -39,9 +39,12 @@ namespace dyt {
 
 struct Geom {
   int64_t M;      // rows (packs of VEC rows on the packed path)
-  int64_t N;      // columns: the row pitch in elements (VEC x Nc on the packed path)
+  int64_t N;      // elements of a row (VEC x Nc on the packed path): the partials' pitch
   int64_t Nc;     // columns of the matrix (= N unless packed)
-  int64_t total;  // elements of the matrix (its rows x Nc): later ones are padding
+  int64_t total;  // elements of the matrix (its rows x Nc): later ones are padding (packed path)
+  int64_t ldx;    // row pitches in elements (= N when packed): x,
+  int64_t ldd;    //   dy,
+  int64_t ldo;    //   and the output (y or dx)
   int NV;         // vector-columns per row (N / VEC)
   int RL;         // row lanes per CTA step (1 on the row-per-CTA path)
   int ncc;        // column chunks (of B vector-columns)
@@ -50,6 +53,7 @@ struct Geom {
   int64_t gq;     // M / nrg     (computed on the host: the kernels divide nothing)
   int64_t grem;   // M % nrg
   uint32_t nv_magic;  // ceil(2^32 / NV) for NV >= 2: tid / NV = umulhi(tid, nv_magic), tid < 1024
+  uint32_t rl_magic;  // ceil(2^32 / RL) for RL >= 2: n / RL = umulhi(n, rl_magic) for n < 2^32 / RL
   int l2_prefetch;    // the pipelined kernels prefetch their first rows into L2 (large inputs only)
 };
 
@@ -453,12 +457,12 @@ __global__ void __launch_bounds__(B, 1)
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t row = r0 + (int64_t)u * g.RL;
-        raw[u] = row < re ? IO::load(x + row * g.N + c0) : IO::zero();
+        raw[u] = row < re ? IO::load(x + row * g.ldx + c0) : IO::zero();
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t row = r0 + (int64_t)u * g.RL;
-        if (row < re) IO::store_raw(y + row * g.N + c0, fwd_vector<T, VEC>(raw[u], alpha, gam, bet, bth));
+        if (row < re) IO::store_raw(y + row * g.ldo + c0, fwd_vector<T, VEC>(raw[u], alpha, gam, bet, bth));
       }
     }
   }
@@ -657,15 +661,15 @@ __global__ void __launch_bounds__(B, 1)
         for (int u = 0; u < U; ++u) {
           const int64_t row = r0 + (int64_t)u * g.RL;
           const bool ok = row < re;
-          rx[u] = ok ? IO::load(x + row * g.N + c0) : IO::zero();
-          rdy[u] = ok ? IO::load(dy + row * g.N + c0) : IO::zero();
+          rx[u] = ok ? IO::load(x + row * g.ldx + c0) : IO::zero();
+          rdy[u] = ok ? IO::load(dy + row * g.ldd + c0) : IO::zero();
         }
         float2 ca = make_float2(0.0f, 0.0f);
         if (r0 + (int64_t)(U - 1) * g.RL < re) {  // every row of the step is real
 #pragma unroll
           for (int u = 0; u < U; ++u) {
             const int64_t row = r0 + (int64_t)u * g.RL;
-            IO::store_raw(dx + row * g.N + c0,
+            IO::store_raw(dx + row * g.ldo + c0,
                           bwd_vector<T, VEC, false>(rx[u], rdy[u], alpha, gam, acc, ca, VEC));
           }
         } else {  // ragged last step of the group
@@ -675,7 +679,7 @@ __global__ void __launch_bounds__(B, 1)
             const bool ok = row < re;
             const typename IO::Raw d =
                 bwd_vector<T, VEC, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok ? VEC : 0);
-            if (ok) IO::store_raw(dx + row * g.N + c0, d);
+            if (ok) IO::store_raw(dx + row * g.ldo + c0, d);
           }
         }
         acc_a += (double)ca.x;

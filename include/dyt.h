@@ -78,8 +78,8 @@ typedef enum dyt_status {
  *   beta   [N]   param_dtype, read
  *   y      [M*N] x_dtype, written (may alias x)
  * Each y element is rounded once to x_dtype. For 16-bit x_dtype an element
- * whose binary32 value of gamma*t + beta cancels (|y| < tau |gamma*t|, tau =
- * 2^-12 for bf16 and 2^-9 for fp16) is recomputed in binary64, so every y is
+ * whose binary32 value of gamma*t + beta may have cancelled (|y| < tau |beta|,
+ * tau = 2^-12 for bf16 and 2^-9 for fp16) is recomputed in binary64, so every y is
  * within one unit in the last place of the correctly rounded value.
  * M * N == 0 launches nothing. Null pointers with M * N > 0 give
  * DYT_ERR_INVALID_VALUE.
@@ -124,6 +124,30 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
                         void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
                         dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace,
                         size_t workspace_bytes, dyt_stream_t stream);
+
+/*
+ * dyt_forward and dyt_backward over row-strided matrices: row i of a tensor
+ * starts ld elements after row i - 1 (ld >= N), each with its own pitch
+ * (ldx, ldy; ldx, lddy, lddx). The page's kernels take contiguous rows; this
+ * leading-dimension form has no counterpart there. With the same kernels
+ * (see below) it gives the same bits as the contiguous call on the same rows.
+ * dyt_forward / dyt_backward are these with every pitch = N.
+ * Padding between rows is neither read nor written. When every tensor is
+ * 16-byte aligned and every pitch times the element size is a multiple of
+ * 16 bytes, the vectorised kernels run; adjacent rows (pitch N) are needed
+ * for the packed form of a ragged N, other strided matrices with a ragged N
+ * take the scalar kernels. y may alias x (dx may alias x or dy) only with
+ * equal pitches. A pitch below N, or (M - 1) * ld + N beyond the int64 limit
+ * of byte offsets, gives DYT_ERR_INVALID_VALUE. dyt_backward_workspace_bytes
+ * covers the strided call too.
+ */
+dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, const void *gamma,
+                               const void *beta, void *y, int64_t ldy, int64_t M, int64_t N,
+                               dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream);
+dyt_status dyt_backward_strided(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
+                                const void *gamma, void *dx, int64_t lddx, void *dgamma, void *dbeta,
+                                void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
+                                void *workspace, size_t workspace_bytes, dyt_stream_t stream);
 
 /* Static, human-readable name of a status. Never NULL. */
 const char *dyt_status_string(dyt_status status);

@@ -56,6 +56,13 @@ def test_host_validation_without_a_device():
     assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 0, 3, 3, 0, 0, 0, 0, None) == 1  # null dalpha
     assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 1, 3, 3, 1, 0, 0, 0, None) == 1  # null dgamma/dbeta
     assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 0, -3, 3, 0, 0, 0, 0, None) == 1
+    # row pitches below N, or byte offsets beyond int64, are rejected
+    assert dyt.dyt_forward_strided(0, 3, 0, 0, 0, 0, 4, 5, 4, 0, 0, None) == 1                  # ldx < N
+    assert dyt.dyt_forward_strided(0, 4, 0, 0, 0, 0, 3, 5, 4, 0, 0, None) == 1                  # ldy < N
+    assert dyt.dyt_forward_strided(0, 2**61, 0, 0, 0, 0, 4, 5, 4, 0, 0, None) == 1              # offsets overflow
+    assert dyt.dyt_backward_strided(0, 4, 0, 2, 0, 0, 0, 4, 0, 0, 1, 5, 4, 0, 0, 0, 0, None) == 1  # lddy < N
+    assert dyt.dyt_backward_strided(0, 4, 0, 4, 0, 0, 0, 3, 0, 0, 1, 5, 4, 0, 0, 0, 0, None) == 1  # lddx < N
+    assert dyt.dyt_forward_strided(0, 9, 0, 0, 0, 0, 9, 0, 4, 0, 0, None) == 0                  # empty
     assert dyt.dyt_backward_workspace_bytes(-1, 3, 0, 0) == 0
     assert dyt.dyt_backward_workspace_bytes(0, 3, 0, 0) == 0
     for s in range(5):
@@ -76,6 +83,8 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
     vec = p["vec"]
     pk = p["pack_rows"]
     assert not (p["tma_stages"] and p["async_stages"])
+    # 16-byte aligned adjacent rows always take the 16-byte kernels (packed when N is ragged)
+    assert bool(p["async_stages"] or p["tma_stages"]) == bool(vectorized)
     if p["async_stages"]:    # per-thread copy ring: 16-byte vectors, one per thread
         assert vectorized and vec == 16 // size
         # a ragged N is streamed in packs of vec rows (exactly N vectors each)
@@ -123,3 +132,18 @@ def test_page_narrow_widths_take_the_row_tiled_path():
             p = dyt.dyt_plan_query(65537, N, xd, 0, 1, 1, 148, 1)
             assert p["path"] == 1 and p["rows_per_step"] > 1
     assert dyt.dyt_plan_query(32768, 8192, 1, 0, 1, 1, 148, 1)["path"] == 2
+
+
+def test_multiply_high_quotients_are_exact():
+    # The kernels divide by the row-lane count RL (2..1024) with a host constant
+    # m = ceil(2^32 / RL): q = (n * m) >> 32. Groups hold at most 128 RL rows, so
+    # n < 129 RL; every quotient in that range must be exact (checked at and
+    # around each multiple of RL, where an error would first show).
+    import numpy as np
+    for RL in range(2, 1025):
+        m = ((1 << 32) + RL - 1) // RL
+        k = np.arange(0, 130, dtype=np.uint64)
+        n = np.concatenate([k * RL, k * RL + RL - 1, np.maximum(k * RL, 1) - 1]).astype(np.uint64)
+        n = n[n < 129 * RL + RL]
+        q = (n * np.uint64(m)) >> np.uint64(32)
+        assert np.array_equal(q, n // np.uint64(RL)), RL

@@ -296,6 +296,78 @@ def test_in_place_aliasing(M, N):
     assert np.array_equal(H.to_numpy(x2, "bf16"), ref["dx"])
 
 
+# ---- row-strided matrices: each tensor with its own leading dimension -----------------------------
+
+def _in_wider_rows(src: torch.Tensor, M: int, N: int, pitch: int, fill: float) -> tuple:
+    buf = torch.full((M, pitch), fill, dtype=src.dtype, device="cuda")
+    buf[:, :N] = src.view(M, N)
+    return buf, buf[:, :N]
+
+
+@pytest.mark.parametrize("N,pad,xd", [(64, 8, "bf16"), (64, 3, "bf16"), (100, 4, "f32"), (17, 3, "f32"),
+                                      (4096, 64, "bf16"), (255, 1, "f32"), (8, 8, "f16"), (1000, 24, "f16")])
+def test_strided_rows(N, pad, xd):
+    import elementwise_reduction_b200 as dyt
+    M = 3001
+    inp = make(M, N, xd, "f32")
+    t = H.gpu_inputs(inp, xd, "f32")
+    _, x = _in_wider_rows(t["x"], M, N, N + pad, float("nan"))      # padding is never read
+    _, dy = _in_wider_rows(t["dy"], M, N, N + 2 * pad, float("nan"))
+    ybuf, y = _in_wider_rows(torch.zeros(M * N, dtype=x.dtype, device="cuda"), M, N, N + 3 * pad, 7.0)
+    dxbuf, dx = _in_wider_rows(torch.zeros(M * N, dtype=x.dtype, device="cuda"), M, N, N + 4 * pad, 7.0)
+    dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=y)
+    info_f = dyt.dyt_last_launch_info()
+    _, dalpha, dgamma, dbeta = dyt.backward(x, dy, t["alpha"], t["gamma"], dx=dx)
+    info_b = dyt.dyt_last_launch_info()
+    torch.cuda.synchronize()
+    assert (ybuf[:, N:] == 7).all() and (dxbuf[:, N:] == 7).all()  # padding is never written
+    out = {"y": H.to_numpy(y.contiguous(), xd), "dx": H.to_numpy(dx.contiguous(), xd),
+           "dgamma": H.to_numpy(dgamma, "f32"), "dbeta": H.to_numpy(dbeta, "f32"), "dalpha": float(dalpha.item())}
+    H.compare_all(inp, out, M, N, xd, "f32")
+    size = 4 if xd == "f32" else 2
+    vec = 16 // size
+    vectorised = N % vec == 0 and all((p * size) % 16 == 0 for p in (N + pad, N + 2 * pad, N + 3 * pad, N + 4 * pad))
+    assert info_f["vec"] == info_b["vec"] == (vec if vectorised else 1)
+    assert info_b["pack_rows"] == 1
+    if vectorised:  # the same kernels as the contiguous call: the same bits
+        ref, _ = H.run_cuda(inp, M, N, xd, "f32")
+        for k in ("y", "dx", "dgamma", "dbeta"):
+            assert np.array_equal(out[k], ref[k]), k
+        assert out["dalpha"] == ref["dalpha"]
+
+
+def test_strided_in_place_and_autograd():
+    import elementwise_reduction_b200 as dyt
+    M, N = 1000, 256
+    inp = make(M, N, "bf16", "f32")
+    ref, _ = H.run_cuda(inp, M, N, "bf16", "f32")
+    t = H.gpu_inputs(inp, "bf16", "f32")
+    buf, x = _in_wider_rows(t["x"], M, N, N + 64, 0.0)
+    dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=x)  # y over x, same pitch
+    assert np.array_equal(H.to_numpy(x.contiguous(), "bf16"), ref["y"])
+    # autograd on a strided view: no copy of x, gradients as from the contiguous call
+    _, x = _in_wider_rows(t["x"], M, N, N + 64, 0.0)
+    x.requires_grad_(True)
+    m = dyt.DyT(N, device="cuda")
+    with torch.no_grad():
+        m.alpha.copy_(t["alpha"]); m.gamma.copy_(t["gamma"]); m.beta.copy_(t["beta"])
+    y = m(x)
+    y.backward(t["dy"].view(M, N))
+    assert np.array_equal(H.to_numpy(y.detach(), "bf16"), ref["y"])
+    assert np.array_equal(H.to_numpy(x.grad.contiguous(), "bf16"), ref["dx"])
+    assert np.array_equal(H.to_numpy(m.gamma.grad, "f32"), ref["dgamma"])
+
+
+def test_rows_must_be_evenly_spaced():
+    import elementwise_reduction_b200 as dyt
+    x = torch.zeros(4, 6, 32, device="cuda")[:, 1:3]  # leading dimensions do not collapse
+    one = torch.ones(32, device="cuda")
+    with pytest.raises(ValueError):
+        dyt.forward(x, one[:1], one, one)
+    with pytest.raises(ValueError):
+        dyt.forward(torch.zeros(32, 8, device="cuda").t(), one[:1], one, one)
+
+
 @pytest.mark.parametrize("M,N,xd", [(65537, 32, "bf16"), (3001, 4096, "bf16"), (20000, 255, "f32")])
 def test_backward_is_bitwise_deterministic(M, N, xd):
     inp = make(M, N, xd, "f32")

@@ -147,3 +147,17 @@ def test_multiply_high_quotients_are_exact():
         n = n[n < 129 * RL + RL]
         q = (n * np.uint64(m)) >> np.uint64(32)
         assert np.array_equal(q, n // np.uint64(RL)), RL
+
+
+def test_package_refuses_to_load_without_the_cuda_library(tmp_path):
+    # A copy of the Python package with no libdyt.so next to it must fail on
+    # import: there is no fallback implementation to run instead.
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "elementwise_reduction_b200")
+    dst = tmp_path / "elementwise_reduction_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "csrc", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import elementwise_reduction_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "libdyt.so is missing" in r.stderr

@@ -68,11 +68,21 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(read=None) -> str:
+    """Hash of the kernel sources with comments and blank space removed, so that
+    only a change of the code itself invalidates the recorded traffic.
+    read(path) -> text (default: the file on disk)."""
+    import re
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(p, encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(p)
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"(?m)//.*$", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,5 +1,6 @@
 // C ABI of the fused DyT layer (declared in include/dyt.h): argument checks,
-// launch planning and kernel dispatch. All device work is in dyt_kernels.cuh.
+// launch planning and kernel dispatch. All device work is in the kernels of
+// dyt_kernels.cuh, dyt_async.cuh and dyt_tma.cuh.
 #include <cuda_runtime.h>
 
 #include <cstdint>

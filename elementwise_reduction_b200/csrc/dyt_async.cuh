@@ -1,14 +1,16 @@
-// Per-thread asynchronous-copy DyT kernels for sm_100a (16-byte aligned rows).
+// Per-thread asynchronous-copy DyT kernels for sm_100a (16-byte vectors).
 //
-// Same decomposition, thread mapping, arithmetic and reduction order as the
-// register-path kernels in dyt_kernels.cuh. Each thread streams the rows it
-// owns (its VEC columns of rows rl, rl + RL, ... of the group) into a private
-// ring of S shared-memory slots with 16-byte asynchronous copies
-// (cp.async.cg, L2 only), S - 1 rows ahead of the row it computes, and reads
-// each slot back after cp.async.wait_group. A thread only ever reads slots it
-// filled itself, so no barrier is needed between threads; the data in flight
-// (up to (S - 1) x 32 bytes per thread) costs no registers. Each thread visits
-// exactly its real rows, so no padded lane is ever computed.
+// Same decomposition, thread mapping and arithmetic as the register-path
+// kernels in dyt_kernels.cuh; the row lanes of a CTA are added in a different
+// (also fixed) order when NV divides 32. Each thread streams the rows it owns
+// (its VEC columns of rows rl, rl + RL, ... of the group) into a private ring
+// of S shared-memory slots with 16-byte asynchronous copies (cp.async.cg, L2
+// only), S - 1 rows ahead of the row it computes, and reads each slot back
+// after cp.async.wait_group. A thread only ever reads slots it filled itself,
+// so no barrier is needed between threads; the data in flight (up to
+// (S - 1) x 32 bytes per thread) costs no registers. Each thread visits
+// exactly its real rows; only the one vector that straddles the end of a
+// packed matrix holds padding, which is masked after the arithmetic.
 #pragma once
 
 #include <cuda_runtime.h>

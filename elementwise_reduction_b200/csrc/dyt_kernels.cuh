@@ -321,10 +321,12 @@ __device__ __forceinline__ float param(const P *p, int64_t i) {
   return to_f32<P>(ld_scalar(p + i));
 }
 
-// First statement of every main kernel: wait until the preceding grid in the
-// stream has completed and its memory is visible (a no-op without a
-// programmatic predecessor), then let the next grid get scheduled. The kernels
-// touch no global memory before this, so programmatic launch keeps stream order.
+// Start of every main kernel: wait until the preceding grid in the stream has
+// completed and its memory is visible (a no-op without a programmatic
+// predecessor), then let the next grid get scheduled. The kernels read and
+// write no global memory before this (the pipelined kernels only issue L2
+// prefetch hints, which change no memory state), so programmatic launch keeps
+// stream order.
 __device__ __forceinline__ void pdl_prologue() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

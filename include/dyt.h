@@ -21,8 +21,10 @@
  *   device memory on the host or synchronises. The caller owns every buffer,
  *   the workspace included; the library allocates nothing and keeps no state
  *   other than the calling thread's last-launch record.
- * - Layout: x, dy, y and dx are contiguous row-major M x N arrays (row stride
- *   N elements). gamma, beta, dgamma and dbeta hold N elements; alpha and
+ * - Layout: x, dy, y and dx are row-major M x N arrays, contiguous (row
+ *   stride N elements) for dyt_forward / dyt_backward and with a row pitch
+ *   per tensor for the *_strided entry points. gamma, beta, dgamma and dbeta
+ *   hold N elements; alpha and
  *   dalpha hold one. Any alignment is accepted; 16-byte aligned tensors take
  *   the vectorised path, for any N (a ragged N is streamed in packs of
  *   16 / element-size rows, which always span whole 16-byte vectors).

@@ -144,6 +144,7 @@ struct Plan {
   bool tma;
   bool async;
   bool packed;  // ragged N on 16-byte aligned rows: packs of vec rows (see dyt_kernels.cuh)
+  bool too_big; // the group or item count would not fit the kernels' int indices
   dyt::TmaGeom tg;
   size_t smem;  // dynamic shared memory of the pipelined kernel
   size_t ws_dg, ws_db, ws_da, ws_total;  // workspace byte offsets / sizes
@@ -194,6 +195,10 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, int sms, 
   // the fill so every CTA gets the same number of items.
   const int64_t max_rows = (int64_t)g.RL * kMaxRowsPerLane;
   if (ceil_div(M, nrg) > max_rows) nrg = ceil_div(ceil_div(M, max_rows), fill) * fill;
+  // Shapes this large cannot be allocated on any device, but the plan must not
+  // wrap around for them either.
+  p.too_big = nrg * g.ncc > (int64_t)INT32_MAX;
+  if (p.too_big) nrg = 1;
   g.nrg = (int)nrg;
   g.nitems = (int)(nrg * g.ncc);
   g.gq = M / nrg;
@@ -413,6 +418,7 @@ dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjac
   }
   *out = make_plan(M, N, use_tma ? kTmaVec : vec, backward, sms, occ, use_async ? kAsyncBlock : kBlock, packed,
                    (int64_t)sizeof(T));
+  if (out->too_big) return DYT_ERR_INVALID_VALUE;
   out->tma = false;
   out->async = use_async;
   if (use_tma) plan_tma(*out, sizeof(T), backward, static_smem);
@@ -678,6 +684,7 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
   const int vec = pc.vec;
   Plan p = make_plan(M, N, use_tma ? kTmaVec : vec, backward != 0, sm_count, ctas_per_sm,
                      use_async ? kAsyncBlock : kBlock, packed, (int64_t)dsize(x_dtype));
+  if (p.too_big) return DYT_ERR_INVALID_VALUE;
   p.tma = false;
   p.async = use_async;
   if (p.async) p.unroll = 1;

@@ -125,6 +125,17 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
     assert p["workspace_bytes"] == 2 * al(p["row_groups"] * Np * 4) + al(p["grid"] * 8)
 
 
+def test_plans_whose_counts_overflow_are_rejected():
+    dyt = _lib()
+    # 2^40 rows of 300 unaligned fp32 columns: 3 row lanes of at most 128 rows
+    # per group would need about 2.9e9 groups, more than an int holds
+    with pytest.raises(dyt.DytError) as e:
+        dyt.dyt_plan_query(2**40, 300, 0, 0, 1, 0, 148, 1)
+    assert e.value.status == 1
+    p = dyt.dyt_plan_query(2**20, 300, 0, 0, 1, 0, 148, 1)
+    assert p["row_lanes"] == 3 and p["row_groups"] == -(-(-(-2**20 // (3 * 128))) // 148) * 148
+
+
 def test_page_narrow_widths_take_the_row_tiled_path():
     dyt = _lib()
     for N in (16, 17, 32, 64, 100, 128, 255, 256):

@@ -201,6 +201,31 @@ def test_saturated_arguments_keep_tiny_gradients(xd):
         assert np.count_nonzero(H.decode(out["dx"], xd)) > M * N // 4
 
 
+@pytest.mark.parametrize("xd", ["bf16", "f32"])
+def test_subnormal_exponentials_scattered_in_ordinary_vectors(xd):
+    # Mostly ordinary |alpha x|, with single elements at 44..51.9 (exp(-2|z|) a
+    # nonzero binary32 subnormal), 53..80 (exp(-2|z|) rounds to 0) and +-inf,
+    # spread so that most 16-byte vectors hold at most one of them.
+    M, N = 512, 256
+    inp = make(M, N, xd, "f32", alpha=1.0)
+    rng = np.random.default_rng(11)
+    X = H.decode(inp["x"], xd).astype(np.float64)
+    idx = rng.permutation(M * N)
+    win, far, inf = idx[:2000], idx[2000:3000], idx[3000:3100]
+    X[win] = rng.uniform(44.0, 51.9, win.size) * rng.choice([-1.0, 1.0], win.size)
+    X[far] = rng.uniform(53.0, 80.0, far.size) * rng.choice([-1.0, 1.0], far.size)
+    X[inf] = np.inf * rng.choice([-1.0, 1.0], inf.size)
+    inp["x"] = oracle.round_to(X, xd) if xd != "f32" else X.astype(np.float32)
+    DY = H.decode(inp["dy"], xd).astype(np.float64)
+    DY[win] = rng.uniform(1e3, 1e4, win.size)  # lifts dx above bf16's smallest subnormal
+    inp["dy"] = oracle.round_to(DY, xd) if xd != "f32" else DY.astype(np.float32)
+    out, _ = H.run_cuda(inp, M, N, xd, "f32")
+    H.compare_all(inp, out, M, N, xd, "f32")
+    dx = H.decode(out["dx"], xd)
+    if xd == "bf16":  # the window's tiny gradients are kept, not flushed
+        assert np.count_nonzero(dx[win]) > win.size // 2
+
+
 def test_empty_shapes():
     import elementwise_reduction_b200 as dyt
     x = torch.empty(0, 7, device="cuda")

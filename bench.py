@@ -489,7 +489,7 @@ def run_ours(args, w):
         line["shapes"] = other_shapes(w, args, dev)
     if world == 1 and not args.no_latency:
         line["latency_us"] = call_latency(args, dev)
-    if not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline:  # the oracle's baseline belongs to the 1-GPU line
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
 

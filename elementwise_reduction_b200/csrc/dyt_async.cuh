@@ -243,57 +243,66 @@ __global__ void __launch_bounds__(B, 1)
       int64_t n = thread_rows(g, rb, re, ln.rl, first);
       const int nl = last_vector_real<VEC, PK>(g, first, c0, n);
       const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
+      const int nn = (int)n;  // at most 128: the host caps a group at 128 rows per lane
       const int64_t sx = (int64_t)g.RL * g.ldx, sd = (int64_t)g.RL * g.ldd, so = (int64_t)g.RL * g.ldo;
-      const T *px = x + first * g.ldx + c0;
+      const T *px = x + first * g.ldx + c0;  // the next rows to copy (advanced, not re-derived)
       const T *pd = dy + first * g.ldd + c0;
       T *pdx = dx + first * g.ldo + c0;
       // Rows first, parameters second: the gamma loads overlap the copies.
+      // Row r lives in slot r mod S; the loop below is unrolled by S so that
+      // every slot index is a constant.
 #pragma unroll
       for (int k = 0; k < S - 1; ++k) {
-        if (k < n) {
+        if (k < nn) {
           if (PK) {
-            const uint32_t b = k == n - 1 ? last_bytes : 16u;
-            cp_async16_zfill(slot0 + (2 * k) * B, px + k * sx, b);
-            cp_async16_zfill(slot0 + (2 * k + 1) * B, pd + k * sd, b);
+            const uint32_t b = k == nn - 1 ? last_bytes : 16u;
+            cp_async16_zfill(slot0 + (2 * k) * B, px, b);
+            cp_async16_zfill(slot0 + (2 * k + 1) * B, pd, b);
           } else {
-            cp_async16(slot0 + (2 * k) * B, px + k * sx);
-            cp_async16(slot0 + (2 * k + 1) * B, pd + k * sd);
+            cp_async16(slot0 + (2 * k) * B, px);
+            cp_async16(slot0 + (2 * k + 1) * B, pd);
           }
         }
+        px += sx;
+        pd += sd;
         cp_async_commit();
       }
       int64_t col[VEC];
       vector_columns<VEC, PK>(c0, g.Nc, col);
 #pragma unroll
       for (int e = 0; e < VEC; ++e) gam[e] = 4.0f * param(gamma, col[e]);  // 4 gamma (see bwd_vector)
-      int s_rd = 0, s_wr = S - 1;
-      for (int64_t k = 0; k < n; ++k) {
-        const int64_t kn = k + S - 1;
-        if (kn < n) {
-          if (PK) {
-            const uint32_t b = kn == n - 1 ? last_bytes : 16u;
-            cp_async16_zfill(slot0 + (2 * s_wr) * B, px + kn * sx, b);
-            cp_async16_zfill(slot0 + (2 * s_wr + 1) * B, pd + kn * sd, b);
-          } else {
-            cp_async16(slot0 + (2 * s_wr) * B, px + kn * sx);
-            cp_async16(slot0 + (2 * s_wr + 1) * B, pd + kn * sd);
+      for (int k0 = 0; k0 < nn; k0 += S) {
+#pragma unroll
+        for (int j = 0; j < S; ++j) {
+          const int k = k0 + j;
+          if (k >= nn) break;
+          if (k + S - 1 < nn) {  // rows k + S - 1 into slot (j + S - 1) mod S
+            const int sw = (j + S - 1) % S;
+            if (PK) {
+              const uint32_t b = k + S - 1 == nn - 1 ? last_bytes : 16u;
+              cp_async16_zfill(slot0 + (2 * sw) * B, px, b);
+              cp_async16_zfill(slot0 + (2 * sw + 1) * B, pd, b);
+            } else {
+              cp_async16(slot0 + (2 * sw) * B, px);
+              cp_async16(slot0 + (2 * sw + 1) * B, pd);
+            }
           }
+          px += sx;
+          pd += sd;
+          cp_async_commit();
+          cp_async_wait<S - 1>();
+          const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
+          const typename IO::Raw rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
+          float2 ca = make_float2(0.0f, 0.0f);
+          if (PK && k == nn - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
+            store_first<T, VEC>(pdx, bwd_vector<T, VEC, true>(rx, rd, alpha, gam, acc, ca, nl), nl);
+          } else {
+            IO::store_raw(pdx, bwd_vector<T, VEC, false>(rx, rd, alpha, gam, acc, ca, VEC));
+          }
+          acc_a += (double)ca.x;
+          acc_a += (double)ca.y;
+          pdx += so;
         }
-        cp_async_commit();
-        cp_async_wait<S - 1>();
-        const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + (2 * s_rd) * B);
-        const typename IO::Raw rd = *(const typename IO::Raw *)(slot0 + (2 * s_rd + 1) * B);
-        float2 ca = make_float2(0.0f, 0.0f);
-        if (PK && k == n - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
-          store_first<T, VEC>(pdx, bwd_vector<T, VEC, true>(rx, rd, alpha, gam, acc, ca, nl), nl);
-        } else {
-          IO::store_raw(pdx, bwd_vector<T, VEC, false>(rx, rd, alpha, gam, acc, ca, VEC));
-        }
-        acc_a += (double)ca.x;
-        acc_a += (double)ca.y;
-        pdx += so;
-        s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
-        s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
       }
       cp_async_wait<0>();
     }

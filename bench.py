@@ -225,6 +225,48 @@ def cpu_baseline(w, seconds_budget=10.0):
             "rows_per_s": passes * rows / dt}
 
 
+def cpu_baseline_threads(w, seconds_budget=5.0):
+    """The same oracle fanned out over row blocks, one thread per host core in
+    this process's affinity set (its C calls release the interpreter lock).
+    Only the timing harness is parallel: each block is an ordinary oracle call
+    on its rows, and the blocks' parameter-gradient sums would be added
+    afterwards (N values, not timed). Repeated full passes until the budget
+    has elapsed."""
+    import concurrent.futures
+
+    import oracle
+    from synth import workloads
+
+    cores = len(os.sched_getaffinity(0))
+    rows = oracle_sample_rows(w, seconds_budget * cores)
+    ws = workloads.Workload(w.name, rows, w.N, w.x_dtype, w.p_dtype, w.alpha, w.x_std, w.dy_std,
+                            w.gamma_mean, w.gamma_std, w.beta_mean, w.beta_std, w.nonzero, w.seed)
+    inp = workloads.make_inputs(ws)
+    N = w.N
+    edges = [rows * i // cores for i in range(cores + 1)]
+    blocks = [(a, b) for a, b in zip(edges[:-1], edges[1:]) if b > a]
+
+    def run(block):
+        a, b = block
+        x, dy = inp["x"][a * N:b * N], inp["dy"][a * N:b * N]
+        oracle.forward(x, inp["alpha"], inp["gamma"], inp["beta"], b - a, N, w.x_dtype, w.p_dtype)
+        oracle.backward(x, dy, inp["alpha"], inp["gamma"], b - a, N, w.x_dtype, w.p_dtype)
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(blocks)) as ex:
+        passes, t0 = 0, time.perf_counter()
+        while True:
+            list(ex.map(run, blocks))
+            passes += 1
+            dt = time.perf_counter() - t0
+            if dt >= seconds_budget:
+                break
+    nbytes = passes * (ws.fwd_bytes() + ws.bwd_bytes())
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": len(blocks), "kind": "oracle, row blocks on threads",
+            "sample": f"first {rows} of {w.M} rows (x {N} columns) in {len(blocks)} row blocks, forward + backward, "
+                      f"{passes} pass(es), {dt:.2f} s",
+            "rows_per_s": passes * rows / dt}
+
+
 # ---- the reference arm: the oracle as it stands ------------------------------------------------
 
 def run_reference(args, w):
@@ -491,6 +533,7 @@ def run_ours(args, w):
         line["latency_us"] = call_latency(args, dev)
     if world == 1 and not args.no_cpu_baseline:  # the oracle's baseline belongs to the 1-GPU line
         line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline_threads"] = cpu_baseline_threads(w)
     print(json.dumps(line), flush=True)
 
 

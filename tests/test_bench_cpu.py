@@ -68,3 +68,13 @@ def test_traffic_csv_is_averaged_per_launch(tmp_path, monkeypatch):
     assert abs(d["dyt_backward"]["bytes_per_launch"] - 12.042e6) < 1
     assert all(v["source_hash"] == bench.kernel_source_hash() for v in d.values())
     assert "at::" not in json.dumps(d)
+
+
+def test_threaded_oracle_baseline_uses_the_host_cores():
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import workloads
+
+    d = bench.cpu_baseline_threads(workloads.WORKLOADS["c1_f32_1024x64"], seconds_budget=0.5)
+    assert d["unit"] == "GB/s" and d["value"] > 0 and d["kind"].startswith("oracle")
+    assert 1 <= d["cores"] <= len(os.sched_getaffinity(0))

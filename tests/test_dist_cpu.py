@@ -28,13 +28,13 @@ def _inputs(M, N):
     return workloads.make_inputs(w)
 
 
-def _rank(rank: int, port: int, M: int, N: int, q):
+def _rank(rank: int, port: int, M: int, N: int, q, world: int = WORLD):
     import oracle
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         inp = _inputs(M, N)
-        b, e = shard_rows(M, WORLD, rank)
+        b, e = shard_rows(M, world, rank)
         r = oracle.backward(inp["x"][b * N:e * N], inp["dy"][b * N:e * N], inp["alpha"], inp["gamma"],
                             e - b, N, "f32", "f32", want_dx=False)
         dg = torch.tensor(r["dgamma"], dtype=torch.float32)
@@ -58,16 +58,17 @@ def test_shard_rows_is_a_balanced_partition():
         shard_rows(5, 2, 2)
 
 
-def test_two_gloo_ranks_sum_to_the_whole_matrix():
+@pytest.mark.parametrize("world,M", [(WORLD, 1001), (3, 1000)])
+def test_gloo_ranks_sum_to_the_whole_matrix(world, M):
     import oracle
-    M, N = 1001, 24
+    N = 24
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, port, M, N, q)) for r in range(WORLD)]
+    procs = [ctx.Process(target=_rank, args=(r, port, M, N, q, world)) for r in range(world)]
     for p in procs:
         p.start()
-    got = [q.get(timeout=120) for _ in range(WORLD)]
+    got = [q.get(timeout=120) for _ in range(world)]
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -77,4 +78,37 @@ def test_two_gloo_ranks_sum_to_the_whole_matrix():
         assert np.all(np.abs(dg - full["dgamma"]) <= 2e-6 + 1e-5 * full["mag_dgamma"])
         assert np.all(np.abs(db - full["dbeta"]) <= 2e-6 + 1e-5 * full["mag_dbeta"])
         assert abs(da - full["dalpha"]) <= 1e-5 * full["mag_dalpha"]
-    assert np.array_equal(got[0][1], got[1][1])
+    for r in range(1, world):
+        assert np.array_equal(got[0][1], got[r][1])
+
+
+def _single_rank(port: int, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        out = []
+        for dt in (torch.float32, torch.bfloat16, torch.float16):
+            g = torch.linspace(-3, 5, 7).to(dt)
+            b = torch.linspace(2, -1, 7).to(dt)
+            a = torch.tensor([0.375]).to(dt)
+            dg, db, da = g.clone(), b.clone(), a.clone()
+            allreduce_param_grads(dg, db, da)  # one rank: the sum is the identity
+            out.append((str(dt), torch.equal(dg, g), torch.equal(db, b), torch.equal(da, a),
+                        dg.dtype == dt))
+        q.put(out)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gradient_exchange_keeps_each_parameter_dtype():
+    # The 2N + 1 gradients travel as one binary32 vector; 16-bit parameter
+    # gradients come back in their own dtype, unchanged by a one-rank sum.
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_single_rank, args=(_free_port(), q))
+    p.start()
+    out = q.get(timeout=120)
+    p.join(timeout=60)
+    assert p.exitcode == 0
+    for name, *oks in out:
+        assert all(oks), name

@@ -186,8 +186,9 @@ dyt_status dyt_last_launch_info(dyt_launch_info *out);
 /*
  * The launch plan dyt_forward (backward = 0) or dyt_backward (backward != 0)
  * would use for this shape on a device with `sm_count` SMs running
- * `ctas_per_sm` CTAs of the kernel each, with 16-byte aligned tensors
- * (vectorized != 0) or not. Host arithmetic only: touches no device, so the
+ * `ctas_per_sm` CTAs of the kernel each, for contiguous tensors that are
+ * 16-byte aligned (vectorized != 0; a ragged N then gets the packed form,
+ * out->pack_rows > 1) or not. Host arithmetic only: touches no device, so the
  * planning is testable without a GPU. out->kernels is the number of kernels
  * the call would launch and out->workspace_bytes the workspace it needs.
  * Errors: as the shape checks of dyt_forward, or DYT_ERR_INVALID_VALUE for

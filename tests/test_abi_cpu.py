@@ -172,3 +172,14 @@ def test_package_refuses_to_load_without_the_cuda_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import elementwise_reduction_b200"], cwd=tmp_path,
                        capture_output=True, text=True, timeout=120)
     assert r.returncode != 0 and "libdyt.so is missing" in r.stderr
+
+
+def test_binding_scratch_size_matches_the_header():
+    # The Python binding keeps its own copy of DYT_NOALLOC_SCRATCH_BYTES (ctypes
+    # cannot read a #define); it must equal the header's value.
+    dyt = _lib()
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+DYT_NOALLOC_SCRATCH_BYTES\s+\(([^)]*)\)", text)
+    assert m, "DYT_NOALLOC_SCRATCH_BYTES not found in include/dyt.h"
+    value = eval(re.sub(r"(\d+)u\b", r"\1", m.group(1)), {"__builtins__": {}})
+    assert value == dyt._abi.NOALLOC_SCRATCH_BYTES

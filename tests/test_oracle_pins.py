@@ -293,3 +293,56 @@ def test_decode_matches_library_converters():
     d = oracle.decode(h, "f16")
     ok = ~np.isnan(h)
     assert np.array_equal(d[ok], h[ok].astype(np.float64))
+
+
+# ---- the sum magnitudes that scale the gradient tolerances ---------------------------------------
+#
+# The oracle also returns S = sum |term| for each gradient sum (dgamma's terms dy t,
+# dbeta's dy, dalpha's gamma dy (1 - t^2) x). These set the tolerance of every sum
+# comparison, so they are pinned here by an independent computation: numpy's tanh
+# and cosh, and math.fsum (a correctly rounded sum), on the same decoded inputs.
+
+
+def _magnitudes_by_fsum(x, dy, alpha, g, M, N):
+    X, DY = x.astype(np.float64).reshape(M, N), dy.astype(np.float64).reshape(M, N)
+    G = g.astype(np.float64)
+    z = float(alpha) * X
+    t = np.tanh(z)
+    sech2 = 1.0 / np.cosh(z) ** 2
+    mg = np.array([math.fsum(np.abs(DY[:, j] * t[:, j])) for j in range(N)])
+    mb = np.array([math.fsum(np.abs(DY[:, j])) for j in range(N)])
+    ma = math.fsum(np.abs(G[None, :] * DY * sech2 * X).ravel())
+    return mg, mb, ma
+
+
+@pytest.mark.parametrize("M,N,alpha,seed", [(23, 11, 0.7, 1), (64, 5, 2.5, 2), (7, 40, 0.05, 3)])
+def test_sum_magnitudes_match_an_independent_fsum(M, N, alpha, seed):
+    x, dy, a, g, _ = _inputs(M, N, alpha=alpha, seed=seed)
+    r = oracle.backward(x, dy, a, g, M, N, "f32", "f32")
+    mg, mb, ma = _magnitudes_by_fsum(x, dy, a[0], g, M, N)
+    # index-order binary64 sums of at most 64 * 40 terms: within 1e-12 relative
+    np.testing.assert_allclose(r["mag_dgamma"], mg, rtol=1e-12, atol=0)
+    np.testing.assert_allclose(r["mag_dbeta"], mb, rtol=1e-12, atol=0)
+    assert abs(r["mag_dalpha"] - ma) <= 1e-12 * ma
+    # the triangle inequality: a magnitude never falls below its sum's absolute value
+    assert np.all(r["mag_dgamma"] >= np.abs(r["dgamma"]))
+    assert np.all(r["mag_dbeta"] >= np.abs(r["dbeta"]))
+    assert r["mag_dalpha"] >= abs(r["dalpha"])
+    # and with terms of both signs it lies strictly above it
+    assert np.all(r["mag_dbeta"] > np.abs(r["dbeta"]))
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+def test_sum_magnitudes_equal_the_sums_when_all_terms_share_a_sign(sign):
+    # x > 0, dy of one sign, gamma > 0, alpha > 0: every term of each sum has the
+    # sign of dy, so sum |term| and |sum term| add the same values in the same order.
+    M, N = 50, 9
+    x = np.abs(synth.normal(M * N, "f32", 0.0, 1.0, 21, 1, nonzero=True))
+    dy = (sign * np.abs(synth.normal(M * N, "f32", 0.0, 1.0, 21, 2, nonzero=True))).astype(np.float32)
+    g = np.abs(synth.normal(N, "f32", 1.0, 0.1, 21, 3)).astype(np.float32)
+    a = np.array([0.9], dtype=np.float32)
+    r = oracle.backward(x, dy, a, g, M, N, "f32", "f32")
+    assert np.array_equal(r["mag_dgamma"], np.abs(r["dgamma"]))
+    assert np.array_equal(r["mag_dbeta"], np.abs(r["dbeta"]))
+    assert r["mag_dalpha"] == abs(r["dalpha"])
+    assert np.all(np.sign(r["dbeta"]) == sign)

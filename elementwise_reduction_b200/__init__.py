@@ -13,15 +13,14 @@ from __future__ import annotations
 import torch
 
 from . import _abi
-from ._abi import (DYT_BF16, DYT_F16, DYT_F32, DytError, dyt_backward, dyt_backward_strided,
-                   dyt_backward_workspace_bytes, dyt_device_error, dyt_forward, dyt_forward_strided,
-                   dyt_last_launch_info, dyt_plan_query, dyt_selftest_wait_timeout, dyt_status_string)
+from ._abi import (DYT_BF16, DYT_F16, DYT_F32, DytError, dyt_backward, dyt_backward_ex, dyt_backward_noalloc,
+                   dyt_backward_strided, dyt_backward_workspace_bytes, dyt_forward, dyt_forward_ex,
+                   dyt_forward_strided, dyt_last_launch_info, dyt_plan_query, dyt_status_string)
 
 __all__ = ["forward", "backward", "workspace", "DyT", "DyTFunction", "dyt_forward", "dyt_backward",
-           "dyt_forward_strided", "dyt_backward_strided", "row_pitch",
-           "dyt_backward_workspace_bytes", "dyt_status_string", "dyt_last_launch_info", "dyt_plan_query",
-           "dyt_device_error", "dyt_selftest_wait_timeout", "DytError",
-           "DTYPE_CODE", "DYT_F32", "DYT_BF16", "DYT_F16"]
+           "dyt_forward_strided", "dyt_backward_strided", "dyt_forward_ex", "dyt_backward_ex",
+           "dyt_backward_noalloc", "row_pitch", "dyt_backward_workspace_bytes", "dyt_status_string",
+           "dyt_last_launch_info", "dyt_plan_query", "DytError", "DTYPE_CODE", "DYT_F32", "DYT_BF16", "DYT_F16"]
 
 DTYPE_CODE = {torch.float32: DYT_F32, torch.bfloat16: DYT_BF16, torch.float16: DYT_F16}
 
@@ -84,7 +83,8 @@ def _stream(device, stream):
 def forward(x: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
             out: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
     """y = gamma * tanh(alpha * x) + beta in x's dtype (one kernel launch). x and out
-    may be row-strided views (dense rows, evenly spaced): no copy is made."""
+    may be row-strided views (dense rows, evenly spaced): no copy is made. alpha,
+    gamma and beta may each have their own dtype."""
     for t, w in ((alpha, "alpha"), (gamma, "gamma"), (beta, "beta")):
         _cuda_contig(t, w)
     ldx = _rows(x, "x")
@@ -94,9 +94,9 @@ def forward(x: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor, beta: tor
         raise ValueError("out must match x in shape and dtype")
     ldy = _rows(y, "out")
     with torch.cuda.device(x.device):
-        st = dyt_forward_strided(x.data_ptr(), ldx, alpha.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
-                                 y.data_ptr(), ldy, M, N, _code(x, "x"), _code(gamma, "gamma"),
-                                 _stream(x.device, stream))
+        st = dyt_forward_ex(x.data_ptr(), ldx, alpha.data_ptr(), gamma.data_ptr(), beta.data_ptr(), y.data_ptr(),
+                            ldy, M, N, _code(x, "x"), _code(alpha, "alpha"), _code(gamma, "gamma"),
+                            _code(beta, "beta"), _stream(x.device, stream))
     _abi._check(st, "dyt_forward")
     return y
 
@@ -110,30 +110,40 @@ def workspace(x: torch.Tensor, gamma: torch.Tensor) -> torch.Tensor:
 
 
 def backward(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor,
-             dx: torch.Tensor | None = None, dgamma: torch.Tensor | None = None,
+             beta: torch.Tensor | None = None, dx: torch.Tensor | None = None, dgamma: torch.Tensor | None = None,
              dbeta: torch.Tensor | None = None, dalpha: torch.Tensor | None = None,
              ws: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None):
-    """(dx, dalpha, dgamma, dbeta): dx in x's dtype, the others in gamma's dtype.
-    x, dy and dx may be row-strided views (dense rows, evenly spaced)."""
+    """(dx, dalpha, dgamma, dbeta): dx in x's dtype and each parameter gradient in
+    its parameter's dtype (dbeta in beta's, or gamma's when beta is not given;
+    beta's values are not read). x, dy and dx may be row-strided views (dense
+    rows, evenly spaced)."""
     for t, w in ((alpha, "alpha"), (gamma, "gamma")):
         _cuda_contig(t, w)
+    if beta is not None:
+        _cuda_contig(beta, "beta")
     if dy.shape != x.shape or dy.dtype != x.dtype:
         raise ValueError("dy must match x in shape and dtype")
     ldx, lddy = _rows(x, "x"), _rows(dy, "dy")
     M, N = _shape(x, gamma)
+    beta_like = gamma if beta is None else beta
     dx = torch.empty(x.shape, dtype=x.dtype, device=x.device) if dx is None else dx
     if dx.shape != x.shape or dx.dtype != x.dtype:
         raise ValueError("dx must match x in shape and dtype")
     lddx = _rows(dx, "dx")
     dgamma = torch.empty_like(gamma) if dgamma is None else dgamma
-    dbeta = torch.empty_like(gamma) if dbeta is None else dbeta
-    dalpha = torch.empty(1, dtype=gamma.dtype, device=gamma.device) if dalpha is None else dalpha
+    dbeta = torch.empty_like(beta_like) if dbeta is None else dbeta
+    dalpha = torch.empty(1, dtype=alpha.dtype, device=alpha.device) if dalpha is None else dalpha
+    for t, like, w in ((dgamma, gamma, "dgamma"), (dbeta, beta_like, "dbeta"), (dalpha, alpha, "dalpha")):
+        if t.dtype != like.dtype or t.numel() != like.numel():
+            raise ValueError(f"{w} must match its parameter in size and dtype")
+        _cuda_contig(t, w)
     ws = workspace(x, gamma) if ws is None else ws
     with torch.cuda.device(x.device):
-        st = dyt_backward_strided(x.data_ptr(), ldx, dy.data_ptr(), lddy, alpha.data_ptr(), gamma.data_ptr(),
-                                  dx.data_ptr(), lddx, dgamma.data_ptr(), dbeta.data_ptr(), dalpha.data_ptr(), M,
-                                  N, _code(x, "x"), _code(gamma, "gamma"), ws.data_ptr(), ws.numel(),
-                                  _stream(x.device, stream))
+        st = dyt_backward_ex(x.data_ptr(), ldx, dy.data_ptr(), lddy, alpha.data_ptr(), gamma.data_ptr(),
+                             None if beta is None else beta.data_ptr(), dx.data_ptr(), lddx, dgamma.data_ptr(),
+                             dbeta.data_ptr(), dalpha.data_ptr(), M, N, _code(x, "x"), _code(alpha, "alpha"),
+                             _code(gamma, "gamma"), _code(beta_like, "beta"), ws.data_ptr(), ws.numel(),
+                             _stream(x.device, stream))
     _abi._check(st, "dyt_backward")
     return dx, dalpha, dgamma, dbeta
 
@@ -145,14 +155,14 @@ class DyTFunction(torch.autograd.Function):
     def forward(ctx, x, alpha, gamma, beta):
         alpha, gamma, beta = (t.contiguous() for t in (alpha, gamma, beta))
         x = x if row_pitch(x) is not None else x.contiguous()
-        ctx.save_for_backward(x, alpha, gamma)
+        ctx.save_for_backward(x, alpha, gamma, beta)
         return forward(x, alpha, gamma, beta)
 
     @staticmethod
     def backward(ctx, dy):
-        x, alpha, gamma = ctx.saved_tensors
+        x, alpha, gamma, beta = ctx.saved_tensors
         dy = dy if row_pitch(dy) is not None else dy.contiguous()
-        dx, dalpha, dgamma, dbeta = backward(x, dy, alpha, gamma)
+        dx, dalpha, dgamma, dbeta = backward(x, dy, alpha, gamma, beta)
         return dx, dalpha.reshape(alpha.shape), dgamma, dbeta
 
 
@@ -160,13 +170,15 @@ class DyT(torch.nn.Module):
     """DyT(x) = gamma * tanh(alpha * x) + beta over the last dimension.
 
     alpha is one scalar parameter; gamma and beta have one entry per channel.
-    Parameters live in ``param_dtype``; gradients come back in it.
+    gamma and beta live in ``param_dtype``, alpha in ``alpha_dtype`` (default:
+    ``param_dtype``); each gradient comes back in its parameter's dtype.
     """
 
     def __init__(self, num_features: int, alpha_init: float = 0.5, param_dtype=torch.float32,
-                 device=None):
+                 device=None, alpha_dtype=None):
         super().__init__()
-        self.alpha = torch.nn.Parameter(torch.full((1,), alpha_init, dtype=param_dtype, device=device))
+        alpha_dtype = param_dtype if alpha_dtype is None else alpha_dtype
+        self.alpha = torch.nn.Parameter(torch.full((1,), alpha_init, dtype=alpha_dtype, device=device))
         self.gamma = torch.nn.Parameter(torch.ones(num_features, dtype=param_dtype, device=device))
         self.beta = torch.nn.Parameter(torch.zeros(num_features, dtype=param_dtype, device=device))
 

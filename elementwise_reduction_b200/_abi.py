@@ -29,7 +29,7 @@ _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_s
 class LaunchInfo(ctypes.Structure):
     _fields_ = [("op", _i32), ("path", _i32), ("vec", _i32), ("block", _i32), ("grid", _i32),
                 ("row_lanes", _i32), ("rows_per_step", _i32), ("col_chunks", _i32),
-                ("row_groups", _i32), ("kernels", _i32), ("tma_stages", _i32), ("async_stages", _i32),
+                ("row_groups", _i32), ("kernels", _i32), ("async_stages", _i32),
                 ("pack_rows", _i32), ("workspace_bytes", _i64)]
 
     def as_dict(self) -> dict:
@@ -40,14 +40,18 @@ lib.dyt_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp
 lib.dyt_forward.restype = _i32
 lib.dyt_backward_workspace_bytes.argtypes = [_i64, _i64, _i32, _i32]
 lib.dyt_backward_workspace_bytes.restype = _sz
-lib.dyt_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _sz,
-                             _vp]
+lib.dyt_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _sz, _vp]
 lib.dyt_backward.restype = _i32
 lib.dyt_forward_strided.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _vp]
 lib.dyt_forward_strided.restype = _i32
-lib.dyt_backward_strided.argtypes = [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i32,
+lib.dyt_backward_strided.argtypes = [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i32,
                                      _i32, _vp, _sz, _vp]
 lib.dyt_backward_strided.restype = _i32
+lib.dyt_forward_ex.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _vp]
+lib.dyt_forward_ex.restype = _i32
+lib.dyt_backward_ex.argtypes = [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i32,
+                                _i32, _i32, _i32, _vp, _sz, _vp]
+lib.dyt_backward_ex.restype = _i32
 lib.dyt_status_string.argtypes = [_i32]
 lib.dyt_status_string.restype = ctypes.c_char_p
 lib.dyt_last_cuda_error.argtypes = []
@@ -56,13 +60,9 @@ lib.dyt_last_launch_info.argtypes = [ctypes.POINTER(LaunchInfo)]
 lib.dyt_last_launch_info.restype = _i32
 lib.dyt_plan_query.argtypes = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(LaunchInfo)]
 lib.dyt_plan_query.restype = _i32
-lib.dyt_backward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp]
+lib.dyt_backward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp]
 lib.dyt_backward_noalloc.restype = _i32
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # DYT_NOALLOC_SCRATCH_BYTES in include/dyt.h
-lib.dyt_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
-lib.dyt_device_error.restype = _i32
-lib.dyt_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp, _vp]
-lib.dyt_selftest_wait_timeout.restype = _i32
 
 
 class DytError(RuntimeError):
@@ -88,10 +88,10 @@ def dyt_backward_workspace_bytes(M, N, x_dtype, param_dtype) -> int:
     return int(lib.dyt_backward_workspace_bytes(M, N, x_dtype, param_dtype))
 
 
-def dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype, workspace,
+def dyt_backward(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype, workspace,
                  workspace_bytes, stream) -> int:
-    """Raw C-ABI call: pointers as ints. Returns the status code."""
-    return lib.dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
+    """Raw C-ABI call: pointers as ints (beta may be None). Returns the status code."""
+    return lib.dyt_backward(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
                             workspace, workspace_bytes, stream)
 
 
@@ -100,19 +100,34 @@ def dyt_forward_strided(x, ldx, alpha, gamma, beta, y, ldy, M, N, x_dtype, param
     return lib.dyt_forward_strided(x, ldx, alpha, gamma, beta, y, ldy, M, N, x_dtype, param_dtype, stream)
 
 
-def dyt_backward_strided(x, ldx, dy, lddy, alpha, gamma, dx, lddx, dgamma, dbeta, dalpha, M, N, x_dtype,
+def dyt_backward_strided(x, ldx, dy, lddy, alpha, gamma, beta, dx, lddx, dgamma, dbeta, dalpha, M, N, x_dtype,
                          param_dtype, workspace, workspace_bytes, stream) -> int:
     """Raw C-ABI call with row pitches (elements). Returns the status code."""
-    return lib.dyt_backward_strided(x, ldx, dy, lddy, alpha, gamma, dx, lddx, dgamma, dbeta, dalpha, M, N,
+    return lib.dyt_backward_strided(x, ldx, dy, lddy, alpha, gamma, beta, dx, lddx, dgamma, dbeta, dalpha, M, N,
                                     x_dtype, param_dtype, workspace, workspace_bytes, stream)
 
 
-def dyt_backward_noalloc(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
+def dyt_forward_ex(x, ldx, alpha, gamma, beta, y, ldy, M, N, x_dtype, alpha_dtype, gamma_dtype, beta_dtype,
+                   stream) -> int:
+    """Raw C-ABI call with row pitches and one dtype per parameter. Returns the status code."""
+    return lib.dyt_forward_ex(x, ldx, alpha, gamma, beta, y, ldy, M, N, x_dtype, alpha_dtype, gamma_dtype,
+                              beta_dtype, stream)
+
+
+def dyt_backward_ex(x, ldx, dy, lddy, alpha, gamma, beta, dx, lddx, dgamma, dbeta, dalpha, M, N, x_dtype,
+                    alpha_dtype, gamma_dtype, beta_dtype, workspace, workspace_bytes, stream) -> int:
+    """Raw C-ABI call with row pitches and one dtype per parameter (dalpha, dgamma and
+    dbeta come back in alpha_dtype, gamma_dtype, beta_dtype). Returns the status code."""
+    return lib.dyt_backward_ex(x, ldx, dy, lddy, alpha, gamma, beta, dx, lddx, dgamma, dbeta, dalpha, M, N, x_dtype,
+                               alpha_dtype, gamma_dtype, beta_dtype, workspace, workspace_bytes, stream)
+
+
+def dyt_backward_noalloc(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
                          stream) -> int:
     """Raw C-ABI call of the backward that uses the library's built-in scratch
     instead of a workspace (for callers that cannot allocate). Returns the status."""
-    return lib.dyt_backward_noalloc(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
-                                    stream)
+    return lib.dyt_backward_noalloc(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype,
+                                    param_dtype, stream)
 
 
 def dyt_status_string(status: int) -> str:
@@ -125,17 +140,6 @@ def dyt_plan_query(M, N, x_dtype, param_dtype, backward, vectorized, sm_count, c
     _check(lib.dyt_plan_query(M, N, x_dtype, param_dtype, int(backward), int(vectorized), sm_count,
                               ctas_per_sm, ctypes.byref(info)), "dyt_plan_query")
     return info.as_dict()
-
-
-def dyt_device_error(clear: bool = False) -> int:
-    """The sticky device error word of the current device (synchronises)."""
-    w = ctypes.c_uint(0)
-    _check(lib.dyt_device_error(ctypes.byref(w), int(clear)), "dyt_device_error")
-    return int(w.value)
-
-
-def dyt_selftest_wait_timeout(spin_limit: int, gave_up_ptr: int, stream) -> int:
-    return lib.dyt_selftest_wait_timeout(spin_limit, gave_up_ptr, stream)
 
 
 def dyt_last_launch_info() -> dict:

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdyt.so")
 SOURCES = [os.path.join(CSRC, "dyt_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_tma.cuh", "dyt_async.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_async.cuh")] + [
     os.path.join(INCLUDE, "dyt.h")]
 
 NVCC_FLAGS = [

@@ -1,6 +1,7 @@
 // C ABI of the fused DyT layer (declared in include/dyt.h): argument checks,
 // launch planning and kernel dispatch. All device work is in the kernels of
-// dyt_kernels.cuh, dyt_async.cuh and dyt_tma.cuh.
+// dyt_kernels.cuh and dyt_async.cuh.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -10,7 +11,6 @@
 
 #include "dyt.h"
 #include "dyt_kernels.cuh"
-#include "dyt_tma.cuh"
 #include "dyt_async.cuh"
 
 namespace {
@@ -20,65 +20,26 @@ using dyt::Geom;
 thread_local dyt_launch_info t_info = {};
 thread_local int t_cuda_err = 0;
 
-// Tuning constants (compile-time; -D overrides them for sweeps).
-#ifndef DYT_FWD_UNROLL_VEC
-#define DYT_FWD_UNROLL_VEC 2
-#endif
-#ifndef DYT_BWD_UNROLL_VEC
-#define DYT_BWD_UNROLL_VEC 2
-#endif
-#ifndef DYT_FWD_UNROLL_SCALAR
-#define DYT_FWD_UNROLL_SCALAR 8
-#endif
-#ifndef DYT_BWD_UNROLL_SCALAR
-#define DYT_BWD_UNROLL_SCALAR 8
-#endif
-// Pipeline of the 16-byte aligned path: 0 = loads into registers, 1 = CTA-wide
-// bulk-copy (TMA) ring, 2 = per-thread asynchronous-copy ring.
-#ifndef DYT_PIPE
-#define DYT_PIPE 2
-#endif
-#define DYT_USE_TMA (DYT_PIPE == 1)
-#ifndef DYT_ASYNC_STAGES_FWD
-#define DYT_ASYNC_STAGES_FWD 8
-#endif
-#ifndef DYT_ASYNC_STAGES_BWD
-#define DYT_ASYNC_STAGES_BWD 6
-#endif
-#ifndef DYT_TILE_BYTES
-#define DYT_TILE_BYTES 32768
-#endif
-#ifndef DYT_MAX_STAGES
-#define DYT_MAX_STAGES 8
-#endif
+constexpr int kScalarBlock = 1024;      // threads per CTA of the one-element kernels
+constexpr int kScalarUnrollFwd = 8;     // rows in flight per thread there
+constexpr int kScalarUnrollBwd = 8;
+constexpr int kAsyncBlock = 512;        // 16-byte kernels: one CTA per SM, up to 128 registers a thread
+constexpr int kAsyncStagesFwd = 8;      // ring slots per thread (forward: x)
+constexpr int kAsyncStagesBwd = 6;      // ring slots per thread (backward: x and dy)
+// Rows one lane adds per group, at most. The kernels count a thread's rows with
+// a multiply-high by ceil(2^32 / RL), exact for counts below 2^32 / RL; a
+// count stays below 2049 RL, and 2049 RL^2 < 2^32 for every RL <= 1024.
+constexpr int kMaxRowsPerLane = 2048;
 // Inputs read by one launch below which the L2 prefetch of the first rows is
-// skipped (bytes).
-#ifndef DYT_PREFETCH_MIN_BYTES
-#define DYT_PREFETCH_MIN_BYTES (1 << 20)
-#endif
-constexpr int kBlock = 1024;          // threads per CTA of the main kernels
-constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits (iterations)
-constexpr int kMaxDynSmem = 227 * 1024;
-#ifndef DYT_ASYNC_BLOCK
-#define DYT_ASYNC_BLOCK 512
-#endif
-constexpr int kAsyncBlock = DYT_ASYNC_BLOCK;  // one CTA per SM: up to 128 registers a thread
-constexpr int kAsyncStagesFwd = DYT_ASYNC_STAGES_FWD;
-constexpr int kAsyncStagesBwd = DYT_ASYNC_STAGES_BWD;
-constexpr int kMaxRowsPerLane = 128;  // sequential binary32 adds per thread per group
-constexpr int64_t kPrefetchMinBytes = DYT_PREFETCH_MIN_BYTES;
-
-constexpr int kFwdUnrollVec = DYT_FWD_UNROLL_VEC;        // rows in flight per thread, 16-byte access
-constexpr int kBwdUnrollVec = DYT_BWD_UNROLL_VEC;
-constexpr int kFwdUnrollScalar = DYT_FWD_UNROLL_SCALAR;  // rows in flight per thread, scalar access
-constexpr int kBwdUnrollScalar = DYT_BWD_UNROLL_SCALAR;
+// skipped (bytes): smaller inputs are likely resident in L2 already.
+constexpr int64_t kPrefetchMinBytes = 1 << 20;
 
 dyt_status cuda_fail(cudaError_t e) {
   t_cuda_err = (int)e;
   return DYT_ERR_CUDA;
 }
 
-size_t dsize(dyt_dtype d) { return d == DYT_F32 ? 4 : 2; }
+size_t dsize(int d) { return d == DYT_F32 ? 4 : 2; }
 bool valid_dtype(int d) { return d == DYT_F32 || d == DYT_BF16 || d == DYT_F16; }
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -88,6 +49,11 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 std::mutex g_mu;
 std::unordered_map<int, int> g_sms;                   // device -> SM count
 std::unordered_map<uint64_t, int> g_occ;              // (device, kernel) -> CTAs per SM
+std::unordered_map<uint64_t, int> g_smem_ready;       // (device, kernel) -> dynamic shared memory opted in
+
+uint64_t kernel_key(int dev, const void *kernel) {
+  return ((uint64_t)(uint32_t)dev << 48) ^ (uint64_t)(uintptr_t)kernel;
+}
 
 dyt_status current_sms(int *dev_out, int *sms_out) {
   int dev = 0;
@@ -113,7 +79,7 @@ dyt_status current_sms(int *dev_out, int *sms_out) {
 }
 
 dyt_status occupancy(int dev, const void *kernel, int block, int *ctas) {
-  const uint64_t key = ((uint64_t)(uint32_t)dev << 48) ^ (uint64_t)(uintptr_t)kernel;
+  const uint64_t key = kernel_key(dev, kernel);
   {
     std::lock_guard<std::mutex> lk(g_mu);
     auto it = g_occ.find(key);
@@ -132,21 +98,34 @@ dyt_status occupancy(int dev, const void *kernel, int block, int *ctas) {
   return DYT_OK;
 }
 
+// Opt a kernel in to `bytes` of dynamic shared memory, once per device.
+dyt_status prepare_smem(int dev, const void *kernel, int bytes) {
+  const uint64_t key = kernel_key(dev, kernel);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_smem_ready.find(key);
+    if (it != g_smem_ready.end() && it->second >= bytes) return DYT_OK;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_smem_ready[key] = bytes;
+  return DYT_OK;
+}
+
 // ---- launch plan ---------------------------------------------------------------
 
 struct Plan {
   Geom g;
-  int block;  // threads per CTA of the main kernel
-  int vec;
-  int unroll;
+  int block;    // threads per CTA of the main kernel
+  int vec;      // elements per access: 16 / element size, or 1 for the one-element kernels
+  int unroll;   // rows in flight per thread on the one-element kernels (1 on the 16-byte path)
   int grid;
-  int path;
-  bool tma;
-  bool async;
+  int path;     // 1 = row-tiled, 2 = row-per-CTA
+  bool async;   // the 16-byte per-thread copy rings
   bool packed;  // ragged N on 16-byte aligned rows: packs of vec rows (see dyt_kernels.cuh)
   bool too_big; // the group or item count would not fit the kernels' int indices
-  dyt::TmaGeom tg;
-  size_t smem;  // dynamic shared memory of the pipelined kernel
+  size_t smem;  // dynamic shared memory of the 16-byte kernel
   size_t ws_dg, ws_db, ws_da, ws_total;  // workspace byte offsets / sizes
 };
 
@@ -156,23 +135,26 @@ size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 // kernel's occupancy. packed: N is not a multiple of vec, and the matrix is
 // laid out as ceil(M / vec) packs of vec rows, each of pitch vec * N. The
 // plan depends only on (M, N, vec, packed, SM count, occupancy).
-Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, int sms, int ctas_per_sm,
-               int block = kBlock, bool packed = false, int64_t elem_bytes = 4) {
+Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool async, int sms, int ctas_per_sm,
+               bool packed, int64_t elem_bytes) {
   Plan p = {};
-  p.block = block;
+  p.block = async ? kAsyncBlock : kScalarBlock;
   p.vec = vec;
+  p.async = async;
   p.packed = packed;
+  const int block = p.block;
   const int64_t M = packed ? ceil_div(M_rows, (int64_t)vec) : M_rows;
   const int64_t N = packed ? (int64_t)vec * N_cols : N_cols;
-  p.unroll = backward ? (vec > 1 ? kBwdUnrollVec : kBwdUnrollScalar)
-                      : (vec > 1 ? kFwdUnrollVec : kFwdUnrollScalar);
+  p.unroll = async ? 1 : (backward ? kScalarUnrollBwd : kScalarUnrollFwd);
+  p.smem = !async ? 0
+                  : backward ? (size_t)kAsyncStagesBwd * 2 * kAsyncBlock * 16 : (size_t)kAsyncStagesFwd * kAsyncBlock * 16;
   const int64_t NV = N / vec;
   Geom &g = p.g;
   g.M = M;
   g.N = N;
   g.Nc = N_cols;
   g.total = M_rows * N_cols;
-  g.ldx = g.ldd = g.ldo = N;  // adjacent rows; the strided entry points override this
+  g.ldx = g.ldd = g.ldo = N;  // adjacent rows; the strided calls override this
   g.NV = (int)NV;
   if (NV <= block / 2) {
     g.RL = block / (int)NV;
@@ -191,8 +173,8 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, int sms, 
   const int64_t rows_per_lane_min = ceil_div(M, (int64_t)g.RL);
   if (fill > rows_per_lane_min) fill = rows_per_lane_min;
   int64_t nrg = fill;
-  // Cap the rows a lane adds in one group; keep the group count a multiple of
-  // the fill so every CTA gets the same number of items.
+  // Cap the rows a lane visits in one group; keep the group count a multiple
+  // of the fill so every CTA gets the same number of items.
   const int64_t max_rows = (int64_t)g.RL * kMaxRowsPerLane;
   if (ceil_div(M, nrg) > max_rows) nrg = ceil_div(ceil_div(M, max_rows), fill) * fill;
   // Shapes this large cannot be allocated on any device, but the plan must not
@@ -205,47 +187,18 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, int sms, 
   g.grem = M % nrg;
   g.nv_magic = NV >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)NV - 1) / (uint64_t)NV) : 0u;
   g.rl_magic = g.RL >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)g.RL - 1) / (uint64_t)g.RL) : 0u;
-  // L2 prefetch of the first rows (pipelined kernels): worth its issue cost
-  // only when the launch reads enough that its inputs are unlikely to be
-  // resident in L2 already and each CTA's first rows take a DRAM round trip
-  // or more; below kPrefetchMinBytes it is skipped.
   g.l2_prefetch = (int64_t)(backward ? 2 : 1) * M_rows * N_cols * elem_bytes >= kPrefetchMinBytes;
   int64_t grid = fill * g.ncc;
   if (grid > target) grid = target;
   if (grid > g.nitems) grid = g.nitems;
   p.grid = (int)grid;
+  // Workspace: binary64 partial sums of dgamma and dbeta per (group, row of a
+  // pack, column), and of dalpha per CTA.
   p.ws_dg = 0;
-  p.ws_db = align16((size_t)nrg * (size_t)N * sizeof(float));
-  p.ws_da = p.ws_db + align16((size_t)nrg * (size_t)N * sizeof(float));
+  p.ws_db = align16((size_t)nrg * (size_t)N * sizeof(double));
+  p.ws_da = p.ws_db + align16((size_t)nrg * (size_t)N * sizeof(double));
   p.ws_total = p.ws_da + align16((size_t)p.grid * sizeof(double));
   return p;
-}
-
-// Tiles of the pipelined kernels: about DYT_TILE_BYTES per stage, as many
-// stages as fit next to the kernel's static shared memory.
-void plan_tma(Plan &p, size_t elem, bool backward, int static_smem) {
-  const dyt::Geom &g = p.g;
-  const int64_t chunk_cols = g.ncc == 1 ? g.N : (int64_t)kBlock * p.vec;
-  dyt::TmaGeom &tg = p.tg;
-  tg.pitch = (int)(chunk_cols * (int64_t)elem);
-  const int ntensors = backward ? 2 : 1;
-  const int64_t per_u = (int64_t)g.RL * tg.pitch * ntensors;  // bytes per row per lane
-  int64_t U = DYT_TILE_BYTES / per_u;
-  if (U < 1) U = 1;
-  const int64_t rows_per_group = ceil_div(g.M, g.nrg);
-  const int64_t u_cap = ceil_div(rows_per_group, g.RL);
-  if (U > u_cap) U = u_cap;
-  if (U > kMaxRowsPerLane) U = kMaxRowsPerLane;
-  tg.U = (int)U;
-  tg.SR = g.RL * tg.U;
-  const int64_t stage = (int64_t)tg.SR * tg.pitch * ntensors;
-  int64_t S = (kMaxDynSmem - static_smem - 16 * DYT_MAX_STAGES - 64) / stage;
-  if (S > DYT_MAX_STAGES) S = DYT_MAX_STAGES;
-  tg.stages = (int)S;
-  tg.spin = kSpinLimit;
-  p.smem = (size_t)S * stage + 16 * S + 16;
-  p.tma = S >= 2;
-  p.unroll = tg.U;
 }
 
 // ---- kernel tables ---------------------------------------------------------------
@@ -255,44 +208,41 @@ constexpr int vec_of() {
   return 16 / (int)sizeof(T);
 }
 
-template <typename T, typename P>
-const void *fwd_kernel(int vec) {
-  if (vec > 1) return (const void *)dyt::dyt_fwd_kernel<T, P, vec_of<T>(), kFwdUnrollVec, kBlock>;
-  return (const void *)dyt::dyt_fwd_kernel<T, P, 1, kFwdUnrollScalar, kBlock>;
-}
-
-template <typename T, typename P>
-const void *bwd_kernel(int vec) {
-  if (vec > 1) return (const void *)dyt::dyt_bwd_kernel<T, P, vec_of<T>(), kBwdUnrollVec, kBlock>;
-  return (const void *)dyt::dyt_bwd_kernel<T, P, 1, kBwdUnrollScalar, kBlock>;
+template <typename T>
+const void *main_kernel(bool backward, bool async, bool packed) {
+  constexpr int V = vec_of<T>();
+  if (async) {
+    if (backward)
+      return packed ? (const void *)dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, true>
+                    : (const void *)dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, false>;
+    return packed ? (const void *)dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, true>
+                  : (const void *)dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, false>;
+  }
+  return backward ? (const void *)dyt::dyt_bwd_kernel<T, kScalarUnrollBwd, kScalarBlock>
+                  : (const void *)dyt::dyt_fwd_kernel<T, kScalarUnrollFwd, kScalarBlock>;
 }
 
 template <typename F>
-dyt_status with_types(dyt_dtype xd, dyt_dtype pd, F &&f) {
-  auto with_p = [&](auto tx) -> dyt_status {
-    using T = decltype(tx);
-    switch (pd) {
-      case DYT_F32: return f(T{}, float{});
-      case DYT_BF16: return f(T{}, __nv_bfloat16{});
-      case DYT_F16: return f(T{}, __half{});
-    }
-    return DYT_ERR_UNSUPPORTED_DTYPE;
-  };
+dyt_status with_xtype(int xd, F &&f) {
   switch (xd) {
-    case DYT_F32: return with_p(float{});
-    case DYT_BF16: return with_p(__nv_bfloat16{});
-    case DYT_F16: return with_p(__half{});
+    case DYT_F32: return f(float{});
+    case DYT_BF16: return f(__nv_bfloat16{});
+    case DYT_F16: return f(__half{});
   }
   return DYT_ERR_UNSUPPORTED_DTYPE;
 }
 
-dyt_status check_shape(int64_t M, int64_t N, dyt_dtype xd, dyt_dtype pd) {
-  if (!valid_dtype(xd) || !valid_dtype(pd)) return DYT_ERR_UNSUPPORTED_DTYPE;
+dyt_status check_shape(int64_t M, int64_t N, int xd) {
+  if (!valid_dtype(xd)) return DYT_ERR_UNSUPPORTED_DTYPE;
   if (M < 0 || N < 0 || N > INT32_MAX) return DYT_ERR_INVALID_VALUE;
   if (N > 0 && M > INT64_MAX / N / 8) return DYT_ERR_INVALID_VALUE;
   // group and item counts are ints
   if (M > ((int64_t)1 << 40)) return DYT_ERR_INVALID_VALUE;
   return DYT_OK;
+}
+
+dyt_status check_param_dtypes(int ad, int gd, int bd) {
+  return valid_dtype(ad) && valid_dtype(gd) && valid_dtype(bd) ? DYT_OK : DYT_ERR_UNSUPPORTED_DTYPE;
 }
 
 // Row pitches: at least N, and the last element of every tensor addressable.
@@ -320,7 +270,6 @@ dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
     i.rows_per_step = p->g.RL * p->unroll * i.pack_rows;
     i.col_chunks = p->g.ncc;
     i.row_groups = p->g.nrg;
-    i.tma_stages = p->tma ? p->tg.stages : 0;
     i.async_stages = p->async ? (op == 2 ? kAsyncStagesBwd : kAsyncStagesFwd) : 0;
   }
   return i;
@@ -328,106 +277,65 @@ dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
 
 void record(int op, const Plan *p, int kernels, size_t ws) { t_info = describe(op, p, kernels, ws); }
 
-// Columns per thread in the pipelined kernels (their shared-memory reads are
-// 4 elements wide; the bulk copies move whole rows regardless).
-constexpr int kTmaVec = 4;
-
-template <typename T, typename P>
-const void *tma_kernel(bool backward) {
-  return backward ? (const void *)dyt::dyt_bwd_tma_kernel<T, P, kTmaVec, kBlock>
-                  : (const void *)dyt::dyt_fwd_tma_kernel<T, P, kTmaVec, kBlock>;
-}
-
-template <typename T, typename P, bool PK>
-const void *async_kernel(bool backward) {
-  return backward ? (const void *)dyt::dyt_bwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesBwd, PK>
-                  : (const void *)dyt::dyt_fwd_async_kernel<T, P, vec_of<T>(), kAsyncBlock, kAsyncStagesFwd, PK>;
-}
-
-// Static shared memory of a kernel and, once, the opt-in to the largest
-// dynamic shared memory (cached per device and kernel).
-std::unordered_map<uint64_t, int> g_static_smem;
-
-dyt_status prepare_tma_kernel(int dev, const void *kernel, int *static_smem) {
-  const uint64_t key = ((uint64_t)(uint32_t)dev << 48) ^ (uint64_t)(uintptr_t)kernel;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    auto it = g_static_smem.find(key);
-    if (it != g_static_smem.end()) {
-      *static_smem = it->second;
-      return DYT_OK;
-    }
-  }
-  cudaFuncAttributes a;
-  cudaError_t e = cudaFuncGetAttributes(&a, kernel);
-  if (e != cudaSuccess) return cuda_fail(e);
-  const int dyn = kMaxDynSmem - (int)a.sharedSizeBytes;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-  if (e != cudaSuccess) return cuda_fail(e);
-  std::lock_guard<std::mutex> lk(g_mu);
-  g_static_smem[key] = (int)a.sharedSizeBytes;
-  *static_smem = (int)a.sharedSizeBytes;
-  return DYT_OK;
-}
-
-// Plan for given pointers' alignment on the current device.
 // Which kernels a call takes. aligned: every tensor starts on a 16-byte
 // boundary; pitched: every row pitch is a whole number of 16-byte vectors;
 // adjacent: every pitch is N. v: elements per 16-byte vector.
 struct PathChoice {
   bool packed;  // ragged N on adjacent rows: packs of v rows through the 16-byte kernels
-  int vec;      // elements per access: v, or 1 for the scalar kernels
-  bool tma;     // the CTA-wide bulk-copy pipeline (compile-time option)
-  bool async;   // the per-thread asynchronous-copy rings
+  bool async;   // the 16-byte kernels (per-thread copy rings)
+  int vec;      // elements per access: v, or 1 for the one-element kernels
 };
 
 PathChoice choose_path(int64_t N, int v, bool aligned, bool pitched, bool adjacent) {
   PathChoice c;
   // A pack of v adjacent rows is a whole number of vectors whatever N is.
-  c.packed = DYT_PIPE == 2 && aligned && adjacent && N % v != 0;
-  const bool vec_ok = aligned && (c.packed || (pitched && N % v == 0));
-  c.tma = DYT_USE_TMA && vec_ok && adjacent;
-  c.vec = vec_ok && (!DYT_USE_TMA || c.tma) ? v : 1;
-  c.async = DYT_PIPE == 2 && c.vec > 1;
+  c.packed = aligned && adjacent && N % v != 0;
+  c.async = aligned && (c.packed || (pitched && N % v == 0));
+  c.vec = c.async ? v : 1;
   return c;
 }
 
-// aligned, pitched, adjacent: as for choose_path.
-template <typename T, typename P>
+// The plan for tensors of type T with the given layout on the current device.
+template <typename T>
 dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjacent, bool backward, Plan *out) {
   int dev = 0, sms = 0;
   dyt_status st = current_sms(&dev, &sms);
   if (st != DYT_OK) return st;
-  // Ragged rows of an aligned matrix go through the asynchronous-copy
-  // kernels as packs; unaligned matrices take the scalar kernels.
   const PathChoice pc = choose_path(N, vec_of<T>(), aligned, pitched, adjacent);
-  const bool packed = pc.packed, use_tma = pc.tma, use_async = pc.async;
-  const int vec = pc.vec;
-  const void *k = use_tma     ? tma_kernel<T, P>(backward)
-                  : use_async ? (packed ? async_kernel<T, P, true>(backward) : async_kernel<T, P, false>(backward))
-                  : backward  ? bwd_kernel<T, P>(vec)
-                              : fwd_kernel<T, P>(vec);
+  const void *k = main_kernel<T>(backward, pc.async, pc.packed);
   int occ = 1;
-  int static_smem = 0;
-  if (use_tma || use_async) {
-    st = prepare_tma_kernel(dev, k, &static_smem);
+  if (pc.async) {
+    // One CTA per SM by construction (__launch_bounds__(B, 1), ring sized for it).
+    const Plan probe = make_plan(1, 1, pc.vec, backward, true, 1, 1, false, (int64_t)sizeof(T));
+    st = prepare_smem(dev, k, (int)probe.smem);
     if (st != DYT_OK) return st;
   } else {
-    st = occupancy(dev, k, kBlock, &occ);
+    st = occupancy(dev, k, kScalarBlock, &occ);
     if (st != DYT_OK) return st;
   }
-  *out = make_plan(M, N, use_tma ? kTmaVec : vec, backward, sms, occ, use_async ? kAsyncBlock : kBlock, packed,
-                   (int64_t)sizeof(T));
+  *out = make_plan(M, N, pc.vec, backward, pc.async, sms, occ, pc.packed, (int64_t)sizeof(T));
   if (out->too_big) return DYT_ERR_INVALID_VALUE;
-  out->tma = false;
-  out->async = use_async;
-  if (use_tma) plan_tma(*out, sizeof(T), backward, static_smem);
-  if (use_async) {
-    out->smem = backward ? (size_t)kAsyncStagesBwd * 2 * kAsyncBlock * 16 : (size_t)kAsyncStagesFwd * kAsyncBlock * 16;
-    out->unroll = 1;
-  }
   return DYT_OK;
 }
+
+// Programmatic dependent launch: the kernel may be scheduled while its
+// predecessor in the stream drains; its first instruction waits
+// (griddepcontrol.wait) for that predecessor, so stream order holds.
+struct PdlConfig {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg;
+  PdlConfig(unsigned grid, unsigned block, size_t smem, cudaStream_t s) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
 
 }  // namespace
 
@@ -436,13 +344,22 @@ extern "C" {
 dyt_status dyt_forward(const void *x, const void *alpha, const void *gamma, const void *beta, void *y,
                        int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
                        dyt_stream_t stream) {
-  return dyt_forward_strided(x, N, alpha, gamma, beta, y, N, M, N, x_dtype, param_dtype, stream);
+  return dyt_forward_ex(x, N, alpha, gamma, beta, y, N, M, N, x_dtype, param_dtype, param_dtype, param_dtype,
+                        stream);
 }
 
 dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, const void *gamma,
                                const void *beta, void *y, int64_t ldy, int64_t M, int64_t N,
                                dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream) {
-  dyt_status st = check_shape(M, N, x_dtype, param_dtype);
+  return dyt_forward_ex(x, ldx, alpha, gamma, beta, y, ldy, M, N, x_dtype, param_dtype, param_dtype, param_dtype,
+                        stream);
+}
+
+dyt_status dyt_forward_ex(const void *x, int64_t ldx, const void *alpha, const void *gamma, const void *beta,
+                          void *y, int64_t ldy, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype alpha_dtype,
+                          dyt_dtype gamma_dtype, dyt_dtype beta_dtype, dyt_stream_t stream) {
+  dyt_status st = check_shape(M, N, x_dtype);
+  if (st == DYT_OK) st = check_param_dtypes(alpha_dtype, gamma_dtype, beta_dtype);
   if (st != DYT_OK) return st;
   if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, ldy) != DYT_OK) return DYT_ERR_INVALID_VALUE;
   if (M == 0 || N == 0) {
@@ -450,51 +367,29 @@ dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, co
     return DYT_OK;
   }
   if (!x || !alpha || !gamma || !beta || !y) return DYT_ERR_INVALID_VALUE;
-  return with_types(x_dtype, param_dtype, [&](auto tx, auto tp) -> dyt_status {
+  const dyt::Params pr = {alpha, gamma, beta, (int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
+  return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
-    using P = decltype(tp);
     constexpr int V = vec_of<T>();
     Plan p;
-    dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y),
-                                  vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)), ldx == N && ldy == N,
-                                  false, &p);
+    dyt_status s = plan_for<T>(M, N, aligned16(x) && aligned16(y), vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)),
+                               ldx == N && ldy == N, false, &p);
     if (s != DYT_OK) return s;
     if (!p.packed) {
       p.g.ldx = ldx;
       p.g.ldo = ldy;
     }
-    // Programmatic dependent launch: the kernel may be scheduled while its
-    // predecessor in the stream drains; its first instruction waits
-    // (griddepcontrol.wait) for that predecessor, so stream order holds.
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(p.block);
-    cfg.stream = (cudaStream_t)stream;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
+    PdlConfig lc(p.grid, p.block, p.smem, (cudaStream_t)stream);
     cudaError_t e;
-    if (p.tma) {
-      cfg.dynamicSmemBytes = p.smem;
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_tma_kernel<T, P, kTmaVec, kBlock>, (const T *)x, (const P *)alpha,
-                             (const P *)gamma, (const P *)beta, (T *)y, p.g, p.tg);
-    } else if (p.async) {
-      cfg.dynamicSmemBytes = p.smem;
-      if (p.packed)
-        e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, true>,
-                               (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
-      else
-        e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, false>,
-                               (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
-    } else if (p.vec > 1)
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, V, kFwdUnrollVec, kBlock>,
-                             (const T *)x, (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y,
-                             p.g);
+    if (p.async && p.packed)
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, true>,
+                             (const T *)x, pr, (T *)y, p.g);
+    else if (p.async)
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, false>,
+                             (const T *)x, pr, (T *)y, p.g);
     else
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_fwd_kernel<T, P, 1, kFwdUnrollScalar, kBlock>, (const T *)x,
-                             (const P *)alpha, (const P *)gamma, (const P *)beta, (T *)y, p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_kernel<T, kScalarUnrollFwd, kScalarBlock>, (const T *)x, pr,
+                             (T *)y, p.g);
     if (e != cudaSuccess) return cuda_fail(e);
     record(1, &p, 1, 0);
     return DYT_OK;
@@ -502,16 +397,15 @@ dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, co
 }
 
 size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype) {
-  if (check_shape(M, N, x_dtype, param_dtype) != DYT_OK) return 0;
+  if (check_shape(M, N, x_dtype) != DYT_OK || !valid_dtype(param_dtype)) return 0;
   if (M == 0 || N == 0) return 0;
   size_t need = 0;
-  dyt_status st = with_types(x_dtype, param_dtype, [&](auto tx, auto tp) -> dyt_status {
+  dyt_status st = with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
-    using P = decltype(tp);
-    // The vectorised and the scalar plan may differ; cover both.
+    // The 16-byte and the one-element plan may differ; cover both.
     for (int v = 0; v < 2; ++v) {
       Plan p;
-      dyt_status s = plan_for<T, P>(M, N, v == 1, v == 1, true, true, &p);
+      dyt_status s = plan_for<T>(M, N, v == 1, v == 1, true, true, &p);
       if (s != DYT_OK) return s;
       if (p.ws_total > need) need = p.ws_total;
     }
@@ -520,48 +414,60 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
   return st == DYT_OK ? need : 0;
 }
 
-dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const void *gamma, void *dx,
-                        void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
-                        dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace,
-                        size_t workspace_bytes, dyt_stream_t stream) {
-  return dyt_backward_strided(x, N, dy, N, alpha, gamma, dx, N, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
-                              workspace, workspace_bytes, stream);
+dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const void *gamma, const void *beta,
+                        void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
+                        dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace, size_t workspace_bytes,
+                        dyt_stream_t stream) {
+  return dyt_backward_ex(x, N, dy, N, alpha, gamma, beta, dx, N, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype,
+                         param_dtype, param_dtype, workspace, workspace_bytes, stream);
 }
 
 dyt_status dyt_backward_strided(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
-                                const void *gamma, void *dx, int64_t lddx, void *dgamma, void *dbeta,
-                                void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
-                                void *workspace, size_t workspace_bytes, dyt_stream_t stream) {
-  dyt_status st = check_shape(M, N, x_dtype, param_dtype);
+                                const void *gamma, const void *beta, void *dx, int64_t lddx, void *dgamma,
+                                void *dbeta, void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype,
+                                dyt_dtype param_dtype, void *workspace, size_t workspace_bytes,
+                                dyt_stream_t stream) {
+  return dyt_backward_ex(x, ldx, dy, lddy, alpha, gamma, beta, dx, lddx, dgamma, dbeta, dalpha, M, N, x_dtype,
+                         param_dtype, param_dtype, param_dtype, workspace, workspace_bytes, stream);
+}
+
+dyt_status dyt_backward_ex(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
+                           const void *gamma, const void *beta, void *dx, int64_t lddx, void *dgamma, void *dbeta,
+                           void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype alpha_dtype,
+                           dyt_dtype gamma_dtype, dyt_dtype beta_dtype, void *workspace, size_t workspace_bytes,
+                           dyt_stream_t stream) {
+  (void)beta;  // the gradients do not depend on beta; only its dtype (beta_dtype) is used
+  dyt_status st = check_shape(M, N, x_dtype);
+  if (st == DYT_OK) st = check_param_dtypes(alpha_dtype, gamma_dtype, beta_dtype);
   if (st != DYT_OK) return st;
   if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, lddy) != DYT_OK || check_pitch(M, N, lddx) != DYT_OK)
     return DYT_ERR_INVALID_VALUE;
   if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return DYT_ERR_INVALID_VALUE;
   cudaStream_t s = (cudaStream_t)stream;
-  const size_t ps = dsize(param_dtype);
   if (M == 0 || N == 0) {
     // Empty sums: every gradient is +0 (all-zero bits in each dtype).
     cudaError_t e = cudaSuccess;
     if (N > 0) {
-      e = cudaMemsetAsync(dgamma, 0, (size_t)N * ps, s);
-      if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, (size_t)N * ps, s);
+      e = cudaMemsetAsync(dgamma, 0, (size_t)N * dsize(gamma_dtype), s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, (size_t)N * dsize(beta_dtype), s);
     }
-    if (e == cudaSuccess) e = cudaMemsetAsync(dalpha, 0, ps, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dalpha, 0, dsize(alpha_dtype), s);
     if (e != cudaSuccess) return cuda_fail(e);
     record(2, nullptr, 0, 0);
     return DYT_OK;
   }
   if (!x || !dy || !alpha || !gamma || !dx || !workspace) return DYT_ERR_INVALID_VALUE;
   if (!aligned16(workspace)) return DYT_ERR_INVALID_VALUE;
-  return with_types(x_dtype, param_dtype, [&](auto tx, auto tp) -> dyt_status {
+  const dyt::Params pr = {alpha, gamma, nullptr, (int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
+  const dyt::GradOut go = {dgamma, dbeta, dalpha, (int)gamma_dtype, (int)beta_dtype, (int)alpha_dtype};
+  return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
-    using P = decltype(tp);
     constexpr int V = vec_of<T>();
     Plan p;
     const size_t es = sizeof(T);
-    dyt_status r = plan_for<T, P>(M, N, aligned16(x) && aligned16(dy) && aligned16(dx),
-                                  vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es),
-                                  ldx == N && lddy == N && lddx == N, true, &p);
+    dyt_status r = plan_for<T>(M, N, aligned16(x) && aligned16(dy) && aligned16(dx),
+                               vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es),
+                               ldx == N && lddy == N && lddx == N, true, &p);
     if (r != DYT_OK) return r;
     if (!p.packed) {
       p.g.ldx = ldx;
@@ -570,42 +476,21 @@ dyt_status dyt_backward_strided(const void *x, int64_t ldx, const void *dy, int6
     }
     if (workspace_bytes < p.ws_total) return DYT_ERR_WORKSPACE_TOO_SMALL;
     char *ws = (char *)workspace;
-    float *pdg = (float *)(ws + p.ws_dg);
-    float *pdb = (float *)(ws + p.ws_db);
+    double *pdg = (double *)(ws + p.ws_dg);
+    double *pdb = (double *)(ws + p.ws_db);
     double *pda = (double *)(ws + p.ws_da);
 
-    cudaLaunchAttribute pdl[1];  // see dyt_forward
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(p.block);
-    cfg.stream = s;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
+    PdlConfig lc(p.grid, p.block, p.smem, s);
     cudaError_t e;
-    if (p.tma) {
-      cfg.dynamicSmemBytes = p.smem;
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_tma_kernel<T, P, kTmaVec, kBlock>, (const T *)x, (const T *)dy,
-                             (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda, p.g, p.tg);
-    } else if (p.async) {
-      cfg.dynamicSmemBytes = p.smem;
-      if (p.packed)
-        e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, true>,
-                               (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb,
-                               pda, p.g);
-      else
-        e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, false>,
-                               (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb,
-                               pda, p.g);
-    } else if (p.vec > 1)
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, V, kBwdUnrollVec, kBlock>,
-                             (const T *)x, (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx,
-                             pdg, pdb, pda, p.g);
+    if (p.async && p.packed)
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, true>,
+                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
+    else if (p.async)
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, false>,
+                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
     else
-      e = cudaLaunchKernelEx(&cfg, dyt::dyt_bwd_kernel<T, P, 1, kBwdUnrollScalar, kBlock>, (const T *)x,
-                             (const T *)dy, (const P *)alpha, (const P *)gamma, (T *)dx, pdg, pdb, pda,
-                             p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_kernel<T, kScalarUnrollBwd, kScalarBlock>, (const T *)x,
+                             (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
     if (e != cudaSuccess) return cuda_fail(e);
 
     // Stage 2, as a programmatic dependent launch: it may start while stage 1
@@ -617,18 +502,9 @@ dyt_status dyt_backward_strided(const void *x, int64_t ldx, const void *dy, int6
     int L = 1;
     while (L < dyt::kFinThreads && (int64_t)L * 4 < nparts) L <<= 1;
     const int CT = dyt::kFinThreads / L;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t fcfg = {};
-    fcfg.gridDim = dim3((unsigned)ceil_div(N, CT));
-    fcfg.blockDim = dim3(dyt::kFinThreads);
-    fcfg.stream = s;
-    fcfg.attrs = attr;
-    fcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&fcfg, dyt::dyt_finalize_kernel<P>, (const float *)pdg, (const float *)pdb,
-                           (const double *)pda, (P *)dgamma, (P *)dbeta, (P *)dalpha, (int64_t)N,
-                           nparts, p.grid, CT);
+    PdlConfig fc((unsigned)ceil_div(N, CT), dyt::kFinThreads, 0, s);
+    e = cudaLaunchKernelEx(&fc.cfg, dyt::dyt_finalize_kernel, (const double *)pdg, (const double *)pdb,
+                           (const double *)pda, go, (int64_t)N, nparts, p.grid, CT);
     if (e != cudaSuccess) return cuda_fail(e);
     record(2, &p, 2, p.ws_total);
     return DYT_OK;
@@ -648,30 +524,11 @@ const char *dyt_status_string(dyt_status status) {
 
 int dyt_last_cuda_error(void) { return t_cuda_err; }
 
-dyt_status dyt_device_error(unsigned int *word, int clear) {
-  if (!word) return DYT_ERR_INVALID_VALUE;
-  cudaError_t e = cudaMemcpyFromSymbol(word, dyt::g_dyt_device_error, sizeof(unsigned int));
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (clear) {
-    const unsigned int zero = 0;
-    e = cudaMemcpyToSymbol(dyt::g_dyt_device_error, &zero, sizeof(unsigned int));
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  return DYT_OK;
-}
-
-dyt_status dyt_selftest_wait_timeout(unsigned int spin_limit, int *gave_up, dyt_stream_t stream) {
-  if (!gave_up || spin_limit == 0) return DYT_ERR_INVALID_VALUE;
-  dyt::dyt_wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(spin_limit, gave_up);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
-  return DYT_OK;
-}
-
 dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype, int backward,
                           int vectorized, int sm_count, int ctas_per_sm, dyt_launch_info *out) {
   if (!out || sm_count < 1 || ctas_per_sm < 1) return DYT_ERR_INVALID_VALUE;
-  dyt_status st = check_shape(M, N, x_dtype, param_dtype);
+  dyt_status st = check_shape(M, N, x_dtype);
+  if (st == DYT_OK && !valid_dtype(param_dtype)) st = DYT_ERR_UNSUPPORTED_DTYPE;
   if (st != DYT_OK) return st;
   const int op = backward ? 2 : 1;
   if (M == 0 || N == 0) {
@@ -680,15 +537,10 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
   }
   const int v = 16 / (int)dsize(x_dtype);
   const PathChoice pc = choose_path(N, v, vectorized != 0, vectorized != 0, true);  // adjacent rows
-  const bool packed = pc.packed, use_tma = pc.tma, use_async = pc.async;
-  const int vec = pc.vec;
-  Plan p = make_plan(M, N, use_tma ? kTmaVec : vec, backward != 0, sm_count, ctas_per_sm,
-                     use_async ? kAsyncBlock : kBlock, packed, (int64_t)dsize(x_dtype));
+  // The 16-byte kernels always run one CTA per SM.
+  Plan p = make_plan(M, N, pc.vec, backward != 0, pc.async, sm_count, pc.async ? 1 : ctas_per_sm, pc.packed,
+                     (int64_t)dsize(x_dtype));
   if (p.too_big) return DYT_ERR_INVALID_VALUE;
-  p.tma = false;
-  p.async = use_async;
-  if (p.async) p.unroll = 1;
-  if (use_tma) plan_tma(p, dsize(x_dtype), backward != 0, backward ? 17 * 1024 : 256);
   *out = describe(op, &p, backward ? 2 : 1, backward ? p.ws_total : 0);
   return DYT_OK;
 }
@@ -707,30 +559,69 @@ dyt_status dyt_last_launch_info(dyt_launch_info *out) {
 // application owning all device memory, or loops that cannot afford
 // cudaMalloc's implicit synchronisation): the scratch is a fixed file-scope
 // device array. Host code only ever sees a stand-in for its name, so the
-// device address is looked up with cudaGetSymbolAddress, once per device,
-// with that device current, and handed to the kernels.
+// device address is looked up with cudaGetSymbolAddress, with the device
+// current, and handed to the kernels. The lookup runs once per device context
+// and is cached under the driver's unique context id, so a context that
+// cudaDeviceReset ended, and the fresh one that replaces it, never share an
+// address.
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_dyt_noalloc_scratch[DYT_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_noalloc_mu;
-std::unordered_map<int, void *> g_noalloc_ptr;  // device -> address of the array
+std::unordered_map<uint64_t, void *> g_noalloc_ptr;  // context id -> address of the array
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// The driver's unique id of the current context, in *id; false when no
+// context is current yet or the driver cannot say.
+bool context_id(uint64_t *id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = (CtxGetCurrentFn)f;
+    f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (CtxGetIdFn)f;
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long v = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &v) != CUDA_SUCCESS)
+    return false;
+  *id = (uint64_t)v;
+  return true;
+}
+
+// The array's device address in the current context. Looked up once per
+// context; without a context id (no context current yet, or a driver that
+// cannot name it) the lookup runs and is cached only once the id is known.
 dyt_status noalloc_scratch(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  auto it = g_noalloc_ptr.find(dev);
-  if (it != g_noalloc_ptr.end()) {
-    *out = it->second;
-    return DYT_OK;
+  uint64_t id = 0;
+  bool known = context_id(&id);
+  if (known) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    auto it = g_noalloc_ptr.find(id);
+    if (it != g_noalloc_ptr.end()) {
+      *out = it->second;
+      return DYT_OK;
+    }
   }
   void *p = nullptr;
-  e = cudaGetSymbolAddress(&p, g_dyt_noalloc_scratch);
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_dyt_noalloc_scratch);  // also creates the context if needed
   if (e != cudaSuccess) return cuda_fail(e);
-  g_noalloc_ptr[dev] = p;
+  if (!known) known = context_id(&id);
+  if (known) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    g_noalloc_ptr[id] = p;
+  }
   *out = p;
   return DYT_OK;
 }
@@ -738,14 +629,22 @@ dyt_status noalloc_scratch(void **out) {
 }  // namespace
 
 extern "C" dyt_status dyt_backward_noalloc(const void *x, const void *dy, const void *alpha, const void *gamma,
-                                           void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M,
-                                           int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
+                                           const void *beta, void *dx, void *dgamma, void *dbeta, void *dalpha,
+                                           int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
                                            dyt_stream_t stream) {
+  // Shape and dtype errors, and empty shapes (which need no scratch), are
+  // settled before the scratch is looked up.
+  dyt_status st = check_shape(M, N, x_dtype);
+  if (st == DYT_OK && !valid_dtype(param_dtype)) st = DYT_ERR_UNSUPPORTED_DTYPE;
+  if (st != DYT_OK) return st;
+  if (M == 0 || N == 0)
+    return dyt_backward(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype, nullptr,
+                        0, stream);
   void *scratch = nullptr;
-  const dyt_status st = noalloc_scratch(&scratch);
+  st = noalloc_scratch(&scratch);
   if (st != DYT_OK) return st;
   // dyt_backward checks the arguments and rejects, before launching, a shape
   // whose scratch need exceeds the array (DYT_ERR_WORKSPACE_TOO_SMALL).
-  return dyt_backward(x, dy, alpha, gamma, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype, scratch,
+  return dyt_backward(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype, scratch,
                       DYT_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -1,8 +1,10 @@
-// Per-thread asynchronous-copy DyT kernels for sm_100a (16-byte vectors).
+// Per-thread asynchronous-copy DyT kernels for sm_100a (16-byte vectors): the
+// kernels every 16-byte aligned matrix takes.
 //
-// Same decomposition, thread mapping and arithmetic as the register-path
-// kernels in dyt_kernels.cuh; the row lanes of a CTA are added in a different
-// (also fixed) order when NV divides 32. Each thread streams the rows it owns
+// Same decomposition, thread mapping and arithmetic as the one-element
+// kernels in dyt_kernels.cuh; the row lanes of a CTA are added by a register
+// reduce-scatter when NV divides 32, otherwise by the same fixed-order tree.
+// Each thread streams the rows it owns
 // (its VEC columns of rows rl, rl + RL, ... of the group) into a private ring
 // of S shared-memory slots with 16-byte asynchronous copies (cp.async.cg, L2
 // only), S - 1 rows ahead of the row it computes, and reads each slot back
@@ -109,8 +111,9 @@ __device__ __forceinline__ void prefetch_first_rows_l2(const T *p, int64_t ld, c
 }
 
 // Rows of the current item owned by this thread: first row and count. A group
-// has at most 128 RL rows (the host caps it), so the quotient is formed with
-// the host's multiply-high constant, exactly, instead of a 64-bit division.
+// has at most kMaxRowsPerLane * RL rows (the host caps it), so the quotient is
+// formed with the host's multiply-high constant, exactly, instead of a 64-bit
+// division.
 __device__ __forceinline__ int64_t thread_rows(const Geom &g, int64_t rb, int64_t re, int rl, int64_t &first) {
   first = rb + rl;
   if (first >= re) return 0;
@@ -140,17 +143,16 @@ __device__ __forceinline__ int last_vector_real(const Geom &g, int64_t first, in
   return r < VEC ? (int)r : VEC;
 }
 
-template <typename T, typename P, int VEC, int B, int S, bool PK>
+template <typename T, int VEC, int B, int S, bool PK>
 __global__ void __launch_bounds__(B, 1)
-    dyt_fwd_async_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma,
-                         const P *__restrict__ beta, T *y, Geom g) {
+    dyt_fwd_async_kernel(const T *__restrict__ x, Params pr, T *y, Geom g) {
   using IO = VecIO<T, VEC>;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
   extern __shared__ uint4 ring[];  // [S][B]
   prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = param(alpha_p, 0);
+  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
   uint4 *slot0 = ring + threadIdx.x;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(B, 1)
     int64_t col[VEC];
     vector_columns<VEC, PK>(c0, g.Nc, col);
     float gam[VEC], bet[VEC], bth[VEC];
-    fwd_params_at<T, P, VEC>(gamma, beta, col, gam, bet, bth);
+    fwd_params_at<T, VEC>(pr, col, gam, bet, bth);
     int s_rd = 0, s_wr = S - 1;
     for (int64_t k = 0; k < n; ++k) {
       const int64_t kn = k + S - 1;
@@ -203,24 +205,25 @@ __global__ void __launch_bounds__(B, 1)
 
 // ---- backward, stage 1 ----------------------------------------------------------
 
-template <typename T, typename P, int VEC, int B, int S, bool PK>
+template <typename T, int VEC, int B, int S, bool PK>
 __global__ void __launch_bounds__(B, 1)
-    dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
-                         const P *__restrict__ gamma, T *dx, float *__restrict__ part_dg,
-                         float *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
+    dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, Params pr, T *dx,
+                         double *__restrict__ part_dg, double *__restrict__ part_db, double *__restrict__ part_da,
+                         Geom g) {
   using IO = VecIO<T, VEC>;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
-  static_assert(2 * VEC * sizeof(float) <= 2 * S * 16, "the reduction fits in the drained ring");
+  static_assert(2 * VEC * sizeof(double) <= 2 * S * 16, "the reduction fits in the drained ring");
   // [S][2][B] 16-byte slots; after an item's last row the ring is empty and
-  // its first 2 VEC * B floats (at most 32 KB) serve the row-lane reduction.
+  // its first 2 VEC * B binary64 values (at most 64 KB) serve the row-lane
+  // reduction.
   extern __shared__ uint4 ring[];
   __shared__ double red_a[B / 32];
   prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
   prefetch_first_rows_l2<T, VEC, B, S, PK>(dy, g.ldd, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = param(alpha_p, 0);
-  float *red = reinterpret_cast<float *>(ring);
+  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
+  double *red = reinterpret_cast<double *>(ring);
   uint4 *slot0 = ring + threadIdx.x;
   double acc_a = 0.0;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
@@ -235,15 +238,15 @@ __global__ void __launch_bounds__(B, 1)
     BwdAcc<VEC> acc;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      acc.g[e] = 0.0f;
-      acc.b[e] = 0.0f;
+      acc.g[e] = 0.0;
+      acc.b[e] = 0.0;
     }
     if (col_ok) {
       int64_t first;
       int64_t n = thread_rows(g, rb, re, ln.rl, first);
       const int nl = last_vector_real<VEC, PK>(g, first, c0, n);
       const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
-      const int nn = (int)n;  // at most 128: the host caps a group at 128 rows per lane
+      const int nn = (int)n;  // at most kMaxRowsPerLane: the host caps a group's rows per lane
       const int64_t sx = (int64_t)g.RL * g.ldx, sd = (int64_t)g.RL * g.ldd, so = (int64_t)g.RL * g.ldo;
       const T *px = x + first * g.ldx + c0;  // the next rows to copy (advanced, not re-derived)
       const T *pd = dy + first * g.ldd + c0;
@@ -270,7 +273,7 @@ __global__ void __launch_bounds__(B, 1)
       int64_t col[VEC];
       vector_columns<VEC, PK>(c0, g.Nc, col);
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) gam[e] = 4.0f * param(gamma, col[e]);  // 4 gamma (see bwd_vector)
+      for (int e = 0; e < VEC; ++e) gam[e] = 4.0f * load_param(pr.gamma, pr.gamma_dt, col[e]);  // see bwd_vector
       for (int k0 = 0; k0 < nn; k0 += S) {
 #pragma unroll
         for (int j = 0; j < S; ++j) {
@@ -307,8 +310,8 @@ __global__ void __launch_bounds__(B, 1)
       cp_async_wait<0>();
     }
     // ---- item done: per-(group, column) partials ----
-    float *pg = part_dg + (int64_t)rg * g.N;
-    float *pb = part_db + (int64_t)rg * g.N;
+    double *pg = part_dg + (int64_t)rg * g.N;
+    double *pb = part_db + (int64_t)rg * g.N;
     if (g.RL == 1) {
       if (col_ok) {
 #pragma unroll
@@ -322,7 +325,7 @@ __global__ void __launch_bounds__(B, 1)
       if ((32 % g.NV) == 0) {
         // the chunk's columns start at 0 on the row-tiled path (one chunk)
         lane_reduce_warps<VEC, B>(acc.g, acc.b, red, g, ln, 0, pg, pb);
-      } else {  // dgamma and dbeta sums in one tree: 2 VEC floats per thread
+      } else {  // dgamma and dbeta sums in one tree: 2 VEC values per thread
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
           red[e * B + threadIdx.x] = acc.g[e];

@@ -1,10 +1,12 @@
-// Fused DyT forward / backward kernels for sm_100a.
+// Fused DyT forward / backward for sm_100a: the pieces every kernel shares,
+// the kernels for matrices that are not 16-byte aligned (one element per
+// access), and the finalize of the backward.
 //
 // Work decomposition (one 1D persistent grid, the page's Summary "Launch
 // limit": rows never sit on grid dimension 1, so M is unbounded):
 //   - a thread owns one vector-column cv (VEC consecutive columns; VEC = 16
-//     bytes / element size, or 1 for unaligned rows) and keeps its
-//     gamma/beta in registers;
+//     bytes / element size on the 16-byte path, 1 here) and keeps its gamma
+//     and beta in registers;
 //   - packed rows (16-byte aligned matrix, N not a multiple of VEC): VEC
 //     consecutive rows always span exactly N 16-byte vectors, so such a pack
 //     is treated as one row of pitch VEC * N with NV = N vector-columns; the
@@ -13,20 +15,20 @@
 //     fewer than VEC rows: its vectors past the matrix are not read, and the
 //     one vector that straddles the end is zero-filled and masked;
 //   - row-tiled path (NV = N / VEC <= B / 2, the page's narrow rows): RL =
-//     B / NV row lanes share a CTA step, so one step covers RL * U whole rows
+//     B / NV row lanes share a CTA step, so one step covers RL whole rows
 //     (the page's Summary "Small widths": several rows per tile);
 //   - row-per-CTA path (wider rows): RL = 1, every thread works on every row
-//     of the CTA, columns spread across threads; rows wider than B * VEC are
-//     split into column chunks;
+//     of the CTA's group, columns spread across threads; rows wider than
+//     B * VEC are split into column chunks;
 //   - rows are cut into nrg balanced contiguous groups; a work item is
 //     (column chunk, row group) and CTA b takes items b, b + grid, ... (a
 //     static schedule: the same inputs always give the same bits).
-// Backward sums: each thread accumulates its columns in binary32 over at most
-// 128 rows per group (the host sizes the groups so), the
-// row lanes of a CTA are added by a fixed-order tree in shared memory, and
-// each (group, column) partial goes to the workspace; dalpha is carried in
-// binary64 per thread, reduced per CTA in a fixed order. The finalize kernel
-// adds the partials in binary64 in a fixed order.
+// Backward sums: each thread accumulates dgamma and dbeta of its columns in
+// binary64 (the product dy * t is exact there), the row lanes of a CTA are
+// added in binary64 in a fixed order, and each (group, column) partial goes
+// to the workspace in binary64; dalpha is carried in binary64 per thread and
+// reduced per CTA in a fixed order. The finalize adds the partials in
+// binary64 in a fixed order and rounds each gradient once.
 // Lanes outside [0,M) x [0,N) never enter a sum: their contribution is
 // dropped by a select after the arithmetic (the page's Summary, "Padding").
 #pragma once
@@ -54,7 +56,28 @@ struct Geom {
   int64_t grem;   // M % nrg
   uint32_t nv_magic;  // ceil(2^32 / NV) for NV >= 2: tid / NV = umulhi(tid, nv_magic), tid < 1024
   uint32_t rl_magic;  // ceil(2^32 / RL) for RL >= 2: n / RL = umulhi(n, rl_magic) for n < 2^32 / RL
-  int l2_prefetch;    // the pipelined kernels prefetch their first rows into L2 (large inputs only)
+  int l2_prefetch;    // the 16-byte kernels prefetch their first rows into L2 (large inputs only)
+};
+
+// The parameters, each with its own dtype (dyt_dtype codes). beta is read by
+// the forward only.
+struct Params {
+  const void *alpha;
+  const void *gamma;
+  const void *beta;
+  int alpha_dt;
+  int gamma_dt;
+  int beta_dt;
+};
+
+// Where the finalize writes the parameter gradients, each in its parameter's dtype.
+struct GradOut {
+  void *dgamma;
+  void *dbeta;
+  void *dalpha;
+  int gamma_dt;
+  int beta_dt;
+  int alpha_dt;
 };
 
 // Rows [begin, end) of group rg when [0, M) is cut into nrg balanced groups.
@@ -76,24 +99,10 @@ __device__ __forceinline__ void item_split(const Geom &g, int item, int &cc, int
 
 // ---- global memory access --------------------------------------------------
 
-// Streaming 16-byte load through the non-coherent path, not kept in L1.
-__device__ __forceinline__ uint4 ld_stream16(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ void st16(void *p, const uint4 &v) {
   asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
-}
-
-template <typename T>
-__device__ __forceinline__ T ld_scalar(const T *p) {
-  return __ldg(p);
 }
 
 // VEC elements of T as raw storage, with float conversion.
@@ -104,10 +113,9 @@ template <typename T>
 struct VecIO<T, 1> {
   using Raw = T;
   static constexpr int kPairs = 0;
-  static __device__ __forceinline__ Raw load(const T *p) { return ld_scalar(p); }
+  static __device__ __forceinline__ Raw load(const T *p) { return __ldg(p); }
   static __device__ __forceinline__ Raw zero() { return from_f32<T>(0.0f); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[1]) { f[0] = to_f32<T>(r); }
-  static __device__ __forceinline__ void store(T *p, const float (&f)[1]) { *p = from_f32<T>(f[0]); }
   static __device__ __forceinline__ void set(Raw &r, int, T v) { r = v; }
   static __device__ __forceinline__ Raw pack(const float (&f)[1]) { return from_f32<T>(f[0]); }
   static __device__ __forceinline__ void store_raw(T *p, const Raw &r) { *p = r; }
@@ -125,17 +133,11 @@ struct VecIO<float, 4> {
     return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y), __float_as_uint(f[1].x),
                       __float_as_uint(f[1].y));
   }
-  static __device__ __forceinline__ Raw load(const float *p) { return ld_stream16(p); }
-  static __device__ __forceinline__ Raw zero() { return make_uint4(0, 0, 0, 0); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[4]) {
     f[0] = __uint_as_float(r.x);
     f[1] = __uint_as_float(r.y);
     f[2] = __uint_as_float(r.z);
     f[3] = __uint_as_float(r.w);
-  }
-  static __device__ __forceinline__ Raw pack(const float (&f)[4]) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
-                      __float_as_uint(f[3]));
   }
   static __device__ __forceinline__ void set(Raw &r, int e, float v) {
     const uint32_t u = __float_as_uint(v);
@@ -179,8 +181,6 @@ struct VecIO<__nv_bfloat16, 8> {
     }
     return r;
   }
-  static __device__ __forceinline__ Raw load(const __nv_bfloat16 *p) { return ld_stream16(p); }
-  static __device__ __forceinline__ Raw zero() { return make_uint4(0, 0, 0, 0); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[8]) {
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -188,16 +188,6 @@ struct VecIO<__nv_bfloat16, 8> {
       f[2 * w] = __uint_as_float(u << 16);
       f[2 * w + 1] = __uint_as_float(u & 0xFFFF0000u);
     }
-  }
-  static __device__ __forceinline__ Raw pack(const float (&f)[8]) {
-    Raw r;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint32_t u;
-      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f[2 * w + 1]), "f"(f[2 * w]));
-      set_word(r, w, u);
-    }
-    return r;
   }
   static __device__ __forceinline__ void set(Raw &r, int e, __nv_bfloat16 v) {
     const uint32_t b = __bfloat16_as_ushort(v);
@@ -228,8 +218,6 @@ struct VecIO<__half, 8> {
     }
     return r;
   }
-  static __device__ __forceinline__ Raw load(const __half *p) { return ld_stream16(p); }
-  static __device__ __forceinline__ Raw zero() { return make_uint4(0, 0, 0, 0); }
   static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[8]) {
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -237,16 +225,6 @@ struct VecIO<__half, 8> {
       f[2 * w] = __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu)));
       f[2 * w + 1] = __half2float(__ushort_as_half((unsigned short)(u >> 16)));
     }
-  }
-  static __device__ __forceinline__ Raw pack(const float (&f)[8]) {
-    Raw r;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint32_t u;
-      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f[2 * w + 1]), "f"(f[2 * w]));
-      set_word(r, w, u);
-    }
-    return r;
   }
   static __device__ __forceinline__ void set(Raw &r, int e, __half v) {
     const uint32_t b = __half_as_ushort(v);
@@ -256,75 +234,10 @@ struct VecIO<__half, 8> {
   static __device__ __forceinline__ void store_raw(__half *p, const Raw &r) { st16(p, r); }
 };
 
-// Four 16-bit elements (8 bytes): the unit the pipelined kernels read from
-// shared memory and store to global memory.
-template <typename T>
-struct VecIO16x4 {
-  using Raw = uint2;
-  static constexpr int kPairs = 2;
-  static __device__ __forceinline__ float2 lo_hi(uint32_t u);
-  static __device__ __forceinline__ uint32_t pack_pair(float2 f);
-  static __device__ __forceinline__ Raw zero() { return make_uint2(0, 0); }
-  static __device__ __forceinline__ void unpack2(const Raw &r, float2 (&f)[2]) {
-    f[0] = lo_hi(r.x);
-    f[1] = lo_hi(r.y);
-  }
-  static __device__ __forceinline__ void unpack(const Raw &r, float (&f)[4]) {
-    const float2 a = lo_hi(r.x), b = lo_hi(r.y);
-    f[0] = a.x;
-    f[1] = a.y;
-    f[2] = b.x;
-    f[3] = b.y;
-  }
-  static __device__ __forceinline__ Raw pack2(const float2 (&f)[2]) {
-    return make_uint2(pack_pair(f[0]), pack_pair(f[1]));
-  }
-  static __device__ __forceinline__ Raw pack(const float (&f)[4]) {
-    return make_uint2(pack_pair(make_float2(f[0], f[1])), pack_pair(make_float2(f[2], f[3])));
-  }
-  static __device__ __forceinline__ void set(Raw &r, int e, T v) {
-    const uint32_t b = (uint32_t)(*reinterpret_cast<const unsigned short *>(&v));
-    uint32_t &w = (e >> 1) ? r.y : r.x;
-    w = (e & 1) ? ((w & 0x0000FFFFu) | (b << 16)) : ((w & 0xFFFF0000u) | b);
-  }
-  static __device__ __forceinline__ void store_raw(T *p, const Raw &r) {
-    asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(r.x), "r"(r.y) : "memory");
-  }
-};
-template <>
-__device__ __forceinline__ float2 VecIO16x4<__nv_bfloat16>::lo_hi(uint32_t u) {
-  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-}
-template <>
-__device__ __forceinline__ uint32_t VecIO16x4<__nv_bfloat16>::pack_pair(float2 f) {
-  uint32_t u;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f.y), "f"(f.x));
-  return u;
-}
-template <>
-__device__ __forceinline__ float2 VecIO16x4<__half>::lo_hi(uint32_t u) {
-  return __half22float2(*reinterpret_cast<const __half2 *>(&u));
-}
-template <>
-__device__ __forceinline__ uint32_t VecIO16x4<__half>::pack_pair(float2 f) {
-  uint32_t u;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(f.y), "f"(f.x));
-  return u;
-}
-template <>
-struct VecIO<__nv_bfloat16, 4> : VecIO16x4<__nv_bfloat16> {};
-template <>
-struct VecIO<__half, 4> : VecIO16x4<__half> {};
-
-template <typename P>
-__device__ __forceinline__ float param(const P *p, int64_t i) {
-  return to_f32<P>(ld_scalar(p + i));
-}
-
 // Start of every main kernel: wait until the preceding grid in the stream has
 // completed and its memory is visible (a no-op without a programmatic
 // predecessor), then let the next grid get scheduled. The kernels read and
-// write no global memory before this (the pipelined kernels only issue L2
+// write no global memory before this (the 16-byte kernels only issue L2
 // prefetch hints, which change no memory state), so programmatic launch keeps
 // stream order.
 __device__ __forceinline__ void pdl_prologue() {
@@ -355,7 +268,7 @@ __device__ __forceinline__ Lane lane_of(const Geom &g, int tid) {
 
 // ---- forward -----------------------------------------------------------------
 
-// y for one vector of VEC elements (one row, VEC consecutive columns).
+// y for one vector of VEC elements (one row, VEC columns).
 // bth[e] = tau |beta[e]|: below it the binary32 value may have cancelled.
 template <typename T, int VEC>
 __device__ __forceinline__ typename VecIO<T, VEC>::Raw fwd_vector(const typename VecIO<T, VEC>::Raw &rx,
@@ -410,61 +323,50 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw fwd_vector(const typename
   return out;
 }
 
-// gamma, beta and the cancellation thresholds of VEC columns.
-template <typename T, typename P, int VEC>
-__device__ __forceinline__ void fwd_params(const P *gamma, const P *beta, int64_t c0, bool ok, float (&gam)[VEC],
-                                           float (&bet)[VEC], float (&bth)[VEC]) {
+// gamma, beta and the cancellation thresholds of the VEC columns col[e] (not
+// necessarily consecutive).
+template <typename T, int VEC>
+__device__ __forceinline__ void fwd_params_at(const Params &pr, const int64_t (&col)[VEC], float (&gam)[VEC],
+                                              float (&bet)[VEC], float (&bth)[VEC]) {
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
-    gam[e] = ok ? param(gamma, c0 + e) : 0.0f;
-    bet[e] = ok ? param(beta, c0 + e) : 0.0f;
+    gam[e] = load_param(pr.gamma, pr.gamma_dt, col[e]);
+    bet[e] = load_param(pr.beta, pr.beta_dt, col[e]);
     bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
   }
 }
 
-// The same for the VEC columns col[e] (not necessarily consecutive).
-template <typename T, typename P, int VEC>
-__device__ __forceinline__ void fwd_params_at(const P *gamma, const P *beta, const int64_t (&col)[VEC],
-                                              float (&gam)[VEC], float (&bet)[VEC], float (&bth)[VEC]) {
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) {
-    gam[e] = param(gamma, col[e]);
-    bet[e] = param(beta, col[e]);
-    bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
-  }
-}
-
-template <typename T, typename P, int VEC, int U, int B>
+// Forward for matrices that are not 16-byte aligned: one element per access,
+// U rows in flight per thread.
+template <typename T, int U, int B>
 __global__ void __launch_bounds__(B, 1)
-    dyt_fwd_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma,
-                   const P *__restrict__ beta, T *y, Geom g) {
-  using IO = VecIO<T, VEC>;
+    dyt_fwd_kernel(const T *__restrict__ x, Params pr, T *y, Geom g) {
+  using IO = VecIO<T, 1>;
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = param(alpha_p, 0);
+  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
     item_split(g, item, cc, rg);
     int64_t rb, re;
     group_rows(g, rg, rb, re);
     const int cv = cc * B + ln.cv;
-    const bool col_ok = ln.live && cv < g.NV;
-    if (!col_ok) continue;
-    const int64_t c0 = (int64_t)cv * VEC;
-    float gam[VEC], bet[VEC], bth[VEC];
-    fwd_params<T, P, VEC>(gamma, beta, c0, true, gam, bet, bth);
+    if (!(ln.live && cv < g.NV)) continue;
+    const int64_t col[1] = {cv};
+    float gam[1], bet[1], bth[1];
+    fwd_params_at<T, 1>(pr, col, gam, bet, bth);
     const int64_t step = (int64_t)g.RL * U;
     for (int64_t r0 = rb + ln.rl; r0 < re; r0 += step) {
-      typename IO::Raw raw[U];
+      T raw[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t row = r0 + (int64_t)u * g.RL;
-        raw[u] = row < re ? IO::load(x + row * g.ldx + c0) : IO::zero();
+        raw[u] = row < re ? IO::load(x + row * g.ldx + cv) : IO::zero();
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t row = r0 + (int64_t)u * g.RL;
-        if (row < re) IO::store_raw(y + row * g.ldo + c0, fwd_vector<T, VEC>(raw[u], alpha, gam, bet, bth));
+        if (row < re) IO::store_raw(y + row * g.ldo + cv, fwd_vector<T, 1>(raw[u], alpha, gam, bet, bth));
       }
     }
   }
@@ -473,17 +375,17 @@ __global__ void __launch_bounds__(B, 1)
 // ---- backward, stage 1 ---------------------------------------------------------
 
 // Fixed-order tree over the RL row lanes of a CTA: lane rl absorbs lane rl + h,
-// h = ceil(n / 2), until one lane is left. red[] holds VEC * B floats,
-// element-major (red[e * B + thread]) so that a warp touches 32 consecutive
-// banks; afterwards lane 0's entries hold the CTA sums.
-template <int VEC, int B>
-__device__ __forceinline__ void lane_tree(float *red, const Geom &g, const Lane &ln) {
+// h = ceil(n / 2), until one lane is left. red[] holds V * B binary64 values,
+// element-major (red[e * B + thread]); afterwards lane 0's entries hold the CTA
+// sums.
+template <int V, int B>
+__device__ __forceinline__ void lane_tree(double *red, const Geom &g, const Lane &ln) {
   for (int n = g.RL; n > 1;) {
     const int h = (n + 1) >> 1;
     if (ln.live && ln.rl < n - h) {
       const int src = threadIdx.x + h * g.NV;
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] += red[e * B + src];
+      for (int e = 0; e < V; ++e) red[e * B + threadIdx.x] += red[e * B + src];
     }
     __syncthreads();
     n = h;
@@ -500,14 +402,14 @@ __device__ __forceinline__ void lane_tree(float *red, const Geom &g, const Lane 
 // before the offsets run out, the remaining levels are a butterfly (both
 // partners form the same sum). The order of every sum is fixed. Each warp
 // then holds each of its 2 NV VEC sums once; one pass over the warps in order
-// adds them. red[] holds (B / 32) x 2 NV VEC floats. Results go to out_g /
-// out_b (row of the group's partials) at the thread's columns.
+// adds them. red[] holds (B / 32) x 2 NV VEC binary64 values. Results go to
+// out_g / out_b (row of the group's partials) at the thread's columns.
 template <int VEC, int B>
-__device__ __forceinline__ void lane_reduce_warps(const float (&vg)[VEC], const float (&vb)[VEC], float *red,
+__device__ __forceinline__ void lane_reduce_warps(const double (&vg)[VEC], const double (&vb)[VEC], double *red,
                                                   const Geom &g, const Lane &ln, int64_t c0_chunk,
-                                                  float *out_g, float *out_b) {
+                                                  double *out_g, double *out_b) {
   constexpr int V2 = 2 * VEC;
-  float v[V2];
+  double v[V2];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
     v[e] = vg[e];
@@ -526,8 +428,8 @@ __device__ __forceinline__ void lane_reduce_warps(const float (&vg)[VEC], const 
       if (h >= 1) {
 #pragma unroll
         for (int j = 0; j < h; ++j) {
-          const float send = up ? v[j] : v[j + h];
-          const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, off);
+          const double send = up ? v[j] : v[j + h];
+          const double recv = __shfl_xor_sync(0xFFFFFFFFu, send, off);
           v[j] = (up ? v[j + h] : v[j]) + recv;
         }
         start += up ? h : 0;
@@ -539,7 +441,7 @@ __device__ __forceinline__ void lane_reduce_warps(const float (&vg)[VEC], const 
       off <<= 1;
     }
   }
-  const int width = g.NV * VEC;  // floats per warp and sum
+  const int width = g.NV * VEC;  // values per warp and sum
   if (!dup) {
 #pragma unroll
     for (int j = 0; j < V2; ++j) {
@@ -552,22 +454,24 @@ __device__ __forceinline__ void lane_reduce_warps(const float (&vg)[VEC], const 
   __syncthreads();
   if (threadIdx.x < 2 * width) {
     const int which = threadIdx.x / width, k = threadIdx.x - which * width;
-    float sum = 0.0f;
+    double sum = 0.0;
     for (int w = 0; w < B / 32; ++w) sum += red[(2 * w + which) * width + k];
     (which ? out_b : out_g)[c0_chunk + k] = sum;
   }
   __syncthreads();
 }
 
-// Per-thread backward state for VEC columns.
+// Per-thread backward state for VEC columns, in binary64.
 template <int VEC>
 struct BwdAcc {
-  float g[VEC];  // sum of dy * t over this group's rows
-  float b[VEC];  // sum of dy
+  double g[VEC];  // sum of dy * t over this group's rows
+  double b[VEC];  // sum of dy
 };
 
 // One vector (one row, VEC columns): dx out, sums in. g4[e] = 4 gamma[e]
 // (with q = (1 - t^2) / 4, g4 * dy * q rounds exactly as gamma * dy * (1 - t^2)).
+// dgamma and dbeta terms are added in binary64: dy * t is exact there (a
+// product of two binary32 values), so these sums carry only t's own error.
 // MASKED: only the first nvalid elements are real (0 for a padded row, fewer
 // than VEC for the vector that straddles the end of a packed matrix); the
 // others are computed like any other and their results dropped afterwards.
@@ -588,19 +492,22 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       dyt_tanh_qsech2_2(mul2(f2(alpha), x2[h]), t, q);
       const float2 gdys = mul2(mul2(make_float2(g4[2 * h], g4[2 * h + 1]), dy2[h]), q);  // gamma dy (1-t^2)
       dx2[h] = mul2(f2(alpha), gdys);
-      const float2 ag = make_float2(acc.g[2 * h], acc.g[2 * h + 1]);
-      const float2 ab = make_float2(acc.b[2 * h], acc.b[2 * h + 1]);
-      float2 ng = fma2(dy2[h], t, ag), nb = add2(ab, dy2[h]), nca = fma2(gdys, x2[h], ca);
+      const double d0 = (double)dy2[h].x, d1 = (double)dy2[h].y;
+      double ng0 = fma(d0, (double)t.x, acc.g[2 * h]), ng1 = fma(d1, (double)t.y, acc.g[2 * h + 1]);
+      double nb0 = acc.b[2 * h] + d0, nb1 = acc.b[2 * h + 1] + d1;
+      float2 nca = fma2(gdys, x2[h], ca);
       if (MASKED) {  // drop padded elements' results, after the arithmetic
         const bool okx = 2 * h < nvalid, oky = 2 * h + 1 < nvalid;
-        ng = make_float2(okx ? ng.x : ag.x, oky ? ng.y : ag.y);
-        nb = make_float2(okx ? nb.x : ab.x, oky ? nb.y : ab.y);
+        ng0 = okx ? ng0 : acc.g[2 * h];
+        nb0 = okx ? nb0 : acc.b[2 * h];
+        ng1 = oky ? ng1 : acc.g[2 * h + 1];
+        nb1 = oky ? nb1 : acc.b[2 * h + 1];
         nca = make_float2(okx ? nca.x : ca.x, oky ? nca.y : ca.y);
       }
-      acc.g[2 * h] = ng.x;
-      acc.g[2 * h + 1] = ng.y;
-      acc.b[2 * h] = nb.x;
-      acc.b[2 * h + 1] = nb.y;
+      acc.g[2 * h] = ng0;
+      acc.g[2 * h + 1] = ng1;
+      acc.b[2 * h] = nb0;
+      acc.b[2 * h + 1] = nb1;
       ca = nca;
     }
     return IO::pack2(dx2);
@@ -614,7 +521,9 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       dyt_tanh_qsech2(alpha * xf[e], t, q);
       const float gdys = (g4[e] * dyf[e]) * q;
       dxf[e] = alpha * gdys;
-      const float ng = fmaf(dyf[e], t, acc.g[e]), nb = acc.b[e] + dyf[e], nca = fmaf(gdys, xf[e], ca.x);
+      const double d = (double)dyf[e];
+      const double ng = fma(d, (double)t, acc.g[e]), nb = acc.b[e] + d;
+      const float nca = fmaf(gdys, xf[e], ca.x);
       const bool ok = e < nvalid;
       acc.g[e] = (MASKED && !ok) ? acc.g[e] : ng;
       acc.b[e] = (MASKED && !ok) ? acc.b[e] : nb;
@@ -624,20 +533,22 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
   }
 }
 
-template <typename T, typename P, int VEC, int U, int B>
+// Backward stage 1 for matrices that are not 16-byte aligned: one element
+// per access, U rows in flight per thread.
+template <typename T, int U, int B>
 __global__ void __launch_bounds__(B, 1)
-    dyt_bwd_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
-                   const P *__restrict__ gamma, T *dx, float *__restrict__ part_dg,
-                   float *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
-  using IO = VecIO<T, VEC>;
-  __shared__ float red[VEC * B];
+    dyt_bwd_kernel(const T *__restrict__ x, const T *__restrict__ dy, Params pr, T *dx,
+                   double *__restrict__ part_dg, double *__restrict__ part_db, double *__restrict__ part_da,
+                   Geom g) {
+  using IO = VecIO<T, 1>;
+  __shared__ double red[2 * B];
   __shared__ double red_a[B / 32];
   // Let the finalize kernel, launched as a programmatic dependent, get
   // scheduled early; it still waits for this grid to finish before reading.
   pdl_prologue();
 
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = param(alpha_p, 0);
+  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
   double acc_a = 0.0;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
@@ -646,76 +557,56 @@ __global__ void __launch_bounds__(B, 1)
     group_rows(g, rg, rb, re);
     const int cv = cc * B + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
-    const int64_t c0 = (int64_t)cv * VEC;
-    float gam[VEC];
-    BwdAcc<VEC> acc;
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      gam[e] = col_ok ? 4.0f * param(gamma, c0 + e) : 0.0f;  // 4 gamma (see bwd_vector)
-      acc.g[e] = 0.0f;
-      acc.b[e] = 0.0f;
-    }
+    float gam[1] = {col_ok ? 4.0f * load_param(pr.gamma, pr.gamma_dt, cv) : 0.0f};  // 4 gamma (see bwd_vector)
+    BwdAcc<1> acc;
+    acc.g[0] = 0.0;
+    acc.b[0] = 0.0;
     if (col_ok) {
       const int64_t step = (int64_t)g.RL * U;
       for (int64_t r0 = rb + ln.rl; r0 < re; r0 += step) {
-        typename IO::Raw rx[U], rdy[U];
+        T rx[U], rdy[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int64_t row = r0 + (int64_t)u * g.RL;
           const bool ok = row < re;
-          rx[u] = ok ? IO::load(x + row * g.ldx + c0) : IO::zero();
-          rdy[u] = ok ? IO::load(dy + row * g.ldd + c0) : IO::zero();
+          rx[u] = ok ? IO::load(x + row * g.ldx + cv) : IO::zero();
+          rdy[u] = ok ? IO::load(dy + row * g.ldd + cv) : IO::zero();
         }
         float2 ca = make_float2(0.0f, 0.0f);
         if (r0 + (int64_t)(U - 1) * g.RL < re) {  // every row of the step is real
 #pragma unroll
           for (int u = 0; u < U; ++u) {
             const int64_t row = r0 + (int64_t)u * g.RL;
-            IO::store_raw(dx + row * g.ldo + c0,
-                          bwd_vector<T, VEC, false>(rx[u], rdy[u], alpha, gam, acc, ca, VEC));
+            IO::store_raw(dx + row * g.ldo + cv, bwd_vector<T, 1, false>(rx[u], rdy[u], alpha, gam, acc, ca, 1));
           }
         } else {  // ragged last step of the group
 #pragma unroll
           for (int u = 0; u < U; ++u) {
             const int64_t row = r0 + (int64_t)u * g.RL;
             const bool ok = row < re;
-            const typename IO::Raw d =
-                bwd_vector<T, VEC, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok ? VEC : 0);
-            if (ok) IO::store_raw(dx + row * g.ldo + c0, d);
+            const T d = bwd_vector<T, 1, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok ? 1 : 0);
+            if (ok) IO::store_raw(dx + row * g.ldo + cv, d);
           }
         }
         acc_a += (double)ca.x;
-        acc_a += (double)ca.y;
       }
     }
     // Per-(group, column) partials.
-    float *pg = part_dg + (int64_t)rg * g.N;
-    float *pb = part_db + (int64_t)rg * g.N;
+    double *pg = part_dg + (int64_t)rg * g.N;
+    double *pb = part_db + (int64_t)rg * g.N;
     if (g.RL == 1) {
       if (col_ok) {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          pg[c0 + e] = acc.g[e];
-          pb[c0 + e] = acc.b[e];
-        }
+        pg[cv] = acc.g[0];
+        pb[cv] = acc.b[0];
       }
     } else {
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.g[e];
+      red[threadIdx.x] = acc.g[0];
+      red[B + threadIdx.x] = acc.b[0];
       __syncthreads();
-      lane_tree<VEC, B>(red, g, ln);
+      lane_tree<2, B>(red, g, ln);
       if (col_ok && ln.rl == 0) {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) pg[c0 + e] = red[e * B + threadIdx.x];
-      }
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) red[e * B + threadIdx.x] = acc.b[e];
-      __syncthreads();
-      lane_tree<VEC, B>(red, g, ln);
-      if (col_ok && ln.rl == 0) {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) pb[c0 + e] = red[e * B + threadIdx.x];
+        pg[cv] = red[threadIdx.x];
+        pb[cv] = red[B + threadIdx.x];
       }
       __syncthreads();
     }
@@ -741,15 +632,13 @@ __global__ void __launch_bounds__(B, 1)
 // round trip per batch. The lanes of a column are then added by a fixed-order
 // warp butterfly (lanes CT apart share a warp when CT < 32) and the warps'
 // results by one thread per column, in warp order; the sum is rounded once
-// to P. The last block also reduces dalpha, with its loads issued together
-// with the column loads.
+// to the gradient's dtype. The last block also reduces dalpha, with its loads
+// issued together with the column loads.
 constexpr int kFinThreads = 256;
 
-template <typename P>
 __global__ void __launch_bounds__(kFinThreads)
-    dyt_finalize_kernel(const float *__restrict__ part_dg, const float *__restrict__ part_db,
-                        const double *__restrict__ part_da, P *dgamma, P *dbeta, P *dalpha,
-                        int64_t N, int nrg, int nda, int CT) {
+    dyt_finalize_kernel(const double *__restrict__ part_dg, const double *__restrict__ part_db,
+                        const double *__restrict__ part_da, GradOut out, int64_t N, int nrg, int nda, int CT) {
   __shared__ double sg[kFinThreads], sb[kFinThreads], sa[kFinThreads / 32];
   // Wait until the stage-1 grid has finished and its writes are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -764,17 +653,17 @@ __global__ void __launch_bounds__(kFinThreads)
   double a = 0.0, b = 0.0;
   if (col < N) {
     for (int r = lane; r < nrg; r += 4 * L) {
-      float va[4], vb[4];
+      double va[4], vb[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int rk = r + k * L;
-        va[k] = rk < nrg ? part_dg[(int64_t)rk * N + col] : 0.0f;  // + 0 leaves a sum unchanged
-        vb[k] = rk < nrg ? part_db[(int64_t)rk * N + col] : 0.0f;
+        va[k] = rk < nrg ? part_dg[(int64_t)rk * N + col] : 0.0;  // + 0 leaves a sum unchanged
+        vb[k] = rk < nrg ? part_db[(int64_t)rk * N + col] : 0.0;
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        a += (double)va[k];
-        b += (double)vb[k];
+        a += va[k];
+        b += vb[k];
       }
     }
   }
@@ -803,13 +692,13 @@ __global__ void __launch_bounds__(kFinThreads)
       sgc += sg[k * stride + tid];
       sbc += sb[k * stride + tid];
     }
-    dgamma[col] = from_f64<P>(sgc);
-    dbeta[col] = from_f64<P>(sbc);
+    store_param(out.dgamma, out.gamma_dt, col, sgc);
+    store_param(out.dbeta, out.beta_dt, col, sbc);
   }
   if (da_block && tid == 0) {
     double s = 0.0;
     for (int w = 0; w < kFinThreads / 32; ++w) s += sa[w];
-    dalpha[0] = from_f64<P>(s);
+    store_param(out.dalpha, out.alpha_dt, 0, s);
   }
 }
 

@@ -7,6 +7,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "dyt.h"
+
 namespace dyt {
 
 // ---- hardware approximations (special-function unit) ---------------------
@@ -173,6 +175,29 @@ __device__ __forceinline__ __half from_f64<__half>(double v) {
   unsigned short b;
   asm("cvt.rn.f16.f64 %0, %1;" : "=h"(b) : "d"(v));
   return __ushort_as_half(b);
+}
+
+// ---- parameters, whose dtypes are known at run time ------------------------
+//
+// alpha, gamma and beta (and their gradients) each carry their own dtype
+// (dyt_dtype codes). They are read once per work item and written once per
+// call, so a run-time switch costs nothing on the element path.
+
+__device__ __forceinline__ float load_param(const void *p, int dt, int64_t i) {
+  if (dt == DYT_F32) return __ldg(static_cast<const float *>(p) + i);
+  const unsigned short u = __ldg(static_cast<const unsigned short *>(p) + i);
+  return dt == DYT_BF16 ? __uint_as_float((uint32_t)u << 16) : __half2float(__ushort_as_half(u));
+}
+
+// v rounded once (nearest, ties to even) to dtype dt and stored at p[i].
+__device__ __forceinline__ void store_param(void *p, int dt, int64_t i, double v) {
+  if (dt == DYT_F32) {
+    static_cast<float *>(p)[i] = (float)v;
+  } else if (dt == DYT_BF16) {
+    static_cast<__nv_bfloat16 *>(p)[i] = from_f64<__nv_bfloat16>(v);
+  } else {
+    static_cast<__half *>(p)[i] = from_f64<__half>(v);
+  }
 }
 
 // ---- forward output with cancellation refinement ---------------------------

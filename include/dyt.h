@@ -28,10 +28,13 @@
  *   dalpha hold one. Any alignment is accepted; 16-byte aligned tensors take
  *   the vectorised path, for any N (a ragged N is streamed in packs of
  *   16 / element-size rows, which always span whole 16-byte vectors).
- * - Dtypes (the page's Summary, "Precision"): x, dy, y and dx share x_dtype;
- *   alpha, gamma, beta and all three parameter gradients share param_dtype.
- *   y and dx come back in x_dtype, the parameter gradients in param_dtype.
- *   Arithmetic is binary32 with binary64 partial sums.
+ * - Dtypes (the page's Summary, "Precision"): x, dy, y and dx share x_dtype,
+ *   so y and dx come back in x's dtype. Each parameter gradient comes back in
+ *   its parameter's dtype: dalpha in alpha's, dgamma in gamma's, dbeta in
+ *   beta's. The *_ex entry points take the three parameter dtypes one by one;
+ *   the others take one param_dtype for all three. Element arithmetic is
+ *   binary32; the parameter-gradient sums are binary64 throughout, rounded
+ *   once to the gradient's dtype.
  * - Outputs are overwritten, never accumulated into.
  * - Aliasing: y may alias x, and dx may alias x or dy (each element is read
  *   before the same thread writes it). Any other overlap is undefined.
@@ -44,6 +47,10 @@
  *   no failure is reported as DYT_OK.
  * - Results are deterministic: the same inputs on the same device give the
  *   same bits (static schedule, fixed reduction order, no atomics in sums).
+ * - Every argument error is reported by a status code before anything is
+ *   launched. No kernel waits on another CTA, grid or device; the only waits
+ *   are hardware completion waits (a thread's own asynchronous copies, the
+ *   preceding grid in the stream).
  */
 #ifndef DYT_H_
 #define DYT_H_
@@ -101,13 +108,15 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
 /*
  * Backward: recomputes t = tanh(alpha * x) and writes dx, dgamma, dbeta and
  * dalpha. Two kernel launches on `stream`: the fused elementwise pass, which
- * also writes partial sums to the workspace (binary32 per row group and
- * column for dgamma and dbeta, binary64 per CTA for dalpha), and a finalize
- * pass that adds the partials in binary64 in a fixed order and rounds them
- * once to param_dtype.
+ * also writes binary64 partial sums to the workspace (per row group and column
+ * for dgamma and dbeta, per CTA for dalpha), and a finalize pass that adds the
+ * partials in binary64 in a fixed order and rounds each gradient once.
  *   x, dy     [M*N] x_dtype, read
  *   alpha     [1]   param_dtype, read on the device
  *   gamma     [N]   param_dtype, read
+ *   beta      [N]   param_dtype, not read: the gradients do not depend on beta.
+ *                   May be NULL. (It is part of the call so that the layer's
+ *                   parameters travel together; dbeta takes beta's dtype.)
  *   dx        [M*N] x_dtype, written (may alias x or dy)
  *   dgamma    [N]   param_dtype, written
  *   dbeta     [N]   param_dtype, written
@@ -122,10 +131,10 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
  * With M * N == 0: dgamma and dbeta (when N > 0) and dalpha are set to zero,
  * and no workspace is used.
  */
-dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const void *gamma,
+dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const void *gamma, const void *beta,
                         void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
-                        dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace,
-                        size_t workspace_bytes, dyt_stream_t stream);
+                        dyt_dtype x_dtype, dyt_dtype param_dtype, void *workspace, size_t workspace_bytes,
+                        dyt_stream_t stream);
 
 /*
  * dyt_forward and dyt_backward over row-strided matrices: row i of a tensor
@@ -147,9 +156,31 @@ dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, co
                                const void *beta, void *y, int64_t ldy, int64_t M, int64_t N,
                                dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream);
 dyt_status dyt_backward_strided(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
-                                const void *gamma, void *dx, int64_t lddx, void *dgamma, void *dbeta,
-                                void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
-                                void *workspace, size_t workspace_bytes, dyt_stream_t stream);
+                                const void *gamma, const void *beta, void *dx, int64_t lddx, void *dgamma,
+                                void *dbeta, void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype,
+                                dyt_dtype param_dtype, void *workspace, size_t workspace_bytes,
+                                dyt_stream_t stream);
+
+/*
+ * The general forms: row pitches as in the *_strided calls, and one dtype per
+ * parameter (the page's Summary, "Precision": each parameter gradient takes
+ * its own parameter's dtype). alpha is read as alpha_dtype, gamma as
+ * gamma_dtype, beta as beta_dtype; the backward writes dalpha in alpha_dtype,
+ * dgamma in gamma_dtype and dbeta in beta_dtype (beta itself is not read and
+ * may be NULL). Every other entry point above is one of these with all
+ * pitches N and/or all three parameter dtypes equal, and gives the same bits
+ * as this call with those arguments. An invalid dtype code gives
+ * DYT_ERR_UNSUPPORTED_DTYPE; the workspace size does not depend on the
+ * parameter dtypes.
+ */
+dyt_status dyt_forward_ex(const void *x, int64_t ldx, const void *alpha, const void *gamma, const void *beta,
+                          void *y, int64_t ldy, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype alpha_dtype,
+                          dyt_dtype gamma_dtype, dyt_dtype beta_dtype, dyt_stream_t stream);
+dyt_status dyt_backward_ex(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
+                           const void *gamma, const void *beta, void *dx, int64_t lddx, void *dgamma, void *dbeta,
+                           void *dalpha, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype alpha_dtype,
+                           dyt_dtype gamma_dtype, dyt_dtype beta_dtype, void *workspace, size_t workspace_bytes,
+                           dyt_stream_t stream);
 
 /* Static, human-readable name of a status. Never NULL. */
 const char *dyt_status_string(dyt_status status);
@@ -173,8 +204,7 @@ typedef struct dyt_launch_info {
   int col_chunks;    /* column chunks the grid is split into */
   int row_groups;    /* row groups (= partial sums per column) */
   int kernels;       /* kernels this call launched */
-  int tma_stages;    /* shared-memory stages of the CTA-wide bulk-copy pipeline (0 = unused) */
-  int async_stages;  /* per-thread asynchronous-copy ring slots (0 = unused) */
+  int async_stages;  /* per-thread asynchronous-copy ring slots (0 = the one-element kernels) */
   int pack_rows;     /* 1, or vec on the packed path: a 16-byte aligned matrix whose N is not a
                         multiple of vec is streamed as packs of vec rows (vec x N elements,
                         exactly N 16-byte vectors) */
@@ -199,22 +229,6 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
                           dyt_launch_info *out);
 
 /*
- * The device error word of the current device, a sticky bit set: bit 0 means a
- * bounded wait inside a pipelined kernel gave up (its results are not valid).
- * Synchronises with the device. clear != 0 resets the word to 0 afterwards.
- */
-dyt_status dyt_device_error(unsigned int *word, int clear);
-
-/*
- * Self-test of the bounded wait used by the pipelined kernels: enqueues on
- * `stream` one kernel that waits on a barrier phase nothing will complete,
- * giving up after `spin_limit` polls. It writes 1 to *gave_up (a DEVICE int)
- * when the wait gave up and sets bit 0 of the device error word. The kernel
- * always returns; nothing faults or hangs.
- */
-dyt_status dyt_selftest_wait_timeout(unsigned int spin_limit, int *gave_up, dyt_stream_t stream);
-
-/*
  * Backward without a caller-provided workspace (no counterpart in the paper:
  * it exists for callers that cannot allocate device memory themselves, such as
  * code embedded in a host application that owns all device memory through its
@@ -226,8 +240,11 @@ dyt_status dyt_selftest_wait_timeout(unsigned int spin_limit, int *gave_up, dyt_
  * library keeps in device memory (every device that loads the library holds it
  * until the process exits). The call allocates nothing.
  * - The first call on each device looks the array's device address up
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   (cudaGetSymbolAddress) with that device current, and keeps it for that
+ *   device's context; make that first call before any stream capture. After a
+ *   cudaDeviceReset, the next call on the device is such a first call again:
+ *   the address is cached under the driver's context id, never reused across
+ *   contexts.
  * - Shapes whose scratch need (dyt_backward_workspace_bytes) exceeds
  *   DYT_NOALLOC_SCRATCH_BYTES are rejected with DYT_ERR_WORKSPACE_TOO_SMALL
  *   before anything is launched.
@@ -240,8 +257,8 @@ dyt_status dyt_selftest_wait_timeout(unsigned int spin_limit, int *gave_up, dyt_
 #define DYT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 
 dyt_status dyt_backward_noalloc(const void *x, const void *dy, const void *alpha, const void *gamma,
-                                void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M, int64_t N,
-                                dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream);
+                                const void *beta, void *dx, void *dgamma, void *dbeta, void *dalpha, int64_t M,
+                                int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -38,9 +38,9 @@ def _load():
         build()
         lib = ctypes.CDLL(_SO)
         vp, i64, i32, dp = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
-        lib.dyt_oracle_forward.argtypes = [vp, i32, vp, vp, vp, i32, i64, i64, dp]
+        lib.dyt_oracle_forward.argtypes = [vp, i32, vp, i32, vp, i32, vp, i32, i64, i64, dp]
         lib.dyt_oracle_forward.restype = i32
-        lib.dyt_oracle_backward.argtypes = [vp, vp, i32, vp, vp, i32, i64, i64, dp, dp, dp, dp, dp, dp, dp]
+        lib.dyt_oracle_backward.argtypes = [vp, vp, i32, vp, i32, vp, i32, i64, i64, dp, dp, dp, dp, dp, dp, dp]
         lib.dyt_oracle_backward.restype = i32
         lib.dyt_oracle_round.argtypes = [dp, i64, i32, vp]
         lib.dyt_oracle_round.restype = i32
@@ -64,30 +64,37 @@ def _as(a, dtype):
     return a
 
 
-def forward(x, alpha, gamma, beta, M: int, N: int, x_dtype: str, p_dtype: str) -> np.ndarray:
-    """y (binary64, M*N) of the DyT forward."""
+def _pdtypes(p_dtype):
+    """(alpha, gamma, beta) storage dtypes from one name or a 3-tuple of names."""
+    return (p_dtype,) * 3 if isinstance(p_dtype, str) else tuple(p_dtype)
+
+
+def forward(x, alpha, gamma, beta, M: int, N: int, x_dtype: str, p_dtype) -> np.ndarray:
+    """y (binary64, M*N) of the DyT forward. p_dtype: one dtype for alpha, gamma and
+    beta, or a tuple (alpha, gamma, beta) of dtypes."""
     lib = _load()
-    x, alpha, gamma, beta = (_as(x, x_dtype), _as(alpha, p_dtype), _as(gamma, p_dtype),
-                             _as(beta, p_dtype))
+    ad, gd, bd = _pdtypes(p_dtype)
+    x, alpha, gamma, beta = _as(x, x_dtype), _as(alpha, ad), _as(gamma, gd), _as(beta, bd)
     y = np.empty(M * N, dtype=np.float64)
-    rc = lib.dyt_oracle_forward(_ptr(x), DTYPE_CODES[x_dtype], _ptr(alpha), _ptr(gamma), _ptr(beta),
-                                DTYPE_CODES[p_dtype], M, N, _ptr(y))
+    rc = lib.dyt_oracle_forward(_ptr(x), DTYPE_CODES[x_dtype], _ptr(alpha), DTYPE_CODES[ad], _ptr(gamma),
+                                DTYPE_CODES[gd], _ptr(beta), DTYPE_CODES[bd], M, N, _ptr(y))
     if rc:
         raise ValueError("dyt_oracle_forward rejected its arguments")
     return y
 
 
-def backward(x, dy, alpha, gamma, M: int, N: int, x_dtype: str, p_dtype: str, want_dx: bool = True):
+def backward(x, dy, alpha, gamma, M: int, N: int, x_dtype: str, p_dtype, want_dx: bool = True):
     """dict with dx (binary64 M*N, or None), dgamma, dbeta (N), dalpha (float) and the
-    magnitude of each sum (mag_dgamma, mag_dbeta, mag_dalpha)."""
+    magnitude of each sum (mag_dgamma, mag_dbeta, mag_dalpha). p_dtype as for forward."""
     lib = _load()
-    x, dy, alpha, gamma = (_as(x, x_dtype), _as(dy, x_dtype), _as(alpha, p_dtype), _as(gamma, p_dtype))
+    ad, gd, _ = _pdtypes(p_dtype)
+    x, dy, alpha, gamma = _as(x, x_dtype), _as(dy, x_dtype), _as(alpha, ad), _as(gamma, gd)
     dx = np.empty(M * N, dtype=np.float64) if want_dx else None
     dg, db = np.empty(N), np.empty(N)
     mg, mb = np.empty(N), np.empty(N)
     da, ma = np.empty(1), np.empty(1)
-    rc = lib.dyt_oracle_backward(_ptr(x), _ptr(dy), DTYPE_CODES[x_dtype], _ptr(alpha), _ptr(gamma),
-                                 DTYPE_CODES[p_dtype], M, N, _ptr(dx), _ptr(dg), _ptr(db), _ptr(da),
+    rc = lib.dyt_oracle_backward(_ptr(x), _ptr(dy), DTYPE_CODES[x_dtype], _ptr(alpha), DTYPE_CODES[ad],
+                                 _ptr(gamma), DTYPE_CODES[gd], M, N, _ptr(dx), _ptr(dg), _ptr(db), _ptr(da),
                                  _ptr(mg), _ptr(mb), _ptr(ma))
     if rc:
         raise ValueError("dyt_oracle_backward rejected its arguments")

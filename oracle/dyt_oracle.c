@@ -80,18 +80,22 @@ static double one_minus_tanh_sq(double z) {
 /* ---- forward ----------------------------------------------------------- */
 
 /* y[i*N + j] = gamma[j] * tanh(alpha * x[i*N + j]) + beta[j], binary64.
+ * alpha, gamma and beta are stored in a_dtype, g_dtype and b_dtype (each
+ * parameter keeps its own dtype, as on the page's Summary, "Precision").
  * Returns 0, or -1 on a bad argument. */
-int dyt_oracle_forward(const void *x, int x_dtype, const void *alpha, const void *gamma,
-                       const void *beta, int p_dtype, int64_t M, int64_t N, double *y) {
-  if (M < 0 || N < 0 || !valid_dtype(x_dtype) || !valid_dtype(p_dtype)) return -1;
+int dyt_oracle_forward(const void *x, int x_dtype, const void *alpha, int a_dtype, const void *gamma,
+                       int g_dtype, const void *beta, int b_dtype, int64_t M, int64_t N, double *y) {
+  if (M < 0 || N < 0 || !valid_dtype(x_dtype) || !valid_dtype(a_dtype) || !valid_dtype(g_dtype) ||
+      !valid_dtype(b_dtype))
+    return -1;
   if (M == 0 || N == 0) return 0;
   if (!x || !alpha || !gamma || !beta || !y) return -1;
   double *g = (double *)malloc((size_t)N * sizeof(double));
   double *b = (double *)malloc((size_t)N * sizeof(double));
   if (!g || !b) { free(g); free(b); return -1; }
-  dyt_oracle_decode(gamma, N, p_dtype, g);
-  dyt_oracle_decode(beta, N, p_dtype, b);
-  const double a = decode_one(alpha, 0, p_dtype);
+  dyt_oracle_decode(gamma, N, g_dtype, g);
+  dyt_oracle_decode(beta, N, b_dtype, b);
+  const double a = decode_one(alpha, 0, a_dtype);
   for (int64_t i = 0; i < M; ++i) {
     for (int64_t j = 0; j < N; ++j) {
       const double xv = decode_one(x, i * N + j, x_dtype);
@@ -112,13 +116,14 @@ int dyt_oracle_forward(const void *x, int x_dtype, const void *alpha, const void
  * absolute values of its terms: mag_dgamma[j] = sum_i |dy*t|, mag_dbeta[j] =
  * sum_i |dy|, mag_dalpha = sum |gamma*dy*(1-t^2)*x|. They set the error scale
  * of a floating-point sum.
+ * alpha and gamma are stored in a_dtype and g_dtype.
  * Returns 0, or -1 on a bad argument.
  */
-int dyt_oracle_backward(const void *x, const void *dy, int x_dtype, const void *alpha,
-                        const void *gamma, int p_dtype, int64_t M, int64_t N, double *dx,
+int dyt_oracle_backward(const void *x, const void *dy, int x_dtype, const void *alpha, int a_dtype,
+                        const void *gamma, int g_dtype, int64_t M, int64_t N, double *dx,
                         double *dgamma, double *dbeta, double *dalpha, double *mag_dgamma,
                         double *mag_dbeta, double *mag_dalpha) {
-  if (M < 0 || N < 0 || !valid_dtype(x_dtype) || !valid_dtype(p_dtype)) return -1;
+  if (M < 0 || N < 0 || !valid_dtype(x_dtype) || !valid_dtype(a_dtype) || !valid_dtype(g_dtype)) return -1;
   if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return -1;
   for (int64_t j = 0; j < N; ++j) {
     dgamma[j] = 0.0;
@@ -132,8 +137,8 @@ int dyt_oracle_backward(const void *x, const void *dy, int x_dtype, const void *
   if (!x || !dy || !alpha || !gamma) return -1;
   double *g = (double *)malloc((size_t)N * sizeof(double));
   if (!g) return -1;
-  dyt_oracle_decode(gamma, N, p_dtype, g);
-  const double a = decode_one(alpha, 0, p_dtype);
+  dyt_oracle_decode(gamma, N, g_dtype, g);
+  const double a = decode_one(alpha, 0, a_dtype);
   double da = 0.0, da_mag = 0.0;
   for (int64_t i = 0; i < M; ++i) {
     for (int64_t j = 0; j < N; ++j) {

@@ -25,7 +25,8 @@ class Workload:
     M: int
     N: int
     x_dtype: str          # x, dy, y, dx
-    p_dtype: str          # alpha, gamma, beta and their gradients
+    p_dtype: object       # alpha, gamma, beta and their gradients: one dtype name, or a tuple
+                          # (alpha, gamma, beta) of names
     alpha: float
     x_std: float = 1.0
     dy_std: float = 1.0
@@ -40,16 +41,21 @@ class Workload:
     def elements(self) -> int:
         return self.M * self.N
 
+    @property
+    def param_dtypes(self) -> tuple:
+        """(alpha, gamma, beta) dtype names."""
+        return (self.p_dtype,) * 3 if isinstance(self.p_dtype, str) else tuple(self.p_dtype)
+
     def fwd_bytes(self) -> int:
         """Algorithmic bytes of one forward: x in, y out, gamma, beta, alpha in."""
-        sx, sp = ITEMSIZE[self.x_dtype], ITEMSIZE[self.p_dtype]
-        return 2 * self.M * self.N * sx + (2 * self.N + 1) * sp
+        sa, sg, sb = (ITEMSIZE[d] for d in self.param_dtypes)
+        return 2 * self.M * self.N * ITEMSIZE[self.x_dtype] + self.N * (sg + sb) + sa
 
     def bwd_bytes(self) -> int:
         """Algorithmic bytes of one backward: x, dy in, dx out, gamma, alpha in,
         dgamma, dbeta, dalpha out."""
-        sx, sp = ITEMSIZE[self.x_dtype], ITEMSIZE[self.p_dtype]
-        return 3 * self.M * self.N * sx + (3 * self.N + 2) * sp
+        sa, sg, sb = (ITEMSIZE[d] for d in self.param_dtypes)
+        return 3 * self.M * self.N * ITEMSIZE[self.x_dtype] + self.N * (2 * sg + sb) + 2 * sa
 
     def with_shape(self, M: int | None = None, N: int | None = None) -> "Workload":
         return replace(self, M=self.M if M is None else M, N=self.N if N is None else N,
@@ -81,8 +87,8 @@ def make_params(w: Workload) -> dict:
         "beta": normal(w.N, "f64", w.beta_mean, w.beta_std, w.seed, STREAM_BETA),
     }
     # Parameters are drawn through binary32 (f64 storage holds the binary32 value) and
-    # then encoded in the parameter dtype.
-    return {k: encode(v, w.p_dtype) for k, v in p.items()}
+    # then encoded in each parameter's dtype.
+    return {k: encode(p[k], dt) for k, dt in zip(("alpha", "gamma", "beta"), w.param_dtypes)}
 
 
 def encode(v64: np.ndarray, dtype: str) -> np.ndarray:

@@ -30,8 +30,19 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for f in ("dyt_forward", "dyt_backward", "dyt_backward_workspace_bytes", "dyt_status_string",
-              "dyt_last_launch_info", "dyt_plan_query"):
+              "dyt_last_launch_info", "dyt_plan_query", "dyt_forward_ex", "dyt_backward_ex"):
         assert f in names
+
+
+def test_backward_takes_beta_after_gamma():
+    # dyt_backward(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, ...)
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    for name in ("dyt_backward", "dyt_backward_strided", "dyt_backward_noalloc", "dyt_backward_ex"):
+        m = re.search(r"dyt_status\s+" + name + r"\s*\(([^)]*)\)", text)
+        assert m, name
+        params = [p.strip().split()[-1].lstrip("*") for p in m.group(1).split(",")]
+        assert params[params.index("gamma") + 1] == "beta", (name, params)
+        assert params.index("beta") < params.index("dx"), (name, params)
 
 
 def test_library_exports_every_declared_function():
@@ -53,15 +64,22 @@ def test_host_validation_without_a_device():
     assert dyt.dyt_forward(0, 0, 0, 0, 0, 2**62, 2**20, 0, 0, None) == 1  # M*N*size overflows
     assert dyt.dyt_forward(0, 0, 0, 0, 0, 0, 5, 0, 0, None) == 0          # empty: nothing to do
     assert dyt.dyt_last_launch_info()["kernels"] == 0
-    assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 0, 3, 3, 0, 0, 0, 0, None) == 1  # null dalpha
-    assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 1, 3, 3, 1, 0, 0, 0, None) == 1  # null dgamma/dbeta
-    assert dyt.dyt_backward(0, 0, 0, 0, 0, 0, 0, 0, -3, 3, 0, 0, 0, 0, None) == 1
+    assert dyt.dyt_backward(0, 0, 0, 0, None, 0, 0, 0, 0, 3, 3, 0, 0, 0, 0, None) == 1  # null dalpha
+    assert dyt.dyt_backward(0, 0, 0, 0, None, 0, 0, 0, 1, 3, 3, 1, 0, 0, 0, None) == 1  # null dgamma/dbeta
+    assert dyt.dyt_backward(0, 0, 0, 0, None, 0, 0, 0, 0, -3, 3, 0, 0, 0, 0, None) == 1
+    assert dyt.dyt_backward(0, 0, 0, 0, None, 0, 0, 0, 0, 3, 3, 0, 5, 0, 0, None) == 2  # bad param dtype
+    # one dtype per parameter: each code is checked
+    for bad in ((3, 0, 0), (0, 3, 0), (0, 0, -1)):
+        assert dyt.dyt_forward_ex(0, 4, 0, 0, 0, 0, 4, 4, 4, 0, *bad, None) == 2
+        assert dyt.dyt_backward_ex(0, 4, 0, 4, 0, 0, None, 0, 4, 0, 0, 0, 4, 4, 0, *bad, 0, 0, None) == 2
+    assert dyt.dyt_forward_ex(0, 4, 0, 0, 0, 0, 4, 0, 4, 1, 1, 2, 0, None) == 0  # empty: nothing to do
+    assert dyt.dyt_backward_noalloc(0, 0, 0, 0, None, 0, 0, 0, 0, -1, 3, 0, 0, None) == 1
     # row pitches below N, or byte offsets beyond int64, are rejected
     assert dyt.dyt_forward_strided(0, 3, 0, 0, 0, 0, 4, 5, 4, 0, 0, None) == 1                  # ldx < N
     assert dyt.dyt_forward_strided(0, 4, 0, 0, 0, 0, 3, 5, 4, 0, 0, None) == 1                  # ldy < N
     assert dyt.dyt_forward_strided(0, 2**61, 0, 0, 0, 0, 4, 5, 4, 0, 0, None) == 1              # offsets overflow
-    assert dyt.dyt_backward_strided(0, 4, 0, 2, 0, 0, 0, 4, 0, 0, 1, 5, 4, 0, 0, 0, 0, None) == 1  # lddy < N
-    assert dyt.dyt_backward_strided(0, 4, 0, 4, 0, 0, 0, 3, 0, 0, 1, 5, 4, 0, 0, 0, 0, None) == 1  # lddx < N
+    assert dyt.dyt_backward_strided(0, 4, 0, 2, 0, 0, None, 0, 4, 0, 0, 1, 5, 4, 0, 0, 0, 0, None) == 1  # lddy < N
+    assert dyt.dyt_backward_strided(0, 4, 0, 4, 0, 0, None, 0, 3, 0, 0, 1, 5, 4, 0, 0, 0, 0, None) == 1  # lddx < N
     assert dyt.dyt_forward_strided(0, 9, 0, 0, 0, 0, 9, 0, 4, 0, 0, None) == 0                  # empty
     assert dyt.dyt_backward_workspace_bytes(-1, 3, 0, 0) == 0
     assert dyt.dyt_backward_workspace_bytes(0, 3, 0, 0) == 0
@@ -82,27 +100,21 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
     size = 4 if xd == 0 else 2
     vec = p["vec"]
     pk = p["pack_rows"]
-    assert not (p["tma_stages"] and p["async_stages"])
     # 16-byte aligned adjacent rows always take the 16-byte kernels (packed when N is ragged)
-    assert bool(p["async_stages"] or p["tma_stages"]) == bool(vectorized)
+    assert bool(p["async_stages"]) == bool(vectorized)
     if p["async_stages"]:    # per-thread copy ring: 16-byte vectors, one per thread
-        assert vectorized and vec == 16 // size
+        assert vec == 16 // size
         # a ragged N is streamed in packs of vec rows (exactly N vectors each)
         assert pk == (vec if N % vec else 1)
+        ctas = sms             # the 16-byte kernels run one CTA per SM
     else:
-        assert pk == 1
-    if p["tma_stages"]:      # bulk-copy pipeline: 16-byte rows, 4 columns per thread
-        assert vectorized and (N * size) % 16 == 0 and vec == 4
-        assert 2 <= p["tma_stages"] <= 8
-    else:
-        assert vec in (1, 16 // size)
-        if vec > 1:
-            assert vectorized and (N % vec == 0 or pk == vec)
+        assert vec == 1 and pk == 1
+        ctas = sms * occ
     Mp, Np = -(-M // pk), pk * N                   # (packed) rows and their pitch
     nv = Np // vec
     B = p["block"]
-    assert B in (512, 1024) and p["kernels"] == 2
-    assert 1 <= p["grid"] <= sms * occ            # persistent 1D grid: never beyond one wave
+    assert B == (512 if p["async_stages"] else 1024) and p["kernels"] == 2
+    assert 1 <= p["grid"] <= ctas                  # persistent 1D grid: never beyond one wave
     if p["path"] == 1:                             # row-tiled: several rows per CTA step
         assert p["row_lanes"] == B // nv >= 2 and p["col_chunks"] == 1
     else:                                          # row-per-CTA: columns across the CTA
@@ -111,29 +123,31 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
         assert p["rows_per_step"] == p["row_lanes"] * pk
     items = p["row_groups"] * p["col_chunks"]
     assert p["grid"] <= items
-    # every lane adds at most 128 (packed) rows per group (bounded binary32 error)
+    # every lane visits at most 2048 (packed) rows per group: the kernels' exact
+    # multiply-high row counts need it
     rows_per_group = -(-Mp // p["row_groups"])
-    assert -(-rows_per_group // p["row_lanes"]) <= 128
+    assert -(-rows_per_group // p["row_lanes"]) <= 2048
     # every CTA gets the same number of work items, unless there are more
     # column chunks than CTAs
-    if p["col_chunks"] <= sms * occ:
+    if p["col_chunks"] <= ctas:
         assert items % p["grid"] == 0
-        assert p["grid"] > (sms * occ) // 2 or p["grid"] == items
-    # workspace: binary32 dgamma and dbeta partials per group and row position
+        assert p["grid"] > ctas // 2 or p["grid"] == items
+    # workspace: binary64 dgamma and dbeta partials per group and row position
     # (pack_rows x N of them) + binary64 dalpha per CTA
     al = lambda v: (v + 15) // 16 * 16
-    assert p["workspace_bytes"] == 2 * al(p["row_groups"] * Np * 4) + al(p["grid"] * 8)
+    assert p["workspace_bytes"] == 2 * al(p["row_groups"] * Np * 8) + al(p["grid"] * 8)
 
 
 def test_plans_whose_counts_overflow_are_rejected():
     dyt = _lib()
-    # 2^40 rows of 300 unaligned fp32 columns: 3 row lanes of at most 128 rows
-    # per group would need about 2.9e9 groups, more than an int holds
+    # 2^40 rows of 5000 unaligned fp32 columns: 5 column chunks of 1024 threads
+    # and groups of at most 2048 rows would need about 2.7e9 work items, more
+    # than an int holds
     with pytest.raises(dyt.DytError) as e:
-        dyt.dyt_plan_query(2**40, 300, 0, 0, 1, 0, 148, 1)
+        dyt.dyt_plan_query(2**40, 5000, 0, 0, 1, 0, 148, 1)
     assert e.value.status == 1
     p = dyt.dyt_plan_query(2**20, 300, 0, 0, 1, 0, 148, 1)
-    assert p["row_lanes"] == 3 and p["row_groups"] == -(-(-(-2**20 // (3 * 128))) // 148) * 148
+    assert p["row_lanes"] == 3 and p["row_groups"] == -(-(-(-2**20 // (3 * 2048))) // 148) * 148
 
 
 def test_page_narrow_widths_take_the_row_tiled_path():
@@ -147,15 +161,15 @@ def test_page_narrow_widths_take_the_row_tiled_path():
 
 def test_multiply_high_quotients_are_exact():
     # The kernels divide by the row-lane count RL (2..1024) with a host constant
-    # m = ceil(2^32 / RL): q = (n * m) >> 32. Groups hold at most 128 RL rows, so
-    # n < 129 RL; every quotient in that range must be exact (checked at and
-    # around each multiple of RL, where an error would first show).
+    # m = ceil(2^32 / RL): q = (n * m) >> 32. Groups hold at most 2048 RL rows,
+    # so n < 2049 RL + RL; every quotient in that range must be exact (checked
+    # at and around each multiple of RL, where an error would first show).
     import numpy as np
     for RL in range(2, 1025):
         m = ((1 << 32) + RL - 1) // RL
-        k = np.arange(0, 130, dtype=np.uint64)
+        k = np.arange(0, 2051, dtype=np.uint64)
         n = np.concatenate([k * RL, k * RL + RL - 1, np.maximum(k * RL, 1) - 1]).astype(np.uint64)
-        n = n[n < 129 * RL + RL]
+        n = n[n < 2050 * RL]
         q = (n * np.uint64(m)) >> np.uint64(32)
         assert np.array_equal(q, n // np.uint64(RL)), RL
 

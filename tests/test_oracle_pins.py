@@ -346,3 +346,22 @@ def test_sum_magnitudes_equal_the_sums_when_all_terms_share_a_sign(sign):
     assert np.array_equal(r["mag_dbeta"], np.abs(r["dbeta"]))
     assert r["mag_dalpha"] == abs(r["dalpha"])
     assert np.all(np.sign(r["dbeta"]) == sign)
+
+
+def test_each_parameter_is_decoded_in_its_own_dtype():
+    # alpha in bf16, gamma in fp16, beta in fp32: the oracle must give the same
+    # values as with every parameter held exactly in binary64 (decoding is exact).
+    M, N = 13, 21
+    x, dy, _, _, _ = _inputs(M, N)
+    a16 = oracle.round_to(np.array([0.8125]), "bf16")
+    g16 = oracle.round_to(synth.normal(N, "f64", 1.0, 0.3, 31, 3), "f16")
+    b32 = synth.normal(N, "f32", 0.0, 0.3, 31, 4)
+    mixed = ("bf16", "f16", "f32")
+    a64, g64, b64 = oracle.decode(a16, "bf16"), oracle.decode(g16, "f16"), b32.astype(np.float64)
+    y = oracle.forward(x, a16, g16, b32, M, N, "f32", mixed)
+    assert np.array_equal(y, oracle.forward(x, a64, g64, b64, M, N, "f32", "f64"))
+    r = oracle.backward(x, dy, a16, g16, M, N, "f32", mixed)
+    r64 = oracle.backward(x, dy, a64, g64, M, N, "f32", "f64")
+    for k in ("dx", "dgamma", "dbeta", "mag_dgamma", "mag_dbeta"):
+        assert np.array_equal(r[k], r64[k]), k
+    assert r["dalpha"] == r64["dalpha"] and r["mag_dalpha"] == r64["mag_dalpha"]

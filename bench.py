@@ -2,6 +2,10 @@
 
 One step = one forward and one backward (dx, dgamma, dbeta, dalpha) of the
 workload over one batch of synthetic input. Prints ONE JSON line on rank 0.
+The headline workload is the largest configuration (32768 x 8192 bf16); the
+line's `shapes` block times every other workload and layout variant the same
+way, each with its roofline entry, replay percentiles, clocks and the oracle's
+CPU time next to it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -18,6 +22,7 @@ is more than twice the L2 size, so no step reads another's data from L2.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -203,8 +208,7 @@ def run_oracle_sample(w, rows: int, min_seconds: float = 0.0):
     import oracle
     from synth import workloads
 
-    ws = workloads.Workload(w.name, rows, w.N, w.x_dtype, w.p_dtype, w.alpha, w.x_std, w.dy_std,
-                            w.gamma_mean, w.gamma_std, w.beta_mean, w.beta_std, w.nonzero, w.seed)
+    ws = dataclasses.replace(w, M=rows)
     inp = workloads.make_inputs(ws)
     passes, t0 = 0, time.perf_counter()
     while True:
@@ -239,8 +243,7 @@ def cpu_baseline_threads(w, seconds_budget=5.0):
 
     cores = len(os.sched_getaffinity(0))
     rows = oracle_sample_rows(w, seconds_budget * cores)
-    ws = workloads.Workload(w.name, rows, w.N, w.x_dtype, w.p_dtype, w.alpha, w.x_std, w.dy_std,
-                            w.gamma_mean, w.gamma_std, w.beta_mean, w.beta_std, w.nonzero, w.seed)
+    ws = dataclasses.replace(w, M=rows)
     inp = workloads.make_inputs(ws)
     N = w.N
     edges = [rows * i // cores for i in range(cores + 1)]
@@ -287,7 +290,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": workload_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"first {rows} of {w.M} rows per step, forward + backward, "
                                    "single-threaded binary64 C oracle"},
@@ -296,10 +299,96 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w):
+def workload_config(w, gpus: int):
+    """The workload as both arms name it (the same dict in both)."""
     return {"workload": w.name, "M": w.M, "N": w.N, "x_dtype": w.x_dtype, "param_dtype": w.p_dtype,
             "alpha": w.alpha, "x_std": w.x_std, "dy_std": w.dy_std, "gamma": f"N({w.gamma_mean},{w.gamma_std})",
-            "beta": f"N({w.beta_mean},{w.beta_std})", "seed": w.seed}
+            "beta": f"N({w.beta_mean},{w.beta_std})", "seed": w.seed, "parallelism": f"rows{gpus}"}
+
+
+# ---- device buffers and timing -------------------------------------------------------------------
+
+def _to_torch(a, dtype, device):
+    import torch
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dtype == "bf16" else torch.from_numpy(a)
+    return t if str(device) == "cpu" else t.to(device)
+
+
+def _matrix(src, w, dev):
+    """An M x N device matrix holding src, starting w.offset elements past a 16-byte
+    boundary (0 for the workloads themselves)."""
+    import torch
+    t = _to_torch(src, w.x_dtype, "cpu")
+    buf = torch.empty(w.M * w.N + w.offset + 8, dtype=t.dtype, device=dev)
+    m = buf[w.offset:w.offset + w.M * w.N].view(w.M, w.N)
+    m.copy_(t.view(w.M, w.N))
+    return m
+
+
+def _empty_like_matrix(m, w):
+    import torch
+    buf = torch.empty(w.M * w.N + w.offset + 8, dtype=m.dtype, device=m.device)
+    return buf[w.offset:w.offset + w.M * w.N].view(w.M, w.N)
+
+
+def _sets(w, inp, dev, L2):
+    """Buffer sets for back-to-back calls: enough that the data touched between two
+    uses of one set exceeds 3x the L2 size, so no call reads another's data from L2."""
+    import torch
+    from synth import workloads
+    set_bytes = 4 * w.M * w.N * workloads.ITEMSIZE[w.x_dtype]  # x, dy, y, dx
+    nsets = int(min(64, max(1, -(-3 * L2 // set_bytes))))
+    x0, dy0 = _matrix(inp["x"], w, dev), _matrix(inp["dy"], w, dev)
+    ad, gd, bd = w.param_dtypes
+    a, g, b = _to_torch(inp["alpha"], ad, dev), _to_torch(inp["gamma"], gd, dev), _to_torch(inp["beta"], bd, dev)
+    sets = []
+    for i in range(nsets):
+        x = x0 if i == 0 else _empty_like_matrix(x0, w).copy_(x0)
+        d = dy0 if i == 0 else _empty_like_matrix(dy0, w).copy_(dy0)
+        sets.append({"x": x, "dy": d, "y": _empty_like_matrix(x0, w), "dx": _empty_like_matrix(x0, w),
+                     "dg": torch.empty_like(g), "db": torch.empty_like(b), "da": torch.empty_like(a)})
+    return sets, (a, g, b), set_bytes, nsets
+
+
+def _graph(stream, fn, n):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fn(i)
+    return g
+
+
+def _time_replays(g, stream, dev, K, clock_index, clocks=True, min_replays=7, min_seconds=0.3,
+                  max_replays=400):
+    """Per-call device time (us) of a K-call graph over repeated replays (CUDA events on
+    the launching stream), with the SM clocks sampled while it runs."""
+    import torch
+    g.replay()
+    torch.cuda.synchronize(dev)
+    per = []
+    with ClockSampler(clock_index, enabled=clocks) as clk:
+        t_end = time.perf_counter() + min_seconds
+        while len(per) < min_replays or (time.perf_counter() < t_end and len(per) < max_replays):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            e1.synchronize()
+            per.append(e0.elapsed_time(e1) * 1e3 / K)
+        while time.perf_counter() < t_end:  # keep the load on for the clock samples
+            g.replay()
+            torch.cuda.synchronize(dev)
+    q = np.percentile(per, [10, 50, 90])
+    return {"us_p10": float(q[0]), "us_p50": float(q[1]), "us_p90": float(q[2]), "replays": len(per),
+            "clocks": clk.summary()}
+
+
+def _roofline(nbytes, us, peak, peak_kind, traffic):
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+            "peak_kind": peak_kind, "traffic": traffic, "algorithmic_bytes_per_launch": nbytes}
 
 
 # ---- our arm ------------------------------------------------------------------------------------
@@ -310,11 +399,6 @@ def run_ours(args, w):
 
     import elementwise_reduction_b200 as dyt
     from synth import workloads
-
-    def to_torch(a, dtype, device):
-        a = np.ascontiguousarray(a)
-        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dtype == "bf16" else torch.from_numpy(a)
-        return t if str(device) == "cpu" else t.to(device)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -328,32 +412,16 @@ def run_ours(args, w):
     M, N = w.M, w.N
     inp = workloads.make_inputs(w)
     L2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    set_bytes = 4 * M * N * workloads.ITEMSIZE[w.x_dtype]  # x, dy, y, dx
-    nsets = int(min(64, max(1, -(-3 * L2 // set_bytes))))
-    x0 = to_torch(inp["x"], w.x_dtype, dev).view(M, N)
-    dy0 = to_torch(inp["dy"], w.x_dtype, dev).view(M, N)
-    alpha = to_torch(inp["alpha"], w.p_dtype, dev)
-    gamma = to_torch(inp["gamma"], w.p_dtype, dev)
-    beta = to_torch(inp["beta"], w.p_dtype, dev)
-    sets = []
-    for i in range(nsets):
-        x = x0 if i == 0 else x0.clone()
-        d = dy0 if i == 0 else dy0.clone()
-        sets.append({"x": x, "dy": d, "y": torch.empty_like(x), "dx": torch.empty_like(x),
-                     "dg": torch.empty_like(gamma), "db": torch.empty_like(gamma),
-                     "da": torch.empty(1, dtype=gamma.dtype, device=dev)})
-    ws = dyt.workspace(x0, gamma)
+    sets, (alpha, gamma, beta), set_bytes, nsets = _sets(w, inp, dev, L2)
+    ws = dyt.workspace(sets[0]["x"], gamma)
     grads = torch.empty(2 * N + 1, dtype=torch.float32, device=dev)
     from elementwise_reduction_b200.dist import allreduce_param_grads
-
-    def allreduce_grads(s):
-        allreduce_param_grads(s["dg"], s["db"], s["da"], buf=grads)
 
     def fwd(s):
         dyt.forward(s["x"], alpha, gamma, beta, out=s["y"])
 
     def bwd(s, ws_=None):
-        dyt.backward(s["x"], s["dy"], alpha, gamma, dx=s["dx"], dgamma=s["dg"], dbeta=s["db"],
+        dyt.backward(s["x"], s["dy"], alpha, gamma, beta, dx=s["dx"], dgamma=s["dg"], dbeta=s["db"],
                      dalpha=s["da"], ws=ws if ws_ is None else ws_)
 
     def step(i):
@@ -361,7 +429,7 @@ def run_ours(args, w):
         fwd(s)
         bwd(s)
         if world > 1:
-            allreduce_grads(s)
+            allreduce_param_grads(s["dg"], s["db"], s["da"], buf=grads)
 
     stream = torch.cuda.Stream(dev)
     torch.cuda.synchronize(dev)
@@ -369,19 +437,10 @@ def run_ours(args, w):
         for i in range(args.warmup):
             step(i)
         torch.cuda.synchronize(dev)
-        launch_info_fwd = None
-
-        def capture(fn, n):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for i in range(n):
-                    fn(i)
-            return g
-
-        g_step = capture(step, args.steps)
-        g_fwd = capture(lambda i: fwd(sets[i % nsets]), args.steps)
+        g_step = _graph(stream, step, args.steps)
+        g_fwd = _graph(stream, lambda i: fwd(sets[i % nsets]), args.steps)
         launch_info_fwd = dyt.dyt_last_launch_info()
-        g_bwd = capture(lambda i: bwd(sets[i % nsets]), args.steps)
+        g_bwd = _graph(stream, lambda i: bwd(sets[i % nsets]), args.steps)
         launch_info_bwd = dyt.dyt_last_launch_info()
         for g in (g_step, g_fwd, g_bwd):  # untimed replay: first-launch costs
             g.replay()
@@ -429,21 +488,21 @@ def run_ours(args, w):
     # independent). Every step still copies in its own inputs and copies out
     # its own results.
     e2e_steps = args.e2e_steps or max(3, min(args.steps, int(2e9 // max(1, set_bytes)) or 3))
-    hx = to_torch(inp["x"], w.x_dtype, "cpu").view(M, N).pin_memory()
-    hdy = to_torch(inp["dy"], w.x_dtype, "cpu").view(M, N).pin_memory()
+    hx = _to_torch(inp["x"], w.x_dtype, "cpu").view(M, N).pin_memory()
+    hdy = _to_torch(inp["dy"], w.x_dtype, "cpu").view(M, N).pin_memory()
     lanes = []
     for j in range(2):
-        d = sets[j] if j < nsets else {"x": torch.empty_like(x0), "dy": torch.empty_like(x0),
-                                       "y": torch.empty_like(x0), "dx": torch.empty_like(x0),
-                                       "dg": torch.empty_like(gamma), "db": torch.empty_like(gamma),
-                                       "da": torch.empty(1, dtype=gamma.dtype, device=dev)}
-        hy = torch.empty_like(hx).pin_memory()
+        x0 = sets[0]["x"]
+        d = sets[j] if j < nsets else {"x": _empty_like_matrix(x0, w), "dy": _empty_like_matrix(x0, w),
+                                       "y": _empty_like_matrix(x0, w), "dx": _empty_like_matrix(x0, w),
+                                       "dg": torch.empty_like(gamma), "db": torch.empty_like(beta),
+                                       "da": torch.empty_like(alpha)}
         lanes.append({"dev": d, "ws": dyt.workspace(x0, gamma), "stream": stream if j == 0 else torch.cuda.Stream(dev),
                       "grads": torch.empty(2 * N + 1, dtype=torch.float32, device=dev),
-                      "hy": hy, "hdx": torch.empty_like(hx).pin_memory(),
+                      "hy": torch.empty_like(hx).pin_memory(), "hdx": torch.empty_like(hx).pin_memory(),
                       "hdg": torch.empty(N, dtype=gamma.dtype).pin_memory(),
-                      "hdb": torch.empty(N, dtype=gamma.dtype).pin_memory(),
-                      "hda": torch.empty(1, dtype=gamma.dtype).pin_memory()})
+                      "hdb": torch.empty(N, dtype=beta.dtype).pin_memory(),
+                      "hda": torch.empty(1, dtype=alpha.dtype).pin_memory()})
 
     def e2e_step(i):
         ln = lanes[i % 2]
@@ -480,9 +539,11 @@ def run_ours(args, w):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
     sx = workloads.ITEMSIZE[w.x_dtype]
-    sp = workloads.ITEMSIZE[w.p_dtype]
+    sa, sg, sb = (workloads.ITEMSIZE[d] for d in w.param_dtypes)
     h2d = 2 * M * N * sx
-    d2h = 2 * M * N * sx + (2 * N + 1) * sp
+    d2h = 2 * M * N * sx + N * (sg + sb) + sa
+    del lanes, sets, ws
+    torch.cuda.empty_cache()
 
     # ---- numbers ----
     fb, bb = w.fwd_bytes(), w.bwd_bytes()
@@ -494,13 +555,9 @@ def run_ours(args, w):
     bw_fwd, bw_bwd = fb / t_fwd / 1e9, bb / t_bwd / 1e9
     dominant = "bwd" if t_bwd >= t_fwd else "fwd"
     traffic = committed_traffic(w.name, "dyt_backward" if dominant == "bwd" else "dyt_fwd_kernel")
-    roofline = {
-        "bound": "hbm", "kernel": "dyt_backward (stage-1 + finalize)" if dominant == "bwd" else "dyt_forward",
-        "achieved": bw_bwd if dominant == "bwd" else bw_fwd, "peak": peak, "unit": "GB/s",
-        "frac": (bw_bwd if dominant == "bwd" else bw_fwd) / peak, "peak_kind": peak_kind,
-        "traffic": traffic,
-        "algorithmic_bytes_per_launch": bb if dominant == "bwd" else fb,
-    }
+    roofline = _roofline(bb if dominant == "bwd" else fb, (t_bwd if dominant == "bwd" else t_fwd) * 1e6, peak,
+                         peak_kind, traffic)
+    roofline["kernel"] = "dyt_backward (stage 1 + finalize)" if dominant == "bwd" else "dyt_forward"
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -509,9 +566,11 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(workload_config(w), io_dtype=w.x_dtype, parallelism=f"rows{world}",
-                       l2=f"{nsets} rotating buffer sets, {nsets * set_bytes / 2**20:.0f} MiB touched per "
-                          f"cycle vs L2 {L2 / 2**20:.0f} MiB"),
+        "config": workload_config(w, world),
+        "l2": f"{nsets} rotating buffer set(s), {nsets * set_bytes / 2**20:.0f} MiB touched per cycle vs L2 "
+              f"{L2 / 2**20:.0f} MiB (inputs larger than L2)" if set_bytes > L2 else
+              f"{nsets} rotating buffer sets, {nsets * set_bytes / 2**20:.0f} MiB touched per cycle vs L2 "
+              f"{L2 / 2**20:.0f} MiB",
         "pct_of_peak": 100.0 * value / world / peak,
         "rows_per_s": M * world / (ms_per_step * 1e-3),
         "fwd": {"us": t_fwd * 1e6, "GB_s": bw_fwd, "frac": bw_fwd / peak, "rows_per_s": M / t_fwd,
@@ -528,7 +587,7 @@ def run_ours(args, w):
     if world > 1:
         dist.destroy_process_group()
     if world == 1 and not args.no_shapes:
-        line["shapes"] = other_shapes(w, args, dev)
+        line["shapes"] = shape_table(args, dev, local, cpu=not args.no_cpu_baseline)
     if world == 1 and not args.no_latency:
         line["latency_us"] = call_latency(args, dev)
     if world == 1 and not args.no_cpu_baseline:  # the oracle's baseline belongs to the 1-GPU line
@@ -552,17 +611,13 @@ def call_latency(args, dev, calls=30):
     flush = torch.empty(2 * L2, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
     state = {}
-    for name, w in workloads.WORKLOADS.items():
+    for name, w in {**workloads.WORKLOADS, **workloads.VARIANTS}.items():
         inp = workloads.make_inputs(w)
-
-        def dev_t(a, dt):
-            a = np.ascontiguousarray(a)
-            t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dt == "bf16" else torch.from_numpy(a)
-            return t.to(dev)
-
-        x = dev_t(inp["x"], w.x_dtype).view(w.M, w.N)
-        st = {"x": x, "dy": dev_t(inp["dy"], w.x_dtype).view(w.M, w.N), "y": torch.empty_like(x),
-              "dx": torch.empty_like(x), "p": [dev_t(inp[k], w.p_dtype) for k in ("alpha", "gamma", "beta")],
+        x = _matrix(inp["x"], w, dev)
+        ad, gd, bd = w.param_dtypes
+        st = {"x": x, "dy": _matrix(inp["dy"], w, dev), "y": _empty_like_matrix(x, w),
+              "dx": _empty_like_matrix(x, w),
+              "p": [_to_torch(inp[k], dt, dev) for k, dt in zip(("alpha", "gamma", "beta"), (ad, gd, bd))],
               "ws": None, "t": {"fwd": [], "bwd": []}}
         st["ws"] = dyt.workspace(x, st["p"][1])
         state[name] = st
@@ -577,7 +632,7 @@ def call_latency(args, dev, calls=30):
                     if op == "fwd":
                         dyt.forward(st["x"], a, g, b, out=st["y"])
                     else:
-                        dyt.backward(st["x"], st["dy"], a, g, dx=st["dx"], ws=st["ws"])
+                        dyt.backward(st["x"], st["dy"], a, g, b, dx=st["dx"], ws=st["ws"])
                     e1.record(stream)
                     e1.synchronize()
                     if i >= 2:
@@ -591,67 +646,60 @@ def call_latency(args, dev, calls=30):
     return out
 
 
-def other_shapes(w0, args, dev):
-    """Forward and backward throughput of the other workloads (the metric is quoted per
-    shape), each timed like the main one: a CUDA graph of K calls over rotating buffer
-    sets that exceed L2."""
+def shape_table(args, dev, clock_index, cpu=True):
+    """Every workload and layout variant, forward and backward, each timed like the
+    headline: a CUDA graph of K calls over rotating buffer sets that exceed L2,
+    replayed at least 7 times (p10 / p50 / p90 of the per-call time) with the SM
+    clocks sampled during the replays. Each line carries its roofline entry and,
+    next to it, the oracle on the host cores on a bounded sample of the same
+    workload. For the narrow shapes, a plain PyTorch copy (the forward's bytes)
+    and a three-operand add (the backward's bytes) timed the same way give the
+    floor a memory-bound kernel of these sizes meets in this setting."""
     import torch
 
     import elementwise_reduction_b200 as dyt
     from synth import workloads
 
     out = {}
-    peak, _ = hbm_peak()
+    peak, peak_kind = hbm_peak()
     L2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    for name, w in workloads.WORKLOADS.items():
-        if name == w0.name:
-            continue
+    K = args.steps
+    for name, w in {**workloads.WORKLOADS, **workloads.VARIANTS}.items():
         inp = workloads.make_inputs(w)
-        M, N = w.M, w.N
-
-        def dev_t(a, dt):
-            a = np.ascontiguousarray(a)
-            t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dt == "bf16" else torch.from_numpy(a)
-            return t.to(dev)
-
-        x0, dy0 = dev_t(inp["x"], w.x_dtype).view(M, N), dev_t(inp["dy"], w.x_dtype).view(M, N)
-        a, g, b = (dev_t(inp[k], w.p_dtype) for k in ("alpha", "gamma", "beta"))
-        set_bytes = 4 * M * N * workloads.ITEMSIZE[w.x_dtype]
-        nsets = int(min(64, max(1, -(-3 * L2 // set_bytes))))
-        sets = [{"x": x0.clone(), "dy": dy0.clone(), "y": torch.empty_like(x0), "dx": torch.empty_like(x0),
-                 "dg": torch.empty_like(g), "db": torch.empty_like(g),
-                 "da": torch.empty(1, dtype=g.dtype, device=dev)} for _ in range(nsets)]
-        ws = dyt.workspace(x0, g)
+        sets, (a, g, b), _, nsets = _sets(w, inp, dev, L2)
+        ws = dyt.workspace(sets[0]["x"], g)
         stream = torch.cuda.Stream(dev)
-        K = args.steps
         res = {}
         with torch.cuda.stream(stream):
-            for op in ("fwd", "bwd"):
-                def call(i, op=op):
-                    s = sets[i % nsets]
-                    if op == "fwd":
-                        dyt.forward(s["x"], a, g, b, out=s["y"])
-                    else:
-                        dyt.backward(s["x"], s["dy"], a, g, dx=s["dx"], dgamma=s["dg"], dbeta=s["db"],
-                                     dalpha=s["da"], ws=ws)
+            calls = {
+                "fwd": lambda i: dyt.forward(sets[i % nsets]["x"], a, g, b, out=sets[i % nsets]["y"]),
+                "bwd": lambda i: dyt.backward(sets[i % nsets]["x"], sets[i % nsets]["dy"], a, g, b,
+                                              dx=sets[i % nsets]["dx"], dgamma=sets[i % nsets]["dg"],
+                                              dbeta=sets[i % nsets]["db"], dalpha=sets[i % nsets]["da"], ws=ws),
+            }
+            if w.M * w.N * workloads.ITEMSIZE[w.x_dtype] < (64 << 20):  # narrow shapes: library floors
+                calls["copy_floor"] = lambda i: sets[i % nsets]["y"].copy_(sets[i % nsets]["x"])
+                calls["add3_floor"] = lambda i: torch.add(sets[i % nsets]["x"], sets[i % nsets]["dy"],
+                                                          out=sets[i % nsets]["dx"])
+            for op, call in calls.items():
                 for i in range(3):
                     call(i)
-                graph = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(graph, stream=stream):
-                    for i in range(K):
-                        call(i)
-                graph.replay()
-                torch.cuda.synchronize(dev)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                graph.replay()
-                e1.record(stream)
-                torch.cuda.synchronize(dev)
-                t = e0.elapsed_time(e1) / K * 1e-3
-                nbytes = w.fwd_bytes() if op == "fwd" else w.bwd_bytes()
-                res[op] = {"us": t * 1e6, "GB_s": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
-                           "rows_per_s": M / t}
+                info = dyt.dyt_last_launch_info() if op in ("fwd", "bwd") else None
+                graph = _graph(stream, call, K)
+                t = _time_replays(graph, stream, dev, K, clock_index, clocks=not args.no_clocks)
                 del graph
+                nbytes = w.fwd_bytes() if op in ("fwd", "copy_floor") else w.bwd_bytes()
+                kernel = {"fwd": "dyt_fwd_kernel", "bwd": "dyt_backward"}.get(op)
+                t["roofline"] = _roofline(nbytes, t["us_p50"], peak, peak_kind,
+                                          committed_traffic(name, kernel) if kernel else None)
+                t["rows_per_s"] = w.M / (t["us_p50"] * 1e-6)
+                if info is not None:
+                    t["launch"] = {k: info[k] for k in ("path", "vec", "grid", "row_lanes", "row_groups",
+                                                        "pack_rows", "kernels")}
+                res[op] = t
+        if cpu:
+            res["cpu_baseline"] = cpu_baseline(w, seconds_budget=2.0)
+            res["cpu_baseline_threads"] = cpu_baseline_threads(w, seconds_budget=1.5)
         out[name] = res
         del sets, ws
         torch.cuda.empty_cache()
@@ -663,7 +711,7 @@ def main():
     from synth import workloads
 
     name = args.workload or workloads.DEFAULT_BENCH
-    w = workloads.WORKLOADS[name]
+    w = {**workloads.WORKLOADS, **workloads.VARIANTS}[name]
     if args.record_traffic:
         record_traffic(args.record_traffic, w.name, args.ncu_command)
         return

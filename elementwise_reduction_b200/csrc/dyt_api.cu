@@ -131,6 +131,12 @@ struct Plan {
 
 size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
+// Dynamic shared memory of a 16-byte kernel: its per-thread ring of 16-byte
+// slots (the backward holds x and dy in each slot pair).
+size_t async_smem(bool backward) {
+  return backward ? (size_t)kAsyncStagesBwd * 2 * kAsyncBlock * 16 : (size_t)kAsyncStagesFwd * kAsyncBlock * 16;
+}
+
 // vec: elements per access (1 or 16 / element size). ctas_per_sm from the
 // kernel's occupancy. packed: N is not a multiple of vec, and the matrix is
 // laid out as ceil(M / vec) packs of vec rows, each of pitch vec * N. The
@@ -146,8 +152,7 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool asyn
   const int64_t M = packed ? ceil_div(M_rows, (int64_t)vec) : M_rows;
   const int64_t N = packed ? (int64_t)vec * N_cols : N_cols;
   p.unroll = async ? 1 : (backward ? kScalarUnrollBwd : kScalarUnrollFwd);
-  p.smem = !async ? 0
-                  : backward ? (size_t)kAsyncStagesBwd * 2 * kAsyncBlock * 16 : (size_t)kAsyncStagesFwd * kAsyncBlock * 16;
+  p.smem = async ? async_smem(backward) : 0;
   const int64_t NV = N / vec;
   Geom &g = p.g;
   g.M = M;
@@ -306,8 +311,7 @@ dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjac
   int occ = 1;
   if (pc.async) {
     // One CTA per SM by construction (__launch_bounds__(B, 1), ring sized for it).
-    const Plan probe = make_plan(1, 1, pc.vec, backward, true, 1, 1, false, (int64_t)sizeof(T));
-    st = prepare_smem(dev, k, (int)probe.smem);
+    st = prepare_smem(dev, k, (int)async_smem(backward));
     if (st != DYT_OK) return st;
   } else {
     st = occupancy(dev, k, kScalarBlock, &occ);

@@ -36,6 +36,7 @@ class Workload:
     beta_std: float = 0.1
     nonzero: bool = False  # redraw x and dy values that are exactly zero
     seed: int = 0
+    offset: int = 0        # elements by which x, dy, y and dx start past a 16-byte boundary
 
     @property
     def elements(self) -> int:
@@ -76,8 +77,20 @@ WORKLOADS = {
     ]
 }
 
-# The configuration whose throughput the benchmark line reports by default.
-DEFAULT_BENCH = "c2_bf16_65537x32"
+# Layout variants of the workloads above: the same values with every activation
+# tensor starting one element past a 16-byte boundary, which sends them through
+# the one-element kernels.
+VARIANTS = {
+    w.name: w
+    for w in [
+        replace(WORKLOADS["c2_bf16_65537x32"], name="c2_bf16_65537x32_off1", offset=1),
+        replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_off1", offset=1),
+    ]
+}
+
+# The configuration whose throughput the benchmark line reports by default: the
+# largest one, where the layer moves the most bytes.
+DEFAULT_BENCH = "c5_bf16_32768x8192"
 
 
 def make_params(w: Workload) -> dict:

@@ -163,22 +163,38 @@ def gpu_inputs(inp: dict, x_dtype: str, p_dtype) -> dict:
     return d
 
 
-def run_cuda(inp: dict, M: int, N: int, x_dtype: str, p_dtype, fwd: bool = True, bwd: bool = True):
+def _at_offset(t: torch.Tensor, M: int, N: int, offset: int) -> torch.Tensor:
+    """An M x N copy of t whose first element lies `offset` elements past a 16-byte boundary."""
+    buf = torch.empty(M * N + offset + 8, dtype=t.dtype, device=t.device)
+    m = buf[offset:offset + M * N].view(M, N)
+    m.copy_(t.view(M, N))
+    return m
+
+
+def run_cuda(inp: dict, M: int, N: int, x_dtype: str, p_dtype, fwd: bool = True, bwd: bool = True,
+             offset: int = 0):
     """Run the C-ABI forward and backward on the device; outputs back as numpy storage.
-    p_dtype: one dtype name for alpha, gamma and beta, or a tuple (alpha, gamma, beta)."""
+    p_dtype: one dtype name for alpha, gamma and beta, or a tuple (alpha, gamma, beta).
+    offset: elements by which x, dy, y and dx start past a 16-byte boundary."""
     import elementwise_reduction_b200 as dyt
 
     ad, gd, bd = param_dtypes(p_dtype)
     t = gpu_inputs(inp, x_dtype, p_dtype)
     x = t["x"].view(M, N) if M * N else t["x"]
+    if offset and M * N:
+        x = _at_offset(x, M, N, offset)
     out, info = {}, {}
     if fwd:
-        y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"])
+        y = _at_offset(torch.empty_like(x), M, N, offset) if offset and M * N else None
+        y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=y)
         info["fwd"] = dyt.dyt_last_launch_info()
         out["y"] = to_numpy(y, x_dtype)
     if bwd:
         dy = t["dy"].view(M, N) if M * N else t["dy"]
-        dx, da, dg, db = dyt.backward(x, dy, t["alpha"], t["gamma"], t["beta"])
+        dxo = None
+        if offset and M * N:
+            dy, dxo = _at_offset(dy, M, N, offset), _at_offset(torch.empty_like(x), M, N, offset)
+        dx, da, dg, db = dyt.backward(x, dy, t["alpha"], t["gamma"], t["beta"], dx=dxo)
         info["bwd"] = dyt.dyt_last_launch_info()
         out.update(dx=to_numpy(dx, x_dtype), dgamma=to_numpy(dg, gd), dbeta=to_numpy(db, bd),
                    dalpha=float(decode(to_numpy(da, ad), ad)[0]))

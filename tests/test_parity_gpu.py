@@ -566,3 +566,16 @@ def test_workload_full_size(name):
         assert stats["dgamma"]["n_over_strict_elementwise"] == 0
     if w.N <= 256:
         assert info["bwd"]["path"] == 1
+
+
+@pytest.mark.parametrize("name", list(workloads.VARIANTS))
+def test_unaligned_variant_full_size(name):
+    # The workload's values with every activation tensor one element past a
+    # 16-byte boundary: the one-element kernels, checked on every element.
+    w = workloads.VARIANTS[name]
+    inp = workloads.make_inputs(w)
+    out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype, offset=w.offset)
+    assert info["fwd"]["vec"] == 1 and info["bwd"]["vec"] == 1
+    stats = H.compare_all(inp, out, w.M, w.N, w.x_dtype, w.p_dtype)
+    print(name, info, stats)
+    assert stats["dbeta"]["n_over_strict_elementwise"] == 0

@@ -132,9 +132,13 @@ struct Plan {
 size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
 // Dynamic shared memory of a 16-byte kernel: its per-thread ring of 16-byte
-// slots (the backward holds x and dy in each slot pair).
-size_t async_smem(bool backward) {
-  return backward ? (size_t)kAsyncStagesBwd * 2 * kAsyncBlock * 16 : (size_t)kAsyncStagesFwd * kAsyncBlock * 16;
+// slots (the backward holds x and dy in each slot pair) and, in a backward
+// over 16-bit activations, each thread's binary64 dgamma totals (16-byte
+// vectors of elem_bytes-byte elements).
+size_t async_smem(bool backward, size_t elem_bytes) {
+  if (!backward) return (size_t)kAsyncStagesFwd * kAsyncBlock * 16;
+  const size_t totals = elem_bytes == 4 ? 0 : (16 / elem_bytes) * (size_t)kAsyncBlock * sizeof(double);
+  return (size_t)kAsyncStagesBwd * 2 * kAsyncBlock * 16 + totals;
 }
 
 // vec: elements per access (1 or 16 / element size). ctas_per_sm from the
@@ -152,7 +156,7 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool asyn
   const int64_t M = packed ? ceil_div(M_rows, (int64_t)vec) : M_rows;
   const int64_t N = packed ? (int64_t)vec * N_cols : N_cols;
   p.unroll = async ? 1 : (backward ? kScalarUnrollBwd : kScalarUnrollFwd);
-  p.smem = async ? async_smem(backward) : 0;
+  p.smem = async ? async_smem(backward, (size_t)elem_bytes) : 0;
   const int64_t NV = N / vec;
   Geom &g = p.g;
   g.M = M;
@@ -311,7 +315,7 @@ dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjac
   int occ = 1;
   if (pc.async) {
     // One CTA per SM by construction (__launch_bounds__(B, 1), ring sized for it).
-    st = prepare_smem(dev, k, (int)async_smem(backward));
+    st = prepare_smem(dev, k, (int)async_smem(backward, sizeof(T)));
     if (st != DYT_OK) return st;
   } else {
     st = occupancy(dev, k, kScalarBlock, &occ);

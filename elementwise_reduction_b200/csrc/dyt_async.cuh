@@ -211,11 +211,15 @@ __global__ void __launch_bounds__(B, 1)
                          double *__restrict__ part_dg, double *__restrict__ part_db, double *__restrict__ part_da,
                          Geom g) {
   using IO = VecIO<T, VEC>;
+  constexpr bool EXACT_G = ExactGamma<T>::value;
+  constexpr int kRunBlocks = kGammaRunRows / S;  // unrolled blocks of S rows per binary32 dgamma run
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
   static_assert(2 * VEC * sizeof(double) <= 2 * S * 16, "the reduction fits in the drained ring");
+  static_assert(kRunBlocks >= 1, "a dgamma run holds at least one block");
   // [S][2][B] 16-byte slots; after an item's last row the ring is empty and
   // its first 2 VEC * B binary64 values (at most 64 KB) serve the row-lane
-  // reduction.
+  // reduction. Without EXACT_G, [VEC][B] binary64 dgamma totals follow the
+  // ring (each thread's own, flushed from its binary32 runs).
   extern __shared__ uint4 ring[];
   __shared__ double red_a[B / 32];
   prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
@@ -224,6 +228,7 @@ __global__ void __launch_bounds__(B, 1)
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
   double *red = reinterpret_cast<double *>(ring);
+  double *gtot = reinterpret_cast<double *>(ring + 2 * S * B) + threadIdx.x;  // [e * B]
   uint4 *slot0 = ring + threadIdx.x;
   double acc_a = 0.0;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
@@ -235,11 +240,12 @@ __global__ void __launch_bounds__(B, 1)
     const bool col_ok = ln.live && cv < g.NV;
     const int64_t c0 = (int64_t)cv * VEC;
     float gam[VEC];
-    BwdAcc<VEC> acc;
+    BwdAcc<VEC, EXACT_G> acc;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
-      acc.g[e] = 0.0;
+      acc.g[e] = 0;
       acc.b[e] = 0.0;
+      if (!EXACT_G) gtot[e * B] = 0.0;
     }
     if (col_ok) {
       int64_t first;
@@ -272,9 +278,10 @@ __global__ void __launch_bounds__(B, 1)
       }
       int64_t col[VEC];
       vector_columns<VEC, PK>(c0, g.Nc, col);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) gam[e] = 4.0f * load_param(pr.gamma, pr.gamma_dt, col[e]);  // see bwd_vector
+      load_params<VEC>(pr.gamma, pr.gamma_dt, col, 4.0f, gam);  // 4 gamma (see bwd_vector)
+      int run = 0;  // blocks in the current binary32 dgamma run
       for (int k0 = 0; k0 < nn; k0 += S) {
+        float2 ca = make_float2(0.0f, 0.0f);  // this block's dalpha terms (at most S VEC / 2 per lane)
 #pragma unroll
         for (int j = 0; j < S; ++j) {
           const int k = k0 + j;
@@ -296,27 +303,37 @@ __global__ void __launch_bounds__(B, 1)
           cp_async_wait<S - 1>();
           const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
           const typename IO::Raw rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
-          float2 ca = make_float2(0.0f, 0.0f);
           if (PK && k == nn - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
-            store_first<T, VEC>(pdx, bwd_vector<T, VEC, true>(rx, rd, alpha, gam, acc, ca, nl), nl);
+            store_first<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, nl), nl);
           } else {
-            IO::store_raw(pdx, bwd_vector<T, VEC, false>(rx, rd, alpha, gam, acc, ca, VEC));
+            IO::store_raw(pdx, bwd_vector<T, VEC, false, EXACT_G>(rx, rd, alpha, gam, acc, ca, VEC));
           }
-          acc_a += (double)ca.x;
-          acc_a += (double)ca.y;
           pdx += so;
+        }
+        acc_a += (double)ca.x;
+        acc_a += (double)ca.y;
+        if (!EXACT_G && ++run == kRunBlocks) {  // end of a binary32 dgamma run
+          run = 0;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            gtot[e * B] += (double)acc.g[e];
+            acc.g[e] = 0;
+          }
         }
       }
       cp_async_wait<0>();
     }
     // ---- item done: per-(group, column) partials ----
+    double ag[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) ag[e] = EXACT_G ? (double)acc.g[e] : gtot[e * B] + (double)acc.g[e];
     double *pg = part_dg + (int64_t)rg * g.N;
     double *pb = part_db + (int64_t)rg * g.N;
     if (g.RL == 1) {
       if (col_ok) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          pg[c0 + e] = acc.g[e];
+          pg[c0 + e] = ag[e];
           pb[c0 + e] = acc.b[e];
         }
       }
@@ -324,11 +341,11 @@ __global__ void __launch_bounds__(B, 1)
       __syncthreads();  // every thread's ring is drained: reuse it for the reduction
       if ((32 % g.NV) == 0) {
         // the chunk's columns start at 0 on the row-tiled path (one chunk)
-        lane_reduce_warps<VEC, B>(acc.g, acc.b, red, g, ln, 0, pg, pb);
+        lane_reduce_warps<VEC, B>(ag, acc.b, red, g, ln, 0, pg, pb);
       } else {  // dgamma and dbeta sums in one tree: 2 VEC values per thread
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          red[e * B + threadIdx.x] = acc.g[e];
+          red[e * B + threadIdx.x] = ag[e];
           red[(VEC + e) * B + threadIdx.x] = acc.b[e];
         }
         __syncthreads();

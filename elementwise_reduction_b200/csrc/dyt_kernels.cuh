@@ -23,17 +23,21 @@
 //   - rows are cut into nrg balanced contiguous groups; a work item is
 //     (column chunk, row group) and CTA b takes items b, b + grid, ... (a
 //     static schedule: the same inputs always give the same bits).
-// Backward sums: each thread accumulates dgamma and dbeta of its columns in
-// binary64 (the product dy * t is exact there), the row lanes of a CTA are
-// added in binary64 in a fixed order, and each (group, column) partial goes
-// to the workspace in binary64; dalpha is carried in binary64 per thread and
-// reduced per CTA in a fixed order. The finalize adds the partials in
-// binary64 in a fixed order and rounds each gradient once.
+// Backward sums: each thread accumulates dbeta of its columns in binary64, and
+// dgamma in binary64 (binary32 activations) or in binary32 runs of at most
+// kGammaRunRows rows flushed into binary64 (16-bit activations); the row
+// lanes of a CTA are added in binary64 in a fixed order, and each (group,
+// column) partial goes to the workspace in binary64; dalpha is carried in
+// binary64 per thread (binary32 within a few rows) and reduced per CTA in a
+// fixed order. The finalize adds the partials in binary64 in a fixed order and
+// rounds each gradient once.
 // Lanes outside [0,M) x [0,N) never enter a sum: their contribution is
 // dropped by a select after the arithmetic (the page's Summary, "Padding").
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "dyt_math.cuh"
 
@@ -328,12 +332,10 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw fwd_vector(const typename
 template <typename T, int VEC>
 __device__ __forceinline__ void fwd_params_at(const Params &pr, const int64_t (&col)[VEC], float (&gam)[VEC],
                                               float (&bet)[VEC], float (&bth)[VEC]) {
+  load_params<VEC>(pr.gamma, pr.gamma_dt, col, 1.0f, gam);
+  load_params<VEC>(pr.beta, pr.beta_dt, col, 1.0f, bet);
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) {
-    gam[e] = load_param(pr.gamma, pr.gamma_dt, col[e]);
-    bet[e] = load_param(pr.beta, pr.beta_dt, col[e]);
-    bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
-  }
+  for (int e = 0; e < VEC; ++e) bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
 }
 
 // Forward for matrices that are not 16-byte aligned: one element per access,
@@ -461,25 +463,42 @@ __device__ __forceinline__ void lane_reduce_warps(const double (&vg)[VEC], const
   __syncthreads();
 }
 
-// Per-thread backward state for VEC columns, in binary64.
-template <int VEC>
+// Whether a kernel over activations of type T adds the dgamma terms in
+// binary64 (exact products dy * t, no rounding of the running sum). The
+// 16-bit kernels carry twice the elements per byte, and a binary32 -> binary64
+// conversion per term would take the special-function pipe (shared with the
+// exp2 and reciprocal of tanh) past its rate: they add dgamma in binary32
+// runs of at most kGammaRunRows rows, each flushed into a binary64 total.
+template <typename T>
+struct ExactGamma {
+  static constexpr bool value = sizeof(T) == 4;
+};
+constexpr int kGammaRunRows = 126;
+
+// Per-thread backward state for VEC columns. dbeta is always a binary64 sum:
+// its terms dy are exact there, so the sum carries no rounding error until the
+// final one. dgamma is binary64 (EXACT_G) or the current binary32 run.
+template <int VEC, bool EXACT_G>
 struct BwdAcc {
-  double g[VEC];  // sum of dy * t over this group's rows
+  using GT = typename std::conditional<EXACT_G, double, float>::type;
+  GT g[VEC];      // sum of dy * t over this group's rows (or the current run)
   double b[VEC];  // sum of dy
 };
 
 // One vector (one row, VEC columns): dx out, sums in. g4[e] = 4 gamma[e]
 // (with q = (1 - t^2) / 4, g4 * dy * q rounds exactly as gamma * dy * (1 - t^2)).
-// dgamma and dbeta terms are added in binary64: dy * t is exact there (a
-// product of two binary32 values), so these sums carry only t's own error.
+// dbeta's terms dy, and with EXACT_G dgamma's terms dy * t (a product of two
+// binary32 values), are exact in binary64; ca collects the dalpha terms of the
+// row in binary32 (the caller moves it into binary64 every few rows).
 // MASKED: only the first nvalid elements are real (0 for a padded row, fewer
 // than VEC for the vector that straddles the end of a packed matrix); the
 // others are computed like any other and their results dropped afterwards.
-template <typename T, int VEC, bool MASKED>
+template <typename T, int VEC, bool MASKED, bool EXACT_G>
 __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename VecIO<T, VEC>::Raw &rx,
                                                                  const typename VecIO<T, VEC>::Raw &rdy,
                                                                  float alpha, const float (&g4)[VEC],
-                                                                 BwdAcc<VEC> &acc, float2 &ca, int nvalid) {
+                                                                 BwdAcc<VEC, EXACT_G> &acc, float2 &ca,
+                                                                 int nvalid) {
   using IO = VecIO<T, VEC>;
   if constexpr (IO::kPairs > 0) {
     constexpr int H = IO::kPairs;
@@ -493,7 +512,16 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       const float2 gdys = mul2(mul2(make_float2(g4[2 * h], g4[2 * h + 1]), dy2[h]), q);  // gamma dy (1-t^2)
       dx2[h] = mul2(f2(alpha), gdys);
       const double d0 = (double)dy2[h].x, d1 = (double)dy2[h].y;
-      double ng0 = fma(d0, (double)t.x, acc.g[2 * h]), ng1 = fma(d1, (double)t.y, acc.g[2 * h + 1]);
+      using GT = typename BwdAcc<VEC, EXACT_G>::GT;
+      GT ng0, ng1;
+      if constexpr (EXACT_G) {
+        ng0 = fma(d0, (double)t.x, acc.g[2 * h]);
+        ng1 = fma(d1, (double)t.y, acc.g[2 * h + 1]);
+      } else {
+        const float2 ng = fma2(dy2[h], t, make_float2(acc.g[2 * h], acc.g[2 * h + 1]));
+        ng0 = ng.x;
+        ng1 = ng.y;
+      }
       double nb0 = acc.b[2 * h] + d0, nb1 = acc.b[2 * h + 1] + d1;
       float2 nca = fma2(gdys, x2[h], ca);
       if (MASKED) {  // drop padded elements' results, after the arithmetic
@@ -521,6 +549,7 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       dyt_tanh_qsech2(alpha * xf[e], t, q);
       const float gdys = (g4[e] * dyf[e]) * q;
       dxf[e] = alpha * gdys;
+      static_assert(EXACT_G, "the one-element kernels add dgamma in binary64");
       const double d = (double)dyf[e];
       const double ng = fma(d, (double)t, acc.g[e]), nb = acc.b[e] + d;
       const float nca = fmaf(gdys, xf[e], ca.x);
@@ -558,7 +587,7 @@ __global__ void __launch_bounds__(B, 1)
     const int cv = cc * B + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
     float gam[1] = {col_ok ? 4.0f * load_param(pr.gamma, pr.gamma_dt, cv) : 0.0f};  // 4 gamma (see bwd_vector)
-    BwdAcc<1> acc;
+    BwdAcc<1, true> acc;
     acc.g[0] = 0.0;
     acc.b[0] = 0.0;
     if (col_ok) {
@@ -577,14 +606,14 @@ __global__ void __launch_bounds__(B, 1)
 #pragma unroll
           for (int u = 0; u < U; ++u) {
             const int64_t row = r0 + (int64_t)u * g.RL;
-            IO::store_raw(dx + row * g.ldo + cv, bwd_vector<T, 1, false>(rx[u], rdy[u], alpha, gam, acc, ca, 1));
+            IO::store_raw(dx + row * g.ldo + cv, bwd_vector<T, 1, false, true>(rx[u], rdy[u], alpha, gam, acc, ca, 1));
           }
         } else {  // ragged last step of the group
 #pragma unroll
           for (int u = 0; u < U; ++u) {
             const int64_t row = r0 + (int64_t)u * g.RL;
             const bool ok = row < re;
-            const T d = bwd_vector<T, 1, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok ? 1 : 0);
+            const T d = bwd_vector<T, 1, true, true>(rx[u], rdy[u], alpha, gam, acc, ca, ok ? 1 : 0);
             if (ok) IO::store_raw(dx + row * g.ldo + cv, d);
           }
         }
@@ -640,8 +669,10 @@ __global__ void __launch_bounds__(kFinThreads)
     dyt_finalize_kernel(const double *__restrict__ part_dg, const double *__restrict__ part_db,
                         const double *__restrict__ part_da, GradOut out, int64_t N, int nrg, int nda, int CT) {
   __shared__ double sg[kFinThreads], sb[kFinThreads], sa[kFinThreads / 32];
-  // Wait until the stage-1 grid has finished and its writes are visible.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // Wait until the stage-1 grid has finished and its writes are visible, then
+  // let the next grid in the stream get scheduled (it waits for this one to
+  // finish before touching memory).
+  pdl_prologue();
   const int tid = threadIdx.x;
   const int L = kFinThreads / CT;
   const int lane = tid / CT, c = tid - lane * CT;

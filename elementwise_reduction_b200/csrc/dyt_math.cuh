@@ -189,6 +189,34 @@ __device__ __forceinline__ float load_param(const void *p, int dt, int64_t i) {
   return dt == DYT_BF16 ? __uint_as_float((uint32_t)u << 16) : __half2float(__ushort_as_half(u));
 }
 
+// The parameter values at indices col[0..V) as binary32, scaled by `scale`
+// (exact: a power of two). One dispatch on the dtype for all V loads, so the
+// loads are issued back to back and their latencies overlap.
+template <int V>
+__device__ __forceinline__ void load_params(const void *p, int dt, const int64_t (&col)[V], float scale,
+                                            float (&out)[V]) {
+  if (dt == DYT_F32) {
+    const float *q = static_cast<const float *>(p);
+    float v[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) v[e] = __ldg(q + col[e]);
+#pragma unroll
+    for (int e = 0; e < V; ++e) out[e] = scale * v[e];
+  } else {
+    const unsigned short *q = static_cast<const unsigned short *>(p);
+    unsigned short v[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) v[e] = __ldg(q + col[e]);
+    if (dt == DYT_BF16) {
+#pragma unroll
+      for (int e = 0; e < V; ++e) out[e] = scale * __uint_as_float((uint32_t)v[e] << 16);
+    } else {
+#pragma unroll
+      for (int e = 0; e < V; ++e) out[e] = scale * __half2float(__ushort_as_half(v[e]));
+    }
+  }
+}
+
 // v rounded once (nearest, ties to even) to dtype dt and stored at p[i].
 __device__ __forceinline__ void store_param(void *p, int dt, int64_t i, double v) {
   if (dt == DYT_F32) {

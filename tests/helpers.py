@@ -11,7 +11,10 @@ Tolerances (stated once, used by every parity test):
                      bounds the relative error of the kernels' binary32 t, and
                      |sum dy (t_gpu - t)| <= eps_t sum |dy t| = eps_t S. With alpha
                      = 0 or +-inf every t is exact (0 or +-1) and the bound is the
-                     stated one.
+                     stated one. Over 16-bit activations the kernels add dgamma in
+                     binary32 runs of at most 126 rows (then binary64), which adds
+                     126 2^-24 S: in all at most 8.2e-6 S, within the 1e-5 S that
+                     the sum-magnitude reading allows.
                      16-bit parameter gradients also pass within one unit of the
                      correctly rounded oracle value.
   dalpha             |g - o| <= 1e-5 S, S = sum of |term| (exact when S = 0).
@@ -103,6 +106,7 @@ def check_elementwise(got: np.ndarray, o64: np.ndarray, dtype: str, what: str) -
 
 
 T_REL_ERR = 2.0 ** -20.5  # relative error bound of the kernels' binary32 tanh (checked by a sweep test)
+GAMMA_RUN_ERR = 126 * 2.0 ** -24  # binary32 dgamma runs of the 16-bit kernels: at most 126 roundings
 
 
 def t_is_exact(alpha: float) -> bool:
@@ -258,7 +262,8 @@ def compare_all(inp: dict, out: dict, M: int, N: int, x_dtype: str, p_dtype, row
     if "dgamma" in out:
         r = oracle.backward(inp["x"], inp["dy"], inp["alpha"], inp["gamma"], M, N, x_dtype, p_dtype,
                             want_dx=False)
-        t_err = 0.0 if t_is_exact(_alpha_value(inp, p_dtype)) else T_REL_ERR
+        t_err = (0.0 if t_is_exact(_alpha_value(inp, p_dtype)) else T_REL_ERR) + \
+            (0.0 if x_dtype == "f32" else GAMMA_RUN_ERR)
         stats["dgamma"] = check_sums(out["dgamma"], r["dgamma"], r["mag_dgamma"], gd, "dgamma", M, t_err)
         stats["dbeta"] = check_sums(out["dbeta"], r["dbeta"], r["mag_dbeta"], bd, "dbeta", M)
         stats["dalpha"] = check_scalar_sum(out["dalpha"], r["dalpha"], r["mag_dalpha"], "dalpha", ad)

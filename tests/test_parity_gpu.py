@@ -562,7 +562,7 @@ def test_workload_full_size(name):
     stats = H.compare_all(inp, out, w.M, w.N, w.x_dtype, w.p_dtype)
     print(name, info, stats)
     assert stats["dbeta"]["n_over_strict_elementwise"] == 0
-    if H.t_is_exact(w.alpha):
+    if H.t_is_exact(w.alpha) and w.x_dtype == "f32":  # binary64 dgamma terms, each exact
         assert stats["dgamma"]["n_over_strict_elementwise"] == 0
     if w.N <= 256:
         assert info["bwd"]["path"] == 1

@@ -415,21 +415,47 @@ def run_ours(args, w):
     sets, (alpha, gamma, beta), set_bytes, nsets = _sets(w, inp, dev, L2)
     ws = dyt.workspace(sets[0]["x"], gamma)
     grads = torch.empty(2 * N + 1, dtype=torch.float32, device=dev)
-    from elementwise_reduction_b200.dist import allreduce_param_grads
+    from elementwise_reduction_b200.dist import FusedGradientSum, allreduce_param_grads
+
+    def make_exchange():
+        """The fused cross-rank gradient sum, or None (every rank then falls back to the
+        all-reduce of the rounded gradients): the ranks decide together."""
+        if world == 1:
+            return None, None
+        ex, why = None, None
+        try:
+            ex = FusedGradientSum(sets[0]["x"], sets[0]["dy"], sets[0]["dx"], gamma)
+        except Exception as e:  # e.g. memory that CUDA IPC cannot share
+            why = f"{type(e).__name__}: {e}"
+        ok = torch.tensor([0 if ex is None else 1], dtype=torch.int32, device=dev)
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN)
+        if int(ok.item()) == 0:
+            if ex is not None:
+                ex.close()
+            return None, why or "another rank could not map the peer workspaces"
+        return ex, None
+
+    exchange, exchange_note = make_exchange()
+    sched = FusedGradientSum.schedule(max(2, args.steps)) if exchange is not None else None
 
     def fwd(s):
         dyt.forward(s["x"], alpha, gamma, beta, out=s["y"])
 
-    def bwd(s, ws_=None):
+    def bwd(s, ws_=None, i=None, ex=None, gbuf=None):
+        ex = exchange if ex is None else ex
+        if ex is not None:  # stage 1, barrier, finalize over every rank's partials
+            ex(s["x"], s["dy"], alpha, gamma, beta, s["dx"], s["dg"], s["db"], s["da"],
+               buffer=None if i is None else sched[i % len(sched)])
+            return
         dyt.backward(s["x"], s["dy"], alpha, gamma, beta, dx=s["dx"], dgamma=s["dg"], dbeta=s["db"],
                      dalpha=s["da"], ws=ws if ws_ is None else ws_)
+        if world > 1:
+            allreduce_param_grads(s["dg"], s["db"], s["da"], buf=grads if gbuf is None else gbuf)
 
     def step(i):
         s = sets[i % nsets]
         fwd(s)
-        bwd(s)
-        if world > 1:
-            allreduce_param_grads(s["dg"], s["db"], s["da"], buf=grads)
+        bwd(s, i=i)
 
     stream = torch.cuda.Stream(dev)
     torch.cuda.synchronize(dev)
@@ -437,10 +463,12 @@ def run_ours(args, w):
         for i in range(args.warmup):
             step(i)
         torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()  # every rank's eager calls are done before any replay reuses a workspace
         g_step = _graph(stream, step, args.steps)
         g_fwd = _graph(stream, lambda i: fwd(sets[i % nsets]), args.steps)
         launch_info_fwd = dyt.dyt_last_launch_info()
-        g_bwd = _graph(stream, lambda i: bwd(sets[i % nsets]), args.steps)
+        g_bwd = _graph(stream, lambda i: bwd(sets[i % nsets], i=i), args.steps)
         launch_info_bwd = dyt.dyt_last_launch_info()
         for g in (g_step, g_fwd, g_bwd):  # untimed replay: first-launch costs
             g.replay()
@@ -480,6 +508,9 @@ def run_ours(args, w):
                 torch.cuda.synchronize(dev)
         clocks = clk.summary()
         del g_step, g_fwd, g_bwd  # graphs that may hold NCCL calls go before the process group
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
 
     # ---- end to end through the public API: pinned host buffers in, results out ----
     # Consecutive steps alternate between two streams, each with its own device
@@ -498,6 +529,7 @@ def run_ours(args, w):
                                        "dg": torch.empty_like(gamma), "db": torch.empty_like(beta),
                                        "da": torch.empty_like(alpha)}
         lanes.append({"dev": d, "ws": dyt.workspace(x0, gamma), "stream": stream if j == 0 else torch.cuda.Stream(dev),
+                      "ex": exchange if j == 0 or exchange is None else FusedGradientSum(x0, x0, x0, gamma),
                       "grads": torch.empty(2 * N + 1, dtype=torch.float32, device=dev),
                       "hy": torch.empty_like(hx).pin_memory(), "hdx": torch.empty_like(hx).pin_memory(),
                       "hdg": torch.empty(N, dtype=gamma.dtype).pin_memory(),
@@ -511,9 +543,7 @@ def run_ours(args, w):
             d["x"].copy_(hx, non_blocking=True)
             d["dy"].copy_(hdy, non_blocking=True)
             fwd(d)
-            bwd(d, ln["ws"])
-            if world > 1:
-                allreduce_param_grads(d["dg"], d["db"], d["da"], buf=ln["grads"])
+            bwd(d, ln["ws"], ex=ln["ex"], gbuf=ln["grads"])
             ln["hy"].copy_(d["y"], non_blocking=True)
             ln["hdx"].copy_(d["dx"], non_blocking=True)
             ln["hdg"].copy_(d["dg"], non_blocking=True)
@@ -542,6 +572,14 @@ def run_ours(args, w):
     sa, sg, sb = (workloads.ITEMSIZE[d] for d in w.param_dtypes)
     h2d = 2 * M * N * sx
     d2h = 2 * M * N * sx + N * (sg + sb) + sa
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()  # no rank still reads a peer's workspace
+    for ln in lanes:
+        if ln["ex"] is not None and ln["ex"] is not exchange:
+            ln["ex"].close()
+    if exchange is not None:
+        exchange.close()
     del lanes, sets, ws
     torch.cuda.empty_cache()
 
@@ -581,7 +619,11 @@ def run_ours(args, w):
         "e2e": {"value": (fb + bb) * world * e2e_steps / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": ms_e2e / e2e_steps},
-        "gpu_launches": args.steps * (launch_info_fwd["kernels"] + launch_info_bwd["kernels"]),
+        "gpu_launches": args.steps * (launch_info_fwd["kernels"] + (2 if world > 1 and exchange is not None
+                                                                     else launch_info_bwd["kernels"])),
+        "grad_exchange": None if world == 1 else (
+            "finalize over every rank's partials through peer pointers, after a one-element NCCL all-reduce"
+            if exchange is not None else f"NCCL all-reduce of the rounded gradients ({exchange_note})"),
         "clocks": clocks,
     }
     if world > 1:

@@ -13,14 +13,19 @@ from __future__ import annotations
 import torch
 
 from . import _abi
-from ._abi import (DYT_BF16, DYT_F16, DYT_F32, DytError, dyt_backward, dyt_backward_ex, dyt_backward_noalloc,
-                   dyt_backward_strided, dyt_backward_workspace_bytes, dyt_forward, dyt_forward_ex,
-                   dyt_forward_strided, dyt_last_launch_info, dyt_plan_query, dyt_status_string)
+from ._abi import (DYT_BF16, DYT_F16, DYT_F32, MAX_RANKS, DytError, dyt_backward, dyt_backward_ex,
+                   dyt_backward_noalloc, dyt_backward_partials, dyt_backward_strided, dyt_backward_workspace_bytes,
+                   dyt_finalize_partials, dyt_forward, dyt_forward_ex, dyt_forward_strided, dyt_ipc_close,
+                   dyt_ipc_export, dyt_ipc_import, dyt_last_launch_info, dyt_partials_layout_query, dyt_plan_query,
+                   dyt_status_string)
 
-__all__ = ["forward", "backward", "workspace", "DyT", "DyTFunction", "dyt_forward", "dyt_backward",
-           "dyt_forward_strided", "dyt_backward_strided", "dyt_forward_ex", "dyt_backward_ex",
-           "dyt_backward_noalloc", "row_pitch", "dyt_backward_workspace_bytes", "dyt_status_string",
-           "dyt_last_launch_info", "dyt_plan_query", "DytError", "DTYPE_CODE", "DYT_F32", "DYT_BF16", "DYT_F16"]
+__all__ = ["forward", "backward", "workspace", "backward_partials", "partials_layout", "finalize_partials", "DyT",
+           "DyTFunction", "dyt_forward", "dyt_backward", "dyt_forward_strided", "dyt_backward_strided",
+           "dyt_forward_ex", "dyt_backward_ex", "dyt_backward_noalloc", "dyt_backward_partials",
+           "dyt_partials_layout_query", "dyt_finalize_partials", "dyt_ipc_export", "dyt_ipc_import",
+           "dyt_ipc_close", "row_pitch", "dyt_backward_workspace_bytes", "dyt_status_string",
+           "dyt_last_launch_info", "dyt_plan_query", "DytError", "DTYPE_CODE", "DYT_F32", "DYT_BF16", "DYT_F16",
+           "MAX_RANKS"]
 
 DTYPE_CODE = {torch.float32: DYT_F32, torch.bfloat16: DYT_BF16, torch.float16: DYT_F16}
 
@@ -146,6 +151,58 @@ def backward(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, gamma: torc
                              _stream(x.device, stream))
     _abi._check(st, "dyt_backward")
     return dx, dalpha, dgamma, dbeta
+
+
+def backward_partials(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor,
+                      ws: torch.Tensor, dx: torch.Tensor | None = None,
+                      stream: torch.cuda.Stream | None = None):
+    """Stage 1 of the backward: (dx, layout). dx in x's dtype; the binary64 partial
+    sums of the parameter gradients stay in ws, where `layout` (a dict) says."""
+    for t, w in ((alpha, "alpha"), (gamma, "gamma")):
+        _cuda_contig(t, w)
+    if dy.shape != x.shape or dy.dtype != x.dtype:
+        raise ValueError("dy must match x in shape and dtype")
+    ldx, lddy = _rows(x, "x"), _rows(dy, "dy")
+    M, N = _shape(x, gamma)
+    dx = torch.empty(x.shape, dtype=x.dtype, device=x.device) if dx is None else dx
+    if dx.shape != x.shape or dx.dtype != x.dtype:
+        raise ValueError("dx must match x in shape and dtype")
+    lddx = _rows(dx, "dx")
+    with torch.cuda.device(x.device):
+        st, layout = dyt_backward_partials(x.data_ptr(), ldx, dy.data_ptr(), lddy, alpha.data_ptr(), gamma.data_ptr(),
+                                           dx.data_ptr(), lddx, M, N, _code(x, "x"), _code(alpha, "alpha"),
+                                           _code(gamma, "gamma"), ws.data_ptr(), ws.numel(),
+                                           _stream(x.device, stream))
+    _abi._check(st, "dyt_backward_partials")
+    return dx, layout
+
+
+def partials_layout(x: torch.Tensor, dy: torch.Tensor, dx: torch.Tensor, N: int) -> dict:
+    """The partials layout backward_partials reports for these tensors (no launch)."""
+    M = x.numel() // N if N else 0
+    with torch.cuda.device(x.device):
+        return dyt_partials_layout_query(x.data_ptr(), _rows(x, "x"), dy.data_ptr(), _rows(dy, "dy"), dx.data_ptr(),
+                                         _rows(dx, "dx"), M, N, _code(x, "x"))
+
+
+def finalize_partials(workspaces, layouts, alpha: torch.Tensor, gamma: torch.Tensor,
+                      beta: torch.Tensor | None = None, dgamma: torch.Tensor | None = None,
+                      dbeta: torch.Tensor | None = None, dalpha: torch.Tensor | None = None,
+                      stream: torch.cuda.Stream | None = None):
+    """(dalpha, dgamma, dbeta) from the partials of several stage-1 launches:
+    workspaces are device pointers (ints) the current device can read, one per
+    rank, layouts their layouts, summed in that order and rounded once."""
+    N = gamma.numel()
+    beta_like = gamma if beta is None else beta
+    dgamma = torch.empty_like(gamma) if dgamma is None else dgamma
+    dbeta = torch.empty_like(beta_like) if dbeta is None else dbeta
+    dalpha = torch.empty(1, dtype=alpha.dtype, device=alpha.device) if dalpha is None else dalpha
+    with torch.cuda.device(gamma.device):
+        st = dyt_finalize_partials(list(workspaces), list(layouts), N, dgamma.data_ptr(), dbeta.data_ptr(),
+                                   dalpha.data_ptr(), _code(alpha, "alpha"), _code(gamma, "gamma"),
+                                   _code(beta_like, "beta"), _stream(gamma.device, stream))
+    _abi._check(st, "dyt_finalize_partials")
+    return dalpha, dgamma, dbeta
 
 
 class DyTFunction(torch.autograd.Function):

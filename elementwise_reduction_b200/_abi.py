@@ -60,6 +60,51 @@ lib.dyt_last_launch_info.argtypes = [ctypes.POINTER(LaunchInfo)]
 lib.dyt_last_launch_info.restype = _i32
 lib.dyt_plan_query.argtypes = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(LaunchInfo)]
 lib.dyt_plan_query.restype = _i32
+class PartialsLayout(ctypes.Structure):
+    """dyt_partials_layout: where a stage-1 launch left its binary64 partials."""
+    _fields_ = [("bytes", _i64), ("off_dgamma", _i64), ("off_dbeta", _i64), ("off_dalpha", _i64),
+                ("rows", ctypes.c_int32), ("dalpha_parts", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+    @classmethod
+    def from_dict(cls, d: dict) -> "PartialsLayout":
+        return cls(**{name: d[name] for name, _ in cls._fields_})
+
+
+class IpcHandle(ctypes.Structure):
+    """dyt_ipc_handle: a CUDA IPC memory handle and a byte offset in its allocation."""
+    _fields_ = [("bytes", ctypes.c_ubyte * 64), ("offset", _i64)]
+
+    def to_bytes(self) -> bytes:
+        return bytes(self.bytes) + int(self.offset).to_bytes(8, "little", signed=True)
+
+    @classmethod
+    def from_bytes(cls, b: bytes) -> "IpcHandle":
+        h = cls()
+        ctypes.memmove(h.bytes, b[:64], 64)
+        h.offset = int.from_bytes(b[64:72], "little", signed=True)
+        return h
+
+
+MAX_RANKS = 8  # DYT_MAX_RANKS in include/dyt.h
+
+lib.dyt_backward_partials.argtypes = [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _vp,
+                                      _sz, ctypes.POINTER(PartialsLayout), _vp]
+lib.dyt_backward_partials.restype = _i32
+lib.dyt_partials_layout_query.argtypes = [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _i32,
+                                          ctypes.POINTER(PartialsLayout)]
+lib.dyt_partials_layout_query.restype = _i32
+lib.dyt_finalize_partials.argtypes = [ctypes.POINTER(_vp), ctypes.POINTER(PartialsLayout), _i32, _i64, _vp, _vp, _vp,
+                                      _i32, _i32, _i32, _vp]
+lib.dyt_finalize_partials.restype = _i32
+lib.dyt_ipc_export.argtypes = [_vp, ctypes.POINTER(IpcHandle)]
+lib.dyt_ipc_export.restype = _i32
+lib.dyt_ipc_import.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(_vp)]
+lib.dyt_ipc_import.restype = _i32
+lib.dyt_ipc_close.argtypes = [_vp, ctypes.POINTER(IpcHandle)]
+lib.dyt_ipc_close.restype = _i32
 lib.dyt_backward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp]
 lib.dyt_backward_noalloc.restype = _i32
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # DYT_NOALLOC_SCRATCH_BYTES in include/dyt.h
@@ -128,6 +173,53 @@ def dyt_backward_noalloc(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M
     instead of a workspace (for callers that cannot allocate). Returns the status."""
     return lib.dyt_backward_noalloc(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype,
                                     param_dtype, stream)
+
+
+def dyt_backward_partials(x, ldx, dy, lddy, alpha, gamma, dx, lddx, M, N, x_dtype, alpha_dtype, gamma_dtype,
+                          workspace, workspace_bytes, stream):
+    """Raw C-ABI call of stage 1. Returns (status, layout dict)."""
+    lay = PartialsLayout()
+    st = lib.dyt_backward_partials(x, ldx, dy, lddy, alpha, gamma, dx, lddx, M, N, x_dtype, alpha_dtype, gamma_dtype,
+                                   workspace, workspace_bytes, ctypes.byref(lay), stream)
+    return st, lay.as_dict()
+
+
+def dyt_partials_layout_query(x, ldx, dy, lddy, dx, lddx, M, N, x_dtype) -> dict:
+    """The partials layout stage 1 would report for these tensors (host arithmetic only)."""
+    lay = PartialsLayout()
+    _check(lib.dyt_partials_layout_query(x, ldx, dy, lddy, dx, lddx, M, N, x_dtype, ctypes.byref(lay)),
+           "dyt_partials_layout_query")
+    return lay.as_dict()
+
+
+def dyt_finalize_partials(workspaces, layouts, N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype,
+                          stream) -> int:
+    """Raw C-ABI call: workspaces a list of device pointers (ints), layouts a list of dicts."""
+    n = len(workspaces)
+    ws = (_vp * max(1, n))(*workspaces)
+    lays = (PartialsLayout * max(1, n))(*[PartialsLayout.from_dict(d) for d in layouts])
+    return lib.dyt_finalize_partials(ws, lays, n, N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype,
+                                     stream)
+
+
+def dyt_ipc_export(ptr: int) -> bytes:
+    """72 bytes: the CUDA IPC handle of ptr's allocation and ptr's offset in it."""
+    h = IpcHandle()
+    _check(lib.dyt_ipc_export(ptr, ctypes.byref(h)), "dyt_ipc_export")
+    return h.to_bytes()
+
+
+def dyt_ipc_import(handle: bytes) -> int:
+    """A device pointer (int) to the exported bytes, readable from the current device."""
+    h = IpcHandle.from_bytes(handle)
+    p = _vp()
+    _check(lib.dyt_ipc_import(ctypes.byref(h), ctypes.byref(p)), "dyt_ipc_import")
+    return int(p.value)
+
+
+def dyt_ipc_close(ptr: int, handle: bytes) -> None:
+    h = IpcHandle.from_bytes(handle)
+    _check(lib.dyt_ipc_close(ptr, ctypes.byref(h)), "dyt_ipc_close")
 
 
 def dyt_status_string(status: int) -> str:

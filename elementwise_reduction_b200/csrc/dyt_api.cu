@@ -345,6 +345,131 @@ struct PdlConfig {
   }
 };
 
+using MemGetAddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+// The partials' layout in the workspace of a backward plan.
+dyt_partials_layout layout_of(const Plan &p) {
+  dyt_partials_layout l = {};
+  l.bytes = (int64_t)p.ws_total;
+  l.off_dgamma = (int64_t)p.ws_dg;
+  l.off_dbeta = (int64_t)p.ws_db;
+  l.off_dalpha = (int64_t)p.ws_da;
+  // (nrg x pack rows) rows of N: a packed row group holds vec partial rows,
+  // one per row of the pack, in pack order.
+  l.rows = p.g.nrg * (p.packed ? p.vec : 1);
+  l.dalpha_parts = p.grid;
+  return l;
+}
+
+// The layout facts of a backward call's tensors: aligned, pitched, adjacent (see choose_path).
+struct LayoutArgs {
+  bool aligned, pitched, adjacent;
+};
+template <typename T>
+LayoutArgs stage1_layout_args(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *dx,
+                              int64_t lddx, int64_t N) {
+  const size_t es = sizeof(T);
+  return {aligned16(x) && aligned16(dy) && aligned16(dx),
+          vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es), ldx == N && lddy == N && lddx == N};
+}
+template <typename T>
+dyt_status plan_for(int64_t M, int64_t N, LayoutArgs a, bool backward, Plan *out) {
+  return plan_for<T>(M, N, a.aligned, a.pitched, a.adjacent, backward, out);
+}
+
+// Every gradient +0 (all-zero bits in each dtype): the empty sums.
+dyt_status zero_gradients(int64_t N, void *dgamma, void *dbeta, void *dalpha, dyt_dtype ad, dyt_dtype gd,
+                          dyt_dtype bd, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  if (N > 0) {
+    e = cudaMemsetAsync(dgamma, 0, (size_t)N * dsize(gd), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, (size_t)N * dsize(bd), s);
+  }
+  if (e == cudaSuccess) e = cudaMemsetAsync(dalpha, 0, dsize(ad), s);
+  return e == cudaSuccess ? DYT_OK : cuda_fail(e);
+}
+
+// Stage 1 of the backward (M, N > 0, arguments checked): dx and the binary64
+// partial sums in the workspace, laid out as *lay describes.
+dyt_status bwd_stage1(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha, const void *gamma,
+                      void *dx, int64_t lddx, int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype alpha_dtype,
+                      dyt_dtype gamma_dtype, void *workspace, size_t workspace_bytes, cudaStream_t s, Plan *plan,
+                      dyt_partials_layout *lay) {
+  if (!x || !dy || !alpha || !gamma || !dx || !workspace) return DYT_ERR_INVALID_VALUE;
+  if (!aligned16(workspace)) return DYT_ERR_INVALID_VALUE;
+  const dyt::Params pr = {alpha, gamma, nullptr, (int)alpha_dtype, (int)gamma_dtype, DYT_F32};
+  return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
+    using T = decltype(tx);
+    constexpr int V = vec_of<T>();
+    Plan &p = *plan;
+    dyt_status r = plan_for<T>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
+    if (r != DYT_OK) return r;
+    if (!p.packed) {
+      p.g.ldx = ldx;
+      p.g.ldd = lddy;
+      p.g.ldo = lddx;
+    }
+    if (workspace_bytes < p.ws_total) return DYT_ERR_WORKSPACE_TOO_SMALL;
+    char *ws = (char *)workspace;
+    double *pdg = (double *)(ws + p.ws_dg);
+    double *pdb = (double *)(ws + p.ws_db);
+    double *pda = (double *)(ws + p.ws_da);
+    PdlConfig lc(p.grid, p.block, p.smem, s);
+    cudaError_t e;
+    if (p.async && p.packed)
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, true>,
+                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
+    else if (p.async)
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, false>,
+                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
+    else
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_kernel<T, kScalarUnrollBwd, kScalarBlock>, (const T *)x,
+                             (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *lay = layout_of(p);
+    return DYT_OK;
+  });
+}
+
+// Stage 2 (N > 0, dtypes checked): the partials of `nranks` workspaces summed
+// in binary64 in a fixed order (rank by rank), each gradient rounded once.
+// Launched as a programmatic dependent: it may start while its predecessor in
+// the stream drains and waits (griddepcontrol.wait) for its results.
+dyt_status bwd_finalize(const void *const *wss, const dyt_partials_layout *lay, int nranks, int64_t N, void *dgamma,
+                        void *dbeta, void *dalpha, dyt_dtype ad, dyt_dtype gd, dyt_dtype bd, cudaStream_t s) {
+  dyt::PartsSet ps = {};
+  ps.nranks = nranks;
+  int64_t rows_max = 0;
+  for (int r = 0; r < nranks; ++r) {
+    const dyt_partials_layout &l = lay[r];
+    if (l.rows < 0 || l.dalpha_parts < 0) return DYT_ERR_INVALID_VALUE;
+    if (l.rows > 0 || l.dalpha_parts > 0) {
+      const char *w = (const char *)wss[r];
+      if (!w || !aligned16(w)) return DYT_ERR_INVALID_VALUE;
+      const int64_t part_bytes = (int64_t)l.rows * N * (int64_t)sizeof(double);
+      if (l.off_dgamma < 0 || l.off_dbeta < 0 || l.off_dalpha < 0 || l.off_dgamma + part_bytes > l.bytes ||
+          l.off_dbeta + part_bytes > l.bytes || l.off_dalpha + (int64_t)l.dalpha_parts * 8 > l.bytes)
+        return DYT_ERR_INVALID_VALUE;
+      ps.r[r].dg = (const double *)(w + l.off_dgamma);
+      ps.r[r].db = (const double *)(w + l.off_dbeta);
+      ps.r[r].da = (const double *)(w + l.off_dalpha);
+    }
+    ps.r[r].rows = l.rows;
+    ps.r[r].nda = l.dalpha_parts;
+    if (l.rows > rows_max) rows_max = l.rows;
+  }
+  // Lanes per column: enough that each lane reads at most four partials of a
+  // rank. Every rank that finalizes the same layouts picks the same L, so all
+  // get the same bits.
+  int L = 1;
+  while (L < dyt::kFinThreads && (int64_t)L * 4 < rows_max) L <<= 1;
+  const int CT = dyt::kFinThreads / L;
+  const dyt::GradOut go = {dgamma, dbeta, dalpha, (int)gd, (int)bd, (int)ad};
+  PdlConfig fc((unsigned)ceil_div(N, CT), dyt::kFinThreads, 0, s);
+  const cudaError_t e = cudaLaunchKernelEx(&fc.cfg, dyt::dyt_finalize_kernel, ps, go, (int64_t)N, CT);
+  return e == cudaSuccess ? DYT_OK : cuda_fail(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -451,72 +576,123 @@ dyt_status dyt_backward_ex(const void *x, int64_t ldx, const void *dy, int64_t l
   if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, lddy) != DYT_OK || check_pitch(M, N, lddx) != DYT_OK)
     return DYT_ERR_INVALID_VALUE;
   if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return DYT_ERR_INVALID_VALUE;
-  cudaStream_t s = (cudaStream_t)stream;
   if (M == 0 || N == 0) {
-    // Empty sums: every gradient is +0 (all-zero bits in each dtype).
-    cudaError_t e = cudaSuccess;
-    if (N > 0) {
-      e = cudaMemsetAsync(dgamma, 0, (size_t)N * dsize(gamma_dtype), s);
-      if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, (size_t)N * dsize(beta_dtype), s);
-    }
-    if (e == cudaSuccess) e = cudaMemsetAsync(dalpha, 0, dsize(alpha_dtype), s);
-    if (e != cudaSuccess) return cuda_fail(e);
-    record(2, nullptr, 0, 0);
+    st = zero_gradients(N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype, (cudaStream_t)stream);
+    if (st == DYT_OK) record(2, nullptr, 0, 0);
+    return st;
+  }
+  Plan p;
+  dyt_partials_layout lay;
+  st = bwd_stage1(x, ldx, dy, lddy, alpha, gamma, dx, lddx, M, N, x_dtype, alpha_dtype, gamma_dtype, workspace,
+                  workspace_bytes, (cudaStream_t)stream, &p, &lay);
+  if (st != DYT_OK) return st;
+  const void *wss[1] = {workspace};
+  st = bwd_finalize(wss, &lay, 1, N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype,
+                    (cudaStream_t)stream);
+  if (st != DYT_OK) return st;
+  record(2, &p, 2, p.ws_total);
+  return DYT_OK;
+}
+
+dyt_status dyt_backward_partials(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
+                                 const void *gamma, void *dx, int64_t lddx, int64_t M, int64_t N, dyt_dtype x_dtype,
+                                 dyt_dtype alpha_dtype, dyt_dtype gamma_dtype, void *workspace,
+                                 size_t workspace_bytes, dyt_partials_layout *layout, dyt_stream_t stream) {
+  if (!layout) return DYT_ERR_INVALID_VALUE;
+  dyt_status st = check_shape(M, N, x_dtype);
+  if (st == DYT_OK) st = check_param_dtypes(alpha_dtype, gamma_dtype, DYT_F32);
+  if (st != DYT_OK) return st;
+  if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, lddy) != DYT_OK || check_pitch(M, N, lddx) != DYT_OK)
+    return DYT_ERR_INVALID_VALUE;
+  if (M == 0 || N == 0) {  // no rows: no partials (a rank with an empty shard adds nothing)
+    *layout = dyt_partials_layout{};
+    record(3, nullptr, 0, 0);
     return DYT_OK;
   }
-  if (!x || !dy || !alpha || !gamma || !dx || !workspace) return DYT_ERR_INVALID_VALUE;
-  if (!aligned16(workspace)) return DYT_ERR_INVALID_VALUE;
-  const dyt::Params pr = {alpha, gamma, nullptr, (int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
-  const dyt::GradOut go = {dgamma, dbeta, dalpha, (int)gamma_dtype, (int)beta_dtype, (int)alpha_dtype};
+  Plan p;
+  st = bwd_stage1(x, ldx, dy, lddy, alpha, gamma, dx, lddx, M, N, x_dtype, alpha_dtype, gamma_dtype, workspace,
+                  workspace_bytes, (cudaStream_t)stream, &p, layout);
+  if (st == DYT_OK) record(3, &p, 1, p.ws_total);
+  return st;
+}
+
+dyt_status dyt_partials_layout_query(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *dx,
+                                     int64_t lddx, int64_t M, int64_t N, dyt_dtype x_dtype,
+                                     dyt_partials_layout *layout) {
+  if (!layout) return DYT_ERR_INVALID_VALUE;
+  dyt_status st = check_shape(M, N, x_dtype);
+  if (st != DYT_OK) return st;
+  if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, lddy) != DYT_OK || check_pitch(M, N, lddx) != DYT_OK)
+    return DYT_ERR_INVALID_VALUE;
+  if (M == 0 || N == 0) {
+    *layout = dyt_partials_layout{};
+    return DYT_OK;
+  }
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
-    constexpr int V = vec_of<T>();
     Plan p;
-    const size_t es = sizeof(T);
-    dyt_status r = plan_for<T>(M, N, aligned16(x) && aligned16(dy) && aligned16(dx),
-                               vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es),
-                               ldx == N && lddy == N && lddx == N, true, &p);
-    if (r != DYT_OK) return r;
-    if (!p.packed) {
-      p.g.ldx = ldx;
-      p.g.ldd = lddy;
-      p.g.ldo = lddx;
-    }
-    if (workspace_bytes < p.ws_total) return DYT_ERR_WORKSPACE_TOO_SMALL;
-    char *ws = (char *)workspace;
-    double *pdg = (double *)(ws + p.ws_dg);
-    double *pdb = (double *)(ws + p.ws_db);
-    double *pda = (double *)(ws + p.ws_da);
-
-    PdlConfig lc(p.grid, p.block, p.smem, s);
-    cudaError_t e;
-    if (p.async && p.packed)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, true>,
-                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
-    else if (p.async)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, false>,
-                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
-    else
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_kernel<T, kScalarUnrollBwd, kScalarBlock>, (const T *)x,
-                             (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
-    if (e != cudaSuccess) return cuda_fail(e);
-
-    // Stage 2, as a programmatic dependent launch: it may start while stage 1
-    // drains and waits (griddepcontrol.wait) for stage 1's results.
-    // The partials form (nrg x pack rows) rows of N columns: a packed row group
-    // holds vec partial rows, one per row of the pack, in pack order.
-    const int nparts = p.g.nrg * (p.packed ? p.vec : 1);
-    // Lanes per column: enough that each lane reads at most four partials.
-    int L = 1;
-    while (L < dyt::kFinThreads && (int64_t)L * 4 < nparts) L <<= 1;
-    const int CT = dyt::kFinThreads / L;
-    PdlConfig fc((unsigned)ceil_div(N, CT), dyt::kFinThreads, 0, s);
-    e = cudaLaunchKernelEx(&fc.cfg, dyt::dyt_finalize_kernel, (const double *)pdg, (const double *)pdb,
-                           (const double *)pda, go, (int64_t)N, nparts, p.grid, CT);
-    if (e != cudaSuccess) return cuda_fail(e);
-    record(2, &p, 2, p.ws_total);
-    return DYT_OK;
+    const dyt_status r = plan_for<T>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
+    if (r == DYT_OK) *layout = layout_of(p);
+    return r;
   });
+}
+
+dyt_status dyt_finalize_partials(const void *const *workspaces, const dyt_partials_layout *layouts, int nranks,
+                                 int64_t N, void *dgamma, void *dbeta, void *dalpha, dyt_dtype alpha_dtype,
+                                 dyt_dtype gamma_dtype, dyt_dtype beta_dtype, dyt_stream_t stream) {
+  if (!workspaces || !layouts || nranks < 1 || nranks > DYT_MAX_RANKS) return DYT_ERR_INVALID_VALUE;
+  dyt_status st = check_param_dtypes(alpha_dtype, gamma_dtype, beta_dtype);
+  if (st != DYT_OK) return st;
+  if (N < 0 || N > INT32_MAX) return DYT_ERR_INVALID_VALUE;
+  if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return DYT_ERR_INVALID_VALUE;
+  if (N == 0)
+    return zero_gradients(N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype, (cudaStream_t)stream);
+  st = bwd_finalize(workspaces, layouts, nranks, N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype,
+                    (cudaStream_t)stream);
+  if (st == DYT_OK) record(4, nullptr, 1, 0);
+  return st;
+}
+
+dyt_status dyt_ipc_export(const void *ptr, dyt_ipc_handle *out) {
+  if (!ptr || !out) return DYT_ERR_INVALID_VALUE;
+  static MemGetAddressRangeFn get_range = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_range = (MemGetAddressRangeFn)f;
+  });
+  if (!get_range) return cuda_fail(cudaErrorNotSupported);
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (get_range(&base, &size, (CUdeviceptr)(uintptr_t)ptr) != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  cudaIpcMemHandle_t h;
+  const cudaError_t e = cudaIpcGetMemHandle(&h, (void *)(uintptr_t)base);
+  if (e != cudaSuccess) return cuda_fail(e);
+  static_assert(sizeof(h) == sizeof(out->bytes), "CUDA IPC handles are 64 bytes");
+  memcpy(out->bytes, &h, sizeof(h));
+  out->offset = (int64_t)((uintptr_t)ptr - (uintptr_t)base);
+  return DYT_OK;
+}
+
+dyt_status dyt_ipc_import(const dyt_ipc_handle *handle, void **ptr) {
+  if (!handle || !ptr || handle->offset < 0) return DYT_ERR_INVALID_VALUE;
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle->bytes, sizeof(h));
+  void *base = nullptr;
+  const cudaError_t e = cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *ptr = (char *)base + handle->offset;
+  return DYT_OK;
+}
+
+dyt_status dyt_ipc_close(void *ptr, const dyt_ipc_handle *handle) {
+  if (!ptr || !handle || handle->offset < 0) return DYT_ERR_INVALID_VALUE;
+  const cudaError_t e = cudaIpcCloseMemHandle((char *)ptr - handle->offset);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DYT_OK;
 }
 
 const char *dyt_status_string(dyt_status status) {

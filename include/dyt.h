@@ -182,6 +182,79 @@ dyt_status dyt_backward_ex(const void *x, int64_t ldx, const void *dy, int64_t l
                            dyt_dtype gamma_dtype, dyt_dtype beta_dtype, void *workspace, size_t workspace_bytes,
                            dyt_stream_t stream);
 
+/*
+ * The backward in two halves, for a row-sharded backward over several GPUs.
+ * The page's gradients are sums over ALL rows (Summary, "Padding" and
+ * "Precision"), so ranks that each hold some rows of x and dy must add their
+ * partial sums once; here that addition is the finalize itself, reading every
+ * rank's binary64 partials through peer pointers, in rank order, rounding once.
+ * dyt_backward is dyt_backward_partials followed by dyt_finalize_partials over
+ * its one workspace, and gives the same bits.
+ *
+ * dyt_backward_partials: stage 1 only. Writes dx and leaves binary64 partial
+ * sums in the workspace (at least dyt_backward_workspace_bytes bytes); *layout
+ * receives where they are. Arguments as for dyt_backward_ex (no beta). M * N ==
+ * 0 launches nothing and gives an empty layout (rows = dalpha_parts = 0).
+ *
+ * dyt_partials_layout_query: the layout dyt_backward_partials would report for
+ * these tensors on the current device, without launching or reading anything
+ * (the pointers are looked at for their alignment only). Ranks exchange these
+ * once, so that every rank finalizes with the same layouts.
+ *
+ * dyt_finalize_partials: dgamma, dbeta (when N > 0) and dalpha from the
+ * partials of nranks (1 <= nranks <= DYT_MAX_RANKS) workspaces. workspaces is a
+ * HOST array of pointers the current device can read (its own workspace, or
+ * another GPU's through dyt_ipc_import); layouts the matching host array.
+ * Every column is summed per rank in a fixed order, the ranks' totals are
+ * added in rank order, and each gradient is rounded once to its dtype. Ranks
+ * that pass the same workspaces and layouts in the same order get the same
+ * bits. One kernel launch; the caller orders it after every rank's
+ * dyt_backward_partials (on other GPUs: a barrier such as a one-element NCCL
+ * all-reduce on the stream) and keeps the workspaces untouched until every
+ * rank's finalize has run. Layouts that point outside their own `bytes` give
+ * DYT_ERR_INVALID_VALUE.
+ */
+#define DYT_MAX_RANKS 8
+
+typedef struct dyt_partials_layout {
+  int64_t bytes;        /* workspace bytes the partials occupy */
+  int64_t off_dgamma;   /* byte offsets, in the workspace, of the dgamma partials, */
+  int64_t off_dbeta;    /*   the dbeta partials */
+  int64_t off_dalpha;   /*   and the dalpha partials */
+  int32_t rows;         /* partial rows: N binary64 values each, for dgamma and for dbeta */
+  int32_t dalpha_parts; /* binary64 dalpha partials */
+} dyt_partials_layout;
+
+dyt_status dyt_backward_partials(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *alpha,
+                                 const void *gamma, void *dx, int64_t lddx, int64_t M, int64_t N, dyt_dtype x_dtype,
+                                 dyt_dtype alpha_dtype, dyt_dtype gamma_dtype, void *workspace,
+                                 size_t workspace_bytes, dyt_partials_layout *layout, dyt_stream_t stream);
+dyt_status dyt_partials_layout_query(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *dx,
+                                     int64_t lddx, int64_t M, int64_t N, dyt_dtype x_dtype,
+                                     dyt_partials_layout *layout);
+dyt_status dyt_finalize_partials(const void *const *workspaces, const dyt_partials_layout *layouts, int nranks,
+                                 int64_t N, void *dgamma, void *dbeta, void *dalpha, dyt_dtype alpha_dtype,
+                                 dyt_dtype gamma_dtype, dyt_dtype beta_dtype, dyt_stream_t stream);
+
+/*
+ * Sharing a workspace with the other processes of a node (CUDA IPC), so that
+ * their finalize can read its partials over NVLink with plain loads.
+ * dyt_ipc_export: a handle for the device allocation holding ptr, and ptr's
+ * byte offset in it (the memory must come from cudaMalloc, directly or through
+ * a caching allocator that uses it). dyt_ipc_import: in another process, a
+ * pointer to the same bytes, readable from the current device (peer access is
+ * enabled on first use). dyt_ipc_close: releases an imported pointer.
+ * Failures report DYT_ERR_CUDA (dyt_last_cuda_error gives the reason).
+ */
+typedef struct dyt_ipc_handle {
+  unsigned char bytes[64]; /* the CUDA IPC memory handle of the allocation */
+  int64_t offset;          /* the pointer's byte offset in that allocation */
+} dyt_ipc_handle;
+
+dyt_status dyt_ipc_export(const void *ptr, dyt_ipc_handle *out);
+dyt_status dyt_ipc_import(const dyt_ipc_handle *handle, void **ptr);
+dyt_status dyt_ipc_close(void *ptr, const dyt_ipc_handle *handle);
+
 /* Static, human-readable name of a status. Never NULL. */
 const char *dyt_status_string(dyt_status status);
 
@@ -193,7 +266,8 @@ int dyt_last_cuda_error(void);
  * dyt_backward call, so tests can check which path ran.
  */
 typedef struct dyt_launch_info {
-  int op;            /* 1 = forward, 2 = backward, 0 = none yet */
+  int op;            /* 1 = forward, 2 = backward, 3 = backward stage 1 (dyt_backward_partials),
+                        4 = finalize (dyt_finalize_partials), 0 = none yet */
   int path;          /* 0 = nothing launched, 1 = row-tiled (several rows per CTA step),
                         2 = row-per-CTA (one row per CTA step, columns across threads) */
   int vec;           /* elements per vector access (1 = scalar) */

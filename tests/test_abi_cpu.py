@@ -74,6 +74,19 @@ def test_host_validation_without_a_device():
         assert dyt.dyt_backward_ex(0, 4, 0, 4, 0, 0, None, 0, 4, 0, 0, 0, 4, 4, 0, *bad, 0, 0, None) == 2
     assert dyt.dyt_forward_ex(0, 4, 0, 0, 0, 0, 4, 0, 4, 1, 1, 2, 0, None) == 0  # empty: nothing to do
     assert dyt.dyt_backward_noalloc(0, 0, 0, 0, None, 0, 0, 0, 0, -1, 3, 0, 0, None) == 1
+    # stage 1 and the finalize of several ranks
+    st, lay = dyt.dyt_backward_partials(0, 4, 0, 4, 0, 0, 0, 4, 0, 4, 0, 0, 0, 0, 0, None)
+    assert st == 0 and lay["rows"] == 0 and lay["dalpha_parts"] == 0      # no rows: no partials
+    assert dyt.dyt_backward_partials(0, 4, 0, 4, 0, 0, 0, 4, -1, 4, 0, 0, 0, 0, 0, None)[0] == 1
+    assert dyt.dyt_backward_partials(0, 4, 0, 4, 0, 0, 0, 4, 3, 4, 0, 7, 0, 0, 0, None)[0] == 2
+    empty = {"bytes": 0, "off_dgamma": 0, "off_dbeta": 0, "off_dalpha": 0, "rows": 0, "dalpha_parts": 0}
+    assert dyt.dyt_finalize_partials([], [], 4, 1, 1, 1, 0, 0, 0, None) == 1                # no ranks
+    assert dyt.dyt_finalize_partials([0] * 9, [empty] * 9, 4, 1, 1, 1, 0, 0, 0, None) == 1   # more than 8
+    assert dyt.dyt_finalize_partials([0], [empty], 4, 1, 1, 1, 0, 5, 0, None) == 2          # bad dtype
+    assert dyt.dyt_finalize_partials([0], [empty], 4, 0, 1, 1, 0, 0, 0, None) == 1          # null dgamma
+    bad = dict(empty, rows=3, bytes=64)                                                     # partials past `bytes`
+    assert dyt.dyt_finalize_partials([16], [bad], 4, 1, 1, 1, 0, 0, 0, None) == 1
+    assert dyt.dyt_finalize_partials([0], [dict(empty, rows=1, bytes=1 << 20)], 4, 1, 1, 1, 0, 0, 0, None) == 1
     # row pitches below N, or byte offsets beyond int64, are rejected
     assert dyt.dyt_forward_strided(0, 3, 0, 0, 0, 0, 4, 5, 4, 0, 0, None) == 1                  # ldx < N
     assert dyt.dyt_forward_strided(0, 4, 0, 0, 0, 0, 3, 5, 4, 0, 0, None) == 1                  # ldy < N

@@ -112,3 +112,131 @@ def test_gradient_exchange_keeps_each_parameter_dtype():
     assert p.exitcode == 0
     for name, *oks in out:
         assert all(oks), name
+
+
+# ---- the fused cross-rank sum: its protocol on CPU ranks ----------------------------------------
+#
+# FusedGradientSum drives the device through an `ops` object. Here the ops are
+# the oracle: stage 1 leaves the shard's binary64 column sums (one partial row
+# per rank) in a numpy buffer, the barrier is a gloo all-reduce, and the
+# finalize's peer loads are a gloo gather of every rank's buffer of that call,
+# summed in rank order like the kernel does. This checks the protocol: layouts
+# and handles exchanged once, buffers rotated so no consecutive calls share
+# one, every rank adding the ranks' totals in rank order with one rounding.
+
+
+class _OracleOps:
+    def __init__(self, rank, N):
+        self.rank, self.N, self.used, self.closed = rank, N, [], []
+
+    def layout(self, x, dy, dx, N):
+        return {"bytes": 8 * (2 * N + 1), "off_dgamma": 0, "off_dbeta": 8 * N, "off_dalpha": 16 * N, "rows": 1,
+                "dalpha_parts": 1}
+
+    def workspace(self, x, gamma):
+        return np.zeros(2 * self.N + 1)
+
+    def pointer(self, buf):
+        return ("own", self.rank, id(buf))
+
+    def export(self, buf):
+        return (self.rank, id(buf))
+
+    def import_(self, handle):
+        return ("peer",) + tuple(handle)
+
+    def close(self, ptr, handle):
+        self.closed.append(handle)
+
+    def partials(self, x, dy, alpha, gamma, dx, buf, stream):
+        import oracle
+        M = x.size // self.N
+        r = oracle.backward(x, dy, alpha, gamma, M, self.N, "f32", "f32", want_dx=False)
+        buf[:self.N], buf[self.N:2 * self.N], buf[2 * self.N] = r["dgamma"], r["dbeta"], r["dalpha"]
+        self.used.append(next(i for i, b in enumerate(self.fgs.buffers) if b is buf))
+        return self.layout(x, dy, dx, self.N)
+
+    def barrier(self, group, stream):
+        dist.all_reduce(torch.zeros(1), group=group)
+
+    def finalize(self, ptrs, layouts, alpha, gamma, beta, dgamma, dbeta, dalpha, stream):
+        mine = next(b for b in self.fgs.buffers if ("own", self.rank, id(b)) == ptrs[self.rank])
+        every = [torch.zeros(2 * self.N + 1, dtype=torch.float64) for _ in ptrs]
+        dist.all_gather(every, torch.from_numpy(mine.copy()))  # stands in for the peer loads
+        total = every[0].clone()
+        for t in every[1:]:
+            total += t  # the ranks' totals in rank order, binary64
+        dgamma.copy_(total[:self.N]), dbeta.copy_(total[self.N:2 * self.N]), dalpha.copy_(total[2 * self.N:])
+
+
+def _fused_rank(rank: int, port: int, world: int, M: int, N: int, calls: int, q):
+    from elementwise_reduction_b200.dist import FusedGradientSum
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        inp = _inputs(M, N)
+        b, e = shard_rows(M, world, rank)
+        x, dy = inp["x"][b * N:e * N], inp["dy"][b * N:e * N]
+        ops = _OracleOps(rank, N)
+        fgs = FusedGradientSum.__new__(FusedGradientSum)
+        ops.fgs = fgs
+        gamma = torch.from_numpy(inp["gamma"])
+        fgs.__init__(x, dy, None, gamma, ops=ops)
+        outs = []
+        for _ in range(calls):
+            dg, db, da = torch.empty(N), torch.empty(N), torch.empty(1)
+            fgs(x, dy, inp["alpha"], inp["gamma"], None, None, dg, db, da)
+            outs.append((dg.numpy().copy(), db.numpy().copy(), float(da.item())))
+        fgs.close()
+        q.put((rank, outs, ops.used, len(ops.closed)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,M", [(2, 1001), (3, 1000), (4, 7)])
+def test_fused_sum_protocol_on_gloo_ranks(world, M):
+    import oracle
+    N, calls = 24, 4
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_fused_rank, args=(r, port, world, M, N, calls, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted([q.get(timeout=180) for _ in range(world)])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    inp = _inputs(M, N)
+    # the ranks' totals, each the oracle's binary64 sum over that rank's rows,
+    # added in rank order and rounded once to binary32
+    totals = []
+    for r in range(world):
+        b, e = shard_rows(M, world, r)
+        t = oracle.backward(inp["x"][b * N:e * N], inp["dy"][b * N:e * N], inp["alpha"], inp["gamma"], e - b, N,
+                            "f32", "f32", want_dx=False)
+        totals.append(np.concatenate([t["dgamma"], t["dbeta"], [t["dalpha"]]]))
+    want = totals[0].copy()
+    for t in totals[1:]:
+        want += t
+    want32 = want.astype(np.float32)
+    full = oracle.backward(inp["x"], inp["dy"], inp["alpha"], inp["gamma"], M, N, "f32", "f32", want_dx=False)
+    for rank, outs, used, closed in got:
+        assert used == [0, 1, 2, 0][:calls]          # three buffers in rotation
+        assert closed == 3 * (world - 1)             # every imported peer buffer released
+        for dg, db, da in outs:                      # same bits on every rank and call
+            assert np.array_equal(dg, want32[:N]) and np.array_equal(db, want32[N:2 * N])
+            assert da == float(want32[2 * N])
+            assert np.all(np.abs(db - full["dbeta"]) <= 2e-6 + 1e-5 * np.abs(full["dbeta"]))
+            assert abs(da - full["dalpha"]) <= 1e-5 * full["mag_dalpha"]
+
+
+def test_replay_schedule_never_reuses_a_buffer_back_to_back():
+    from elementwise_reduction_b200.dist import FusedGradientSum
+    for k in range(2, 40):
+        s = FusedGradientSum.schedule(k)
+        assert len(s) == k and set(s) <= {0, 1, 2}
+        cyc = s + s  # two replays back to back
+        assert all(cyc[i] != cyc[i + 1] for i in range(len(cyc) - 1)), (k, s)
+    with pytest.raises(ValueError):
+        FusedGradientSum.schedule(1)

@@ -496,6 +496,61 @@ def test_fp32_sums_meet_the_elementwise_bound(M, N, alpha):
         assert st["dgamma"]["n_over_strict_elementwise"] == 0
 
 
+@pytest.mark.parametrize("R,M,N,xd", [(1, 3001, 64, "bf16"), (2, 65537, 32, "bf16"), (3, 10007, 100, "f32"),
+                                      (8, 4099, 17, "f32"), (4, 5, 4096, "bf16"), (8, 5, 64, "f16"),
+                                      (3, 20000, 255, "f32")])
+def test_partials_of_several_ranks_sum_in_one_finalize(R, M, N, xd):
+    # R ranks of a row-sharded backward, emulated on one GPU: each rank's stage 1
+    # runs on its own rows into its own workspace, then one finalize reads every
+    # rank's partials in rank order, as each rank's finalize does through peer
+    # pointers. Shards whose rows start off a 16-byte boundary take the
+    # one-element kernels; shards with no rows add nothing.
+    import elementwise_reduction_b200 as dyt
+    from elementwise_reduction_b200.dist import shard_rows
+    inp = make(M, N, xd, "f32")
+    t = H.gpu_inputs(inp, xd, "f32")
+    x, dy = t["x"].view(M, N), t["dy"].view(M, N)
+    dx = torch.empty_like(x)
+    wss, lays = [], []
+    for r in range(R):
+        b, e = shard_rows(M, R, r)
+        xs, dys, dxs = x[b:e], dy[b:e], dx[b:e]
+        ws = dyt.workspace(xs, t["gamma"])
+        _, lay = dyt.backward_partials(xs, dys, t["alpha"], t["gamma"], ws, dx=dxs)
+        assert lay == dyt.partials_layout(xs, dys, dxs, N)
+        wss.append(ws)
+        lays.append(lay)
+    ptrs = [w.data_ptr() for w in wss]
+    da, dg, db = dyt.finalize_partials(ptrs, lays, t["alpha"], t["gamma"], t["beta"])
+    torch.cuda.synchronize()
+    out = {"dx": H.to_numpy(dx, xd), "dgamma": H.to_numpy(dg, "f32"), "dbeta": H.to_numpy(db, "f32"),
+           "dalpha": float(da.item())}
+    st = H.compare_all(inp, out, M, N, xd, "f32")
+    assert st["dbeta"]["n_over_strict_elementwise"] == 0
+    da2, dg2, db2 = dyt.finalize_partials(ptrs, lays, t["alpha"], t["gamma"], t["beta"])  # same bits again
+    assert torch.equal(dg, dg2) and torch.equal(db, db2) and torch.equal(da, da2)
+    if R == 1:  # one rank: exactly the single-GPU backward
+        ref = dyt.backward(x, dy, t["alpha"], t["gamma"], t["beta"])
+        for a, b in zip((dx, da, dg, db), ref):
+            assert torch.equal(a, b)
+
+
+def test_finalize_rejects_layouts_outside_their_workspace():
+    import elementwise_reduction_b200 as dyt
+    M, N = 100, 64
+    x = torch.randn(M, N, device="cuda")
+    g = torch.ones(N, device="cuda")
+    a = torch.tensor([0.5], device="cuda")
+    ws = dyt.workspace(x, g)
+    _, lay = dyt.backward_partials(x, x, a, g, ws)
+    bad = dict(lay, rows=lay["rows"] + 1000)
+    with pytest.raises(dyt.DytError) as e:
+        dyt.finalize_partials([ws.data_ptr()], [bad], a, g)
+    assert e.value.status == 1
+    with pytest.raises(dyt.DytError):
+        dyt.finalize_partials([ws.data_ptr()] * 9, [lay] * 9, a, g)  # more than 8 ranks
+
+
 def test_autograd_module_matches_oracle():
     import elementwise_reduction_b200 as dyt
     M, N = 512, 384

@@ -56,6 +56,7 @@ def parse():
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--no-shapes", action="store_true", help="skip the per-shape table of the other workloads")
     p.add_argument("--no-latency", action="store_true", help="skip the per-call cold-L2 latency percentiles")
+    p.add_argument("--no-sustained", action="store_true", help="skip the 1 s back-to-back replay of the step")
     p.add_argument("--record-traffic", metavar="NCU_CSV", default=None,
                    help="store DRAM bytes per launch from an ncu --csv capture of dram__bytes_read.sum and "
                         "dram__bytes_write.sum into profiles/dram_traffic.json for --workload, then exit")
@@ -151,47 +152,94 @@ def record_traffic(csv_path: str, workload: str, command: str) -> None:
 # ---- clocks sampled during the timed region ---------------------------------------------------
 
 class ClockSampler:
+    """SM clock, power and throttle reasons of one GPU, sampled every few ms while
+    the `with` block runs: through NVML (the GPU matched by UUID), else by
+    polling nvidia-smi every 100 ms."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int, enabled: bool = True):
-        self.index, self.enabled, self.rows, self.proc = index, enabled, [], None
+    def __init__(self, index: int, enabled: bool = True, period_s: float = 0.005):
+        self.index, self.enabled, self.period = index, enabled, period_s
+        self.rows = []  # (host time, sm MHz, max sm MHz, watts, [reasons])
+        self.proc, self.thread, self._stop = None, None, threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
 
     def __enter__(self):
-        if self.enabled:
+        if not self.enabled:
+            return self
+        try:
+            nv, h = self._nvml_handle()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            reasons_of = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        w = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        bits = reasons_of(h)
+                        self.rows.append((time.time(), float(sm), float(mx), w,
+                                          [n for b, n in self.REASONS.items() if bits & b]))
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+        except Exception:
             try:
                 self.proc = subprocess.Popen(
                     ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
                      "--format=csv,noheader,nounits", "-lms", "100"],
                     stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-                self.thread = threading.Thread(target=self._read, daemon=True)
+                self.thread = threading.Thread(target=self._read_smi, daemon=True)
                 self.thread.start()
             except Exception:
                 self.proc = None
         return self
 
-    def _read(self):
+    def _read_smi(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.proc.stdout:
-            self.rows.append([c.strip() for c in line.split(",")])
+            r = [c.strip() for c in line.split(",")]
+            try:
+                self.rows.append((time.time(), float(r[1]), float(r[2]), float(r[3]),
+                                  [n for n, v in zip(names, r[5:9]) if v.lower() == "active"]))
+            except (ValueError, IndexError):
+                pass
 
     def __exit__(self, *exc):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
-    def summary(self):
-        if not self.rows:
+    def summary(self, t0: float | None = None, t1: float | None = None):
+        rows = [r for r in self.rows if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
+        if not rows:
             return None
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+        sm = [r[1] for r in rows]
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": max(r[2] for r in rows),
+                "power_w": statistics.median(r[3] for r in rows),
+                "reasons": sorted({n for r in rows for n in r[4]}), "samples": len(rows)}
 
 
 # ---- CPU baseline: the oracle on a bounded sample ---------------------------------------------
@@ -360,29 +408,41 @@ def _graph(stream, fn, n):
     return g
 
 
-def _time_replays(g, stream, dev, K, clock_index, clocks=True, min_replays=7, min_seconds=0.3,
-                  max_replays=400):
-    """Per-call device time (us) of a K-call graph over repeated replays (CUDA events on
-    the launching stream), with the SM clocks sampled while it runs."""
+def _time_replays(g, stream, dev, K, clock_index, clocks=True, idle_s=0.4, min_seconds=0.6, min_replays=7,
+                  max_replays=2000):
+    """Per-call device time (us) of a K-call graph over repeated replays (CUDA events
+    on the launching stream), after `idle_s` without load so that the GPU starts
+    below its power limit. `burst`: the median of the first three replays;
+    `sustained`: the median over the second half of the window, when a kernel that
+    draws the power limit has reached its capped clock. p10 / p50 / p90 over all.
+    Clocks, power and throttle reasons are sampled throughout."""
     import torch
     g.replay()
     torch.cuda.synchronize(dev)
-    per = []
+    time.sleep(idle_s)
+    rec = []
     with ClockSampler(clock_index, enabled=clocks) as clk:
+        t_start = time.time()
         t_end = time.perf_counter() + min_seconds
-        while len(per) < min_replays or (time.perf_counter() < t_end and len(per) < max_replays):
+        while len(rec) < min_replays or (time.perf_counter() < t_end and len(rec) < max_replays):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t = time.time()
             e0.record(stream)
             g.replay()
             e1.record(stream)
             e1.synchronize()
-            per.append(e0.elapsed_time(e1) * 1e3 / K)
-        while time.perf_counter() < t_end:  # keep the load on for the clock samples
+            rec.append((t, e0.elapsed_time(e1) * 1e3 / K))
+        while time.perf_counter() < t_end:  # keep the load on for the whole window
             g.replay()
             torch.cuda.synchronize(dev)
+        t_stop = time.time()
+    per = np.array([r[1] for r in rec])
     q = np.percentile(per, [10, 50, 90])
+    t_half = rec[len(rec) // 2][0]
     return {"us_p10": float(q[0]), "us_p50": float(q[1]), "us_p90": float(q[2]), "replays": len(per),
-            "clocks": clk.summary()}
+            "burst_us": float(np.median(per[:3])), "sustained_us": float(np.median(per[len(per) // 2:])),
+            "clocks": clk.summary(t_start, t_stop), "clocks_burst": clk.summary(t_start, t_start + 0.05),
+            "clocks_sustained": clk.summary(t_half, t_stop)}
 
 
 def _roofline(nbytes, us, peak, peak_kind, traffic):
@@ -493,20 +553,16 @@ def run_ours(args, w):
             return ms
 
         with ClockSampler(local, enabled=not args.no_clocks) as clk:
-            # Keep the GPU under the same load for ~0.3 s around the timed replays so
-            # that the sampled clocks (every 100 ms) describe the timed region.
-            t_end = time.perf_counter() + 0.3
-            while time.perf_counter() < t_end:
-                g_step.replay()
-                torch.cuda.synchronize(dev)
-            ms_step = timed(g_step)
+            t0 = time.time()
+            ms_step = timed(g_step)  # the timed region: K steps, clocks sampled every 5 ms
+            t1 = time.time()
             ms_fwd = timed(g_fwd)
             ms_bwd = timed(g_bwd)
-            t_end = time.perf_counter() + 0.15
-            while time.perf_counter() < t_end:
-                g_step.replay()
-                torch.cuda.synchronize(dev)
-        clocks = clk.summary()
+        clocks = clk.summary(t0, t1) or clk.summary()
+        # The same step graph replayed back to back for about a second: what a long
+        # run of this layer alone gets once the GPU sits at its power limit.
+        sustained = _time_replays(g_step, stream, dev, args.steps, local, clocks=not args.no_clocks, idle_s=0.0,
+                                  min_seconds=1.0) if world == 1 and not args.no_sustained else None
         del g_step, g_fwd, g_bwd  # graphs that may hold NCCL calls go before the process group
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -626,6 +682,11 @@ def run_ours(args, w):
             if exchange is not None else f"NCCL all-reduce of the rounded gradients ({exchange_note})"),
         "clocks": clocks,
     }
+    if sustained is not None:
+        ms_s = sustained["sustained_us"] * 1e-3
+        line["sustained"] = {"ms_per_step": ms_s, "value": step_bytes / (ms_s * 1e-3) / 1e9, "unit": "GB/s",
+                             "clocks": sustained["clocks_sustained"],
+                             "note": "the step graph replayed back to back for 1 s; second half"}
     if world > 1:
         dist.destroy_process_group()
     if world == 1 and not args.no_shapes:
@@ -691,12 +752,14 @@ def call_latency(args, dev, calls=30):
 def shape_table(args, dev, clock_index, cpu=True):
     """Every workload and layout variant, forward and backward, each timed like the
     headline: a CUDA graph of K calls over rotating buffer sets that exceed L2,
-    replayed at least 7 times (p10 / p50 / p90 of the per-call time) with the SM
-    clocks sampled during the replays. Each line carries its roofline entry and,
-    next to it, the oracle on the host cores on a bounded sample of the same
-    workload. For the narrow shapes, a plain PyTorch copy (the forward's bytes)
-    and a three-operand add (the backward's bytes) timed the same way give the
-    floor a memory-bound kernel of these sizes meets in this setting."""
+    replayed for 0.6 s after an idle gap (burst: the first replays; sustained:
+    the second half, once a power-hungry kernel sits at its power limit; p10 /
+    p50 / p90 over all) with the SM clocks, power and throttle reasons sampled
+    during the replays. Each line carries its roofline entry (burst, and
+    sustained) and, next to it, the oracle on the host cores on a bounded sample
+    of the same workload. A plain PyTorch copy (the forward's bytes) and a
+    three-operand add (the backward's bytes), timed the same way, give what a
+    library kernel moving the same bytes meets in this setting."""
     import torch
 
     import elementwise_reduction_b200 as dyt
@@ -719,10 +782,10 @@ def shape_table(args, dev, clock_index, cpu=True):
                                               dx=sets[i % nsets]["dx"], dgamma=sets[i % nsets]["dg"],
                                               dbeta=sets[i % nsets]["db"], dalpha=sets[i % nsets]["da"], ws=ws),
             }
-            if w.M * w.N * workloads.ITEMSIZE[w.x_dtype] < (64 << 20):  # narrow shapes: library floors
-                calls["copy_floor"] = lambda i: sets[i % nsets]["y"].copy_(sets[i % nsets]["x"])
-                calls["add3_floor"] = lambda i: torch.add(sets[i % nsets]["x"], sets[i % nsets]["dy"],
-                                                          out=sets[i % nsets]["dx"])
+            # library floors: the same bytes moved by a PyTorch copy and a three-operand add
+            calls["copy_floor"] = lambda i: sets[i % nsets]["y"].copy_(sets[i % nsets]["x"])
+            calls["add3_floor"] = lambda i: torch.add(sets[i % nsets]["x"], sets[i % nsets]["dy"],
+                                                      out=sets[i % nsets]["dx"])
             for op, call in calls.items():
                 for i in range(3):
                     call(i)
@@ -732,9 +795,10 @@ def shape_table(args, dev, clock_index, cpu=True):
                 del graph
                 nbytes = w.fwd_bytes() if op in ("fwd", "copy_floor") else w.bwd_bytes()
                 kernel = {"fwd": "dyt_fwd_kernel", "bwd": "dyt_backward"}.get(op)
-                t["roofline"] = _roofline(nbytes, t["us_p50"], peak, peak_kind,
+                t["roofline"] = _roofline(nbytes, t["burst_us"], peak, peak_kind,
                                           committed_traffic(name, kernel) if kernel else None)
-                t["rows_per_s"] = w.M / (t["us_p50"] * 1e-6)
+                t["roofline_sustained"] = _roofline(nbytes, t["sustained_us"], peak, peak_kind, None)
+                t["rows_per_s"] = w.M / (t["burst_us"] * 1e-6)
                 if info is not None:
                     t["launch"] = {k: info[k] for k in ("path", "vec", "grid", "row_lanes", "row_groups",
                                                         "pack_rows", "kernels")}

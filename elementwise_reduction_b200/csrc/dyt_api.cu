@@ -217,18 +217,38 @@ constexpr int vec_of() {
   return 16 / (int)sizeof(T);
 }
 
-template <typename T>
+template <typename T, typename P>
 const void *main_kernel(bool backward, bool async, bool packed) {
   constexpr int V = vec_of<T>();
   if (async) {
     if (backward)
-      return packed ? (const void *)dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, true>
-                    : (const void *)dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, false>;
-    return packed ? (const void *)dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, true>
-                  : (const void *)dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, false>;
+      return packed ? (const void *)dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, true>
+                    : (const void *)dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, false>;
+    return packed ? (const void *)dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, true>
+                  : (const void *)dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, false>;
   }
-  return backward ? (const void *)dyt::dyt_bwd_kernel<T, kScalarUnrollBwd, kScalarBlock>
-                  : (const void *)dyt::dyt_fwd_kernel<T, kScalarUnrollFwd, kScalarBlock>;
+  return backward ? (const void *)dyt::dyt_bwd_kernel<T, P, kScalarUnrollBwd, kScalarBlock>
+                  : (const void *)dyt::dyt_fwd_kernel<T, P, kScalarUnrollFwd, kScalarBlock>;
+}
+
+// The parameter type of the kernels for these parameter dtypes: the shared
+// dtype when all are equal (typed, read-only loads), else void (a run-time
+// switch per parameter). f receives a Tag<P>.
+template <typename P>
+struct Tag {
+  using type = P;
+};
+template <typename F>
+dyt_status with_ptype(int ad, int gd, int bd, F &&f) {
+  if (ad == gd && gd == bd) {
+    switch (ad) {
+      case DYT_F32: return f(Tag<float>{});
+      case DYT_BF16: return f(Tag<__nv_bfloat16>{});
+      case DYT_F16: return f(Tag<__half>{});
+    }
+    return DYT_ERR_UNSUPPORTED_DTYPE;
+  }
+  return f(Tag<void>{});
 }
 
 template <typename F>
@@ -305,13 +325,13 @@ PathChoice choose_path(int64_t N, int v, bool aligned, bool pitched, bool adjace
 }
 
 // The plan for tensors of type T with the given layout on the current device.
-template <typename T>
+template <typename T, typename P>
 dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjacent, bool backward, Plan *out) {
   int dev = 0, sms = 0;
   dyt_status st = current_sms(&dev, &sms);
   if (st != DYT_OK) return st;
   const PathChoice pc = choose_path(N, vec_of<T>(), aligned, pitched, adjacent);
-  const void *k = main_kernel<T>(backward, pc.async, pc.packed);
+  const void *k = main_kernel<T, P>(backward, pc.async, pc.packed);
   int occ = 1;
   if (pc.async) {
     // One CTA per SM by construction (__launch_bounds__(B, 1), ring sized for it).
@@ -372,9 +392,9 @@ LayoutArgs stage1_layout_args(const void *x, int64_t ldx, const void *dy, int64_
   return {aligned16(x) && aligned16(dy) && aligned16(dx),
           vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es), ldx == N && lddy == N && lddx == N};
 }
-template <typename T>
+template <typename T, typename P>
 dyt_status plan_for(int64_t M, int64_t N, LayoutArgs a, bool backward, Plan *out) {
-  return plan_for<T>(M, N, a.aligned, a.pitched, a.adjacent, backward, out);
+  return plan_for<T, P>(M, N, a.aligned, a.pitched, a.adjacent, backward, out);
 }
 
 // Every gradient +0 (all-zero bits in each dtype): the empty sums.
@@ -397,12 +417,15 @@ dyt_status bwd_stage1(const void *x, int64_t ldx, const void *dy, int64_t lddy, 
                       dyt_partials_layout *lay) {
   if (!x || !dy || !alpha || !gamma || !dx || !workspace) return DYT_ERR_INVALID_VALUE;
   if (!aligned16(workspace)) return DYT_ERR_INVALID_VALUE;
-  const dyt::Params pr = {alpha, gamma, nullptr, (int)alpha_dtype, (int)gamma_dtype, DYT_F32};
+  const dyt::ParamTypes pt = {(int)alpha_dtype, (int)gamma_dtype, (int)gamma_dtype};
+  // beta is not read: the kernels' parameter type follows alpha and gamma.
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
+    return with_ptype(alpha_dtype, gamma_dtype, gamma_dtype, [&](auto tp) -> dyt_status {
+    using P = typename decltype(tp)::type;
     constexpr int V = vec_of<T>();
     Plan &p = *plan;
-    dyt_status r = plan_for<T>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
+    dyt_status r = plan_for<T, P>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
     if (r != DYT_OK) return r;
     if (!p.packed) {
       p.g.ldx = ldx;
@@ -414,20 +437,22 @@ dyt_status bwd_stage1(const void *x, int64_t ldx, const void *dy, int64_t lddy, 
     double *pdg = (double *)(ws + p.ws_dg);
     double *pdb = (double *)(ws + p.ws_db);
     double *pda = (double *)(ws + p.ws_da);
+    const P *pa = (const P *)alpha, *pg = (const P *)gamma;
     PdlConfig lc(p.grid, p.block, p.smem, s);
     cudaError_t e;
     if (p.async && p.packed)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, true>,
-                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, true>,
+                             (const T *)x, (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
     else if (p.async)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesBwd, false>,
-                             (const T *)x, (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, false>,
+                             (const T *)x, (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
     else
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_kernel<T, kScalarUnrollBwd, kScalarBlock>, (const T *)x,
-                             (const T *)dy, pr, (T *)dx, pdg, pdb, pda, p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_kernel<T, P, kScalarUnrollBwd, kScalarBlock>, (const T *)x,
+                             (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
     if (e != cudaSuccess) return cuda_fail(e);
     *lay = layout_of(p);
     return DYT_OK;
+    });
   });
 }
 
@@ -500,32 +525,37 @@ dyt_status dyt_forward_ex(const void *x, int64_t ldx, const void *alpha, const v
     return DYT_OK;
   }
   if (!x || !alpha || !gamma || !beta || !y) return DYT_ERR_INVALID_VALUE;
-  const dyt::Params pr = {alpha, gamma, beta, (int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
+  const dyt::ParamTypes pt = {(int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
+    return with_ptype(alpha_dtype, gamma_dtype, beta_dtype, [&](auto tp) -> dyt_status {
+    using P = typename decltype(tp)::type;
     constexpr int V = vec_of<T>();
     Plan p;
-    dyt_status s = plan_for<T>(M, N, aligned16(x) && aligned16(y), vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)),
-                               ldx == N && ldy == N, false, &p);
+    dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y),
+                                  vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)), ldx == N && ldy == N, false,
+                                  &p);
     if (s != DYT_OK) return s;
     if (!p.packed) {
       p.g.ldx = ldx;
       p.g.ldo = ldy;
     }
+    const P *pa = (const P *)alpha, *pg = (const P *)gamma, *pb = (const P *)beta;
     PdlConfig lc(p.grid, p.block, p.smem, (cudaStream_t)stream);
     cudaError_t e;
     if (p.async && p.packed)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, true>,
-                             (const T *)x, pr, (T *)y, p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, true>,
+                             (const T *)x, pa, pg, pb, pt, (T *)y, p.g);
     else if (p.async)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, V, kAsyncBlock, kAsyncStagesFwd, false>,
-                             (const T *)x, pr, (T *)y, p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, false>,
+                             (const T *)x, pa, pg, pb, pt, (T *)y, p.g);
     else
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_kernel<T, kScalarUnrollFwd, kScalarBlock>, (const T *)x, pr,
-                             (T *)y, p.g);
+      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_kernel<T, P, kScalarUnrollFwd, kScalarBlock>, (const T *)x, pa,
+                             pg, pb, pt, (T *)y, p.g);
     if (e != cudaSuccess) return cuda_fail(e);
     record(1, &p, 1, 0);
     return DYT_OK;
+    });
   });
 }
 
@@ -538,7 +568,7 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
     // The 16-byte and the one-element plan may differ; cover both.
     for (int v = 0; v < 2; ++v) {
       Plan p;
-      dyt_status s = plan_for<T>(M, N, v == 1, v == 1, true, true, &p);
+      dyt_status s = plan_for<T, float>(M, N, v == 1, v == 1, true, true, &p);  // the plan does not depend on P
       if (s != DYT_OK) return s;
       if (p.ws_total > need) need = p.ws_total;
     }
@@ -631,7 +661,7 @@ dyt_status dyt_partials_layout_query(const void *x, int64_t ldx, const void *dy,
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
     Plan p;
-    const dyt_status r = plan_for<T>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
+    const dyt_status r = plan_for<T, float>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
     if (r == DYT_OK) *layout = layout_of(p);
     return r;
   });

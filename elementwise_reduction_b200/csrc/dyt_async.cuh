@@ -143,16 +143,17 @@ __device__ __forceinline__ int last_vector_real(const Geom &g, int64_t first, in
   return r < VEC ? (int)r : VEC;
 }
 
-template <typename T, int VEC, int B, int S, bool PK>
+template <typename T, typename P, int VEC, int B, int S, bool PK>
 __global__ void __launch_bounds__(B, 1)
-    dyt_fwd_async_kernel(const T *__restrict__ x, Params pr, T *y, Geom g) {
+    dyt_fwd_async_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma_p,
+                         const P *__restrict__ beta_p, ParamTypes pt, T *y, Geom g) {
   using IO = VecIO<T, VEC>;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
   extern __shared__ uint4 ring[];  // [S][B]
   prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
+  const float alpha = load_param<P>(alpha_p, pt.alpha, 0);
   uint4 *slot0 = ring + threadIdx.x;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(B, 1)
     int64_t col[VEC];
     vector_columns<VEC, PK>(c0, g.Nc, col);
     float gam[VEC], bet[VEC], bth[VEC];
-    fwd_params_at<T, VEC>(pr, col, gam, bet, bth);
+    fwd_params_at<T, VEC, P>(gamma_p, beta_p, pt, col, gam, bet, bth);
     int s_rd = 0, s_wr = S - 1;
     for (int64_t k = 0; k < n; ++k) {
       const int64_t kn = k + S - 1;
@@ -205,11 +206,11 @@ __global__ void __launch_bounds__(B, 1)
 
 // ---- backward, stage 1 ----------------------------------------------------------
 
-template <typename T, int VEC, int B, int S, bool PK>
+template <typename T, typename P, int VEC, int B, int S, bool PK>
 __global__ void __launch_bounds__(B, 1)
-    dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, Params pr, T *dx,
-                         double *__restrict__ part_dg, double *__restrict__ part_db, double *__restrict__ part_da,
-                         Geom g) {
+    dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
+                         const P *__restrict__ gamma_p, ParamTypes pt, T *dx, double *__restrict__ part_dg,
+                         double *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
   using IO = VecIO<T, VEC>;
   constexpr bool EXACT_G = ExactGamma<T>::value;
   constexpr int kRunBlocks = kGammaRunRows / S;  // unrolled blocks of S rows per binary32 dgamma run
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(B, 1)
   prefetch_first_rows_l2<T, VEC, B, S, PK>(dy, g.ldd, g);
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
+  const float alpha = load_param<P>(alpha_p, pt.alpha, 0);
   double *red = reinterpret_cast<double *>(ring);
   double *gtot = reinterpret_cast<double *>(ring + 2 * S * B) + threadIdx.x;  // [e * B]
   uint4 *slot0 = ring + threadIdx.x;
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(B, 1)
       }
       int64_t col[VEC];
       vector_columns<VEC, PK>(c0, g.Nc, col);
-      load_params<VEC>(pr.gamma, pr.gamma_dt, col, 4.0f, gam);  // 4 gamma (see bwd_vector)
+      load_params<VEC, P>(gamma_p, pt.gamma, col, 4.0f, gam);  // 4 gamma (see bwd_vector)
       int run = 0;  // blocks in the current binary32 dgamma run
       for (int k0 = 0; k0 < nn; k0 += S) {
         float2 ca = make_float2(0.0f, 0.0f);  // this block's dalpha terms (at most S VEC / 2 per lane)

@@ -63,15 +63,13 @@ struct Geom {
   int l2_prefetch;    // the 16-byte kernels prefetch their first rows into L2 (large inputs only)
 };
 
-// The parameters, each with its own dtype (dyt_dtype codes). beta is read by
-// the forward only.
-struct Params {
-  const void *alpha;
-  const void *gamma;
-  const void *beta;
-  int alpha_dt;
-  int gamma_dt;
-  int beta_dt;
+// The parameters' dtypes (dyt_dtype codes), read by the kernels instantiated
+// with P = void (parameters of different dtypes); beta is read by the forward
+// only.
+struct ParamTypes {
+  int alpha;
+  int gamma;
+  int beta;
 };
 
 // Where the finalize writes the parameter gradients, each in its parameter's dtype.
@@ -329,24 +327,26 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw fwd_vector(const typename
 
 // gamma, beta and the cancellation thresholds of the VEC columns col[e] (not
 // necessarily consecutive).
-template <typename T, int VEC>
-__device__ __forceinline__ void fwd_params_at(const Params &pr, const int64_t (&col)[VEC], float (&gam)[VEC],
+template <typename T, int VEC, typename P>
+__device__ __forceinline__ void fwd_params_at(const P *__restrict__ gamma, const P *__restrict__ beta,
+                                              const ParamTypes &pt, const int64_t (&col)[VEC], float (&gam)[VEC],
                                               float (&bet)[VEC], float (&bth)[VEC]) {
-  load_params<VEC>(pr.gamma, pr.gamma_dt, col, 1.0f, gam);
-  load_params<VEC>(pr.beta, pr.beta_dt, col, 1.0f, bet);
+  load_params<VEC, P>(gamma, pt.gamma, col, 1.0f, gam);
+  load_params<VEC, P>(beta, pt.beta, col, 1.0f, bet);
 #pragma unroll
   for (int e = 0; e < VEC; ++e) bth[e] = fabsf(bet[e]) * CancelGuard<T>::kTau;
 }
 
 // Forward for matrices that are not 16-byte aligned: one element per access,
 // U rows in flight per thread.
-template <typename T, int U, int B>
+template <typename T, typename P, int U, int B>
 __global__ void __launch_bounds__(B, 1)
-    dyt_fwd_kernel(const T *__restrict__ x, Params pr, T *y, Geom g) {
+    dyt_fwd_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma_p,
+                   const P *__restrict__ beta_p, ParamTypes pt, T *y, Geom g) {
   using IO = VecIO<T, 1>;
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
+  const float alpha = load_param<P>(alpha_p, pt.alpha, 0);
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
     item_split(g, item, cc, rg);
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(B, 1)
     if (!(ln.live && cv < g.NV)) continue;
     const int64_t col[1] = {cv};
     float gam[1], bet[1], bth[1];
-    fwd_params_at<T, 1>(pr, col, gam, bet, bth);
+    fwd_params_at<T, 1, P>(gamma_p, beta_p, pt, col, gam, bet, bth);
     const int64_t step = (int64_t)g.RL * U;
     for (int64_t r0 = rb + ln.rl; r0 < re; r0 += step) {
       T raw[U];
@@ -564,11 +564,11 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
 
 // Backward stage 1 for matrices that are not 16-byte aligned: one element
 // per access, U rows in flight per thread.
-template <typename T, int U, int B>
+template <typename T, typename P, int U, int B>
 __global__ void __launch_bounds__(B, 1)
-    dyt_bwd_kernel(const T *__restrict__ x, const T *__restrict__ dy, Params pr, T *dx,
-                   double *__restrict__ part_dg, double *__restrict__ part_db, double *__restrict__ part_da,
-                   Geom g) {
+    dyt_bwd_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
+                   const P *__restrict__ gamma_p, ParamTypes pt, T *dx, double *__restrict__ part_dg,
+                   double *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
   using IO = VecIO<T, 1>;
   __shared__ double red[2 * B];
   __shared__ double red_a[B / 32];
@@ -577,7 +577,7 @@ __global__ void __launch_bounds__(B, 1)
   pdl_prologue();
 
   const Lane ln = lane_of(g, threadIdx.x);
-  const float alpha = load_param(pr.alpha, pr.alpha_dt, 0);
+  const float alpha = load_param<P>(alpha_p, pt.alpha, 0);
   double acc_a = 0.0;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(B, 1)
     group_rows(g, rg, rb, re);
     const int cv = cc * B + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
-    float gam[1] = {col_ok ? 4.0f * load_param(pr.gamma, pr.gamma_dt, cv) : 0.0f};  // 4 gamma (see bwd_vector)
+    float gam[1] = {col_ok ? 4.0f * load_param<P>(gamma_p, pt.gamma, cv) : 0.0f};  // 4 gamma (see bwd_vector)
     BwdAcc<1, true> acc;
     acc.g[0] = 0.0;
     acc.b[0] = 0.0;

@@ -600,7 +600,14 @@ def test_tanh_and_sech2_accuracy_sweep():
     print("max rel err t: 2^%.2f" % np.log2(rel_t.max()), " backward t: 2^%.2f" % np.log2(rel_tb.max()),
           " 1-t^2: 2^%.2f" % np.log2(rel_s.max()))
     assert rel_t.max() <= H.T_REL_ERR, rel_t.max()
-    assert rel_tb.max() <= H.T_REL_ERR, rel_tb.max()  # the bound the dgamma tolerance uses
+    # the bound the dgamma tolerance uses: relative, plus an absolute part where
+    # |alpha x| < 0.5 (the backward's t takes the exp form for every argument)
+    err_tb = np.abs(t_bwd - np.tanh(X))
+    assert (err_tb <= H.T_REL_ERR * np.abs(np.tanh(X)) + H.T_ABS_ERR).all(), \
+        (err_tb / (H.T_REL_ERR * np.abs(np.tanh(X)) + H.T_ABS_ERR)).max()
+    big = np.abs(X) >= 0.5
+    assert rel_tb[big].max() <= H.T_REL_ERR, rel_tb[big].max()
+    print("backward t: max abs err below 0.5: 2^%.2f" % np.log2(err_tb[~big].max()))
     bound_s = 2.0 ** -20 + 2.0 * np.abs(X[ok]) * 2.0 ** -24
     assert (rel_s <= bound_s).all(), (rel_s / bound_s).max()
 

@@ -454,8 +454,8 @@ __device__ __forceinline__ void lane_reduce_warps(const double (&vg)[VEC], const
     }
   }
   __syncthreads();
-  if (threadIdx.x < 2 * width) {
-    const int which = threadIdx.x / width, k = threadIdx.x - which * width;
+  for (int i = threadIdx.x; i < 2 * width; i += B) {  // 2 width can exceed B (NV = 32 with B = 256)
+    const int which = i / width, k = i - which * width;
     double sum = 0.0;
     for (int w = 0; w < B / 32; ++w) sum += red[(2 * w + which) * width + k];
     (which ? out_b : out_g)[c0_chunk + k] = sum;

@@ -363,21 +363,21 @@ def _to_torch(a, dtype, device):
     return t if str(device) == "cpu" else t.to(device)
 
 
-def _matrix(src, w, dev):
-    """An M x N device matrix holding src, starting w.offset elements past a 16-byte
+def _matrix(src, w, dev, off):
+    """An M x N device matrix holding src, starting `off` elements past a 16-byte
     boundary (0 for the workloads themselves)."""
     import torch
     t = _to_torch(src, w.x_dtype, "cpu")
-    buf = torch.empty(w.M * w.N + w.offset + 8, dtype=t.dtype, device=dev)
-    m = buf[w.offset:w.offset + w.M * w.N].view(w.M, w.N)
+    buf = torch.empty(w.M * w.N + off + 8, dtype=t.dtype, device=dev)
+    m = buf[off:off + w.M * w.N].view(w.M, w.N)
     m.copy_(t.view(w.M, w.N))
     return m
 
 
-def _empty_like_matrix(m, w):
+def _empty_like_matrix(m, w, off):
     import torch
-    buf = torch.empty(w.M * w.N + w.offset + 8, dtype=m.dtype, device=m.device)
-    return buf[w.offset:w.offset + w.M * w.N].view(w.M, w.N)
+    buf = torch.empty(w.M * w.N + off + 8, dtype=m.dtype, device=m.device)
+    return buf[off:off + w.M * w.N].view(w.M, w.N)
 
 
 def _sets(w, inp, dev, L2):
@@ -387,14 +387,15 @@ def _sets(w, inp, dev, L2):
     from synth import workloads
     set_bytes = 4 * w.M * w.N * workloads.ITEMSIZE[w.x_dtype]  # x, dy, y, dx
     nsets = int(min(64, max(1, -(-3 * L2 // set_bytes))))
-    x0, dy0 = _matrix(inp["x"], w, dev), _matrix(inp["dy"], w, dev)
+    x0, dy0 = _matrix(inp["x"], w, dev, w.x_off), _matrix(inp["dy"], w, dev, w.offset)
     ad, gd, bd = w.param_dtypes
     a, g, b = _to_torch(inp["alpha"], ad, dev), _to_torch(inp["gamma"], gd, dev), _to_torch(inp["beta"], bd, dev)
     sets = []
     for i in range(nsets):
-        x = x0 if i == 0 else _empty_like_matrix(x0, w).copy_(x0)
-        d = dy0 if i == 0 else _empty_like_matrix(dy0, w).copy_(dy0)
-        sets.append({"x": x, "dy": d, "y": _empty_like_matrix(x0, w), "dx": _empty_like_matrix(x0, w),
+        x = x0 if i == 0 else _empty_like_matrix(x0, w, w.x_off).copy_(x0)
+        d = dy0 if i == 0 else _empty_like_matrix(dy0, w, w.offset).copy_(dy0)
+        sets.append({"x": x, "dy": d, "y": _empty_like_matrix(x0, w, w.offset),
+                     "dx": _empty_like_matrix(x0, w, w.offset),
                      "dg": torch.empty_like(g), "db": torch.empty_like(b), "da": torch.empty_like(a)})
     return sets, (a, g, b), set_bytes, nsets
 
@@ -580,8 +581,9 @@ def run_ours(args, w):
     lanes = []
     for j in range(2):
         x0 = sets[0]["x"]
-        d = sets[j] if j < nsets else {"x": _empty_like_matrix(x0, w), "dy": _empty_like_matrix(x0, w),
-                                       "y": _empty_like_matrix(x0, w), "dx": _empty_like_matrix(x0, w),
+        d = sets[j] if j < nsets else {"x": _empty_like_matrix(x0, w, w.x_off), "dy": _empty_like_matrix(x0, w, w.offset),
+                                       "y": _empty_like_matrix(x0, w, w.offset),
+                                       "dx": _empty_like_matrix(x0, w, w.offset),
                                        "dg": torch.empty_like(gamma), "db": torch.empty_like(beta),
                                        "da": torch.empty_like(alpha)}
         lanes.append({"dev": d, "ws": dyt.workspace(x0, gamma), "stream": stream if j == 0 else torch.cuda.Stream(dev),
@@ -716,10 +718,10 @@ def call_latency(args, dev, calls=30):
     state = {}
     for name, w in {**workloads.WORKLOADS, **workloads.VARIANTS}.items():
         inp = workloads.make_inputs(w)
-        x = _matrix(inp["x"], w, dev)
+        x = _matrix(inp["x"], w, dev, w.x_off)
         ad, gd, bd = w.param_dtypes
-        st = {"x": x, "dy": _matrix(inp["dy"], w, dev), "y": _empty_like_matrix(x, w),
-              "dx": _empty_like_matrix(x, w),
+        st = {"x": x, "dy": _matrix(inp["dy"], w, dev, w.offset), "y": _empty_like_matrix(x, w, w.offset),
+              "dx": _empty_like_matrix(x, w, w.offset),
               "p": [_to_torch(inp[k], dt, dev) for k, dt in zip(("alpha", "gamma", "beta"), (ad, gd, bd))],
               "ws": None, "t": {"fwd": [], "bwd": []}}
         st["ws"] = dyt.workspace(x, st["p"][1])

@@ -30,7 +30,7 @@ class LaunchInfo(ctypes.Structure):
     _fields_ = [("op", _i32), ("path", _i32), ("vec", _i32), ("block", _i32), ("grid", _i32),
                 ("row_lanes", _i32), ("rows_per_step", _i32), ("col_chunks", _i32),
                 ("row_groups", _i32), ("kernels", _i32), ("async_stages", _i32),
-                ("pack_rows", _i32), ("workspace_bytes", _i64)]
+                ("pack_rows", _i32), ("shifted", _i32), ("shift", _i32), ("workspace_bytes", _i64)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -58,7 +58,7 @@ lib.dyt_last_cuda_error.argtypes = []
 lib.dyt_last_cuda_error.restype = _i32
 lib.dyt_last_launch_info.argtypes = [ctypes.POINTER(LaunchInfo)]
 lib.dyt_last_launch_info.restype = _i32
-lib.dyt_plan_query.argtypes = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(LaunchInfo)]
+lib.dyt_plan_query.argtypes = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(LaunchInfo)]
 lib.dyt_plan_query.restype = _i32
 class PartialsLayout(ctypes.Structure):
     """dyt_partials_layout: where a stage-1 launch left its binary64 partials."""
@@ -226,10 +226,14 @@ def dyt_status_string(status: int) -> str:
     return lib.dyt_status_string(status).decode()
 
 
-def dyt_plan_query(M, N, x_dtype, param_dtype, backward, vectorized, sm_count, ctas_per_sm) -> dict:
-    """The launch plan for a shape on a hypothetical device (host arithmetic only)."""
+def dyt_plan_query(M, N, x_dtype, param_dtype, backward, layout, sm_count, ctas_per_sm, shift=0) -> dict:
+    """The launch plan for a shape on a hypothetical device (host arithmetic only).
+
+    layout: 0 = rows that are not whole 16-byte vectors (one-element kernels),
+    1 = contiguous and 16-byte aligned, 2 = contiguous with the output `shift`
+    elements past a 16-byte boundary (the shifted kernels)."""
     info = LaunchInfo()
-    _check(lib.dyt_plan_query(M, N, x_dtype, param_dtype, int(backward), int(vectorized), sm_count,
+    _check(lib.dyt_plan_query(M, N, x_dtype, param_dtype, int(backward), int(layout), int(shift), sm_count,
                               ctas_per_sm, ctypes.byref(info)), "dyt_plan_query")
     return info.as_dict()
 

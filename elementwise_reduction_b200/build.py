@@ -15,16 +15,13 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdyt.so")
-SOURCES = [os.path.join(CSRC, "dyt_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_async.cuh")] + [
+SOURCES = [os.path.join(CSRC, f) for f in ("dyt_api.cu", "dyt_inst_f32.cu", "dyt_inst_bf16.cu", "dyt_inst_f16.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_async.cuh", "dyt_finalize.cuh",
+                                                  "dyt_select.cuh", "dyt_select_impl.cuh")] + [
     os.path.join(INCLUDE, "dyt.h")]
 
-NVCC_FLAGS = [
-    "-std=c++17", "-O3", "-lineinfo",
-    "-gencode", "arch=compute_100a,code=sm_100a",
-    "-Xcompiler", "-fPIC", "-shared",
-    "-I", INCLUDE, "-I", CSRC,
-]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = ["-std=c++17", "-O3", "-lineinfo", *ARCH, "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 
 
 def nvcc() -> str:
@@ -35,16 +32,29 @@ def nvcc() -> str:
 def build(force: bool = False, verbose: bool = False, defines=(), out: str | None = None) -> str:
     """Compile libdyt.so if any source is newer than it. Returns its path.
 
+    The translation units (the C ABI, and the kernels of each activation dtype)
+    compile in parallel and are linked into one shared library.
     defines: extra -D tuning overrides; out: another output path (for sweeps).
     """
+    import concurrent.futures
+    import tempfile
+
     out = out or LIB
     if not force and not defines and os.path.exists(out):
         built = os.path.getmtime(out)
         if all(os.path.getmtime(d) <= built for d in DEPS):
             return out
-    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), *[f"-D{d}" for d in defines],
-           "-o", out + ".tmp", *SOURCES, "-lcudart"]
-    subprocess.check_call(cmd)
+    with tempfile.TemporaryDirectory() as tmp:
+        def compile_one(src: str) -> str:
+            obj = os.path.join(tmp, os.path.basename(src) + ".o")
+            cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), *[f"-D{d}" for d in defines],
+                   "-c", "-o", obj, src]
+            subprocess.check_call(cmd)
+            return obj
+
+        with concurrent.futures.ThreadPoolExecutor(len(SOURCES)) as pool:
+            objs = list(pool.map(compile_one, SOURCES))
+        subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", out + ".tmp", *objs, "-lcudart"])
     os.replace(out + ".tmp", out)
     return out
 

@@ -10,38 +10,17 @@
 #include <unordered_map>
 
 #include "dyt.h"
-#include "dyt_kernels.cuh"
-#include "dyt_async.cuh"
+#include "dyt_finalize.cuh"
+#include "dyt_select.cuh"
 
 namespace {
 
 using dyt::Geom;
+using namespace dyt::launch;
 
 thread_local dyt_launch_info t_info = {};
 thread_local int t_cuda_err = 0;
 
-constexpr int kScalarBlock = 1024;      // threads per CTA of the one-element kernels
-constexpr int kScalarUnrollFwd = 8;     // rows in flight per thread there
-constexpr int kScalarUnrollBwd = 8;
-constexpr int kAsyncBlock = 512;        // 16-byte kernels: one CTA per SM, up to 128 registers a thread
-constexpr int kAsyncStagesFwd = 8;      // ring slots per thread (forward: x)
-constexpr int kAsyncStagesBwd = 6;      // ring slots per thread (backward: x and dy)
-// The backward over narrow rows (at most kNarrowMaxNV 16-byte vectors per row)
-// runs 256-thread CTAs with deeper rings: each thread then visits twice the
-// rows, and the per-thread fixed work (group bounds, ring prologue, parameter
-// loads, the row-lane reduction) is spread over twice the elements. Measured
-// on B200: 65537 x 32 bf16 9.2 -> 8.2 us, 100003 x 17 fp32 11.3 -> 10.0 us,
-// 100003 x 100 fp32 26.9 -> 25.0 us; 128 threads and 12 slots were slower.
-constexpr int kAsyncBlockNarrow = 256;
-constexpr int kAsyncStagesBwdNarrow = 8;
-constexpr int kNarrowMaxNV = 64;
-// Rows one lane adds per group, at most. The kernels count a thread's rows with
-// a multiply-high by ceil(2^32 / RL), exact for counts below 2^32 / RL; a
-// count stays below 2049 RL, and 2049 RL^2 < 2^32 for every RL <= 1024.
-constexpr int kMaxRowsPerLane = 2048;
-// Inputs read by one launch below which the L2 prefetch of the first rows is
-// skipped (bytes): smaller inputs are likely resident in L2 already.
-constexpr int64_t kPrefetchMinBytes = 1 << 20;
 
 dyt_status cuda_fail(cudaError_t e) {
   t_cuda_err = (int)e;
@@ -51,6 +30,12 @@ dyt_status cuda_fail(cudaError_t e) {
 size_t dsize(int d) { return d == DYT_F32 ? 4 : 2; }
 bool valid_dtype(int d) { return d == DYT_F32 || d == DYT_BF16 || d == DYT_F16; }
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+// A pointer to whole elements of `bytes` bytes (the kernels' loads need it).
+bool elem_aligned(const void *p, size_t bytes) { return ((uintptr_t)p & (bytes - 1)) == 0; }
+// Elements between the 16-byte boundary below p and p.
+int shift_of(const void *p, size_t elem) { return (int)(((uintptr_t)p & 15u) / elem); }
+// Two pointers at the same offset past a 16-byte boundary.
+bool same_offset(const void *a, const void *b) { return (((uintptr_t)a ^ (uintptr_t)b) & 15u) == 0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ---- per-device facts and per-kernel occupancy (cached, thread-safe) -------
@@ -132,7 +117,10 @@ struct Plan {
   int grid;
   int path;     // 1 = row-tiled, 2 = row-per-CTA
   bool async;   // the 16-byte per-thread copy rings
-  bool packed;  // ragged N on 16-byte aligned rows: packs of vec rows (see dyt_kernels.cuh)
+  bool packed;  // the packed-layout kernels: a ragged N (packs of vec rows) or the shifted kernels
+  bool shifted; // the shifted kernels: contiguous tensors not all 16-byte aligned (see dyt_async.cuh)
+  int shm;      // their mode: 0 = not shifted, else 1 | 2 (x's vectors cut out of two chunks) | 4 (dy's)
+  int pack_rows;  // matrix rows per row of the packed layout: vec for a ragged N, else 1
   bool too_big; // the group or item count would not fit the kernels' int indices
   size_t smem;  // dynamic shared memory of the 16-byte kernel
   size_t ws_dg, ws_db, ws_da, ws_total;  // workspace byte offsets / sizes
@@ -147,34 +135,42 @@ size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 size_t async_stages(bool backward, int block) {
   return !backward ? kAsyncStagesFwd : block == kAsyncBlockNarrow ? kAsyncStagesBwdNarrow : kAsyncStagesBwd;
 }
-size_t async_smem(bool backward, int block, size_t elem_bytes) {
-  if (!backward) return (size_t)kAsyncStagesFwd * block * 16;
+// The shifted kernels hold two 16-byte chunks per slot and tensor.
+size_t async_smem(bool backward, int block, size_t elem_bytes, bool shifted) {
+  const size_t ch = shifted ? 2 : 1;
+  if (!backward) return (size_t)kAsyncStagesFwd * ch * block * 16;
   const size_t totals = elem_bytes == 4 ? 0 : (16 / elem_bytes) * (size_t)block * sizeof(double);
-  return async_stages(true, block) * 2 * block * 16 + totals;
+  return async_stages(true, block) * 2 * ch * block * 16 + totals;
 }
 
 // vec: elements per access (1 or 16 / element size). ctas_per_sm from the
-// kernel's occupancy. packed: N is not a multiple of vec, and the matrix is
-// laid out as ceil(M / vec) packs of vec rows, each of pitch vec * N. The
-// plan depends only on (M, N, vec, packed, SM count, occupancy).
+// kernel's occupancy. ragged: N is not a multiple of vec, and the matrix is
+// laid out as packs of vec rows, each of pitch vec * N. shifted: the shifted
+// kernels, whose packed layout (packs of vec rows for a ragged N, else of one
+// row) starts the matrix at position sh, the output's offset past a 16-byte
+// boundary in elements. The plan depends only on these arguments.
 Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool async, int sms, int ctas_per_sm,
-               bool packed, int64_t elem_bytes) {
+               bool ragged, bool shifted, int sh, int64_t elem_bytes) {
   Plan p = {};
   p.vec = vec;
   p.async = async;
-  p.packed = packed;
-  const int64_t M = packed ? ceil_div(M_rows, (int64_t)vec) : M_rows;
-  const int64_t N = packed ? (int64_t)vec * N_cols : N_cols;
+  p.packed = ragged || shifted;
+  p.shifted = shifted;
+  p.pack_rows = ragged ? vec : 1;
+  const int64_t end = M_rows * N_cols + (shifted ? sh : 0);  // the matrix's end in the (packed) layout
+  const int64_t N = (int64_t)p.pack_rows * N_cols;
+  const int64_t M = p.packed ? ceil_div(end, N) : M_rows;
   const int64_t NV = N / vec;
   p.block = !async ? kScalarBlock : backward && NV <= kNarrowMaxNV ? kAsyncBlockNarrow : kAsyncBlock;
   const int block = p.block;
   p.unroll = async ? 1 : (backward ? kScalarUnrollBwd : kScalarUnrollFwd);
-  p.smem = async ? async_smem(backward, block, (size_t)elem_bytes) : 0;
+  p.smem = async ? async_smem(backward, block, (size_t)elem_bytes, shifted) : 0;
   Geom &g = p.g;
   g.M = M;
   g.N = N;
   g.Nc = N_cols;
-  g.total = M_rows * N_cols;
+  g.total = end;
+  g.sh = shifted ? sh : 0;
   g.ldx = g.ldd = g.ldo = N;  // adjacent rows; the strided calls override this
   g.NV = (int)NV;
   if (NV <= block / 2) {
@@ -224,27 +220,10 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool asyn
 
 // ---- kernel tables ---------------------------------------------------------------
 
-template <typename T>
-constexpr int vec_of() {
-  return 16 / (int)sizeof(T);
-}
-
 template <typename T, typename P>
-const void *main_kernel(bool backward, bool async, bool packed, int block) {
-  constexpr int V = vec_of<T>();
-  if (async) {
-    if (backward && block == kAsyncBlockNarrow)
-      return packed
-                 ? (const void *)dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlockNarrow, kAsyncStagesBwdNarrow, true>
-                 : (const void *)dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlockNarrow, kAsyncStagesBwdNarrow, false>;
-    if (backward)
-      return packed ? (const void *)dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, true>
-                    : (const void *)dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, false>;
-    return packed ? (const void *)dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, true>
-                  : (const void *)dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, false>;
-  }
-  return backward ? (const void *)dyt::dyt_bwd_kernel<T, P, kScalarUnrollBwd, kScalarBlock>
-                  : (const void *)dyt::dyt_fwd_kernel<T, P, kScalarUnrollFwd, kScalarBlock>;
+const void *main_kernel(bool backward, bool async, bool packed, int shm, int block) {
+  return backward ? (const void *)bwd_kernel_of<T, P>(async, packed, shm, block)
+                  : (const void *)fwd_kernel_of<T, P>(async, packed, shm);
 }
 
 // The parameter type of the kernels for these parameter dtypes: the shared
@@ -311,7 +290,9 @@ dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
     i.block = p->block;
     i.grid = p->grid;
     i.row_lanes = p->g.RL;
-    i.pack_rows = p->packed ? p->vec : 1;
+    i.pack_rows = p->pack_rows;
+    i.shifted = p->shifted ? 1 : 0;
+    i.shift = p->g.sh;
     i.rows_per_step = p->g.RL * p->unroll * i.pack_rows;
     i.col_chunks = p->g.ncc;
     i.row_groups = p->g.nrg;
@@ -324,39 +305,49 @@ void record(int op, const Plan *p, int kernels, size_t ws) { t_info = describe(o
 
 // Which kernels a call takes. aligned: every tensor starts on a 16-byte
 // boundary; pitched: every row pitch is a whole number of 16-byte vectors;
-// adjacent: every pitch is N. v: elements per 16-byte vector.
+// adjacent: every pitch is N. v: elements per 16-byte vector. Every pointer
+// is a whole number of elements (checked before).
 struct PathChoice {
-  bool packed;  // ragged N on adjacent rows: packs of v rows through the 16-byte kernels
-  bool async;   // the 16-byte kernels (per-thread copy rings)
-  int vec;      // elements per access: v, or 1 for the one-element kernels
+  bool ragged;   // ragged N on adjacent rows: packs of v rows through the 16-byte kernels
+  bool shifted;  // adjacent rows not all 16-byte aligned: the shifted 16-byte kernels
+  bool async;    // the 16-byte kernels (per-thread copy rings)
+  int vec;       // elements per access: v, or 1 for the one-element kernels
 };
 
 PathChoice choose_path(int64_t N, int v, bool aligned, bool pitched, bool adjacent) {
   PathChoice c;
+  c.shifted = !aligned && adjacent;
   // A pack of v adjacent rows is a whole number of vectors whatever N is.
-  c.packed = aligned && adjacent && N % v != 0;
-  c.async = aligned && (c.packed || (pitched && N % v == 0));
+  c.ragged = adjacent && N % v != 0;
+  c.async = c.shifted || (aligned && (c.ragged || (pitched && N % v == 0)));
+  if (!c.async) c.ragged = false;
   c.vec = c.async ? v : 1;
   return c;
 }
 
-// The plan for tensors of type T with the given layout on the current device.
+// The plan for tensors of type T with the given layout on the current device;
+// sh: the output's offset past a 16-byte boundary, in elements; win: for the
+// shifted kernels, 2 if x's offset differs from the output's, | 4 if dy's does.
 template <typename T, typename P>
-dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjacent, bool backward, Plan *out) {
+dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjacent, int sh, int win,
+                    bool backward, Plan *out) {
   int dev = 0, sms = 0;
   dyt_status st = current_sms(&dev, &sms);
   if (st != DYT_OK) return st;
   const PathChoice pc = choose_path(N, vec_of<T>(), aligned, pitched, adjacent);
   if (pc.async) {
     // One CTA per SM by construction (__launch_bounds__(B, 1), ring sized for it).
-    *out = make_plan(M, N, pc.vec, backward, true, sms, 1, pc.packed, (int64_t)sizeof(T));
+    *out = make_plan(M, N, pc.vec, backward, true, sms, 1, pc.ragged, pc.shifted, sh, (int64_t)sizeof(T));
     if (out->too_big) return DYT_ERR_INVALID_VALUE;
-    return prepare_smem(dev, main_kernel<T, P>(backward, true, pc.packed, out->block), (int)out->smem);
+    // dy alone off the output's offset runs the kernel that cuts both inputs
+    out->shm = !out->shifted ? 0 : (win & 4) ? 7 : 1 | (win & 2);
+    return prepare_smem(dev, main_kernel<T, P>(backward, true, out->packed, out->shm, out->block),
+                        (int)out->smem);
   }
   int occ = 1;
-  st = occupancy(dev, main_kernel<T, P>(backward, false, false, kScalarBlock), kScalarBlock, &occ);
+  st = occupancy(dev, main_kernel<T, P>(backward, false, false, 0, kScalarBlock), kScalarBlock, &occ);
   if (st != DYT_OK) return st;
-  *out = make_plan(M, N, pc.vec, backward, pc.async, sms, occ, pc.packed, (int64_t)sizeof(T));
+  *out = make_plan(M, N, pc.vec, backward, false, sms, occ, false, false, 0, (int64_t)sizeof(T));
   if (out->too_big) return DYT_ERR_INVALID_VALUE;
   return DYT_OK;
 }
@@ -389,27 +380,36 @@ dyt_partials_layout layout_of(const Plan &p) {
   l.off_dgamma = (int64_t)p.ws_dg;
   l.off_dbeta = (int64_t)p.ws_db;
   l.off_dalpha = (int64_t)p.ws_da;
-  // (nrg x pack rows) rows of N: a packed row group holds vec partial rows,
-  // one per row of the pack, in pack order.
-  l.rows = p.g.nrg * (p.packed ? p.vec : 1);
+  // (nrg x pack rows) rows of N: a packed row group holds pack_rows partial
+  // rows, one per row of the pack, in pack order.
+  l.rows = p.g.nrg * p.pack_rows;
   l.dalpha_parts = p.grid;
   return l;
 }
 
-// The layout facts of a backward call's tensors: aligned, pitched, adjacent (see choose_path).
+// The layout facts of a backward call's tensors: aligned, pitched, adjacent
+// (see choose_path), the output's offset past a 16-byte boundary and which
+// inputs' offsets differ from it (see plan_for).
 struct LayoutArgs {
   bool aligned, pitched, adjacent;
+  int sh, win;
 };
 template <typename T>
 LayoutArgs stage1_layout_args(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *dx,
                               int64_t lddx, int64_t N) {
   const size_t es = sizeof(T);
   return {aligned16(x) && aligned16(dy) && aligned16(dx),
-          vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es), ldx == N && lddy == N && lddx == N};
+          vec_pitch(ldx, es) && vec_pitch(lddy, es) && vec_pitch(lddx, es), ldx == N && lddy == N && lddx == N,
+          shift_of(dx, es), (same_offset(x, dx) ? 0 : 2) | (same_offset(dy, dx) ? 0 : 4)};
 }
 template <typename T, typename P>
 dyt_status plan_for(int64_t M, int64_t N, LayoutArgs a, bool backward, Plan *out) {
-  return plan_for<T, P>(M, N, a.aligned, a.pitched, a.adjacent, backward, out);
+  return plan_for<T, P>(M, N, a.aligned, a.pitched, a.adjacent, a.sh, a.win, backward, out);
+}
+
+// The gradient pointers hold whole elements of their dtypes.
+bool grads_aligned(const void *dgamma, const void *dbeta, const void *dalpha, int ad, int gd, int bd) {
+  return elem_aligned(dgamma, dsize(gd)) && elem_aligned(dbeta, dsize(bd)) && elem_aligned(dalpha, dsize(ad));
 }
 
 // Every gradient +0 (all-zero bits in each dtype): the empty sums.
@@ -432,13 +432,16 @@ dyt_status bwd_stage1(const void *x, int64_t ldx, const void *dy, int64_t lddy, 
                       dyt_partials_layout *lay) {
   if (!x || !dy || !alpha || !gamma || !dx || !workspace) return DYT_ERR_INVALID_VALUE;
   if (!aligned16(workspace)) return DYT_ERR_INVALID_VALUE;
+  const size_t es = dsize(x_dtype);
+  if (!elem_aligned(x, es) || !elem_aligned(dy, es) || !elem_aligned(dx, es) ||
+      !elem_aligned(alpha, dsize(alpha_dtype)) || !elem_aligned(gamma, dsize(gamma_dtype)))
+    return DYT_ERR_INVALID_VALUE;
   const dyt::ParamTypes pt = {(int)alpha_dtype, (int)gamma_dtype, (int)gamma_dtype};
   // beta is not read: the kernels' parameter type follows alpha and gamma.
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
     return with_ptype(alpha_dtype, gamma_dtype, gamma_dtype, [&](auto tp) -> dyt_status {
     using P = typename decltype(tp)::type;
-    constexpr int V = vec_of<T>();
     Plan &p = *plan;
     dyt_status r = plan_for<T, P>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
     if (r != DYT_OK) return r;
@@ -454,25 +457,8 @@ dyt_status bwd_stage1(const void *x, int64_t ldx, const void *dy, int64_t lddy, 
     double *pda = (double *)(ws + p.ws_da);
     const P *pa = (const P *)alpha, *pg = (const P *)gamma;
     PdlConfig lc(p.grid, p.block, p.smem, s);
-    cudaError_t e;
-    const bool narrow = p.block == kAsyncBlockNarrow;
-    if (p.async && narrow && p.packed)
-      e = cudaLaunchKernelEx(&lc.cfg,
-                             dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlockNarrow, kAsyncStagesBwdNarrow, true>,
-                             (const T *)x, (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
-    else if (p.async && narrow)
-      e = cudaLaunchKernelEx(&lc.cfg,
-                             dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlockNarrow, kAsyncStagesBwdNarrow, false>,
-                             (const T *)x, (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
-    else if (p.async && p.packed)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, true>,
-                             (const T *)x, (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
-    else if (p.async)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesBwd, false>,
-                             (const T *)x, (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
-    else
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_bwd_kernel<T, P, kScalarUnrollBwd, kScalarBlock>, (const T *)x,
-                             (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
+    const cudaError_t e = cudaLaunchKernelEx(&lc.cfg, bwd_kernel_of<T, P>(p.async, p.packed, p.shm, p.block),
+                                             (const T *)x, (const T *)dy, pa, pg, pt, (T *)dx, pdg, pdb, pda, p.g);
     if (e != cudaSuccess) return cuda_fail(e);
     *lay = layout_of(p);
     return DYT_OK;
@@ -549,16 +535,19 @@ dyt_status dyt_forward_ex(const void *x, int64_t ldx, const void *alpha, const v
     return DYT_OK;
   }
   if (!x || !alpha || !gamma || !beta || !y) return DYT_ERR_INVALID_VALUE;
+  const size_t es = dsize(x_dtype);
+  if (!elem_aligned(x, es) || !elem_aligned(y, es) || !elem_aligned(alpha, dsize(alpha_dtype)) ||
+      !elem_aligned(gamma, dsize(gamma_dtype)) || !elem_aligned(beta, dsize(beta_dtype)))
+    return DYT_ERR_INVALID_VALUE;
   const dyt::ParamTypes pt = {(int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
     return with_ptype(alpha_dtype, gamma_dtype, beta_dtype, [&](auto tp) -> dyt_status {
     using P = typename decltype(tp)::type;
-    constexpr int V = vec_of<T>();
     Plan p;
     dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y),
-                                  vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)), ldx == N && ldy == N, false,
-                                  &p);
+                                  vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)), ldx == N && ldy == N,
+                                  shift_of(y, sizeof(T)), same_offset(x, y) ? 0 : 2, false, &p);
     if (s != DYT_OK) return s;
     if (!p.packed) {
       p.g.ldx = ldx;
@@ -566,16 +555,8 @@ dyt_status dyt_forward_ex(const void *x, int64_t ldx, const void *alpha, const v
     }
     const P *pa = (const P *)alpha, *pg = (const P *)gamma, *pb = (const P *)beta;
     PdlConfig lc(p.grid, p.block, p.smem, (cudaStream_t)stream);
-    cudaError_t e;
-    if (p.async && p.packed)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, true>,
-                             (const T *)x, pa, pg, pb, pt, (T *)y, p.g);
-    else if (p.async)
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_async_kernel<T, P, V, kAsyncBlock, kAsyncStagesFwd, false>,
-                             (const T *)x, pa, pg, pb, pt, (T *)y, p.g);
-    else
-      e = cudaLaunchKernelEx(&lc.cfg, dyt::dyt_fwd_kernel<T, P, kScalarUnrollFwd, kScalarBlock>, (const T *)x, pa,
-                             pg, pb, pt, (T *)y, p.g);
+    const cudaError_t e = cudaLaunchKernelEx(&lc.cfg, fwd_kernel_of<T, P>(p.async, p.packed, p.shm),
+                                             (const T *)x, pa, pg, pb, pt, (T *)y, p.g);
     if (e != cudaSuccess) return cuda_fail(e);
     record(1, &p, 1, 0);
     return DYT_OK;
@@ -589,10 +570,14 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
   size_t need = 0;
   dyt_status st = with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
-    // The 16-byte and the one-element plan may differ; cover both.
-    for (int v = 0; v < 2; ++v) {
+    // The aligned, the shifted (one per output offset) and the one-element
+    // plans may differ; cover them all. The plans do not depend on P.
+    constexpr int V = vec_of<T>();
+    for (int v = -2; v < V; ++v) {
       Plan p;
-      dyt_status s = plan_for<T, float>(M, N, v == 1, v == 1, true, true, &p);  // the plan does not depend on P
+      const dyt_status s = v == -2   ? plan_for<T, float>(M, N, true, true, true, 0, 0, true, &p)
+                           : v == -1 ? plan_for<T, float>(M, N, false, false, false, 0, 0, true, &p)
+                                     : plan_for<T, float>(M, N, false, false, true, v, 0, true, &p);
       if (s != DYT_OK) return s;
       if (p.ws_total > need) need = p.ws_total;
     }
@@ -630,6 +615,7 @@ dyt_status dyt_backward_ex(const void *x, int64_t ldx, const void *dy, int64_t l
   if (check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, lddy) != DYT_OK || check_pitch(M, N, lddx) != DYT_OK)
     return DYT_ERR_INVALID_VALUE;
   if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return DYT_ERR_INVALID_VALUE;
+  if (!grads_aligned(dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype)) return DYT_ERR_INVALID_VALUE;
   if (M == 0 || N == 0) {
     st = zero_gradients(N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype, (cudaStream_t)stream);
     if (st == DYT_OK) record(2, nullptr, 0, 0);
@@ -699,6 +685,7 @@ dyt_status dyt_finalize_partials(const void *const *workspaces, const dyt_partia
   if (st != DYT_OK) return st;
   if (N < 0 || N > INT32_MAX) return DYT_ERR_INVALID_VALUE;
   if (!dalpha || (N > 0 && (!dgamma || !dbeta))) return DYT_ERR_INVALID_VALUE;
+  if (!grads_aligned(dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype)) return DYT_ERR_INVALID_VALUE;
   if (N == 0)
     return zero_gradients(N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype, (cudaStream_t)stream);
   st = bwd_finalize(workspaces, layouts, nranks, N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype,
@@ -762,22 +749,25 @@ const char *dyt_status_string(dyt_status status) {
 
 int dyt_last_cuda_error(void) { return t_cuda_err; }
 
-dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype, int backward,
-                          int vectorized, int sm_count, int ctas_per_sm, dyt_launch_info *out) {
+dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype, int backward, int layout,
+                          int shift, int sm_count, int ctas_per_sm, dyt_launch_info *out) {
   if (!out || sm_count < 1 || ctas_per_sm < 1) return DYT_ERR_INVALID_VALUE;
   dyt_status st = check_shape(M, N, x_dtype);
   if (st == DYT_OK && !valid_dtype(param_dtype)) st = DYT_ERR_UNSUPPORTED_DTYPE;
   if (st != DYT_OK) return st;
+  const int v = 16 / (int)dsize(x_dtype);
+  if (layout < 0 || layout > 2 || (layout == 2 && (shift < 0 || shift >= v))) return DYT_ERR_INVALID_VALUE;
   const int op = backward ? 2 : 1;
   if (M == 0 || N == 0) {
     *out = describe(op, nullptr, 0, 0);
     return DYT_OK;
   }
-  const int v = 16 / (int)dsize(x_dtype);
-  const PathChoice pc = choose_path(N, v, vectorized != 0, vectorized != 0, true);  // adjacent rows
+  // layout 0: rows that are not whole 16-byte vectors; 1: contiguous and
+  // 16-byte aligned; 2: contiguous, the output `shift` elements past a boundary.
+  const PathChoice pc = choose_path(N, v, layout == 1, layout == 1, layout != 0);
   // The 16-byte kernels always run one CTA per SM.
-  Plan p = make_plan(M, N, pc.vec, backward != 0, pc.async, sm_count, pc.async ? 1 : ctas_per_sm, pc.packed,
-                     (int64_t)dsize(x_dtype));
+  Plan p = make_plan(M, N, pc.vec, backward != 0, pc.async, sm_count, pc.async ? 1 : ctas_per_sm, pc.ragged,
+                     pc.shifted, layout == 2 ? shift : 0, (int64_t)dsize(x_dtype));
   if (p.too_big) return DYT_ERR_INVALID_VALUE;
   *out = describe(op, &p, backward ? 2 : 1, backward ? p.ws_total : 0);
   return DYT_OK;

@@ -38,11 +38,13 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // Matrix columns of the VEC elements of the vector at offset c0 of a row:
-// c0 + e, or on the packed path (c0 + e) mod Nc, where c0 < VEC * Nc.
+// c0 + e, or on the packed path (c0 + e) mod Nc, where -VEC < c0 < VEC * Nc
+// (the shifted kernels pass the vector's offset minus sh).
 template <int VEC, bool PK>
 __device__ __forceinline__ void vector_columns(int64_t c0, int64_t Nc, int64_t (&col)[VEC]) {
   if constexpr (PK) {
     int64_t c = c0;
+    while (c < 0) c += Nc;    // the shifted layout: c0 - sh, sh < VEC
     while (c >= Nc) c -= Nc;  // at most VEC - 1 times
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
@@ -55,13 +57,13 @@ __device__ __forceinline__ void vector_columns(int64_t c0, int64_t Nc, int64_t (
   }
 }
 
-// The first n (< VEC) elements of a 16-byte vector, one by one: the vector
-// that straddles the end of a packed matrix.
+// The elements of a 16-byte vector whose bit is set in m, one by one: the
+// vectors that straddle the start or the end of a packed matrix.
 template <typename T, int VEC>
-__device__ __forceinline__ void store_first(T *p, const uint4 &r, int n) {
+__device__ __forceinline__ void store_mask(T *p, const uint4 &r, uint32_t m) {
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
-    if (e < n) {
+    if ((m >> e) & 1u) {
       if constexpr (sizeof(T) == 4) {
         *reinterpret_cast<uint32_t *>(p + e) = word_of(r, e);
       } else {
@@ -70,6 +72,148 @@ __device__ __forceinline__ void store_first(T *p, const uint4 &r, int n) {
       }
     }
   }
+}
+
+// ---- shifted kernels: contiguous tensors off 16-byte boundaries ----------------
+//
+// The packed layout is laid over the output with its matrix starting at
+// position sh (the output's offset past a 16-byte boundary, in elements), so
+// every output vector is a whole, aligned 16-byte vector. An input whose
+// offset differs from the output's by d bytes (mod 16) holds the elements of
+// output vector k in bytes [d, d + 16) of its two aligned chunks k and k + 1:
+// both are copied into the thread's slot and the vector is cut out of them.
+
+// What the shifted kernels need of one input tensor.
+struct ShIn {
+  const char *a;     // 16-byte aligned: its first chunk under position 0 of the layout
+  int d;             // byte offset of a vector in its two chunks (0: the vector is one chunk)
+  uintptr_t lo, hi;  // the tensor's bytes [lo, hi)
+};
+
+template <typename T>
+__device__ __forceinline__ ShIn shifted_input(const T *p, const Geom &g) {
+  ShIn s;
+  const uintptr_t f = (uintptr_t)p - (uintptr_t)g.sh * sizeof(T);  // where position 0 falls in this tensor
+  s.d = (int)(f & 15u);
+  s.a = reinterpret_cast<const char *>(f - (uintptr_t)s.d);
+  s.lo = (uintptr_t)p;
+  s.hi = s.lo + (uintptr_t)(g.total - g.sh) * sizeof(T);
+  return s;
+}
+
+// Bytes [d, d + 16) of the 32 bytes lo:hi (two adjacent 16-byte chunks,
+// little-endian words), 0 <= d < 16: the word offset d / 4 by two selects,
+// the byte offset by funnel shifts (a shift of 0 returns the low word).
+__device__ __forceinline__ uint4 window16(const uint4 &lo, const uint4 &hi, int d) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  const int q = d >> 2;
+  const uint32_t r = (uint32_t)(d & 3) * 8u;
+  uint32_t u[6], v[5];
+#pragma unroll
+  for (int i = 0; i < 6; ++i) u[i] = (q & 2) ? w[i + 2] : w[i];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) v[i] = (q & 1) ? u[i + 1] : u[i];
+  return make_uint4(__funnelshift_r(v[0], v[1], r), __funnelshift_r(v[1], v[2], r), __funnelshift_r(v[2], v[3], r),
+                    __funnelshift_r(v[3], v[4], r));
+}
+
+// A 16-byte chunk (at a, 16-byte aligned) of a tensor whose bytes are
+// [lo, hi), elements of ES bytes: copied whole when it lies inside; only its
+// first hi - a bytes (the rest of the slot zero-filled) when the tensor ends in
+// it; element by element from lo when the tensor starts in it; not at all when
+// it holds none of the tensor. Nothing outside [lo, hi) is read. The slot bytes
+// not written hold stale values, which only padded elements take.
+template <int ES>
+__device__ __forceinline__ void copy_chunk_checked(uint4 *slot, const char *a, uintptr_t lo, uintptr_t hi) {
+  const uintptr_t ua = (uintptr_t)a;
+  if (ua >= hi || ua + 16u <= lo) return;
+  if (ua >= lo) {
+    const uintptr_t n = hi - ua;
+    cp_async16_zfill(slot, a, n < 16u ? (uint32_t)n : 16u);
+    return;
+  }
+  const int b1 = hi - ua < 16u ? (int)(hi - ua) : 16;
+  char *dst = reinterpret_cast<char *>(slot);
+  for (int b = (int)(lo - ua); b < b1; b += ES) {
+    if constexpr (ES == 4) *reinterpret_cast<uint32_t *>(dst + b) = *reinterpret_cast<const uint32_t *>(a + b);
+    else *reinterpret_cast<unsigned short *>(dst + b) = *reinterpret_cast<const unsigned short *>(a + b);
+  }
+}
+
+// One input's chunks of a row into its slot (chunk 0 at slot, chunk 1 at
+// slot + B): plain copies on the rows where every copy lies inside the tensor
+// (fast), checked ones elsewhere.
+// W: the kernel cuts windows out of this input (its offset may differ from
+// the output's); without W its vectors are single chunks (d = 0).
+template <typename T, int B, bool W>
+__device__ __forceinline__ void copy_shifted(uint4 *slot, const T *src, const ShIn &s, bool fast) {
+  const char *a = reinterpret_cast<const char *>(src);
+  if (fast) {
+    cp_async16(slot, a);
+    if (W && s.d) cp_async16(slot + B, a + 16);
+  } else {
+    copy_chunk_checked<(int)sizeof(T)>(slot, a, s.lo, s.hi);
+    if (W && s.d) copy_chunk_checked<(int)sizeof(T)>(slot + B, a + 16, s.lo, s.hi);
+  }
+}
+
+// The input vector of a row from its slot.
+template <int B, bool W>
+__device__ __forceinline__ uint4 read_shifted(const uint4 *slot, const ShIn &s) {
+  if constexpr (W) return window16(slot[0], slot[B], s.d);
+  else return *slot;
+}
+
+// Whether row k of a thread is one of its whole-vector rows [k_lo, k_hi).
+__device__ __forceinline__ bool fast_row(int k, int k_lo, int k_hi) {
+  return (unsigned)(k - k_lo) < (unsigned)(k_hi - k_lo);
+}
+
+// Real elements (bits) of the output vector at position pos of the layout:
+// those in [sh, total).
+template <int VEC>
+__device__ __forceinline__ uint32_t shifted_mask(const Geom &g, int64_t pos) {
+  const int lo = pos < g.sh ? (int)(g.sh - pos) : 0;
+  const int64_t rem = g.total - pos;
+  const int hi = rem <= 0 ? 0 : rem < VEC ? (int)rem : VEC;
+  return ((1u << hi) - 1u) & ~((1u << lo) - 1u);
+}
+
+// The L2 prefetch of prefetch_first_rows_l2 for the shifted kernels: the same
+// rows of the layout, clipped to the 16-byte units that lie wholly inside the
+// tensor, so nothing outside it is touched.
+template <typename T, int VEC, int B, int S>
+__device__ __forceinline__ void prefetch_shifted_rows_l2(const ShIn &s, const Geom &g) {
+  if (!g.l2_prefetch || threadIdx.x >= 32 || (int)blockIdx.x >= g.nitems) return;  // warp 0 issues them
+  int cc, rg;
+  item_split(g, blockIdx.x, cc, rg);
+  int64_t rb, re;
+  group_rows(g, rg, rb, re);
+  const int64_t rows = min(re - rb, (int64_t)(S - 1) * g.RL);
+  if (rows <= 0) return;
+  const uintptr_t lo = (s.lo + 15u) & ~(uintptr_t)15, hi = s.hi & ~(uintptr_t)15;
+  constexpr uintptr_t kPiece = 16384;
+  uintptr_t a, e;
+  if (g.ncc == 1) {  // whole rows: one range, cut into pieces
+    a = (uintptr_t)s.a + (uintptr_t)(rb * g.N) * sizeof(T) + threadIdx.x * kPiece;
+    e = (uintptr_t)s.a + (uintptr_t)((rb + rows) * g.N) * sizeof(T);
+    if (e > a + kPiece) e = a + kPiece;
+  } else {  // one column chunk of each row
+    if (threadIdx.x >= rows) return;
+    const int64_t c0 = (int64_t)cc * B * VEC;
+    a = (uintptr_t)s.a + (uintptr_t)((rb + threadIdx.x) * g.N + c0) * sizeof(T);
+    e = a + (uintptr_t)min((int64_t)B * VEC, g.N - c0) * sizeof(T);
+  }
+  if (a < lo) a = lo;
+  if (e > hi) e = hi;
+  if (a < e)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"((uint32_t)(e - a)) : "memory");
+}
+
+// Whether input chunk(s) at a lie inside the tensor from below / from above.
+__device__ __forceinline__ bool shifted_lo_ok(const ShIn &s, const void *a) { return (uintptr_t)a >= s.lo; }
+__device__ __forceinline__ bool shifted_hi_ok(const ShIn &s, const void *a) {
+  return (uintptr_t)a + (s.d ? 32u : 16u) <= s.hi;
 }
 
 // Start pulling into L2 the rows this CTA copies first: those of its first
@@ -143,18 +287,35 @@ __device__ __forceinline__ int last_vector_real(const Geom &g, int64_t first, in
   return r < VEC ? (int)r : VEC;
 }
 
-template <typename T, typename P, int VEC, int B, int S, bool PK>
+// SHM != 0: the shifted kernels (contiguous tensors not all 16-byte aligned;
+// PK holds): ring slots of two chunks, the packed layout laid over the output
+// with its matrix from position g.sh, rows whose copies or output vector reach
+// past a tensor's ends handled one by one (checked copies, masked stores).
+// SHM bit 1: x's offset differs from y's, so its vectors are cut out of two
+// chunks.
+template <typename T, typename P, int VEC, int B, int S, bool PK, int SHM>
 __global__ void __launch_bounds__(B, 1)
     dyt_fwd_async_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma_p,
                          const P *__restrict__ beta_p, ParamTypes pt, T *y, Geom g) {
   using IO = VecIO<T, VEC>;
+  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0;
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
-  extern __shared__ uint4 ring[];  // [S][B]
-  prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
+  static_assert(PK || !SH, "the shifted kernels use the packed layout");
+  constexpr int CH = SH ? 2 : 1;  // 16-byte chunks per slot
+  extern __shared__ uint4 ring[];  // [S][CH][B]
+  ShIn ix = {};
+  if constexpr (SH) {
+    ix = shifted_input(x, g);
+    prefetch_shifted_rows_l2<T, VEC, B, S>(ix, g);
+  } else {
+    prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
+  }
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = load_param<P>(alpha_p, pt.alpha, 0);
   uint4 *slot0 = ring + threadIdx.x;
+  const T *xb = SH ? reinterpret_cast<const T *>(ix.a) : x;  // position 0 of the layout
+  T *yb = SH ? y - g.sh : y;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
     item_split(g, item, cc, rg);
@@ -168,34 +329,54 @@ __global__ void __launch_bounds__(B, 1)
     const int nl = last_vector_real<VEC, PK>(g, first, c0, n);
     const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
     const int64_t sx = (int64_t)g.RL * g.ldx, sy = (int64_t)g.RL * g.ldo;
-    const T *px = x + first * g.ldx + c0;
-    T *py = y + first * g.ldo + c0;
+    const T *px = xb + first * g.ldx + c0;
+    T *py = yb + first * g.ldo + c0;
+    // SH: rows [k_lo, k_hi) copy and store whole vectors; the others (at most
+    // a few at each end of the matrix) go element by element.
+    const int64_t pos0 = first * g.N + c0, dpos = (int64_t)g.RL * g.N;  // layout positions
+    int k_lo = 0, k_hi = (int)n;  // n is at most kMaxRowsPerLane
+    if constexpr (SH) {
+      while (k_lo < n && !(pos0 + k_lo * dpos >= g.sh && shifted_lo_ok(ix, px + k_lo * sx))) ++k_lo;
+      while (k_hi > k_lo &&
+             !(pos0 + (k_hi - 1) * dpos + VEC <= g.total && shifted_hi_ok(ix, px + (k_hi - 1) * sx)))
+        --k_hi;
+    }
     // Rows first, parameters second: the parameter loads overlap the copies.
 #pragma unroll
     for (int k = 0; k < S - 1; ++k) {
       if (k < n) {
-        if (PK) cp_async16_zfill(slot0 + k * B, px + k * sx, k == n - 1 ? last_bytes : 16u);
+        if constexpr (SH) copy_shifted<T, B, WX>(slot0 + k * CH * B, px + k * sx, ix, fast_row(k, k_lo, k_hi));
+        else if (PK) cp_async16_zfill(slot0 + k * B, px + k * sx, k == n - 1 ? last_bytes : 16u);
         else cp_async16(slot0 + k * B, px + k * sx);
       }
       cp_async_commit();
     }
     int64_t col[VEC];
-    vector_columns<VEC, PK>(c0, g.Nc, col);
+    vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
     float gam[VEC], bet[VEC], bth[VEC];
     fwd_params_at<T, VEC, P>(gamma_p, beta_p, pt, col, gam, bet, bth);
     int s_rd = 0, s_wr = S - 1;
     for (int64_t k = 0; k < n; ++k) {
       const int64_t kn = k + S - 1;
       if (kn < n) {
-        if (PK) cp_async16_zfill(slot0 + s_wr * B, px + kn * sx, kn == n - 1 ? last_bytes : 16u);
+        if constexpr (SH) copy_shifted<T, B, WX>(slot0 + s_wr * CH * B, px + kn * sx, ix, fast_row((int)kn, k_lo, k_hi));
+        else if (PK) cp_async16_zfill(slot0 + s_wr * B, px + kn * sx, kn == n - 1 ? last_bytes : 16u);
         else cp_async16(slot0 + s_wr * B, px + kn * sx);
       }
       cp_async_commit();
       cp_async_wait<S - 1>();
-      const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + s_rd * B);
+      typename IO::Raw rx;
+      if constexpr (SH) rx = read_shifted<B, WX>(slot0 + s_rd * CH * B, ix);
+      else rx = *(const typename IO::Raw *)(slot0 + s_rd * B);
       const typename IO::Raw ry = fwd_vector<T, VEC>(rx, alpha, gam, bet, bth);
-      if (PK && k == n - 1 && nl < VEC) store_first<T, VEC>(py, ry, nl);  // zero-filled tail: not stored
-      else IO::store_raw(py, ry);
+      if constexpr (SH) {
+        if (fast_row((int)k, k_lo, k_hi)) IO::store_raw(py, ry);
+        else store_mask<T, VEC>(py, ry, shifted_mask<VEC>(g, pos0 + k * dpos));  // padding: not stored
+      } else if (PK && k == n - 1 && nl < VEC) {
+        store_mask<T, VEC>(py, ry, (1u << nl) - 1u);  // zero-filled tail: not stored
+      } else {
+        IO::store_raw(py, ry);
+      }
       py += sy;
       s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
       s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
@@ -206,31 +387,47 @@ __global__ void __launch_bounds__(B, 1)
 
 // ---- backward, stage 1 ----------------------------------------------------------
 
-template <typename T, typename P, int VEC, int B, int S, bool PK>
+// SHM != 0: as the forward's shifted kernels, x and dy each with their own
+// offset: bit 1 cuts x's vectors out of two chunks, bit 2 dy's.
+template <typename T, typename P, int VEC, int B, int S, bool PK, int SHM>
 __global__ void __launch_bounds__(B, 1)
     dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
                          const P *__restrict__ gamma_p, ParamTypes pt, T *dx, double *__restrict__ part_dg,
                          double *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
   using IO = VecIO<T, VEC>;
+  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0, WD = (SHM & 4) != 0;
   constexpr bool EXACT_G = ExactGamma<T>::value;
   constexpr int kRunBlocks = kGammaRunRows / S;  // unrolled blocks of S rows per binary32 dgamma run
+  constexpr int CH = SH ? 2 : 1;                 // 16-byte chunks per slot
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
+  static_assert(PK || !SH, "the shifted kernels use the packed layout");
   static_assert(2 * VEC * sizeof(double) <= 2 * S * 16, "the reduction fits in the drained ring");
   static_assert(kRunBlocks >= 1, "a dgamma run holds at least one block");
-  // [S][2][B] 16-byte slots; after an item's last row the ring is empty and
-  // its first 2 VEC * B binary64 values (at most 64 KB) serve the row-lane
-  // reduction. Without EXACT_G, [VEC][B] binary64 dgamma totals follow the
-  // ring (each thread's own, flushed from its binary32 runs).
+  // [S][2][CH][B] 16-byte slots (x, then dy); after an item's last row the
+  // ring is empty and its first 2 VEC * B binary64 values (at most 64 KB) serve
+  // the row-lane reduction. Without EXACT_G, [VEC][B] binary64 dgamma totals
+  // follow the ring (each thread's own, flushed from its binary32 runs).
   extern __shared__ uint4 ring[];
   __shared__ double red_a[B / 32];
-  prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
-  prefetch_first_rows_l2<T, VEC, B, S, PK>(dy, g.ldd, g);
+  ShIn ix = {}, id = {};
+  if constexpr (SH) {
+    ix = shifted_input(x, g);
+    id = shifted_input(dy, g);
+    prefetch_shifted_rows_l2<T, VEC, B, S>(ix, g);
+    prefetch_shifted_rows_l2<T, VEC, B, S>(id, g);
+  } else {
+    prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
+    prefetch_first_rows_l2<T, VEC, B, S, PK>(dy, g.ldd, g);
+  }
   pdl_prologue();
   const Lane ln = lane_of(g, threadIdx.x);
   const float alpha = load_param<P>(alpha_p, pt.alpha, 0);
   double *red = reinterpret_cast<double *>(ring);
-  double *gtot = reinterpret_cast<double *>(ring + 2 * S * B) + threadIdx.x;  // [e * B]
+  double *gtot = reinterpret_cast<double *>(ring + 2 * S * CH * B) + threadIdx.x;  // [e * B]
   uint4 *slot0 = ring + threadIdx.x;
+  const T *xb = SH ? reinterpret_cast<const T *>(ix.a) : x;  // position 0 of the layout
+  const T *db = SH ? reinterpret_cast<const T *>(id.a) : dy;
+  T *dxb = SH ? dx - g.sh : dx;
   double acc_a = 0.0;
   for (int item = blockIdx.x; item < g.nitems; item += gridDim.x) {
     int cc, rg;
@@ -255,16 +452,32 @@ __global__ void __launch_bounds__(B, 1)
       const uint32_t last_bytes = (uint32_t)(nl * (int)sizeof(T));
       const int nn = (int)n;  // at most kMaxRowsPerLane: the host caps a group's rows per lane
       const int64_t sx = (int64_t)g.RL * g.ldx, sd = (int64_t)g.RL * g.ldd, so = (int64_t)g.RL * g.ldo;
-      const T *px = x + first * g.ldx + c0;  // the next rows to copy (advanced, not re-derived)
-      const T *pd = dy + first * g.ldd + c0;
-      T *pdx = dx + first * g.ldo + c0;
+      const T *px = xb + first * g.ldx + c0;  // the next rows to copy (advanced, not re-derived)
+      const T *pd = db + first * g.ldd + c0;
+      T *pdx = dxb + first * g.ldo + c0;
+      // SH: rows [k_lo, k_hi) copy and store whole vectors; the others (at
+      // most a few at each end of the matrix) go element by element.
+      const int64_t pos0 = first * g.N + c0, dpos = (int64_t)g.RL * g.N;  // layout positions
+      int k_lo = 0, k_hi = nn;
+      if constexpr (SH) {
+        while (k_lo < nn && !(pos0 + k_lo * dpos >= g.sh && shifted_lo_ok(ix, px + k_lo * sx) &&
+                              shifted_lo_ok(id, pd + k_lo * sd)))
+          ++k_lo;
+        while (k_hi > k_lo && !(pos0 + (k_hi - 1) * dpos + VEC <= g.total && shifted_hi_ok(ix, px + (k_hi - 1) * sx) &&
+                                shifted_hi_ok(id, pd + (k_hi - 1) * sd)))
+          --k_hi;
+      }
       // Rows first, parameters second: the gamma loads overlap the copies.
       // Row r lives in slot r mod S; the loop below is unrolled by S so that
       // every slot index is a constant.
 #pragma unroll
       for (int k = 0; k < S - 1; ++k) {
         if (k < nn) {
-          if (PK) {
+          if constexpr (SH) {
+            const bool fast = fast_row(k, k_lo, k_hi);
+            copy_shifted<T, B, WX>(slot0 + (2 * k) * CH * B, px, ix, fast);
+            copy_shifted<T, B, WD>(slot0 + (2 * k + 1) * CH * B, pd, id, fast);
+          } else if (PK) {
             const uint32_t b = k == nn - 1 ? last_bytes : 16u;
             cp_async16_zfill(slot0 + (2 * k) * B, px, b);
             cp_async16_zfill(slot0 + (2 * k + 1) * B, pd, b);
@@ -278,7 +491,7 @@ __global__ void __launch_bounds__(B, 1)
         cp_async_commit();
       }
       int64_t col[VEC];
-      vector_columns<VEC, PK>(c0, g.Nc, col);
+      vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
       load_params<VEC, P>(gamma_p, pt.gamma, col, 4.0f, gam);  // 4 gamma (see bwd_vector)
       int run = 0;  // blocks in the current binary32 dgamma run
       for (int k0 = 0; k0 < nn; k0 += S) {
@@ -289,7 +502,11 @@ __global__ void __launch_bounds__(B, 1)
           if (k >= nn) break;
           if (k + S - 1 < nn) {  // rows k + S - 1 into slot (j + S - 1) mod S
             const int sw = (j + S - 1) % S;
-            if (PK) {
+            if constexpr (SH) {
+              const bool fast = fast_row(k + S - 1, k_lo, k_hi);
+              copy_shifted<T, B, WX>(slot0 + (2 * sw) * CH * B, px, ix, fast);
+              copy_shifted<T, B, WD>(slot0 + (2 * sw + 1) * CH * B, pd, id, fast);
+            } else if (PK) {
               const uint32_t b = k + S - 1 == nn - 1 ? last_bytes : 16u;
               cp_async16_zfill(slot0 + (2 * sw) * B, px, b);
               cp_async16_zfill(slot0 + (2 * sw + 1) * B, pd, b);
@@ -302,12 +519,22 @@ __global__ void __launch_bounds__(B, 1)
           pd += sd;
           cp_async_commit();
           cp_async_wait<S - 1>();
-          const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
-          const typename IO::Raw rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
-          if (PK && k == nn - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
-            store_first<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, nl), nl);
+          typename IO::Raw rx, rd;
+          if constexpr (SH) {
+            rx = read_shifted<B, WX>(slot0 + (2 * j) * CH * B, ix);
+            rd = read_shifted<B, WD>(slot0 + (2 * j + 1) * CH * B, id);
           } else {
-            IO::store_raw(pdx, bwd_vector<T, VEC, false, EXACT_G>(rx, rd, alpha, gam, acc, ca, VEC));
+            rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
+            rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
+          }
+          if (SH && !fast_row(k, k_lo, k_hi)) {  // padding of the shifted layout: dropped
+            const uint32_t m = shifted_mask<VEC>(g, pos0 + k * dpos);
+            store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
+          } else if (!SH && PK && k == nn - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
+            const uint32_t m = (1u << nl) - 1u;
+            store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
+          } else {
+            IO::store_raw(pdx, bwd_vector<T, VEC, false, EXACT_G>(rx, rd, alpha, gam, acc, ca, 0xFFu));
           }
           pdx += so;
         }
@@ -334,15 +561,16 @@ __global__ void __launch_bounds__(B, 1)
       if (col_ok) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          pg[c0 + e] = ag[e];
-          pb[c0 + e] = acc.b[e];
+          const int64_t at = SH ? shifted_slot(g, c0 + e) : c0 + e;
+          pg[at] = ag[e];
+          pb[at] = acc.b[e];
         }
       }
     } else {
       __syncthreads();  // every thread's ring is drained: reuse it for the reduction
       if ((32 % g.NV) == 0) {
         // the chunk's columns start at 0 on the row-tiled path (one chunk)
-        lane_reduce_warps<VEC, B>(ag, acc.b, red, g, ln, 0, pg, pb);
+        lane_reduce_warps<VEC, B, SH>(ag, acc.b, red, g, ln, 0, pg, pb);
       } else {  // dgamma and dbeta sums in one tree: 2 VEC values per thread
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
@@ -354,8 +582,9 @@ __global__ void __launch_bounds__(B, 1)
         if (col_ok && ln.rl == 0) {
 #pragma unroll
           for (int e = 0; e < VEC; ++e) {
-            pg[c0 + e] = red[e * B + threadIdx.x];
-            pb[c0 + e] = red[(VEC + e) * B + threadIdx.x];
+            const int64_t at = SH ? shifted_slot(g, c0 + e) : c0 + e;
+            pg[at] = red[e * B + threadIdx.x];
+            pb[at] = red[(VEC + e) * B + threadIdx.x];
           }
         }
         __syncthreads();

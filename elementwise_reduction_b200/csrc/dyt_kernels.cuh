@@ -61,6 +61,8 @@ struct Geom {
   uint32_t nv_magic;  // ceil(2^32 / NV) for NV >= 2: tid / NV = umulhi(tid, nv_magic), tid < 1024
   uint32_t rl_magic;  // ceil(2^32 / RL) for RL >= 2: n / RL = umulhi(n, rl_magic) for n < 2^32 / RL
   int l2_prefetch;    // the 16-byte kernels prefetch their first rows into L2 (large inputs only)
+  int sh;             // shifted kernels: the output's offset past a 16-byte boundary, in elements
+                      // (0 .. VEC - 1); its matrix starts at position sh of the packed layout
 };
 
 // The parameters' dtypes (dyt_dtype codes), read by the kernels instantiated
@@ -81,6 +83,15 @@ struct GradOut {
   int beta_dt;
   int alpha_dt;
 };
+
+// Where the shifted kernels keep the partial sums of position q of a packed
+// row. The matrix starts at position sh there, so position q holds column
+// (q - sh) mod Nc; slot q - sh (mod N) holds the same column modulo Nc, which
+// is all the finalize reads (it adds slot j into column j mod Nc).
+__device__ __forceinline__ int64_t shifted_slot(const Geom &g, int64_t q) {
+  const int64_t r = q - g.sh;
+  return r < 0 ? r + g.N : r;
+}
 
 // Rows [begin, end) of group rg when [0, M) is cut into nrg balanced groups.
 __device__ __forceinline__ void group_rows(const Geom &g, int rg, int64_t &begin, int64_t &end) {
@@ -405,8 +416,9 @@ __device__ __forceinline__ void lane_tree(double *red, const Geom &g, const Lane
 // partners form the same sum). The order of every sum is fixed. Each warp
 // then holds each of its 2 NV VEC sums once; one pass over the warps in order
 // adds them. red[] holds (B / 32) x 2 NV VEC binary64 values. Results go to
-// out_g / out_b (row of the group's partials) at the thread's columns.
-template <int VEC, int B>
+// out_g / out_b (row of the group's partials) at the thread's positions
+// (SH: at their shifted_slot).
+template <int VEC, int B, bool SH>
 __device__ __forceinline__ void lane_reduce_warps(const double (&vg)[VEC], const double (&vb)[VEC], double *red,
                                                   const Geom &g, const Lane &ln, int64_t c0_chunk,
                                                   double *out_g, double *out_b) {
@@ -458,7 +470,7 @@ __device__ __forceinline__ void lane_reduce_warps(const double (&vg)[VEC], const
     const int which = i / width, k = i - which * width;
     double sum = 0.0;
     for (int w = 0; w < B / 32; ++w) sum += red[(2 * w + which) * width + k];
-    (which ? out_b : out_g)[c0_chunk + k] = sum;
+    (which ? out_b : out_g)[SH ? shifted_slot(g, c0_chunk + k) : c0_chunk + k] = sum;
   }
   __syncthreads();
 }
@@ -490,15 +502,16 @@ struct BwdAcc {
 // dbeta's terms dy, and with EXACT_G dgamma's terms dy * t (a product of two
 // binary32 values), are exact in binary64; ca collects the dalpha terms of the
 // row in binary32 (the caller moves it into binary64 every few rows).
-// MASKED: only the first nvalid elements are real (0 for a padded row, fewer
-// than VEC for the vector that straddles the end of a packed matrix); the
-// others are computed like any other and their results dropped afterwards.
+// MASKED: only the elements whose bit is set in vmask are real (none for a
+// padded row; the vectors that straddle the start or the end of a packed
+// matrix hold some); the others are computed like any other and their
+// results dropped afterwards.
 template <typename T, int VEC, bool MASKED, bool EXACT_G>
 __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename VecIO<T, VEC>::Raw &rx,
                                                                  const typename VecIO<T, VEC>::Raw &rdy,
                                                                  float alpha, const float (&g4)[VEC],
                                                                  BwdAcc<VEC, EXACT_G> &acc, float2 &ca,
-                                                                 int nvalid) {
+                                                                 uint32_t vmask) {
   using IO = VecIO<T, VEC>;
   if constexpr (IO::kPairs > 0) {
     constexpr int H = IO::kPairs;
@@ -525,7 +538,7 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       double nb0 = acc.b[2 * h] + d0, nb1 = acc.b[2 * h + 1] + d1;
       float2 nca = fma2(gdys, x2[h], ca);
       if (MASKED) {  // drop padded elements' results, after the arithmetic
-        const bool okx = 2 * h < nvalid, oky = 2 * h + 1 < nvalid;
+        const bool okx = (vmask >> (2 * h)) & 1u, oky = (vmask >> (2 * h + 1)) & 1u;
         ng0 = okx ? ng0 : acc.g[2 * h];
         nb0 = okx ? nb0 : acc.b[2 * h];
         ng1 = oky ? ng1 : acc.g[2 * h + 1];
@@ -553,7 +566,7 @@ __device__ __forceinline__ typename VecIO<T, VEC>::Raw bwd_vector(const typename
       const double d = (double)dyf[e];
       const double ng = fma(d, (double)t, acc.g[e]), nb = acc.b[e] + d;
       const float nca = fmaf(gdys, xf[e], ca.x);
-      const bool ok = e < nvalid;
+      const bool ok = (vmask >> e) & 1u;
       acc.g[e] = (MASKED && !ok) ? acc.g[e] : ng;
       acc.b[e] = (MASKED && !ok) ? acc.b[e] : nb;
       ca.x = (MASKED && !ok) ? ca.x : nca;
@@ -650,121 +663,6 @@ __global__ void __launch_bounds__(B, 1)
     for (int w = 0; w < B / 32; ++w) s += red_a[w];
     part_da[blockIdx.x] = s;
   }
-}
-
-// ---- backward, stage 2 -------------------------------------------------------
-
-// The binary64 partial sums that one stage-1 launch left, possibly in another
-// GPU's memory (a peer mapping): rows x N dgamma and dbeta partials, nda dalpha
-// partials.
-constexpr int kMaxRanks = 8;
-struct RankParts {
-  const double *dg;
-  const double *db;
-  const double *da;
-  int rows;
-  int nda;
-};
-struct PartsSet {
-  RankParts r[kMaxRanks];
-  int nranks;
-};
-
-// Block of 256 threads = CT columns x L lanes (L = 256 / CT, chosen on the host
-// so that a lane reads at most a few partials of a rank), thread = lane * CT +
-// column. For each rank in order, lane l adds that rank's partials l, l + L,
-// ... of its column in binary64, in that order; each batch of four is loaded
-// before any is added, so a lane waits for one round trip per batch. The lanes
-// of a column are then added by a fixed-order warp butterfly (lanes CT apart
-// share a warp when CT < 32) and the warps' results by one thread per column,
-// in warp order: the rank's column total. The ranks' totals are added in rank
-// order (the first one starts the sum), and the result is rounded once to the
-// gradient's dtype. The last block also reduces dalpha the same way. With one
-// rank this is the single-GPU finalize; with several it is the cross-GPU sum of
-// a row-sharded backward, each rank's partials read through peer loads.
-constexpr int kFinThreads = 256;
-
-__device__ __forceinline__ double fin_rank_column(const RankParts &rp, int64_t N, int64_t col, int lane, int L,
-                                                  bool ok, double &b_out) {
-  double a = 0.0, b = 0.0;
-  if (ok) {
-    for (int r = lane; r < rp.rows; r += 4 * L) {
-      double va[4], vb[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int rk = r + k * L;
-        va[k] = rk < rp.rows ? rp.dg[(int64_t)rk * N + col] : 0.0;  // + 0 leaves a sum unchanged
-        vb[k] = rk < rp.rows ? rp.db[(int64_t)rk * N + col] : 0.0;
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        a += va[k];
-        b += vb[k];
-      }
-    }
-  }
-  b_out = b;
-  return a;
-}
-
-__global__ void __launch_bounds__(kFinThreads)
-    dyt_finalize_kernel(PartsSet ps, GradOut out, int64_t N, int CT) {
-  __shared__ double sg[kFinThreads], sb[kFinThreads], sa[kFinThreads / 32];
-  // Wait until the stage-1 grid has finished and its writes are visible, then
-  // let the next grid in the stream get scheduled (it waits for this one to
-  // finish before touching memory).
-  pdl_prologue();
-  const int tid = threadIdx.x;
-  const int L = kFinThreads / CT;
-  const int lane = tid / CT, c = tid - lane * CT;
-  const int64_t col = (int64_t)blockIdx.x * CT + c;
-  const bool da_block = blockIdx.x == gridDim.x - 1;
-  const int stride = CT < 32 ? 32 : CT;  // one value per warp and column (CT < 32), else one per lane
-  double tg = 0.0, tb = 0.0, ta = 0.0;   // the ranks' totals so far (threads tid < CT, and 0 for dalpha)
-  for (int r = 0; r < ps.nranks; ++r) {
-    const RankParts &rp = ps.r[r];
-    // dalpha partials: thread i adds i, i + 256, ...; the first is loaded here
-    // and added only after the column loads below are under way.
-    const double da0 = da_block && tid < rp.nda ? rp.da[tid] : 0.0;
-    double b;
-    double a = fin_rank_column(rp, N, col, lane, L, col < N, b);
-    // Lanes of a column within a warp: a butterfly (both partners of an
-    // exchange form the same sum, so every lane ends with identical bits).
-    for (int off = CT; off < 32; off <<= 1) {
-      a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
-      b += __shfl_xor_sync(0xFFFFFFFFu, b, off);
-    }
-    if (r > 0) __syncthreads();  // the previous rank's totals have been read
-    sg[tid] = a;
-    sb[tid] = b;
-    if (da_block) {
-      double da = 0.0 + da0;
-      for (int i = tid + kFinThreads; i < rp.nda; i += kFinThreads) da += rp.da[i];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) da += __shfl_xor_sync(0xFFFFFFFFu, da, off);
-      if ((tid & 31) == 0) sa[tid >> 5] = da;
-    }
-    __syncthreads();
-    if (tid < CT && col < N) {
-      double sgc = 0.0, sbc = 0.0;
-      for (int k = 0; k < kFinThreads / stride; ++k) {
-        sgc += sg[k * stride + tid];
-        sbc += sb[k * stride + tid];
-      }
-      tg = r == 0 ? sgc : tg + sgc;
-      tb = r == 0 ? sbc : tb + sbc;
-    }
-    if (da_block && tid == 0) {
-      double s = 0.0;
-      for (int w = 0; w < kFinThreads / 32; ++w) s += sa[w];
-      ta = r == 0 ? s : ta + s;
-    }
-  }
-  if (tid < CT && col < N) {
-    store_param(out.dgamma, out.gamma_dt, col, tg);
-    store_param(out.dbeta, out.beta_dt, col, tb);
-  }
-  if (da_block && tid == 0) store_param(out.dalpha, out.alpha_dt, 0, ta);
 }
 
 }  // namespace dyt

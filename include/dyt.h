@@ -25,9 +25,14 @@
  *   stride N elements) for dyt_forward / dyt_backward and with a row pitch
  *   per tensor for the *_strided entry points. gamma, beta, dgamma and dbeta
  *   hold N elements; alpha and
- *   dalpha hold one. Any alignment is accepted; 16-byte aligned tensors take
- *   the vectorised path, for any N (a ragged N is streamed in packs of
- *   16 / element-size rows, which always span whole 16-byte vectors).
+ *   dalpha hold one. Every pointer must hold whole elements of its dtype
+ *   (2- or 4-byte aligned; others give DYT_ERR_INVALID_VALUE); beyond that
+ *   any alignment is accepted. 16-byte aligned tensors take the vectorised
+ *   path, for any N (a ragged N is streamed in packs of 16 / element-size
+ *   rows, which always span whole 16-byte vectors). Contiguous tensors that
+ *   are not all 16-byte aligned take the shifted vectorised kernels: whole
+ *   16-byte vectors of the output, each input vector cut out of two aligned
+ *   16-byte chunks; no byte outside a tensor is read or written.
  * - Dtypes (the page's Summary, "Precision"): x, dy, y and dx share x_dtype,
  *   so y and dx come back in x's dtype. Each parameter gradient comes back in
  *   its parameter's dtype: dalpha in alpha's, dgamma in gamma's, dbeta in
@@ -145,9 +150,10 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
  * dyt_forward / dyt_backward are these with every pitch = N.
  * Padding between rows is neither read nor written. When every tensor is
  * 16-byte aligned and every pitch times the element size is a multiple of
- * 16 bytes, the vectorised kernels run; adjacent rows (pitch N) are needed
- * for the packed form of a ragged N, other strided matrices with a ragged N
- * take the scalar kernels. y may alias x (dx may alias x or dy) only with
+ * 16 bytes, the vectorised kernels run. Adjacent rows (pitch N) are needed
+ * for the packed form of a ragged N and for the shifted kernels (tensors not
+ * all 16-byte aligned); other strided matrices with a ragged N or off 16-byte
+ * boundaries take the one-element kernels. y may alias x (dx may alias x or dy) only with
  * equal pitches. A pitch below N, or (M - 1) * ld + N beyond the int64 limit
  * of byte offsets, gives DYT_ERR_INVALID_VALUE. dyt_backward_workspace_bytes
  * covers the strided call too.
@@ -279,9 +285,13 @@ typedef struct dyt_launch_info {
   int row_groups;    /* row groups (= partial sums per column) */
   int kernels;       /* kernels this call launched */
   int async_stages;  /* per-thread asynchronous-copy ring slots (0 = the one-element kernels) */
-  int pack_rows;     /* 1, or vec on the packed path: a 16-byte aligned matrix whose N is not a
+  int pack_rows;     /* 1, or vec on the packed path: a matrix of adjacent rows whose N is not a
                         multiple of vec is streamed as packs of vec rows (vec x N elements,
                         exactly N 16-byte vectors) */
+  int shifted;       /* 1 = the shifted 16-byte kernels (adjacent rows, tensors not all 16-byte
+                        aligned), 0 otherwise */
+  int shift;         /* shifted kernels: the output's offset past a 16-byte boundary, in
+                        elements (0 .. vec - 1); 0 otherwise */
   int64_t workspace_bytes;
 } dyt_launch_info;
 
@@ -290,16 +300,20 @@ dyt_status dyt_last_launch_info(dyt_launch_info *out);
 /*
  * The launch plan dyt_forward (backward = 0) or dyt_backward (backward != 0)
  * would use for this shape on a device with `sm_count` SMs running
- * `ctas_per_sm` CTAs of the kernel each, for contiguous tensors that are
- * 16-byte aligned (vectorized != 0; a ragged N then gets the packed form,
- * out->pack_rows > 1) or not. Host arithmetic only: touches no device, so the
- * planning is testable without a GPU. out->kernels is the number of kernels
- * the call would launch and out->workspace_bytes the workspace it needs.
+ * `ctas_per_sm` CTAs of the kernel each, for tensors laid out as `layout`
+ * says: 0 = rows that are not whole 16-byte vectors (the one-element kernels),
+ * 1 = contiguous and 16-byte aligned (a ragged N gets the packed form,
+ * out->pack_rows > 1), 2 = contiguous with the output `shift` elements past a
+ * 16-byte boundary (the shifted kernels; `shift` is read for layout 2 only).
+ * Host arithmetic only: touches no device, so the planning is testable
+ * without a GPU. out->kernels is the number of kernels the call would launch
+ * and out->workspace_bytes the workspace it needs.
  * Errors: as the shape checks of dyt_forward, or DYT_ERR_INVALID_VALUE for
- * out == NULL or sm_count / ctas_per_sm < 1.
+ * out == NULL, sm_count / ctas_per_sm < 1, a layout outside 0..2 or a shift
+ * outside 0 .. 16 / element size - 1.
  */
 dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,
-                          int backward, int vectorized, int sm_count, int ctas_per_sm,
+                          int backward, int layout, int shift, int sm_count, int ctas_per_sm,
                           dyt_launch_info *out);
 
 /*

@@ -36,7 +36,13 @@ class Workload:
     beta_std: float = 0.1
     nonzero: bool = False  # redraw x and dy values that are exactly zero
     seed: int = 0
-    offset: int = 0        # elements by which x, dy, y and dx start past a 16-byte boundary
+    offset: int = 0        # elements by which dy, y and dx (and x, unless x_offset) start past a
+                           # 16-byte boundary
+    x_offset: int | None = None  # x's own offset, when it differs
+
+    @property
+    def x_off(self) -> int:
+        return self.offset if self.x_offset is None else self.x_offset
 
     @property
     def elements(self) -> int:
@@ -77,14 +83,17 @@ WORKLOADS = {
     ]
 }
 
-# Layout variants of the workloads above: the same values with every activation
-# tensor starting one element past a 16-byte boundary, which sends them through
-# the one-element kernels.
+# Layout variants of the workloads above: the same values with tensors off
+# 16-byte boundaries, which sends them through the shifted 16-byte kernels.
+# _off1: every activation tensor one element past a boundary (each input
+# vector one aligned chunk); _xoff1: x alone, as a sliced input next to fresh
+# outputs (each x vector cut out of two aligned chunks).
 VARIANTS = {
     w.name: w
     for w in [
         replace(WORKLOADS["c2_bf16_65537x32"], name="c2_bf16_65537x32_off1", offset=1),
         replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_off1", offset=1),
+        replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_xoff1", x_offset=1),
     ]
 }
 

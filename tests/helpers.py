@@ -178,20 +178,23 @@ def _at_offset(t: torch.Tensor, M: int, N: int, offset: int) -> torch.Tensor:
 
 
 def run_cuda(inp: dict, M: int, N: int, x_dtype: str, p_dtype, fwd: bool = True, bwd: bool = True,
-             offset: int = 0):
+             offset: int = 0, x_offset: int | None = None):
     """Run the C-ABI forward and backward on the device; outputs back as numpy storage.
     p_dtype: one dtype name for alpha, gamma and beta, or a tuple (alpha, gamma, beta).
-    offset: elements by which x, dy, y and dx start past a 16-byte boundary."""
+    offset: elements by which dy, y and dx (and x, unless x_offset is given) start
+    past a 16-byte boundary."""
+    xo = offset if x_offset is None else x_offset
     import elementwise_reduction_b200 as dyt
 
     ad, gd, bd = param_dtypes(p_dtype)
     t = gpu_inputs(inp, x_dtype, p_dtype)
     x = t["x"].view(M, N) if M * N else t["x"]
-    if offset and M * N:
-        x = _at_offset(x, M, N, offset)
+    if xo and M * N:
+        x = _at_offset(x, M, N, xo)
     out, info = {}, {}
     if fwd:
-        y = _at_offset(torch.empty_like(x), M, N, offset) if offset and M * N else None
+        y = _at_offset(torch.empty((M, N), dtype=x.dtype, device=x.device), M, N, offset) if offset and M * N \
+            else None
         y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=y)
         info["fwd"] = dyt.dyt_last_launch_info()
         out["y"] = to_numpy(y, x_dtype)
@@ -199,7 +202,8 @@ def run_cuda(inp: dict, M: int, N: int, x_dtype: str, p_dtype, fwd: bool = True,
         dy = t["dy"].view(M, N) if M * N else t["dy"]
         dxo = None
         if offset and M * N:
-            dy, dxo = _at_offset(dy, M, N, offset), _at_offset(torch.empty_like(x), M, N, offset)
+            dy, dxo = _at_offset(dy, M, N, offset), _at_offset(torch.empty((M, N), dtype=x.dtype,
+                                                                           device=x.device), M, N, offset)
         dx, da, dg, db = dyt.backward(x, dy, t["alpha"], t["gamma"], t["beta"], dx=dxo)
         info["bwd"] = dyt.dyt_last_launch_info()
         out.update(dx=to_numpy(dx, x_dtype), dgamma=to_numpy(dg, gd), dbeta=to_numpy(db, bd),

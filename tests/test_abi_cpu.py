@@ -101,20 +101,43 @@ def test_host_validation_without_a_device():
     assert dyt.dyt_status_string(99) == "DYT_ERR_UNKNOWN"
 
 
+def test_pointers_must_hold_whole_elements():
+    # Every pointer is checked before anything runs, so fake device addresses
+    # suffice: a tensor off its element boundary is an argument error.
+    dyt = _lib()
+    A, W = 1 << 20, 1 << 20  # 16-byte aligned stand-ins (W: the workspace)
+    assert dyt.dyt_forward(A + 1, A, A, A, A, 4, 8, 1, 0, None) == 1                 # bf16 x one byte off
+    assert dyt.dyt_forward(A, A, A, A, A + 3, 4, 8, 1, 0, None) == 1                 # bf16 y
+    assert dyt.dyt_forward(A, A, A + 2, A, A, 4, 8, 1, 0, None) == 1                 # fp32 gamma
+    assert dyt.dyt_forward(A, A, A, A + 6, A, 4, 8, 1, 0, None) == 1                 # fp32 beta
+    assert dyt.dyt_forward_ex(A, 8, A + 1, A, A, A, 8, 4, 8, 1, 1, 0, 0, None) == 1  # bf16 alpha
+    bw = lambda x=A, dy=A, al=A, ga=A, dx=A, dg=A, db=A, da=A: dyt.dyt_backward(
+        x, dy, al, ga, None, dx, dg, db, da, 4, 8, 1, 0, W, 1 << 20, None)
+    assert bw(x=A + 1) == 1 and bw(dy=A + 1) == 1 and bw(dx=A + 1) == 1   # bf16 activations
+    assert bw(al=A + 2) == 1 and bw(ga=A + 2) == 1                        # fp32 parameters
+    assert bw(dg=A + 2) == 1 and bw(db=A + 2) == 1 and bw(da=A + 2) == 1  # fp32 gradients
+    empty = {"bytes": 0, "off_dgamma": 0, "off_dbeta": 0, "off_dalpha": 0, "rows": 0, "dalpha_parts": 0}
+    assert dyt.dyt_finalize_partials([W], [empty], 4, A + 2, A, A, 0, 0, 0, None) == 1
+    assert dyt.dyt_finalize_partials([W], [empty], 4, A, A, A + 1, 1, 1, 1, None) == 1  # bf16 dalpha
+
+
 @pytest.mark.parametrize("M,N,xd", [(1024, 64, 0), (65537, 32, 1), (100003, 17, 0), (100003, 100, 0),
                                     (100003, 255, 0), (16384, 4096, 1), (32768, 8192, 1), (1, 1, 0),
                                     (3, 70000, 2), (10**7, 8, 1), (5, 513, 0), (7, 3, 1), (1, 17, 0),
                                     (100003, 4097, 1), (4099, 1001, 0)])
-@pytest.mark.parametrize("vectorized", [0, 1])
+@pytest.mark.parametrize("layout,shift", [(0, 0), (1, 0), (2, 0), (2, 1), (2, -1)])
 @pytest.mark.parametrize("sms,occ", [(148, 1), (148, 2), (7, 1)])
-def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
+def test_launch_plan_invariants(M, N, xd, layout, shift, sms, occ):
     dyt = _lib()
-    p = dyt.dyt_plan_query(M, N, xd, 0, 1, vectorized, sms, occ)
     size = 4 if xd == 0 else 2
+    sh = shift % (16 // size) if layout == 2 else 0
+    p = dyt.dyt_plan_query(M, N, xd, 0, 1, layout, sms, occ, shift=sh)
     vec = p["vec"]
     pk = p["pack_rows"]
-    # 16-byte aligned adjacent rows always take the 16-byte kernels (packed when N is ragged)
-    assert bool(p["async_stages"]) == bool(vectorized)
+    # adjacent rows always take the 16-byte kernels (packed when N is ragged);
+    # tensors off 16-byte boundaries the shifted ones
+    assert bool(p["async_stages"]) == (layout != 0)
+    assert p["shifted"] == (layout == 2) and p["shift"] == sh
     if p["async_stages"]:    # per-thread copy ring: 16-byte vectors, one per thread
         assert vec == 16 // size
         # a ragged N is streamed in packs of vec rows (exactly N vectors each)
@@ -123,7 +146,8 @@ def test_launch_plan_invariants(M, N, xd, vectorized, sms, occ):
     else:
         assert vec == 1 and pk == 1
         ctas = sms * occ
-    Mp, Np = -(-M // pk), pk * N                   # (packed) rows and their pitch
+    Np = pk * N                                    # pitch of a (packed) row
+    Mp = -(-(M * N + sh) // Np) if layout == 2 else -(-M // pk)  # (packed) rows; shifted: the matrix from position sh
     nv = Np // vec
     B = p["block"]
     # the backward over narrow rows (at most 64 vectors) runs 256-thread CTAs with 8-slot rings

@@ -244,21 +244,100 @@ def test_empty_shapes():
 
 # ---- layout: unaligned pointers, in-place, determinism ------------------------------------------
 
-def test_unaligned_pointers_take_the_scalar_path():
+def _placed(src, M: int, N: int, offset: int, dtype, fill: float):
+    """An M x N tensor `offset` elements past a 16-byte boundary, with guard
+    elements of value `fill` on both sides (a fresh allocation starts on a
+    512-byte boundary)."""
+    buf = torch.full((M * N + offset + 24,), fill, dtype=dtype, device="cuda")
+    m = buf[offset:offset + M * N].view(M, N)
+    if src is not None:
+        m.copy_(src.reshape(M, N))
+    return buf, m
+
+
+def _run_placed(inp, M, N, xd, pd, hx, hd, ho):
+    """Forward and backward with x, dy at offsets hx, hd and y, dx at ho (elements)."""
     import elementwise_reduction_b200 as dyt
-    M, N = 300, 64
+    t = H.gpu_inputs(inp, xd, pd)
+    dt = t["x"].dtype
+    _, x = _placed(t["x"], M, N, hx, dt, float("nan"))
+    _, dy = _placed(t["dy"], M, N, hd, dt, float("nan"))
+    ybuf, y = _placed(None, M, N, ho, dt, 7.0)
+    dxbuf, dx = _placed(None, M, N, ho, dt, 7.0)
+    dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=y)
+    info_f = dyt.dyt_last_launch_info()
+    _, da, dg, db = dyt.backward(x, dy, t["alpha"], t["gamma"], t["beta"], dx=dx)
+    info_b = dyt.dyt_last_launch_info()
+    torch.cuda.synchronize()
+    for buf in (ybuf, dxbuf):  # nothing outside the outputs is written
+        assert (buf[:ho] == 7).all() and (buf[ho + M * N:] == 7).all()
+    ad, gd, bd = H.param_dtypes(pd)
+    out = {"y": H.to_numpy(y, xd), "dx": H.to_numpy(dx, xd), "dgamma": H.to_numpy(dg, gd),
+           "dbeta": H.to_numpy(db, bd), "dalpha": float(H.decode(H.to_numpy(da, ad), ad)[0])}
+    return out, info_f, info_b
+
+
+# Contiguous tensors off 16-byte boundaries take the shifted 16-byte kernels:
+# each output vector whole, each input vector cut out of two aligned chunks
+# (x and dy each at their own offset), the first and last vectors element by
+# element. NaN guards around the inputs fail any read outside them; guards
+# around the outputs any write outside them.
+@pytest.mark.parametrize("xd", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("M,N", [(1, 1), (3, 3), (7, 8), (33, 17), (129, 64), (65, 255), (9, 1001), (5, 4100),
+                                 (2049, 32)])
+@pytest.mark.parametrize("hx,hd,ho", [(1, 1, 1), (1, 0, 0), (0, 0, 1), (3, 5, 7), (7, 1, 2), (0, 7, 0), (2, 2, 6)])
+def test_unaligned_tensors_take_the_shifted_kernels(xd, M, N, hx, hd, ho):
+    vec = 4 if xd == "f32" else 8
+    hx, hd, ho = hx % vec, hd % vec, ho % vec
+    if hx == hd == ho == 0:
+        pytest.skip("aligned")
+    inp = make(M, N, xd, "f32")
+    out, info_f, info_b = _run_placed(inp, M, N, xd, "f32", hx, hd, ho)
+    # the forward sees x and y only
+    for info, shifted in ((info_f, hx or ho), (info_b, True)):
+        assert info["vec"] == vec and info["shifted"] == bool(shifted) and info["shift"] == (ho if shifted else 0)
+        assert info["pack_rows"] == (vec if N % vec else 1)
+    H.compare_all(inp, out, M, N, xd, "f32")
+    # every element's arithmetic is the aligned kernels': the same bits
+    ref, _ = H.run_cuda(inp, M, N, xd, "f32")
+    assert np.array_equal(out["y"], ref["y"]) and np.array_equal(out["dx"], ref["dx"])
+
+
+@pytest.mark.parametrize("xd,pd", [("bf16", ("bf16", "f32", "f16")), ("f16", "f16"), ("f32", "bf16")])
+def test_shifted_kernels_with_parameter_dtypes(xd, pd):
+    M, N = 1537, 100
+    inp = make(M, N, xd, pd)
+    out, info_f, info_b = _run_placed(inp, M, N, xd, pd, 3, 1, 1)
+    assert info_f["shifted"] == info_b["shifted"] == 1
+    H.compare_all(inp, out, M, N, xd, pd)
+
+
+@pytest.mark.parametrize("N", [17, 1001])
+def test_shifted_kernels_with_infinite_alpha(N):
+    # the padded elements of the first and last vectors would give
+    # tanh(inf * 0) = NaN if they entered a sum
+    M = 4099
+    inp = make(M, N, "f32", "f32", alpha=float("inf"), nonzero=True)
+    out, _, info_b = _run_placed(inp, M, N, "f32", "f32", 1, 2, 3)
+    assert info_b["shifted"] == 1
+    stats = H.compare_all(inp, out, M, N, "f32", "f32")
+    assert stats["dgamma"]["n_over_strict_elementwise"] == 0 and stats["dbeta"]["n_over_strict_elementwise"] == 0
+
+
+def test_shifted_in_place():
+    import elementwise_reduction_b200 as dyt
+    M, N = 1001, 255
     inp = make(M, N, "bf16", "f32")
+    ref, _ = H.run_cuda(inp, M, N, "bf16", "f32")
     t = H.gpu_inputs(inp, "bf16", "f32")
-    buf = torch.empty(M * N + 1, dtype=torch.bfloat16, device="cuda")
-    buf[1:] = t["x"]
-    x = buf[1:].view(M, N)  # 2-byte offset: not 16-byte aligned
-    y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"])
-    assert dyt.dyt_last_launch_info()["vec"] == 1
-    dx, da, dg, db = dyt.backward(x, t["dy"].view(M, N), t["alpha"], t["gamma"])
-    assert dyt.dyt_last_launch_info()["vec"] == 1
-    out = {"y": H.to_numpy(y, "bf16"), "dx": H.to_numpy(dx, "bf16"), "dgamma": H.to_numpy(dg, "f32"),
-           "dbeta": H.to_numpy(db, "f32"), "dalpha": float(da.item())}
-    H.compare_all(inp, out, M, N, "bf16", "f32")
+    _, x = _placed(t["x"], M, N, 3, torch.bfloat16, 0.0)
+    dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=x)  # y over x
+    assert dyt.dyt_last_launch_info()["shifted"] == 1
+    assert np.array_equal(H.to_numpy(x, "bf16"), ref["y"])
+    _, x = _placed(t["x"], M, N, 3, torch.bfloat16, 0.0)
+    _, dy = _placed(t["dy"], M, N, 5, torch.bfloat16, 0.0)
+    dyt.backward(x, dy, t["alpha"], t["gamma"], dx=dy)  # dx over dy
+    assert np.array_equal(H.to_numpy(dy, "bf16"), ref["dx"])
 
 
 # Ragged widths of aligned tensors are streamed in packs of 16 / size rows; the
@@ -285,23 +364,6 @@ def test_infinite_alpha_in_the_straddling_vector(N):
     H.compare_all(inp, out, M, N, "f32", "f32")
     assert np.isfinite(H.decode(out["dgamma"], "f32")).all()
     assert np.isfinite(H.decode(out["dbeta"], "f32")).all()
-
-
-def test_unaligned_ragged_rows_take_the_scalar_path():
-    import elementwise_reduction_b200 as dyt
-    M, N = 301, 17
-    inp = make(M, N, "f32", "f32")
-    t = H.gpu_inputs(inp, "f32", "f32")
-    buf = torch.empty(M * N + 1, dtype=torch.float32, device="cuda")
-    buf[1:] = t["x"]
-    x = buf[1:].view(M, N)  # 4-byte offset: not 16-byte aligned
-    y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"])
-    info = dyt.dyt_last_launch_info()
-    assert info["vec"] == 1 and info["pack_rows"] == 1
-    dx, da, dg, db = dyt.backward(x, t["dy"].view(M, N), t["alpha"], t["gamma"])
-    out = {"y": H.to_numpy(y, "f32"), "dx": H.to_numpy(dx, "f32"), "dgamma": H.to_numpy(dg, "f32"),
-           "dbeta": H.to_numpy(db, "f32"), "dalpha": float(da.item())}
-    H.compare_all(inp, out, M, N, "f32", "f32")
 
 
 @pytest.mark.parametrize("M,N", [(1000, 256), (1001, 255)])
@@ -633,11 +695,12 @@ def test_workload_full_size(name):
 @pytest.mark.parametrize("name", list(workloads.VARIANTS))
 def test_unaligned_variant_full_size(name):
     # The workload's values with every activation tensor one element past a
-    # 16-byte boundary: the one-element kernels, checked on every element.
+    # 16-byte boundary: the shifted kernels, checked on every element.
     w = workloads.VARIANTS[name]
     inp = workloads.make_inputs(w)
-    out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype, offset=w.offset)
-    assert info["fwd"]["vec"] == 1 and info["bwd"]["vec"] == 1
+    out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype, offset=w.offset, x_offset=w.x_offset)
+    assert info["fwd"]["shifted"] == 1 and info["bwd"]["shifted"] == 1
+    assert info["fwd"]["shift"] == info["bwd"]["shift"] == w.offset
     stats = H.compare_all(inp, out, w.M, w.N, w.x_dtype, w.p_dtype)
     print(name, info, stats)
     assert stats["dbeta"]["n_over_strict_elementwise"] == 0

@@ -22,8 +22,12 @@ thread_local dyt_launch_info t_info = {};
 thread_local int t_cuda_err = 0;
 
 
+// A CUDA runtime call failed: keep its code for dyt_last_cuda_error and clear
+// the runtime's last-error state, so that the failure, reported by our status,
+// does not surface again in the caller's next CUDA call.
 dyt_status cuda_fail(cudaError_t e) {
   t_cuda_err = (int)e;
+  (void)cudaGetLastError();
   return DYT_ERR_CUDA;
 }
 

@@ -264,7 +264,10 @@ dyt_status dyt_ipc_close(void *ptr, const dyt_ipc_handle *handle);
 /* Static, human-readable name of a status. Never NULL. */
 const char *dyt_status_string(dyt_status status);
 
-/* The cudaError_t value behind the calling thread's last DYT_ERR_CUDA (0 if none). */
+/* The cudaError_t value behind the calling thread's last DYT_ERR_CUDA (0 if
+ * none). When a call returns DYT_ERR_CUDA it has also cleared the CUDA
+ * runtime's last-error state (cudaGetLastError), so the failure is reported
+ * once, by the status; a sticky error (a fault in an earlier kernel) stays. */
 int dyt_last_cuda_error(void);
 
 /*

@@ -41,7 +41,8 @@ METRIC = "DyT fwd+bwd achieved HBM GB/s (and % of B200 peak), rows/s per shape"
 FALLBACK_HBM_GBS = 6650.0
 PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = [os.path.join(ROOT, "elementwise_reduction_b200", "csrc", f)
-                  for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_async.cuh", "dyt_api.cu")]
+                  for f in ("dyt_kernels.cuh", "dyt_math.cuh", "dyt_async.cuh", "dyt_finalize.cuh", "dyt_select.cuh",
+                            "dyt_select_impl.cuh", "dyt_api.cu")]
 
 
 def parse():

@@ -17,6 +17,8 @@
 
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "dyt_kernels.cuh"
 
 namespace dyt {
@@ -362,30 +364,50 @@ __global__ void __launch_bounds__(B, 1)
     float gam[VEC], bet[VEC], bth[VEC];
     fwd_params_at<T, VEC, P>(gamma_p, beta_p, pt, col, gam, bet, bth);
     int s_rd = 0, s_wr = S - 1;
-    for (int64_t k = 0; k < n; ++k) {
-      const int64_t kn = k + S - 1;
-      if (kn < n) {
-        if constexpr (SH) copy_shifted<T, B, WX>(slot0 + s_wr * CH * B, px + kn * sx, ix, fast_row((int)kn, k_lo, k_hi));
-        else if (PK) cp_async16_zfill(slot0 + s_wr * B, px + kn * sx, kn == n - 1 ? last_bytes : 16u);
-        else cp_async16(slot0 + s_wr * B, px + kn * sx);
-      }
-      cp_async_commit();
-      cp_async_wait<S - 1>();
-      typename IO::Raw rx;
-      if constexpr (SH) rx = read_shifted<B, WX>(slot0 + s_rd * CH * B, ix);
-      else rx = *(const typename IO::Raw *)(slot0 + s_rd * B);
-      const typename IO::Raw ry = fwd_vector<T, VEC>(rx, alpha, gam, bet, bth);
-      if constexpr (SH) {
-        if (fast_row((int)k, k_lo, k_hi)) IO::store_raw(py, ry);
+    if constexpr (SH) {
+      // One ring step: copy row k + S - 1, then compute and store row k. CHK:
+      // the step tests whether its rows are whole-vector rows; iterations
+      // [k_lo, k_hi - S + 1) need no test (both rows lie in [k_lo, k_hi)).
+      int64_t k = 0;
+      auto step = [&](auto chk) {
+        constexpr bool CHK = decltype(chk)::value;
+        const int64_t kn = k + S - 1;
+        if (!CHK || kn < n)
+          copy_shifted<T, B, WX>(slot0 + s_wr * CH * B, px + kn * sx, ix, !CHK || fast_row((int)kn, k_lo, k_hi));
+        cp_async_commit();
+        cp_async_wait<S - 1>();
+        const typename IO::Raw ry =
+            fwd_vector<T, VEC>(read_shifted<B, WX>(slot0 + s_rd * CH * B, ix), alpha, gam, bet, bth);
+        if (!CHK || fast_row((int)k, k_lo, k_hi)) IO::store_raw(py, ry);
         else store_mask<T, VEC>(py, ry, shifted_mask<VEC>(g, pos0 + k * dpos));  // padding: not stored
-      } else if (PK && k == n - 1 && nl < VEC) {
-        store_mask<T, VEC>(py, ry, (1u << nl) - 1u);  // zero-filled tail: not stored
-      } else {
-        IO::store_raw(py, ry);
+        py += sy;
+        s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
+        s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
+        ++k;
+      };
+      const int64_t f1 = max((int64_t)k_lo, (int64_t)k_hi - (S - 1));
+      if (f1 - k_lo >= 2 * S) {  // enough unchecked steps to pay for the phases
+        while (k < k_lo) step(std::true_type{});
+        while (k < f1) step(std::false_type{});
       }
-      py += sy;
-      s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
-      s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
+      while (k < n) step(std::true_type{});
+    } else {
+      for (int64_t k = 0; k < n; ++k) {
+        const int64_t kn = k + S - 1;
+        if (kn < n) {
+          if (PK) cp_async16_zfill(slot0 + s_wr * B, px + kn * sx, kn == n - 1 ? last_bytes : 16u);
+          else cp_async16(slot0 + s_wr * B, px + kn * sx);
+        }
+        cp_async_commit();
+        cp_async_wait<S - 1>();
+        const typename IO::Raw rx = *(const typename IO::Raw *)(slot0 + s_rd * B);
+        const typename IO::Raw ry = fwd_vector<T, VEC>(rx, alpha, gam, bet, bth);
+        if (PK && k == n - 1 && nl < VEC) store_mask<T, VEC>(py, ry, (1u << nl) - 1u);  // zero-filled tail: not stored
+        else IO::store_raw(py, ry);
+        py += sy;
+        s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
+        s_wr = s_wr + 1 == S ? 0 : s_wr + 1;
+      }
     }
     cp_async_wait<0>();
   }
@@ -502,47 +524,60 @@ __global__ void __launch_bounds__(B, 1)
       int run = 0;  // blocks in the current binary32 dgamma run
       for (int k0 = 0; k0 < nn; k0 += S) {
         float2 ca = make_float2(0.0f, 0.0f);  // this block's dalpha terms (at most S VEC / 2 per lane)
+        // Rows k0 .. k0 + S - 1. CHK: the rows and their copies are tested
+        // (ends of the matrix, the shifted kernels' partial vectors); the
+        // shifted kernels skip the tests on blocks whose rows and copies all
+        // lie in [k_lo, k_hi).
+        auto block = [&](auto chk) {
+          constexpr bool CHK = decltype(chk)::value;
 #pragma unroll
-        for (int j = 0; j < S; ++j) {
-          const int k = k0 + j;
-          if (k >= nn) break;
-          if (k + S - 1 < nn) {  // rows k + S - 1 into slot (j + S - 1) mod S
-            const int sw = (j + S - 1) % S;
-            if constexpr (SH) {
-              const bool fast = fast_row(k + S - 1, k_lo, k_hi);
-              copy_shifted<T, B, WX>(slot0 + (2 * sw) * CH * B, px, ix, fast);
-              copy_shifted<T, B, WD>(slot0 + (2 * sw + 1) * CH * B, pd, id, fast);
-            } else if (PK) {
-              const uint32_t b = k + S - 1 == nn - 1 ? last_bytes : 16u;
-              cp_async16_zfill(slot0 + (2 * sw) * B, px, b);
-              cp_async16_zfill(slot0 + (2 * sw + 1) * B, pd, b);
-            } else {
-              cp_async16(slot0 + (2 * sw) * B, px);
-              cp_async16(slot0 + (2 * sw + 1) * B, pd);
+          for (int j = 0; j < S; ++j) {
+            const int k = k0 + j;
+            if (CHK && k >= nn) break;
+            if (!CHK || k + S - 1 < nn) {  // rows k + S - 1 into slot (j + S - 1) mod S
+              const int sw = (j + S - 1) % S;
+              if constexpr (SH) {
+                const bool fast = !CHK || fast_row(k + S - 1, k_lo, k_hi);
+                copy_shifted<T, B, WX>(slot0 + (2 * sw) * CH * B, px, ix, fast);
+                copy_shifted<T, B, WD>(slot0 + (2 * sw + 1) * CH * B, pd, id, fast);
+              } else if (PK) {
+                const uint32_t b = k + S - 1 == nn - 1 ? last_bytes : 16u;
+                cp_async16_zfill(slot0 + (2 * sw) * B, px, b);
+                cp_async16_zfill(slot0 + (2 * sw + 1) * B, pd, b);
+              } else {
+                cp_async16(slot0 + (2 * sw) * B, px);
+                cp_async16(slot0 + (2 * sw + 1) * B, pd);
+              }
             }
+            px += sx;
+            pd += sd;
+            cp_async_commit();
+            cp_async_wait<S - 1>();
+            typename IO::Raw rx, rd;
+            if constexpr (SH) {
+              rx = read_shifted<B, WX>(slot0 + (2 * j) * CH * B, ix);
+              rd = read_shifted<B, WD>(slot0 + (2 * j + 1) * CH * B, id);
+            } else {
+              rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
+              rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
+            }
+            if (SH && CHK && !fast_row(k, k_lo, k_hi)) {  // padding of the shifted layout: dropped
+              const uint32_t m = shifted_mask<VEC>(g, pos0 + k * dpos);
+              store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
+            } else if (!SH && PK && k == nn - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
+              const uint32_t m = (1u << nl) - 1u;
+              store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
+            } else {
+              IO::store_raw(pdx, bwd_vector<T, VEC, false, EXACT_G>(rx, rd, alpha, gam, acc, ca, 0xFFu));
+            }
+            pdx += so;
           }
-          px += sx;
-          pd += sd;
-          cp_async_commit();
-          cp_async_wait<S - 1>();
-          typename IO::Raw rx, rd;
-          if constexpr (SH) {
-            rx = read_shifted<B, WX>(slot0 + (2 * j) * CH * B, ix);
-            rd = read_shifted<B, WD>(slot0 + (2 * j + 1) * CH * B, id);
-          } else {
-            rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
-            rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
-          }
-          if (SH && !fast_row(k, k_lo, k_hi)) {  // padding of the shifted layout: dropped
-            const uint32_t m = shifted_mask<VEC>(g, pos0 + k * dpos);
-            store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
-          } else if (!SH && PK && k == nn - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
-            const uint32_t m = (1u << nl) - 1u;
-            store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
-          } else {
-            IO::store_raw(pdx, bwd_vector<T, VEC, false, EXACT_G>(rx, rd, alpha, gam, acc, ca, 0xFFu));
-          }
-          pdx += so;
+        };
+        if constexpr (SH && B >= 512) {  // narrow rows (256-thread CTAs) give each thread few rows
+          if (k0 >= k_lo && k0 + 2 * S - 2 < k_hi) block(std::false_type{});
+          else block(std::true_type{});
+        } else {
+          block(std::true_type{});
         }
         acc_a += (double)ca.x;
         acc_a += (double)ca.y;

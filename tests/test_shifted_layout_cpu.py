@@ -1,0 +1,152 @@
+"""The shifted kernels' addressing, replayed on the host for the library's own plans.
+
+Contiguous tensors off 16-byte boundaries run the 16-byte kernels in the
+shifted layout: the packed layout laid over the output from position sh (the
+output's offset in elements), each input read as one or two aligned 16-byte
+chunks per output vector. This test replays, per thread of the plan that
+dyt_plan_query returns, the rows it visits, the chunks it copies (plain copies
+on its whole-vector rows, checked copies elsewhere), the output elements it
+stores, the columns it assigns and the partial-sum slots it writes, with the
+same arithmetic as the kernels (dyt_async.cuh, shifted kernels), and checks:
+- every byte read lies inside its tensor;
+- every output element is stored exactly once, at its own address;
+- every stored element's input bytes were copied in the same row step;
+- element e of the matrix gets column e mod N;
+- its partial-sum slot is congruent to that column mod N (what the finalize
+  relies on).
+Host arithmetic only: no device is touched.
+"""
+import pytest
+
+from tests.test_abi_cpu import _lib
+
+
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+def replay(dyt, M, N, xd, hx, hd, ho, backward, sms=3):
+    es = 4 if xd == 0 else 2
+    vec = 16 // es
+    p = dyt.dyt_plan_query(M, N, xd, 0, int(backward), 2, sms, 1, shift=ho)
+    assert p["shifted"] == 1 and p["shift"] == ho
+    B, RL, ncc, nrg, grid, pk = (p[k] for k in ("block", "row_lanes", "col_chunks", "row_groups", "grid", "pack_rows"))
+    Np = pk * N                       # pitch of a row of the layout
+    NV = Np // vec                    # 16-byte vectors per row of the layout
+    sh, total = ho, M * N + ho        # the matrix occupies positions [sh, total) of the layout
+    Mp = _cdiv(total, Np)
+    gq, grem = Mp // nrg, Mp % nrg
+    bases = {"x": 1 << 20, "dy": 2 << 20, "o": 3 << 20}  # 16-byte aligned regions, one per tensor
+    lo = {"x": bases["x"] + hx * es, "dy": bases["dy"] + hd * es, "o": bases["o"] + ho * es}
+    hi = {k: v + M * N * es for k, v in lo.items()}
+    ins = ["x", "dy"] if backward else ["x"]
+    frame = {}
+    for k in ins:  # where position 0 of the layout falls in each input: aligned chunk base, byte offset d
+        f = lo[k] - sh * es
+        frame[k] = (f - (f & 15), f & 15)
+    out_base = lo["o"] - sh * es
+    assert out_base % 16 == 0
+    stored = set()
+    for blk in range(grid):
+        for tid in range(B):
+            rl, cvl, live = (tid // NV, tid % NV, tid // NV < RL) if RL > 1 else (0, tid, True)
+            for item in range(blk, nrg * ncc, grid):
+                cc, rg = (0, item) if ncc == 1 else (item % ncc, item // ncc)
+                rb = rg * gq + min(rg, grem)
+                re = rb + gq + (1 if rg < grem else 0)
+                cv = cc * B + cvl
+                if not (live and cv < NV):
+                    continue
+                c0 = cv * vec
+                first = rb + rl
+                n = 0 if first >= re else _cdiv(re - first, RL)
+                assert n <= 2048
+                if n > 0 and total - ((first + (n - 1) * RL) * Np + c0) <= 0:
+                    n -= 1  # a last vector wholly past the matrix is not visited
+                c = c0 - sh
+                while c < 0:
+                    c += N
+                cols = [(c + e) % N for e in range(vec)]
+                pos0, dpos, step = first * Np + c0, RL * Np, RL * Np * es
+
+                def chunk(k, name):
+                    return frame[name][0] + (first * Np + c0) * es + k * step
+
+                def lo_ok(k):
+                    return pos0 + k * dpos >= sh and all(chunk(k, m) >= lo[m] for m in ins)
+
+                def hi_ok(k):
+                    return pos0 + k * dpos + vec <= total and all(
+                        chunk(k, m) + (32 if frame[m][1] else 16) <= hi[m] for m in ins)
+
+                k_lo = 0
+                while k_lo < n and not lo_ok(k_lo):
+                    k_lo += 1
+                k_hi = n
+                while k_hi > k_lo and not hi_ok(k_hi - 1):
+                    k_hi -= 1
+                for k in range(n):
+                    fast = k_lo <= k < k_hi
+                    got = {}
+                    for m in ins:
+                        a, d = chunk(k, m), frame[m][1]
+                        bytes_ = set()
+                        for ca in ([a, a + 16] if d else [a]):
+                            if fast:  # plain 16-byte copy
+                                bytes_.update(range(ca, ca + 16))
+                            elif ca >= hi[m] or ca + 16 <= lo[m]:
+                                continue  # holds none of the tensor: not copied
+                            elif ca >= lo[m]:  # the tensor ends here: its leading bytes, zero-filled slot
+                                bytes_.update(range(ca, ca + min(16, hi[m] - ca)))
+                            else:  # the tensor starts here: element by element from its first byte
+                                assert (lo[m] - ca) % es == 0
+                                bytes_.update(range(lo[m], min(hi[m], ca + 16)))
+                        assert all(lo[m] <= b < hi[m] for b in bytes_), ("read outside", m)
+                        got[m] = (a + d, bytes_)
+                    pos = pos0 + k * dpos
+                    for e in range(vec):
+                        real = sh <= pos + e < total
+                        if fast:
+                            assert real
+                        if not real:
+                            continue  # masked: neither stored nor summed
+                        f = pos + e - sh  # flat index in the matrix
+                        assert out_base + (pos + e) * es == lo["o"] + f * es
+                        assert f not in stored, "stored twice"
+                        stored.add(f)
+                        assert cols[e] == f % N
+                        for m in ins:
+                            start, bytes_ = got[m]
+                            for b in range(start + e * es, start + (e + 1) * es):
+                                assert b in bytes_, "an input byte was not copied"
+                                assert (b - lo[m]) // es == f
+                        q = c0 + e  # partial-sum slot of this position
+                        slot = q - sh if q >= sh else q - sh + Np
+                        assert slot % N == cols[e]
+    assert len(stored) == M * N
+
+
+CASES = [(M, N) for N in (1, 3, 8, 17, 32, 100, 255) for M in (1, 3, 9)] + [(33, 17), (5, 520), (3, 1031)]
+
+
+@pytest.mark.parametrize("xd", [0, 1])
+@pytest.mark.parametrize("M,N", CASES)
+def test_shifted_addressing_stays_inside_every_tensor(xd, M, N):
+    dyt = _lib()
+    vec = 4 if xd == 0 else 8
+    for backward in (False, True):
+        for ho in range(vec):
+            for hx in sorted({0, 1, vec - 1, ho}):
+                for hd in (sorted({0, ho, vec - 1}) if backward else [0]):
+                    replay(dyt, M, N, xd, hx, hd, ho, backward)
+
+
+@pytest.mark.parametrize("M,N,xd", [(3, 4104, 1), (2, 4099, 1), (4, 2051, 0)])
+def test_shifted_addressing_with_column_chunks(M, N, xd):
+    # rows wider than a CTA's vectors: several column chunks per row
+    dyt = _lib()
+    vec = 4 if xd == 0 else 8
+    for ho in (0, 1, vec - 1):
+        for hx in (0, 1):
+            for backward in (False, True):
+                replay(dyt, M, N, xd, hx, hx, ho, backward, sms=5)

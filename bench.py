@@ -366,19 +366,18 @@ def _to_torch(a, dtype, device):
 
 def _matrix(src, w, dev, off):
     """An M x N device matrix holding src, starting `off` elements past a 16-byte
-    boundary (0 for the workloads themselves)."""
-    import torch
+    boundary (0 for the workloads themselves), rows w.pitch elements apart."""
     t = _to_torch(src, w.x_dtype, "cpu")
-    buf = torch.empty(w.M * w.N + off + 8, dtype=t.dtype, device=dev)
-    m = buf[off:off + w.M * w.N].view(w.M, w.N)
+    m = _empty_like_matrix(t, w, off, dev)
     m.copy_(t.view(w.M, w.N))
     return m
 
 
-def _empty_like_matrix(m, w, off):
+def _empty_like_matrix(m, w, off, dev=None):
     import torch
-    buf = torch.empty(w.M * w.N + off + 8, dtype=m.dtype, device=m.device)
-    return buf[off:off + w.M * w.N].view(w.M, w.N)
+    ld = w.pitch or w.N
+    buf = torch.empty(w.M * ld + off + 8, dtype=m.dtype, device=dev or m.device)
+    return buf[off:off + w.M * ld].view(w.M, ld)[:, :w.N]
 
 
 def _sets(w, inp, dev, L2):

@@ -39,6 +39,7 @@ class Workload:
     offset: int = 0        # elements by which dy, y and dx (and x, unless x_offset) start past a
                            # 16-byte boundary
     x_offset: int | None = None  # x's own offset, when it differs
+    pitch: int | None = None     # row pitch (elements) of x, dy, y and dx, when not N
 
     @property
     def x_off(self) -> int:
@@ -87,13 +88,16 @@ WORKLOADS = {
 # 16-byte boundaries, which sends them through the shifted 16-byte kernels.
 # _off1: every activation tensor one element past a boundary (each input
 # vector one aligned chunk); _xoff1: x alone, as a sliced input next to fresh
-# outputs (each x vector cut out of two aligned chunks).
+# outputs (each x vector cut out of two aligned chunks). _pitch4100: rows of
+# 4096 elements 4100 apart (8200 bytes, not whole 16-byte vectors), which the
+# one-element kernels take.
 VARIANTS = {
     w.name: w
     for w in [
         replace(WORKLOADS["c2_bf16_65537x32"], name="c2_bf16_65537x32_off1", offset=1),
         replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_off1", offset=1),
         replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_xoff1", x_offset=1),
+        replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_pitch4100", pitch=4100),
     ]
 }
 

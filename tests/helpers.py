@@ -169,31 +169,34 @@ def gpu_inputs(inp: dict, x_dtype: str, p_dtype) -> dict:
     return d
 
 
-def _at_offset(t: torch.Tensor, M: int, N: int, offset: int) -> torch.Tensor:
-    """An M x N copy of t whose first element lies `offset` elements past a 16-byte boundary."""
-    buf = torch.empty(M * N + offset + 8, dtype=t.dtype, device=t.device)
-    m = buf[offset:offset + M * N].view(M, N)
-    m.copy_(t.view(M, N))
+def _at_offset(t: torch.Tensor, M: int, N: int, offset: int, pitch: int | None = None) -> torch.Tensor:
+    """An M x N copy of t whose first element lies `offset` elements past a 16-byte
+    boundary, rows `pitch` elements apart (default N)."""
+    ld = pitch or N
+    buf = torch.empty(M * ld + offset + 8, dtype=t.dtype, device=t.device)
+    m = buf[offset:offset + M * ld].view(M, ld)[:, :N]
+    m.copy_(t.reshape(M, N))
     return m
 
 
 def run_cuda(inp: dict, M: int, N: int, x_dtype: str, p_dtype, fwd: bool = True, bwd: bool = True,
-             offset: int = 0, x_offset: int | None = None):
+             offset: int = 0, x_offset: int | None = None, pitch: int | None = None):
     """Run the C-ABI forward and backward on the device; outputs back as numpy storage.
     p_dtype: one dtype name for alpha, gamma and beta, or a tuple (alpha, gamma, beta).
     offset: elements by which dy, y and dx (and x, unless x_offset is given) start
-    past a 16-byte boundary."""
+    past a 16-byte boundary; pitch: their row pitch in elements (default N)."""
     xo = offset if x_offset is None else x_offset
+    placed = bool(offset or xo or pitch) and M * N > 0
     import elementwise_reduction_b200 as dyt
 
     ad, gd, bd = param_dtypes(p_dtype)
     t = gpu_inputs(inp, x_dtype, p_dtype)
     x = t["x"].view(M, N) if M * N else t["x"]
-    if xo and M * N:
-        x = _at_offset(x, M, N, xo)
+    if placed:
+        x = _at_offset(x, M, N, xo, pitch)
     out, info = {}, {}
     if fwd:
-        y = _at_offset(torch.empty((M, N), dtype=x.dtype, device=x.device), M, N, offset) if offset and M * N \
+        y = _at_offset(torch.empty((M, N), dtype=x.dtype, device=x.device), M, N, offset, pitch) if placed \
             else None
         y = dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=y)
         info["fwd"] = dyt.dyt_last_launch_info()
@@ -201,9 +204,10 @@ def run_cuda(inp: dict, M: int, N: int, x_dtype: str, p_dtype, fwd: bool = True,
     if bwd:
         dy = t["dy"].view(M, N) if M * N else t["dy"]
         dxo = None
-        if offset and M * N:
-            dy, dxo = _at_offset(dy, M, N, offset), _at_offset(torch.empty((M, N), dtype=x.dtype,
-                                                                           device=x.device), M, N, offset)
+        if placed:
+            dy, dxo = _at_offset(dy, M, N, offset, pitch), _at_offset(torch.empty((M, N), dtype=x.dtype,
+                                                                                  device=x.device), M, N, offset,
+                                                                      pitch)
         dx, da, dg, db = dyt.backward(x, dy, t["alpha"], t["gamma"], t["beta"], dx=dxo)
         info["bwd"] = dyt.dyt_last_launch_info()
         out.update(dx=to_numpy(dx, x_dtype), dgamma=to_numpy(dg, gd), dbeta=to_numpy(db, bd),

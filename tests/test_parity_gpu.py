@@ -694,13 +694,18 @@ def test_workload_full_size(name):
 
 @pytest.mark.parametrize("name", list(workloads.VARIANTS))
 def test_unaligned_variant_full_size(name):
-    # The workload's values with every activation tensor one element past a
-    # 16-byte boundary: the shifted kernels, checked on every element.
+    # The workload's values with tensors off 16-byte boundaries (the shifted
+    # kernels) or rows that are not whole 16-byte vectors (the one-element
+    # kernels), checked on every element.
     w = workloads.VARIANTS[name]
     inp = workloads.make_inputs(w)
-    out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype, offset=w.offset, x_offset=w.x_offset)
-    assert info["fwd"]["shifted"] == 1 and info["bwd"]["shifted"] == 1
-    assert info["fwd"]["shift"] == info["bwd"]["shift"] == w.offset
+    out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype, offset=w.offset, x_offset=w.x_offset,
+                           pitch=w.pitch)
+    if w.pitch:
+        assert info["fwd"]["vec"] == info["bwd"]["vec"] == 1
+    else:
+        assert info["fwd"]["shifted"] == 1 and info["bwd"]["shifted"] == 1
+        assert info["fwd"]["shift"] == info["bwd"]["shift"] == w.offset
     stats = H.compare_all(inp, out, w.M, w.N, w.x_dtype, w.p_dtype)
     print(name, info, stats)
     assert stats["dbeta"]["n_over_strict_elementwise"] == 0

@@ -1,5 +1,6 @@
 // Per-thread asynchronous-copy DyT kernels for sm_100a (16-byte vectors): the
-// kernels every 16-byte aligned matrix takes.
+// kernels every 16-byte aligned matrix takes, and (shifted kernels, below)
+// every contiguous matrix off 16-byte boundaries.
 //
 // Same decomposition, thread mapping and arithmetic as the one-element
 // kernels in dyt_kernels.cuh; the row lanes of a CTA are added by a register
@@ -10,9 +11,10 @@
 // only), S - 1 rows ahead of the row it computes, and reads each slot back
 // after cp.async.wait_group. A thread only ever reads slots it filled itself,
 // so no barrier is needed between threads; the data in flight (up to
-// (S - 1) x 32 bytes per thread) costs no registers. Each thread visits
-// exactly its real rows; only the one vector that straddles the end of a
-// packed matrix holds padding, which is masked after the arithmetic.
+// (S - 1) x 32 bytes per thread, twice that in the shifted kernels) costs no
+// registers. Each thread visits exactly its real rows; only the vectors that
+// straddle the start or the end of a packed matrix hold padding, which is
+// masked after the arithmetic.
 #pragma once
 
 #include <cuda_runtime.h>

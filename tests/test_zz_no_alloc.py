@@ -31,14 +31,23 @@ def _tensor(a: np.ndarray, dtype: str) -> torch.Tensor:
     return t.cuda()
 
 
-def _backward(inp, M, N, xd, pd, noalloc: bool):
-    """One backward through the C ABI; returns (dx, dgamma, dbeta, dalpha) as float64 arrays."""
+def _at(t: torch.Tensor, offset: int) -> torch.Tensor:
+    """A copy of the flat tensor t starting `offset` elements past a 16-byte boundary."""
+    buf = torch.empty(t.numel() + offset + 8, dtype=t.dtype, device=t.device)
+    out = buf[offset:offset + t.numel()]
+    out.copy_(t)
+    return out
+
+
+def _backward(inp, M, N, xd, pd, noalloc: bool, offset: int = 0):
+    """One backward through the C ABI; returns the raw bytes of (dx, dgamma, dbeta, dalpha).
+    offset: elements by which x, dy and dx start past a 16-byte boundary."""
     import elementwise_reduction_b200 as dyt
     from elementwise_reduction_b200 import _abi
 
-    x, dy = _tensor(inp["x"], xd), _tensor(inp["dy"], xd)
+    x, dy = _at(_tensor(inp["x"], xd), offset), _at(_tensor(inp["dy"], xd), offset)
     alpha, gamma = _tensor(inp["alpha"], pd), _tensor(inp["gamma"], pd)
-    dx = torch.full_like(x, float("nan"))
+    dx = _at(torch.full_like(x, float("nan")), offset)
     dg, db = torch.full_like(gamma, float("nan")), torch.full_like(gamma, float("nan"))
     da = torch.full((1,), float("nan"), dtype=gamma.dtype, device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
@@ -47,7 +56,7 @@ def _backward(inp, M, N, xd, pd, noalloc: bool):
                                        dx.data_ptr(), dg.data_ptr(), db.data_ptr(), da.data_ptr(), M, N,
                                        CODE[xd], CODE[pd], stream)
     else:
-        ws = dyt.workspace(x.view(M, N), gamma)
+        ws = dyt.workspace(x.view(M, N), gamma)  # sized for any layout of this shape
         st = _abi.dyt_backward(x.data_ptr(), dy.data_ptr(), alpha.data_ptr(), gamma.data_ptr(), None,
                                dx.data_ptr(), dg.data_ptr(), db.data_ptr(), da.data_ptr(), M, N, CODE[xd],
                                CODE[pd], ws.data_ptr(), ws.numel(), stream)
@@ -68,6 +77,20 @@ def test_noalloc_backward_matches_workspace_backward_call_after_call():
         got = _backward(inp, M, N, xd, pd, noalloc=True)
         for name, g, r in zip(("dx", "dgamma", "dbeta", "dalpha"), got, want):
             assert np.array_equal(g, r), f"{name} differs from the workspace call ({M}x{N} {xd})"
+
+
+def test_noalloc_backward_with_misaligned_tensors():
+    # one element past a 16-byte boundary: the shifted kernels, same bits as
+    # the workspace call on the same tensors
+    from elementwise_reduction_b200 import _abi
+    for M, N, xd in ((65537, 32, "bf16"), (3001, 255, "f32"), (2049, 4096, "bf16")):
+        w = workloads.Workload("noalloc_off1", M, N, xd, "f32", alpha=0.7)
+        inp = workloads.make_inputs(w)
+        want = _backward(inp, M, N, xd, "f32", noalloc=False, offset=1)
+        assert _abi.dyt_last_launch_info()["shifted"] == 1
+        got = _backward(inp, M, N, xd, "f32", noalloc=True, offset=1)
+        for name, g, r in zip(("dx", "dgamma", "dbeta", "dalpha"), got, want):
+            assert np.array_equal(g, r), f"{name} differs from the workspace call ({M}x{N} {xd}, offset 1)"
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():

@@ -11,11 +11,15 @@ CPU time next to it.
 
 Multi-GPU (torchrun, one process per GPU): each rank runs the whole workload
 on its own batch of rows (weak scaling); the parameter gradients are summed
-across ranks with one NCCL all-reduce of 2N+1 values per step, the exchange
-that row sharding of the column sums requires.
+across ranks inside the finalize, which reads every rank's binary64 partials
+through peer pointers after a one-element NCCL all-reduce (or, where the
+workspaces cannot be mapped, by one NCCL all-reduce of the 2N+1 rounded
+gradients): the exchange that row sharding of the column sums requires.
 
-Device timing: CUDA events around a CUDA graph of K steps on the launching
-stream, barrier + synchronize on both sides, max over ranks. The steps cycle
+Device timing: CUDA events around K steps on the launching stream (one GPU: a
+CUDA graph of them; several: launched directly, so that no NCCL collective is
+captured into a graph), barrier + synchronize on both sides, max over ranks.
+The steps cycle
 through enough buffer sets that the data touched between two uses of a set
 is more than twice the L2 size, so no step reads another's data from L2.
 """
@@ -409,6 +413,19 @@ def _graph(stream, fn, n):
     return g
 
 
+class _Eager:
+    """The n calls fn(0) .. fn(n - 1) launched directly on the current stream at
+    each replay(): the multi-rank steps, whose NCCL collectives (the exchange's
+    barrier, or the all-reduce of the gradients) are not captured into graphs."""
+
+    def __init__(self, fn, n):
+        self.fn, self.n = fn, n
+
+    def replay(self):
+        for i in range(self.n):
+            self.fn(i)
+
+
 def _time_replays(g, stream, dev, K, clock_index, clocks=True, idle_s=0.4, min_seconds=0.6, min_replays=7,
                   max_replays=2000):
     """Per-call device time (us) of a K-call graph over repeated replays (CUDA events
@@ -523,14 +540,21 @@ def run_ours(args, w):
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             step(i)
+        # the launch records of one forward and one backward (the backward with
+        # the next buffer of the exchange's schedule, as a further warm-up step)
+        fwd(sets[0])
+        launch_info_fwd = dyt.dyt_last_launch_info()
+        bwd(sets[0], i=args.warmup)
+        launch_info_bwd = dyt.dyt_last_launch_info()
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()  # every rank's eager calls are done before any replay reuses a workspace
-        g_step = _graph(stream, step, args.steps)
-        g_fwd = _graph(stream, lambda i: fwd(sets[i % nsets]), args.steps)
-        launch_info_fwd = dyt.dyt_last_launch_info()
-        g_bwd = _graph(stream, lambda i: bwd(sets[i % nsets], i=i), args.steps)
-        launch_info_bwd = dyt.dyt_last_launch_info()
+        # One rank: CUDA graphs of K calls. Several: the same calls launched
+        # eagerly (no NCCL collective inside a graph).
+        steps_of = (lambda fn: _graph(stream, fn, args.steps)) if world == 1 else (lambda fn: _Eager(fn, args.steps))
+        g_step = steps_of(step)
+        g_fwd = steps_of(lambda i: fwd(sets[i % nsets]))
+        g_bwd = steps_of(lambda i: bwd(sets[i % nsets], i=i))
         for g in (g_step, g_fwd, g_bwd):  # untimed replay: first-launch costs
             g.replay()
         torch.cuda.synchronize(dev)
@@ -564,7 +588,7 @@ def run_ours(args, w):
         # run of this layer alone gets once the GPU sits at its power limit.
         sustained = _time_replays(g_step, stream, dev, args.steps, local, clocks=not args.no_clocks, idle_s=0.0,
                                   min_seconds=1.0) if world == 1 and not args.no_sustained else None
-        del g_step, g_fwd, g_bwd  # graphs that may hold NCCL calls go before the process group
+        del g_step, g_fwd, g_bwd
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()

@@ -495,32 +495,29 @@ def run_ours(args, w):
     grads = torch.empty(2 * N + 1, dtype=torch.float32, device=dev)
     from elementwise_reduction_b200.dist import FusedGradientSum, allreduce_param_grads
 
-    def make_exchange():
+    def make_exchange(x, dy, dx):
         """The fused cross-rank gradient sum, or None (every rank then falls back to the
         all-reduce of the rounded gradients): the ranks decide together."""
         if world == 1:
             return None, None
-        ex, why = None, None
-        try:
-            ex = FusedGradientSum(sets[0]["x"], sets[0]["dy"], sets[0]["dx"], gamma)
-        except Exception as e:  # e.g. memory that CUDA IPC cannot share
-            why = f"{type(e).__name__}: {e}"
-        ok = torch.tensor([0 if ex is None else 1], dtype=torch.int32, device=dev)
+        ex = FusedGradientSum(x, dy, dx, gamma)  # records a local failure in ex.error
+        ok = torch.tensor([1 if ex.error is None else 0], dtype=torch.int32, device=dev)
         dist.all_reduce(ok, op=dist.ReduceOp.MIN)
         if int(ok.item()) == 0:
-            if ex is not None:
-                ex.close()
-            return None, why or "another rank could not map the peer workspaces"
+            ex.close()
+            return None, ex.error or "another rank could not map the peer workspaces"
         return ex, None
 
-    exchange, exchange_note = make_exchange()
+    exchange, exchange_note = make_exchange(sets[0]["x"], sets[0]["dy"], sets[0]["dx"])
     sched = FusedGradientSum.schedule(max(2, args.steps)) if exchange is not None else None
 
     def fwd(s):
         dyt.forward(s["x"], alpha, gamma, beta, out=s["y"])
 
-    def bwd(s, ws_=None, i=None, ex=None, gbuf=None):
-        ex = exchange if ex is None else ex
+    default = object()  # bwd's ex: the run's exchange unless a lane passes its own (None: the all-reduce)
+
+    def bwd(s, ws_=None, i=None, ex=default, gbuf=None):
+        ex = exchange if ex is default else ex
         if ex is not None:  # stage 1, barrier, finalize over every rank's partials
             ex(s["x"], s["dy"], alpha, gamma, beta, s["dx"], s["dg"], s["db"], s["da"],
                buffer=None if i is None else sched[i % len(sched)])
@@ -611,7 +608,7 @@ def run_ours(args, w):
                                        "dg": torch.empty_like(gamma), "db": torch.empty_like(beta),
                                        "da": torch.empty_like(alpha)}
         lanes.append({"dev": d, "ws": dyt.workspace(x0, gamma), "stream": stream if j == 0 else torch.cuda.Stream(dev),
-                      "ex": exchange if j == 0 or exchange is None else FusedGradientSum(x0, x0, x0, gamma),
+                      "ex": exchange if j == 0 or exchange is None else make_exchange(x0, x0, x0)[0],
                       "grads": torch.empty(2 * N + 1, dtype=torch.float32, device=dev),
                       "hy": torch.empty_like(hx).pin_memory(), "hdx": torch.empty_like(hx).pin_memory(),
                       "hdg": torch.empty(N, dtype=gamma.dtype).pin_memory(),

@@ -134,31 +134,50 @@ class FusedGradientSum:
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         from . import MAX_RANKS
-        if self.world > MAX_RANKS:
+        if self.world > MAX_RANKS:  # the same on every rank, before any collective
             raise ValueError(f"at most {MAX_RANKS} ranks")
         self.ops = ops if ops is not None else DeviceOps(x.device)
         self.N = gamma.numel()
+        # Why this rank cannot take part (None: it can). Every rank runs the same
+        # collectives whatever fails locally, so a failure is recorded, not
+        # raised between two collectives; callers agree on `error` (one
+        # collective over all ranks) before the first call.
+        self.error = None
+        self.buffers, self._imported, self.ptrs, self.calls = [], [], [], 0
+        mine, handles = None, None
+        try:
+            mine = self.ops.layout(x, dy, dx, self.N)
+            self.buffers = [self.ops.workspace(x, gamma) for _ in range(self.NBUF)]
+            handles = [self.ops.export(b) for b in self.buffers]
+        except Exception as e:  # e.g. memory that CUDA IPC cannot share
+            self.error = f"{type(e).__name__}: {e}"
+            mine, handles = None, None
         self.layouts = [None] * self.world
-        dist.all_gather_object(self.layouts, self.ops.layout(x, dy, dx, self.N), group=group)
-        self.buffers = [self.ops.workspace(x, gamma) for _ in range(self.NBUF)]
-        handles = [self.ops.export(b) for b in self.buffers]
+        dist.all_gather_object(self.layouts, mine, group=group)
         everyone = [None] * self.world
         dist.all_gather_object(everyone, handles, group=group)
-        self._imported = []
-        self.ptrs = []
-        for b in range(self.NBUF):
-            row = []
-            for r in range(self.world):
-                if r == self.rank:
-                    row.append(self.ops.pointer(self.buffers[b]))
-                else:
-                    p = self.ops.import_(everyone[r][b])
-                    self._imported.append((p, everyone[r][b]))
-                    row.append(p)
-            self.ptrs.append(row)
-        self.calls = 0
+        if self.error is None and any(h is None for h in everyone):
+            self.error = "another rank could not export its workspaces"
+        if self.error is None:
+            try:
+                for b in range(self.NBUF):
+                    row = []
+                    for r in range(self.world):
+                        if r == self.rank:
+                            row.append(self.ops.pointer(self.buffers[b]))
+                        else:
+                            p = self.ops.import_(everyone[r][b])
+                            self._imported.append((p, everyone[r][b]))
+                            row.append(p)
+                    self.ptrs.append(row)
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                self.close()
+                self.ptrs = []
 
     def __call__(self, x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, stream=None, buffer=None):
+        if self.error is not None:
+            raise RuntimeError(f"the fused gradient sum cannot run on this rank: {self.error}")
         b = self.calls % self.NBUF if buffer is None else buffer
         layout = self.ops.partials(x, dy, alpha, gamma, dx, self.buffers[b], stream)
         if layout != self.layouts[self.rank]:

@@ -2,6 +2,7 @@
 own rows (here the oracle stands in for the device kernels), the parameter
 gradients are summed with the one all-reduce the method needs, and the result
 must equal the backward over all rows."""
+import datetime
 import os
 import socket
 
@@ -229,6 +230,69 @@ def test_fused_sum_protocol_on_gloo_ranks(world, M):
             assert da == float(want32[2 * N])
             assert np.all(np.abs(db - full["dbeta"]) <= 2e-6 + 1e-5 * np.abs(full["dbeta"]))
             assert abs(da - full["dalpha"]) <= 1e-5 * full["mag_dalpha"]
+
+
+class _FailingOps(_OracleOps):
+    """_OracleOps whose rank `bad` fails to export (or, with on_import, to import)."""
+
+    def __init__(self, rank, N, bad, on_import):
+        super().__init__(rank, N)
+        self.bad, self.on_import = bad, on_import
+
+    def export(self, buf):
+        if self.rank == self.bad and not self.on_import:
+            raise RuntimeError("cannot share this memory")
+        return super().export(buf)
+
+    def import_(self, handle):
+        if self.rank == self.bad and self.on_import and handle[0] != 0:
+            raise RuntimeError("cannot map that peer")
+        return super().import_(handle)
+
+
+def _failing_rank(rank: int, port: int, world: int, bad: int, on_import: bool, q):
+    from elementwise_reduction_b200.dist import FusedGradientSum
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        N = 8
+        ops = _FailingOps(rank, N, bad, on_import)
+        fgs = FusedGradientSum.__new__(FusedGradientSum)
+        ops.fgs = fgs
+        fgs.__init__(np.zeros(4 * N, dtype=np.float32), None, None, torch.zeros(N), ops=ops)
+        # what the bench does next: one collective over every rank's verdict
+        ok = torch.tensor([1 if fgs.error is None else 0])
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN)
+        fgs.close()
+        q.put((rank, fgs.error, int(ok.item()), len(fgs._imported)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("on_import", [False, True])
+def test_fused_sum_records_a_failing_rank(on_import):
+    # A rank that cannot export (or import) its workspaces records the failure
+    # instead of raising between two collectives: every rank finishes the
+    # construction, and the ranks agree to fall back.
+    world, bad = 3, 1
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_rank, args=(r, port, world, bad, on_import, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted([q.get(timeout=180) for _ in range(world)])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, error, ok, imported in got:
+        assert ok == 0 and imported == 0                   # all fall back; imported peers released
+        if rank == bad:
+            assert "cannot" in error
+        elif not on_import:
+            assert error == "another rank could not export its workspaces"
+        else:
+            assert error is None                           # only the bad rank failed to map
 
 
 def test_replay_schedule_never_reuses_a_buffer_back_to_back():

@@ -596,7 +596,9 @@ def run_ours(args, w):
     # overlap the next step's copies in (the link's two directions are
     # independent). Every step still copies in its own inputs and copies out
     # its own results.
-    e2e_steps = args.e2e_steps or max(3, min(args.steps, int(2e9 // max(1, set_bytes)) or 3))
+    # enough steps that the pipeline's fill and drain (one step's copies in, the
+    # last step's copies out) do not dominate; a c5 step is ~20-30 ms of copies
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 16))
     hx = _to_torch(inp["x"], w.x_dtype, "cpu").view(M, N).pin_memory()
     hdy = _to_torch(inp["dy"], w.x_dtype, "cpu").view(M, N).pin_memory()
     lanes = []
@@ -615,19 +617,34 @@ def run_ours(args, w):
                       "hdb": torch.empty(N, dtype=beta.dtype).pin_memory(),
                       "hda": torch.empty(1, dtype=alpha.dtype).pin_memory()})
 
+    # Copies in one direction run one step after another (each step's copies in
+    # wait for the previous step's, likewise out), so that the link carries one
+    # step's inputs while it returns the previous step's results instead of
+    # splitting one direction between two steps.
+    link = {"in": None, "out": None}
+
     def e2e_step(i):
         ln = lanes[i % 2]
         d = ln["dev"]
-        with torch.cuda.stream(ln["stream"]):
+        st = ln["stream"]
+        with torch.cuda.stream(st):
+            if link["in"] is not None:
+                st.wait_event(link["in"])
             d["x"].copy_(hx, non_blocking=True)
             d["dy"].copy_(hdy, non_blocking=True)
+            link["in"] = torch.cuda.Event()
+            link["in"].record(st)
             fwd(d)
             bwd(d, ln["ws"], ex=ln["ex"], gbuf=ln["grads"])
+            if link["out"] is not None:
+                st.wait_event(link["out"])
             ln["hy"].copy_(d["y"], non_blocking=True)
             ln["hdx"].copy_(d["dx"], non_blocking=True)
             ln["hdg"].copy_(d["dg"], non_blocking=True)
             ln["hdb"].copy_(d["db"], non_blocking=True)
             ln["hda"].copy_(d["da"], non_blocking=True)
+            link["out"] = torch.cuda.Event()
+            link["out"].record(st)
 
     e2e_step(0)
     e2e_step(1)

@@ -153,7 +153,8 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
  * 16 bytes, the vectorised kernels run. Adjacent rows (pitch N) are needed
  * for the packed form of a ragged N and for the shifted kernels (tensors not
  * all 16-byte aligned); other strided matrices with a ragged N or off 16-byte
- * boundaries take the one-element kernels. y may alias x (dx may alias x or dy) only with
+ * boundaries take the one-element kernels. y may alias x (dx may alias x or
+ * dy) only with
  * equal pitches. A pitch below N, or (M - 1) * ld + N beyond the int64 limit
  * of byte offsets, gives DYT_ERR_INVALID_VALUE. dyt_backward_workspace_bytes
  * covers the strided call too.
@@ -279,7 +280,7 @@ typedef struct dyt_launch_info {
                         4 = finalize (dyt_finalize_partials), 0 = none yet */
   int path;          /* 0 = nothing launched, 1 = row-tiled (several rows per CTA step),
                         2 = row-per-CTA (one row per CTA step, columns across threads) */
-  int vec;           /* elements per vector access (1 = scalar) */
+  int vec;           /* elements per vector access (1 = the one-element kernels) */
   int block;         /* threads per CTA */
   int grid;          /* CTAs of the main kernel (1D) */
   int row_lanes;     /* rows (packs of pack_rows rows) one CTA step covers side by side */

@@ -155,9 +155,8 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
  * all 16-byte aligned); other strided matrices with a ragged N or off 16-byte
  * boundaries take the one-element kernels. y may alias x (dx may alias x or
  * dy) only with equal pitches. A pitch below N, or (M - 1) * ld + N beyond
- * the int64 limit
- * of byte offsets, gives DYT_ERR_INVALID_VALUE. dyt_backward_workspace_bytes
- * covers the strided call too.
+ * the int64 limit of byte offsets, gives DYT_ERR_INVALID_VALUE.
+ * dyt_backward_workspace_bytes covers the strided call too.
  */
 dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, const void *gamma,
                                const void *beta, void *y, int64_t ldy, int64_t M, int64_t N,

@@ -1,6 +1,8 @@
 // C ABI of the fused DyT layer (declared in include/dyt.h): argument checks,
 // launch planning and kernel dispatch. All device work is in the kernels of
-// dyt_kernels.cuh and dyt_async.cuh.
+// dyt_async.cuh and dyt_kernels.cuh (stage 1 and the forward, selected through
+// dyt_select.cuh and compiled per activation dtype in dyt_inst_*.cu) and
+// dyt_finalize.cuh (the finalize, compiled here).
 #include <cuda.h>
 #include <cuda_runtime.h>
 

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
@@ -123,9 +124,12 @@ struct Plan {
   int grid;
   int path;     // 1 = row-tiled, 2 = row-per-CTA
   bool async;   // the 16-byte per-thread copy rings
-  bool packed;  // the packed-layout kernels: a ragged N (packs of vec rows) or the shifted kernels
-  bool shifted; // the shifted kernels: contiguous tensors not all 16-byte aligned (see dyt_async.cuh)
+  bool packed;  // the packed-layout kernels: a ragged N (packs of vec rows) or the flat shifted kernels
+  bool shifted; // the shifted kernels: tensors not all 16-byte aligned, or strided rows of a ragged N
+                // (see dyt_async.cuh)
+  bool rowframe;  // of those, the row frame: strided rows, each shifted on its own
   int shm;      // their mode: 0 = not shifted, else 1 | 2 (x's vectors cut out of two chunks) | 4 (dy's)
+                // | 8 (the row frame)
   int pack_rows;  // matrix rows per row of the packed layout: vec for a ragged N, else 1
   bool too_big; // the group or item count would not fit the kernels' int indices
   size_t smem;  // dynamic shared memory of the 16-byte kernel
@@ -151,41 +155,49 @@ size_t async_smem(bool backward, int block, size_t elem_bytes, bool shifted) {
 
 // vec: elements per access (1 or 16 / element size). ctas_per_sm from the
 // kernel's occupancy. ragged: N is not a multiple of vec, and the matrix is
-// laid out as packs of vec rows, each of pitch vec * N. shifted: the shifted
-// kernels, whose packed layout (packs of vec rows for a ragged N, else of one
-// row) starts the matrix at position sh, the output's offset past a 16-byte
-// boundary in elements. The plan depends only on these arguments.
+// laid out as packs of vec rows, each of pitch vec * N. shifted: the flat
+// shifted kernels, whose packed layout (packs of vec rows for a ragged N, else
+// of one row) starts the matrix at position sh, the output's offset past a
+// 16-byte boundary in elements. rowframe: the row frame, each matrix row laid
+// out on its own from position sh of a row of ceil((N + sh) / vec) vectors.
+// The plan depends only on these arguments.
 Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool async, int sms, int ctas_per_sm,
-               bool ragged, bool shifted, int sh, int64_t elem_bytes) {
+               bool ragged, bool shifted, bool rowframe, int sh, int64_t elem_bytes) {
   Plan p = {};
   p.vec = vec;
   p.async = async;
   p.packed = ragged || shifted;
-  p.shifted = shifted;
+  p.shifted = shifted || rowframe;
+  p.rowframe = rowframe;
   p.pack_rows = ragged ? vec : 1;
-  const int64_t end = M_rows * N_cols + (shifted ? sh : 0);  // the matrix's end in the (packed) layout
-  const int64_t N = (int64_t)p.pack_rows * N_cols;
+  // the matrix's end in the (packed) layout; the row frame: a row's end in its frame
+  const int64_t end = rowframe ? N_cols + sh : M_rows * N_cols + (shifted ? sh : 0);
+  const int64_t N = rowframe ? ceil_div(end, (int64_t)vec) * vec : (int64_t)p.pack_rows * N_cols;
   const int64_t M = p.packed ? ceil_div(end, N) : M_rows;
   const int64_t NV = N / vec;
   p.block = !async ? kScalarBlock : backward && NV <= kNarrowMaxNV ? kAsyncBlockNarrow : kAsyncBlock;
   const int block = p.block;
   p.unroll = async ? 1 : (backward ? kScalarUnrollBwd : kScalarUnrollFwd);
-  p.smem = async ? async_smem(backward, block, (size_t)elem_bytes, shifted) : 0;
+  p.smem = async ? async_smem(backward, block, (size_t)elem_bytes, p.shifted) : 0;
   Geom &g = p.g;
   g.M = M;
   g.N = N;
   g.Nc = N_cols;
   g.total = end;
-  g.sh = shifted ? sh : 0;
+  g.sh = p.shifted ? sh : 0;
   g.ldx = g.ldd = g.ldo = N;  // adjacent rows; the strided calls override this
   g.NV = (int)NV;
   if (NV <= block / 2) {
     g.RL = block / (int)NV;
     g.ncc = 1;
+    g.cw = block;
     p.path = 1;
   } else {
     g.RL = 1;
     g.ncc = (int)ceil_div(NV, block);
+    // Chunks of equal width in whole warps: 513 vectors as 288 + 225, not as
+    // 512 + 1, which would leave the CTAs of every second item nearly idle.
+    g.cw = async ? (int)std::min<int64_t>(block, ceil_div(ceil_div(NV, (int64_t)g.ncc), 32) * 32) : block;
     p.path = 2;
   }
   const int64_t target = (int64_t)sms * ctas_per_sm;
@@ -210,16 +222,18 @@ Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool asyn
   g.grem = M % nrg;
   g.nv_magic = NV >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)NV - 1) / (uint64_t)NV) : 0u;
   g.rl_magic = g.RL >= 2 ? (uint32_t)((((uint64_t)1 << 32) + (uint64_t)g.RL - 1) / (uint64_t)g.RL) : 0u;
-  g.l2_prefetch = (int64_t)(backward ? 2 : 1) * M_rows * N_cols * elem_bytes >= kPrefetchMinBytes;
+  // (the row frame's rows are strided: no prefetch)
+  g.l2_prefetch = !rowframe && (int64_t)(backward ? 2 : 1) * M_rows * N_cols * elem_bytes >= kPrefetchMinBytes;
   int64_t grid = fill * g.ncc;
   if (grid > target) grid = target;
   if (grid > g.nitems) grid = g.nitems;
   p.grid = (int)grid;
   // Workspace: binary64 partial sums of dgamma and dbeta per (group, row of a
   // pack, column), and of dalpha per CTA.
+  const size_t width = (size_t)p.pack_rows * (size_t)N_cols;  // partials per group
   p.ws_dg = 0;
-  p.ws_db = align16((size_t)nrg * (size_t)N * sizeof(double));
-  p.ws_da = p.ws_db + align16((size_t)nrg * (size_t)N * sizeof(double));
+  p.ws_db = align16((size_t)nrg * width * sizeof(double));
+  p.ws_da = p.ws_db + align16((size_t)nrg * width * sizeof(double));
   p.ws_total = p.ws_da + align16((size_t)p.grid * sizeof(double));
   return p;
 }
@@ -297,7 +311,7 @@ dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
     i.grid = p->grid;
     i.row_lanes = p->g.RL;
     i.pack_rows = p->pack_rows;
-    i.shifted = p->shifted ? 1 : 0;
+    i.shifted = p->rowframe ? 2 : p->shifted ? 1 : 0;
     i.shift = p->g.sh;
     i.rows_per_step = p->g.RL * p->unroll * i.pack_rows;
     i.col_chunks = p->g.ncc;
@@ -314,10 +328,11 @@ void record(int op, const Plan *p, int kernels, size_t ws) { t_info = describe(o
 // adjacent: every pitch is N. v: elements per 16-byte vector. Every pointer
 // is a whole number of elements (checked before).
 struct PathChoice {
-  bool ragged;   // ragged N on adjacent rows: packs of v rows through the 16-byte kernels
-  bool shifted;  // adjacent rows not all 16-byte aligned: the shifted 16-byte kernels
-  bool async;    // the 16-byte kernels (per-thread copy rings)
-  int vec;       // elements per access: v, or 1 for the one-element kernels
+  bool ragged;    // ragged N on adjacent rows: packs of v rows through the 16-byte kernels
+  bool shifted;   // adjacent rows not all 16-byte aligned: the flat shifted 16-byte kernels
+  bool rowframe;  // strided rows of whole-vector pitches, not all aligned or of a ragged N: the row frame
+  bool async;     // the 16-byte kernels (per-thread copy rings)
+  int vec;        // elements per access: v, or 1 for the one-element kernels
 };
 
 PathChoice choose_path(int64_t N, int v, bool aligned, bool pitched, bool adjacent) {
@@ -325,7 +340,9 @@ PathChoice choose_path(int64_t N, int v, bool aligned, bool pitched, bool adjace
   c.shifted = !aligned && adjacent;
   // A pack of v adjacent rows is a whole number of vectors whatever N is.
   c.ragged = adjacent && N % v != 0;
-  c.async = c.shifted || (aligned && (c.ragged || (pitched && N % v == 0)));
+  // Whole-vector pitches keep every row's offset past a boundary the same.
+  c.rowframe = !adjacent && pitched && (!aligned || N % v != 0);
+  c.async = c.shifted || c.rowframe || (aligned && (c.ragged || (pitched && N % v == 0)));
   if (!c.async) c.ragged = false;
   c.vec = c.async ? v : 1;
   return c;
@@ -343,17 +360,18 @@ dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjac
   const PathChoice pc = choose_path(N, vec_of<T>(), aligned, pitched, adjacent);
   if (pc.async) {
     // One CTA per SM by construction (__launch_bounds__(B, 1), ring sized for it).
-    *out = make_plan(M, N, pc.vec, backward, true, sms, 1, pc.ragged, pc.shifted, sh, (int64_t)sizeof(T));
+    *out = make_plan(M, N, pc.vec, backward, true, sms, 1, pc.ragged, pc.shifted, pc.rowframe, sh,
+                     (int64_t)sizeof(T));
     if (out->too_big) return DYT_ERR_INVALID_VALUE;
     // dy alone off the output's offset runs the kernel that cuts both inputs
-    out->shm = !out->shifted ? 0 : (win & 4) ? 7 : 1 | (win & 2);
+    out->shm = !out->shifted ? 0 : (out->rowframe ? 8 : 0) | ((win & 4) ? 7 : 1 | (win & 2));
     return prepare_smem(dev, main_kernel<T, P>(backward, true, out->packed, out->shm, out->block),
                         (int)out->smem);
   }
   int occ = 1;
   st = occupancy(dev, main_kernel<T, P>(backward, false, false, 0, kScalarBlock), kScalarBlock, &occ);
   if (st != DYT_OK) return st;
-  *out = make_plan(M, N, pc.vec, backward, false, sms, occ, false, false, 0, (int64_t)sizeof(T));
+  *out = make_plan(M, N, pc.vec, backward, false, sms, occ, false, false, false, 0, (int64_t)sizeof(T));
   if (out->too_big) return DYT_ERR_INVALID_VALUE;
   return DYT_OK;
 }
@@ -576,14 +594,17 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
   size_t need = 0;
   dyt_status st = with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
-    // The aligned, the shifted (one per output offset) and the one-element
-    // plans may differ; cover them all. The plans do not depend on P.
+    // The aligned (adjacent or strided), the shifted and the row-frame (one
+    // per output offset) and the one-element plans may differ; cover them
+    // all. The plans do not depend on P.
     constexpr int V = vec_of<T>();
-    for (int v = -2; v < V; ++v) {
+    for (int v = -3; v < 2 * V; ++v) {
       Plan p;
-      const dyt_status s = v == -2   ? plan_for<T, float>(M, N, true, true, true, 0, 0, true, &p)
+      const dyt_status s = v == -3   ? plan_for<T, float>(M, N, true, true, true, 0, 0, true, &p)
+                           : v == -2 ? plan_for<T, float>(M, N, true, true, false, 0, 0, true, &p)
                            : v == -1 ? plan_for<T, float>(M, N, false, false, false, 0, 0, true, &p)
-                                     : plan_for<T, float>(M, N, false, false, true, v, 0, true, &p);
+                           : v < V   ? plan_for<T, float>(M, N, false, false, true, v, 0, true, &p)
+                                     : plan_for<T, float>(M, N, false, true, false, v - V, 0, true, &p);
       if (s != DYT_OK) return s;
       if (p.ws_total > need) need = p.ws_total;
     }
@@ -762,18 +783,21 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
   if (st == DYT_OK && !valid_dtype(param_dtype)) st = DYT_ERR_UNSUPPORTED_DTYPE;
   if (st != DYT_OK) return st;
   const int v = 16 / (int)dsize(x_dtype);
-  if (layout < 0 || layout > 2 || (layout == 2 && (shift < 0 || shift >= v))) return DYT_ERR_INVALID_VALUE;
+  if (layout < 0 || layout > 3 || (layout >= 2 && (shift < 0 || shift >= v))) return DYT_ERR_INVALID_VALUE;
   const int op = backward ? 2 : 1;
   if (M == 0 || N == 0) {
     *out = describe(op, nullptr, 0, 0);
     return DYT_OK;
   }
   // layout 0: rows that are not whole 16-byte vectors; 1: contiguous and
-  // 16-byte aligned; 2: contiguous, the output `shift` elements past a boundary.
-  const PathChoice pc = choose_path(N, v, layout == 1, layout == 1, layout != 0);
+  // 16-byte aligned; 2: contiguous, the output `shift` elements past a
+  // boundary; 3: strided rows of whole-vector pitches, the output `shift`
+  // elements past a boundary.
+  const PathChoice pc = choose_path(N, v, layout == 1 || (layout == 3 && shift == 0), layout == 1 || layout == 3,
+                                    layout == 1 || layout == 2);
   // The 16-byte kernels always run one CTA per SM.
   Plan p = make_plan(M, N, pc.vec, backward != 0, pc.async, sm_count, pc.async ? 1 : ctas_per_sm, pc.ragged,
-                     pc.shifted, layout == 2 ? shift : 0, (int64_t)dsize(x_dtype));
+                     pc.shifted, pc.rowframe, layout >= 2 ? shift : 0, (int64_t)dsize(x_dtype));
   if (p.too_big) return DYT_ERR_INVALID_VALUE;
   *out = describe(op, &p, backward ? 2 : 1, backward ? p.ws_total : 0);
   return DYT_OK;

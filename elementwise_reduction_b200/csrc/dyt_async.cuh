@@ -61,6 +61,19 @@ __device__ __forceinline__ void vector_columns(int64_t c0, int64_t Nc, int64_t (
   }
 }
 
+// Row frame: matrix columns c + e of the VEC elements of a vector starting
+// at column c (c + e may fall in the row's padding, below 0 or at N and
+// beyond: those elements are masked, and get column 0 or N - 1 so that every
+// parameter load stays inside the parameter vectors).
+template <int VEC>
+__device__ __forceinline__ void row_frame_columns(int64_t c, int64_t Nc, int64_t (&col)[VEC]) {
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    const int64_t v = c + e;
+    col[e] = v < 0 ? 0 : v >= Nc ? Nc - 1 : v;
+  }
+}
+
 // The elements of a 16-byte vector whose bit is set in m, one by one: the
 // vectors that straddle the start or the end of a packed matrix.
 template <typename T, int VEC>
@@ -94,14 +107,18 @@ struct ShIn {
   uintptr_t lo, hi;  // the tensor's bytes [lo, hi)
 };
 
+// rf: the row frame (rows ld elements apart, position 0 of row 0's frame
+// sh elements before p); [lo, hi) is then the tensor's span, from its first
+// element to its last: the bytes between its rows (the chunks at a row's two
+// ends reach into them) lie inside it.
 template <typename T>
-__device__ __forceinline__ ShIn shifted_input(const T *p, const Geom &g) {
+__device__ __forceinline__ ShIn shifted_input(const T *p, const Geom &g, int64_t ld, bool rf) {
   ShIn s;
   const uintptr_t f = (uintptr_t)p - (uintptr_t)g.sh * sizeof(T);  // where position 0 falls in this tensor
   s.d = (int)(f & 15u);
   s.a = reinterpret_cast<const char *>(f - (uintptr_t)s.d);
   s.lo = (uintptr_t)p;
-  s.hi = s.lo + (uintptr_t)(g.total - g.sh) * sizeof(T);
+  s.hi = s.lo + (uintptr_t)(rf ? (g.M - 1) * ld + g.Nc : g.total - g.sh) * sizeof(T);
   return s;
 }
 
@@ -210,9 +227,9 @@ __device__ __forceinline__ void prefetch_shifted_rows_l2(const ShIn &s, const Ge
     if (e > a + kPiece) e = a + kPiece;
   } else {  // one column chunk of each row
     if (threadIdx.x >= rows) return;
-    const int64_t c0 = (int64_t)cc * B * VEC;
+    const int64_t c0 = (int64_t)cc * g.cw * VEC;
     a = (uintptr_t)s.a + (uintptr_t)((rb + threadIdx.x) * g.N + c0) * sizeof(T);
-    e = a + (uintptr_t)min((int64_t)B * VEC, g.N - c0) * sizeof(T);
+    e = a + (uintptr_t)min((int64_t)g.cw * VEC, g.N - c0) * sizeof(T);
   }
   if (a < lo) a = lo;
   if (e > hi) e = hi;
@@ -254,9 +271,9 @@ __device__ __forceinline__ void prefetch_first_rows_l2(const T *p, int64_t ld, c
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
     }
   } else if (threadIdx.x < rows) {  // one column chunk of each row
-    const int64_t c0 = (int64_t)cc * B * VEC;
+    const int64_t c0 = (int64_t)cc * g.cw * VEC;
     const int64_t at = (rb + threadIdx.x) * ld + c0;
-    int64_t n = min((int64_t)B * VEC, g.N - c0);
+    int64_t n = min((int64_t)g.cw * VEC, g.N - c0);
     if (PK) n = min(n, g.total - at);  // packed rows are adjacent (ld = N)
     n = (n * (int64_t)sizeof(T)) & ~(int64_t)15;
     if (n > 0)
@@ -302,22 +319,28 @@ __device__ __forceinline__ int last_vector_real(const Geom &g, int64_t first, in
 // with its matrix from position g.sh, rows whose copies or output vector reach
 // past a tensor's ends handled one by one (checked copies, masked stores).
 // SHM bit 1: x's offset differs from y's, so its vectors are cut out of two
-// chunks.
+// chunks. SHM bit 3: the row frame (RF) instead of the flat packed layout:
+// strided rows, each laid out on its own from position sh (see row_frame_*).
 template <typename T, typename P, int VEC, int B, int S, bool PK, int SHM>
 __global__ void __launch_bounds__(B, 1)
     dyt_fwd_async_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma_p,
                          const P *__restrict__ beta_p, ParamTypes pt, T *y, Geom g) {
   using IO = VecIO<T, VEC>;
-  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0;
+  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0, RF = (SHM & 8) != 0;
+  constexpr bool FL = SH && !RF;  // the flat shifted layout
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
-  static_assert(PK || !SH, "the shifted kernels use the packed layout");
+  static_assert(PK == FL || (PK && !SH), "the flat shifted kernels use the packed layout, the row frame does not");
   constexpr int CH = SH ? 2 : 1;  // 16-byte chunks per slot
   extern __shared__ uint4 ring[];  // [S][CH][B]
+  // A launch whose shared memory cannot hold the ring writes nothing (the
+  // host sizes it from the same constants; this only keeps a mismatch from
+  // reaching past the allocation).
+  if (dynamic_smem_bytes() < (uint32_t)(S * CH * B * 16)) return;
   ShIn ix = {};
-  if constexpr (SH) {
-    ix = shifted_input(x, g);
+  if constexpr (SH) ix = shifted_input(x, g, g.ldx, RF);
+  if constexpr (FL) {
     prefetch_shifted_rows_l2<T, VEC, B, S>(ix, g);
-  } else {
+  } else if constexpr (!RF) {
     prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
   }
   pdl_prologue();
@@ -331,7 +354,7 @@ __global__ void __launch_bounds__(B, 1)
     item_split(g, item, cc, rg);
     int64_t rb, re;
     group_rows(g, rg, rb, re);
-    const int cv = cc * B + ln.cv;
+    const int cv = cc * g.cw + ln.cv;
     if (!(ln.live && cv < g.NV)) continue;
     const int64_t c0 = (int64_t)cv * VEC;
     int64_t first;
@@ -341,14 +364,18 @@ __global__ void __launch_bounds__(B, 1)
     const int64_t sx = (int64_t)g.RL * g.ldx, sy = (int64_t)g.RL * g.ldo;
     const T *px = xb + first * g.ldx + c0;
     T *py = yb + first * g.ldo + c0;
-    // SH: rows [k_lo, k_hi) copy and store whole vectors; the others (at most
-    // a few at each end of the matrix) go element by element.
+    // SH: rows [k_lo, k_hi) copy whole chunks (and FL: store whole vectors);
+    // the others (at most a few at each end of the matrix) copy element by
+    // element.
     const int64_t pos0 = first * g.N + c0, dpos = (int64_t)g.RL * g.N;  // layout positions
     int k_lo = 0, k_hi = (int)n;  // n is at most kMaxRowsPerLane
+    // RF: the real elements of the thread's vectors are the same in every row
+    const uint32_t rmask = RF ? shifted_mask<VEC>(g, c0) : 0xFFu;
+    const bool rstore = !RF || rmask == (1u << VEC) - 1u;
     if constexpr (SH) {
-      while (k_lo < n && !(pos0 + k_lo * dpos >= g.sh && shifted_lo_ok(ix, px + k_lo * sx))) ++k_lo;
+      while (k_lo < n && !((RF || pos0 + k_lo * dpos >= g.sh) && shifted_lo_ok(ix, px + k_lo * sx))) ++k_lo;
       while (k_hi > k_lo &&
-             !(pos0 + (k_hi - 1) * dpos + VEC <= g.total && shifted_hi_ok(ix, px + (k_hi - 1) * sx)))
+             !((RF || pos0 + (k_hi - 1) * dpos + VEC <= g.total) && shifted_hi_ok(ix, px + (k_hi - 1) * sx)))
         --k_hi;
     }
     // Rows first, parameters second: the parameter loads overlap the copies.
@@ -362,7 +389,8 @@ __global__ void __launch_bounds__(B, 1)
       cp_async_commit();
     }
     int64_t col[VEC];
-    vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
+    if constexpr (RF) row_frame_columns<VEC>(c0 - g.sh, g.Nc, col);
+    else vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
     float gam[VEC], bet[VEC], bth[VEC];
     fwd_params_at<T, VEC, P>(gamma_p, beta_p, pt, col, gam, bet, bth);
     int s_rd = 0, s_wr = S - 1;
@@ -380,7 +408,8 @@ __global__ void __launch_bounds__(B, 1)
         cp_async_wait<S - 1>();
         const typename IO::Raw ry =
             fwd_vector<T, VEC>(read_shifted<B, WX>(slot0 + s_rd * CH * B, ix), alpha, gam, bet, bth);
-        if (!CHK || fast_row((int)k, k_lo, k_hi)) IO::store_raw(py, ry);
+        if (!rstore) store_mask<T, VEC>(py, ry, rmask);  // RF: the row's padding is not stored
+        else if (RF || !CHK || fast_row((int)k, k_lo, k_hi)) IO::store_raw(py, ry);
         else store_mask<T, VEC>(py, ry, shifted_mask<VEC>(g, pos0 + k * dpos));  // padding: not stored
         py += sy;
         s_rd = s_rd + 1 == S ? 0 : s_rd + 1;
@@ -452,19 +481,21 @@ __global__ void __launch_bounds__(B, 1)
 // ---- backward, stage 1 ----------------------------------------------------------
 
 // SHM != 0: as the forward's shifted kernels, x and dy each with their own
-// offset: bit 1 cuts x's vectors out of two chunks, bit 2 dy's.
+// offset: bit 1 cuts x's vectors out of two chunks, bit 2 dy's; bit 3 the row
+// frame.
 template <typename T, typename P, int VEC, int B, int S, bool PK, int SHM>
 __global__ void __launch_bounds__(B, 1)
     dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
                          const P *__restrict__ gamma_p, ParamTypes pt, T *dx, double *__restrict__ part_dg,
                          double *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
   using IO = VecIO<T, VEC>;
-  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0, WD = (SHM & 4) != 0;
+  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0, WD = (SHM & 4) != 0, RF = (SHM & 8) != 0;
+  constexpr bool FL = SH && !RF;  // the flat shifted layout
   constexpr bool EXACT_G = ExactGamma<T>::value;
   constexpr int kRunBlocks = kGammaRunRows / S;  // unrolled blocks of S rows per binary32 dgamma run
   constexpr int CH = SH ? 2 : 1;                 // 16-byte chunks per slot
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
-  static_assert(PK || !SH, "the shifted kernels use the packed layout");
+  static_assert(PK == FL || (PK && !SH), "the flat shifted kernels use the packed layout, the row frame does not");
   static_assert(2 * VEC * sizeof(double) <= 2 * S * 16, "the reduction fits in the drained ring");
   static_assert(kRunBlocks >= 1, "a dgamma run holds at least one block");
   // [S][2][CH][B] 16-byte slots (x, then dy); after an item's last row the
@@ -473,13 +504,18 @@ __global__ void __launch_bounds__(B, 1)
   // follow the ring (each thread's own, flushed from its binary32 runs).
   extern __shared__ uint4 ring[];
   __shared__ double red_a[B / 32];
+  // A launch whose shared memory cannot hold the ring and the dgamma totals
+  // writes nothing (see the forward).
+  if (dynamic_smem_bytes() < (uint32_t)(2 * S * CH * B * 16 + (EXACT_G ? 0 : VEC * B * 8))) return;
   ShIn ix = {}, id = {};
   if constexpr (SH) {
-    ix = shifted_input(x, g);
-    id = shifted_input(dy, g);
+    ix = shifted_input(x, g, g.ldx, RF);
+    id = shifted_input(dy, g, g.ldd, RF);
+  }
+  if constexpr (FL) {
     prefetch_shifted_rows_l2<T, VEC, B, S>(ix, g);
     prefetch_shifted_rows_l2<T, VEC, B, S>(id, g);
-  } else {
+  } else if constexpr (!RF) {
     prefetch_first_rows_l2<T, VEC, B, S, PK>(x, g.ldx, g);
     prefetch_first_rows_l2<T, VEC, B, S, PK>(dy, g.ldd, g);
   }
@@ -498,7 +534,7 @@ __global__ void __launch_bounds__(B, 1)
     item_split(g, item, cc, rg);
     int64_t rb, re;
     group_rows(g, rg, rb, re);
-    const int cv = cc * B + ln.cv;
+    const int cv = cc * g.cw + ln.cv;
     const bool col_ok = ln.live && cv < g.NV;
     const int64_t c0 = (int64_t)cv * VEC;
     float gam[VEC];
@@ -523,12 +559,15 @@ __global__ void __launch_bounds__(B, 1)
       // most a few at each end of the matrix) go element by element.
       const int64_t pos0 = first * g.N + c0, dpos = (int64_t)g.RL * g.N;  // layout positions
       int k_lo = 0, k_hi = nn;
+      // RF: the real elements of the thread's vectors are the same in every row
+      const uint32_t rmask = RF ? shifted_mask<VEC>(g, c0) : 0xFFu;
+      const bool rstore = !RF || rmask == (1u << VEC) - 1u;
       if constexpr (SH) {
-        while (k_lo < nn && !(pos0 + k_lo * dpos >= g.sh && shifted_lo_ok(ix, px + k_lo * sx) &&
+        while (k_lo < nn && !((RF || pos0 + k_lo * dpos >= g.sh) && shifted_lo_ok(ix, px + k_lo * sx) &&
                               shifted_lo_ok(id, pd + k_lo * sd)))
           ++k_lo;
-        while (k_hi > k_lo && !(pos0 + (k_hi - 1) * dpos + VEC <= g.total && shifted_hi_ok(ix, px + (k_hi - 1) * sx) &&
-                                shifted_hi_ok(id, pd + (k_hi - 1) * sd)))
+        while (k_hi > k_lo && !((RF || pos0 + (k_hi - 1) * dpos + VEC <= g.total) &&
+                                shifted_hi_ok(ix, px + (k_hi - 1) * sx) && shifted_hi_ok(id, pd + (k_hi - 1) * sd)))
           --k_hi;
       }
       // Rows first, parameters second: the gamma loads overlap the copies.
@@ -555,7 +594,8 @@ __global__ void __launch_bounds__(B, 1)
         cp_async_commit();
       }
       int64_t col[VEC];
-      vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
+      if constexpr (RF) row_frame_columns<VEC>(c0 - g.sh, g.Nc, col);
+      else vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
       load_params<VEC, P>(gamma_p, pt.gamma, col, 4.0f, gam);  // 4 gamma (see bwd_vector)
       int run = 0;  // blocks in the current binary32 dgamma run
       for (int k0 = 0; k0 < nn; k0 += S) {
@@ -656,7 +696,9 @@ __global__ void __launch_bounds__(B, 1)
               rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
               rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
             }
-            if (SH && CHK && !fast_row(k, k_lo, k_hi)) {  // padding of the shifted layout: dropped
+            if (!rstore) {  // RF: the row's padding is dropped
+              store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, rmask), rmask);
+            } else if (FL && CHK && !fast_row(k, k_lo, k_hi)) {  // padding of the shifted layout: dropped
               const uint32_t m = shifted_mask<VEC>(g, pos0 + k * dpos);
               store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
             } else if (!SH && PK && k == nn - 1 && nl < VEC) {  // the straddling vector: its zero-filled tail is dropped
@@ -691,22 +733,31 @@ __global__ void __launch_bounds__(B, 1)
     double ag[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) ag[e] = EXACT_G ? (double)acc.g[e] : gtot[e * B] + (double)acc.g[e];
-    double *pg = part_dg + (int64_t)rg * g.N;
-    double *pb = part_db + (int64_t)rg * g.N;
+    // a row of partials holds N (RF: Nc, the columns) values
+    double *pg = part_dg + (int64_t)rg * (RF ? g.Nc : g.N);
+    double *pb = part_db + (int64_t)rg * (RF ? g.Nc : g.N);
     if (g.RL == 1) {
       if (col_ok) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          const int64_t at = SH ? shifted_slot(g, c0 + e) : c0 + e;
-          pg[at] = ag[e];
-          pb[at] = acc.b[e];
+          const int64_t q = c0 + e;
+          if constexpr (RF) {
+            if (q >= g.sh && q - g.sh < g.Nc) {
+              pg[q - g.sh] = ag[e];
+              pb[q - g.sh] = acc.b[e];
+            }
+          } else {
+            const int64_t at = SH ? shifted_slot(g, q) : q;
+            pg[at] = ag[e];
+            pb[at] = acc.b[e];
+          }
         }
       }
     } else {
       __syncthreads();  // every thread's ring is drained: reuse it for the reduction
       if ((32 % g.NV) == 0) {
         // the chunk's columns start at 0 on the row-tiled path (one chunk)
-        lane_reduce_warps<VEC, B, SH>(ag, acc.b, red, g, ln, 0, pg, pb);
+        lane_reduce_warps<VEC, B, RF ? 2 : SH ? 1 : 0>(ag, acc.b, red, g, ln, 0, pg, pb);
       } else {  // dgamma and dbeta sums in one tree: 2 VEC values per thread
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
@@ -718,9 +769,17 @@ __global__ void __launch_bounds__(B, 1)
         if (col_ok && ln.rl == 0) {
 #pragma unroll
           for (int e = 0; e < VEC; ++e) {
-            const int64_t at = SH ? shifted_slot(g, c0 + e) : c0 + e;
-            pg[at] = red[e * B + threadIdx.x];
-            pb[at] = red[(VEC + e) * B + threadIdx.x];
+            const int64_t q = c0 + e;
+            if constexpr (RF) {
+              if (q >= g.sh && q - g.sh < g.Nc) {
+                pg[q - g.sh] = red[e * B + threadIdx.x];
+                pb[q - g.sh] = red[(VEC + e) * B + threadIdx.x];
+              }
+            } else {
+              const int64_t at = SH ? shifted_slot(g, q) : q;
+              pg[at] = red[e * B + threadIdx.x];
+              pb[at] = red[(VEC + e) * B + threadIdx.x];
+            }
           }
         }
         __syncthreads();

@@ -53,7 +53,8 @@ struct Geom {
   int64_t ldo;    //   and the output (y or dx)
   int NV;         // vector-columns per row (N / VEC)
   int RL;         // row lanes per CTA step (1 on the row-per-CTA path)
-  int ncc;        // column chunks (of B vector-columns)
+  int ncc;        // column chunks
+  int cw;         // vector-columns per column chunk (at most B; the 16-byte kernels read it)
   int nrg;        // row groups
   int nitems;     // ncc * nrg
   int64_t gq;     // M / nrg     (computed on the host: the kernels divide nothing)
@@ -247,6 +248,13 @@ struct VecIO<__half, 8> {
   static __device__ __forceinline__ void store_raw(__half *p, const Raw &r) { st16(p, r); }
 };
 
+// Bytes of dynamic shared memory this launch was given.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t r;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+
 // Start of every main kernel: wait until the preceding grid in the stream has
 // completed and its memory is visible (a no-op without a programmatic
 // predecessor), then let the next grid get scheduled. The kernels read and
@@ -262,7 +270,7 @@ __device__ __forceinline__ void pdl_prologue() {
 struct Lane {
   int rl;     // row lane
   int cv;     // vector-column within the chunk
-  bool live;  // false for threads past RL * NV on the row-tiled path
+  bool live;  // false for threads past RL * NV on the row-tiled path, past cw on the other
 };
 
 __device__ __forceinline__ Lane lane_of(const Geom &g, int tid) {
@@ -274,7 +282,7 @@ __device__ __forceinline__ Lane lane_of(const Geom &g, int tid) {
   } else {
     l.rl = 0;
     l.cv = tid;
-    l.live = true;
+    l.live = tid < g.cw;
   }
   return l;
 }
@@ -416,9 +424,10 @@ __device__ __forceinline__ void lane_tree(double *red, const Geom &g, const Lane
 // partners form the same sum). The order of every sum is fixed. Each warp
 // then holds each of its 2 NV VEC sums once; one pass over the warps in order
 // adds them. red[] holds (B / 32) x 2 NV VEC binary64 values. Results go to
-// out_g / out_b (row of the group's partials) at the thread's positions
-// (SH: at their shifted_slot).
-template <int VEC, int B, bool SH>
+// out_g / out_b (row of the group's partials) at the thread's positions; MAP
+// 1: at their shifted_slot (flat shifted layout); MAP 2: at position - sh,
+// padding positions skipped (row frame).
+template <int VEC, int B, int MAP>
 __device__ __forceinline__ void lane_reduce_warps(const double (&vg)[VEC], const double (&vb)[VEC], double *red,
                                                   const Geom &g, const Lane &ln, int64_t c0_chunk,
                                                   double *out_g, double *out_b) {
@@ -470,7 +479,12 @@ __device__ __forceinline__ void lane_reduce_warps(const double (&vg)[VEC], const
     const int which = i / width, k = i - which * width;
     double sum = 0.0;
     for (int w = 0; w < B / 32; ++w) sum += red[(2 * w + which) * width + k];
-    (which ? out_b : out_g)[SH ? shifted_slot(g, c0_chunk + k) : c0_chunk + k] = sum;
+    const int64_t q = c0_chunk + k;
+    if constexpr (MAP == 2) {
+      if (q >= g.sh && q - g.sh < g.Nc) (which ? out_b : out_g)[q - g.sh] = sum;
+    } else {
+      (which ? out_b : out_g)[MAP == 1 ? shifted_slot(g, q) : q] = sum;
+    }
   }
   __syncthreads();
 }

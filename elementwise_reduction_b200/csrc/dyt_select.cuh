@@ -26,7 +26,7 @@ constexpr int kAsyncStagesBwd = 6;      // ring slots per thread (backward: x an
 // 100003 x 100 fp32 26.9 -> 25.0 us; 128 threads and 12 slots were slower.
 constexpr int kAsyncBlockNarrow = 256;
 constexpr int kAsyncStagesBwdNarrow = 8;
-constexpr int kNarrowMaxNV = 64;
+constexpr int kNarrowMaxNV = 32;
 // Rows one lane adds per group, at most. The kernels count a thread's rows with
 // a multiply-high by ceil(2^32 / RL), exact for counts below 2^32 / RL; a
 // count stays below 2049 RL, and 2049 RL^2 < 2^32 for every RL <= 1024.
@@ -48,7 +48,8 @@ using BwdKernel = void (*)(const T *, const T *, const P *, const P *, ParamType
 
 // The forward kernel of a plan: the 16-byte kernels (aligned, packed or
 // shifted) or the one-element kernel. shm: the shifted kernels' mode (0 = not
-// shifted; else 1, | 2 when x's vectors are cut out of two chunks).
+// shifted; else 1, | 2 when x's vectors are cut out of two chunks, | 8 for the
+// row frame).
 template <typename T, typename P>
 FwdKernel<T, P> fwd_kernel_of(bool async, bool packed, int shm);
 

@@ -19,6 +19,8 @@ FwdKernel<T, P> fwd_kernel_of(bool async, bool packed, int shm) {
   switch (shm) {
     case 1: return dyt_fwd_async_kernel<T, P, V, B, S, true, 1>;
     case 3: return dyt_fwd_async_kernel<T, P, V, B, S, true, 3>;
+    case 9: return dyt_fwd_async_kernel<T, P, V, B, S, false, 9>;
+    case 11: return dyt_fwd_async_kernel<T, P, V, B, S, false, 11>;
   }
   return packed ? dyt_fwd_async_kernel<T, P, V, B, S, true, 0> : dyt_fwd_async_kernel<T, P, V, B, S, false, 0>;
 }
@@ -30,6 +32,9 @@ BwdKernel<T, P> bwd_async_of(bool packed, int shm) {
     case 1: return dyt_bwd_async_kernel<T, P, V, B, S, true, 1>;
     case 3: return dyt_bwd_async_kernel<T, P, V, B, S, true, 3>;
     case 7: return dyt_bwd_async_kernel<T, P, V, B, S, true, 7>;
+    case 9: return dyt_bwd_async_kernel<T, P, V, B, S, false, 9>;
+    case 11: return dyt_bwd_async_kernel<T, P, V, B, S, false, 11>;
+    case 15: return dyt_bwd_async_kernel<T, P, V, B, S, false, 15>;
   }
   return packed ? dyt_bwd_async_kernel<T, P, V, B, S, true, 0> : dyt_bwd_async_kernel<T, P, V, B, S, false, 0>;
 }

@@ -148,12 +148,17 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
  * leading-dimension form has no counterpart there. With the same kernels
  * (see below) it gives the same bits as the contiguous call on the same rows.
  * dyt_forward / dyt_backward are these with every pitch = N.
- * Padding between rows is neither read nor written. When every tensor is
- * 16-byte aligned and every pitch times the element size is a multiple of
- * 16 bytes, the vectorised kernels run. Adjacent rows (pitch N) are needed
- * for the packed form of a ragged N and for the shifted kernels (tensors not
- * all 16-byte aligned); other strided matrices with a ragged N or off 16-byte
- * boundaries take the one-element kernels. y may alias x (dx may alias x or
+ * Padding between rows is never written. When every pitch times the
+ * element size is a multiple of 16 bytes, the vectorised kernels run: the
+ * aligned ones for 16-byte aligned tensors and N a multiple of 16 / element
+ * size, else the row frame (each row laid out on its own as the shifted
+ * kernels lay out a contiguous matrix: whole 16-byte vectors of the output,
+ * masked at the row's two ends). The row frame copies the inputs in aligned
+ * 16-byte chunks, so it reads the padding bytes that share a chunk with a
+ * row's first or last elements (always between the tensor's first and last
+ * elements); their values reach no result. The other kernels read no
+ * padding. Pitches that are not whole 16-byte vectors take the one-element
+ * kernels. y may alias x (dx may alias x or
  * dy) only with equal pitches. A pitch below N, or (M - 1) * ld + N beyond
  * the int64 limit of byte offsets, gives DYT_ERR_INVALID_VALUE.
  * dyt_backward_workspace_bytes covers the strided call too.
@@ -291,8 +296,10 @@ typedef struct dyt_launch_info {
   int pack_rows;     /* 1, or vec on the packed path: a matrix of adjacent rows whose N is not a
                         multiple of vec is streamed as packs of vec rows (vec x N elements,
                         exactly N 16-byte vectors) */
-  int shifted;       /* 1 = the shifted 16-byte kernels (adjacent rows, tensors not all 16-byte
-                        aligned), 0 otherwise */
+  int shifted;       /* 1 = the flat shifted 16-byte kernels (adjacent rows, tensors not all
+                        16-byte aligned); 2 = the row frame (strided rows whose pitches are
+                        whole 16-byte vectors, tensors not all 16-byte aligned or N not a
+                        multiple of vec: each row shifted on its own); 0 otherwise */
   int shift;         /* shifted kernels: the output's offset past a 16-byte boundary, in
                         elements (0 .. vec - 1); 0 otherwise */
   int64_t workspace_bytes;
@@ -307,12 +314,15 @@ dyt_status dyt_last_launch_info(dyt_launch_info *out);
  * says: 0 = rows that are not whole 16-byte vectors (the one-element kernels),
  * 1 = contiguous and 16-byte aligned (a ragged N gets the packed form,
  * out->pack_rows > 1), 2 = contiguous with the output `shift` elements past a
- * 16-byte boundary (the shifted kernels; `shift` is read for layout 2 only).
+ * 16-byte boundary (the shifted kernels), 3 = strided rows (pitches not N)
+ * whose pitches are whole 16-byte vectors, the output `shift` elements past a
+ * 16-byte boundary (the row frame unless shift is 0 and N a multiple of vec;
+ * `shift` is read for layouts 2 and 3 only).
  * Host arithmetic only: touches no device, so the planning is testable
  * without a GPU. out->kernels is the number of kernels the call would launch
  * and out->workspace_bytes the workspace it needs.
  * Errors: as the shape checks of dyt_forward, or DYT_ERR_INVALID_VALUE for
- * out == NULL, sm_count / ctas_per_sm < 1, a layout outside 0..2 or a shift
+ * out == NULL, sm_count / ctas_per_sm < 1, a layout outside 0..3 or a shift
  * outside 0 .. 16 / element size - 1.
  */
 dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,

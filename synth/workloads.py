@@ -90,7 +90,9 @@ WORKLOADS = {
 # vector one aligned chunk); _xoff1: x alone, as a sliced input next to fresh
 # outputs (each x vector cut out of two aligned chunks). _pitch4100: rows of
 # 4096 elements 4100 apart (8200 bytes, not whole 16-byte vectors), which the
-# one-element kernels take.
+# one-element kernels take. _pitch4104_off1: rows 4104 apart (whole vectors),
+# every tensor one element past a boundary; _pitch256: rows of 255 fp32
+# elements 256 apart: the row frame, each row shifted on its own.
 VARIANTS = {
     w.name: w
     for w in [
@@ -98,6 +100,8 @@ VARIANTS = {
         replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_off1", offset=1),
         replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_xoff1", x_offset=1),
         replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_pitch4100", pitch=4100),
+        replace(WORKLOADS["c4_bf16_16384x4096"], name="c4_bf16_16384x4096_pitch4104_off1", pitch=4104, offset=1),
+        replace(WORKLOADS["c3_f32_100003x255_inf"], name="c3_f32_100003x255_inf_pitch256", pitch=256),
     ]
 }
 

@@ -125,33 +125,39 @@ def test_pointers_must_hold_whole_elements():
                                     (100003, 255, 0), (16384, 4096, 1), (32768, 8192, 1), (1, 1, 0),
                                     (3, 70000, 2), (10**7, 8, 1), (5, 513, 0), (7, 3, 1), (1, 17, 0),
                                     (100003, 4097, 1), (4099, 1001, 0)])
-@pytest.mark.parametrize("layout,shift", [(0, 0), (1, 0), (2, 0), (2, 1), (2, -1)])
+@pytest.mark.parametrize("layout,shift", [(0, 0), (1, 0), (2, 0), (2, 1), (2, -1), (3, 0), (3, 1), (3, -1)])
 @pytest.mark.parametrize("sms,occ", [(148, 1), (148, 2), (7, 1)])
 def test_launch_plan_invariants(M, N, xd, layout, shift, sms, occ):
     dyt = _lib()
     size = 4 if xd == 0 else 2
-    sh = shift % (16 // size) if layout == 2 else 0
+    sh = shift % (16 // size) if layout >= 2 else 0
     p = dyt.dyt_plan_query(M, N, xd, 0, 1, layout, sms, occ, shift=sh)
     vec = p["vec"]
     pk = p["pack_rows"]
+    # strided rows of whole-vector pitches, off a boundary or of a ragged N:
+    # the row frame
+    rf = layout == 3 and (sh != 0 or N % (16 // size) != 0)
     # adjacent rows always take the 16-byte kernels (packed when N is ragged);
-    # tensors off 16-byte boundaries the shifted ones
+    # tensors off 16-byte boundaries the shifted ones; strided rows of
+    # whole-vector pitches too
     assert bool(p["async_stages"]) == (layout != 0)
-    assert p["shifted"] == (layout == 2) and p["shift"] == sh
+    assert p["shifted"] == (2 if rf else 1 if layout == 2 else 0) and p["shift"] == sh
     if p["async_stages"]:    # per-thread copy ring: 16-byte vectors, one per thread
         assert vec == 16 // size
-        # a ragged N is streamed in packs of vec rows (exactly N vectors each)
-        assert pk == (vec if N % vec else 1)
+        # a ragged N on adjacent rows is streamed in packs of vec rows (exactly
+        # N vectors each)
+        assert pk == (vec if N % vec and layout in (1, 2) else 1)
         ctas = sms             # the 16-byte kernels run one CTA per SM
     else:
         assert vec == 1 and pk == 1
         ctas = sms * occ
-    Np = pk * N                                    # pitch of a (packed) row
+    # pitch of a (packed) row; the row frame: a row's vectors from position sh
+    Np = -(-(N + sh) // vec) * vec if rf else pk * N
     Mp = -(-(M * N + sh) // Np) if layout == 2 else -(-M // pk)  # (packed) rows; shifted: the matrix from position sh
     nv = Np // vec
     B = p["block"]
-    # the backward over narrow rows (at most 64 vectors) runs 256-thread CTAs with 8-slot rings
-    assert B == (1024 if not p["async_stages"] else 256 if nv <= 64 else 512) and p["kernels"] == 2
+    # the backward over narrow rows (at most 32 vectors) runs 256-thread CTAs with 8-slot rings
+    assert B == (1024 if not p["async_stages"] else 256 if nv <= 32 else 512) and p["kernels"] == 2
     if p["async_stages"]:
         assert p["async_stages"] == (8 if B == 256 else 6)
     assert 1 <= p["grid"] <= ctas                  # persistent 1D grid: never beyond one wave
@@ -175,7 +181,7 @@ def test_launch_plan_invariants(M, N, xd, layout, shift, sms, occ):
     # workspace: binary64 dgamma and dbeta partials per group and row position
     # (pack_rows x N of them) + binary64 dalpha per CTA
     al = lambda v: (v + 15) // 16 * 16
-    assert p["workspace_bytes"] == 2 * al(p["row_groups"] * Np * 8) + al(p["grid"] * 8)
+    assert p["workspace_bytes"] == 2 * al(p["row_groups"] * pk * N * 8) + al(p["grid"] * 8)
 
 
 def test_plans_whose_counts_overflow_are_rejected():

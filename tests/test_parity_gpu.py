@@ -399,7 +399,7 @@ def test_strided_rows(N, pad, xd):
     M = 3001
     inp = make(M, N, xd, "f32")
     t = H.gpu_inputs(inp, xd, "f32")
-    _, x = _in_wider_rows(t["x"], M, N, N + pad, float("nan"))      # padding is never read
+    _, x = _in_wider_rows(t["x"], M, N, N + pad, float("nan"))      # padding reaches no result
     _, dy = _in_wider_rows(t["dy"], M, N, N + 2 * pad, float("nan"))
     ybuf, y = _in_wider_rows(torch.zeros(M * N, dtype=x.dtype, device="cuda"), M, N, N + 3 * pad, 7.0)
     dxbuf, dx = _in_wider_rows(torch.zeros(M * N, dtype=x.dtype, device="cuda"), M, N, N + 4 * pad, 7.0)
@@ -414,14 +414,71 @@ def test_strided_rows(N, pad, xd):
     H.compare_all(inp, out, M, N, xd, "f32")
     size = 4 if xd == "f32" else 2
     vec = 16 // size
-    vectorised = N % vec == 0 and all((p * size) % 16 == 0 for p in (N + pad, N + 2 * pad, N + 3 * pad, N + 4 * pad))
-    assert info_f["vec"] == info_b["vec"] == (vec if vectorised else 1)
+    # whole-vector pitches take the 16-byte kernels (aligned tensors and N a
+    # multiple of vec: the plain ones, else the row frame)
+    pitched = all((p * size) % 16 == 0 for p in (N + pad, N + 2 * pad, N + 3 * pad, N + 4 * pad))
+    vectorised = N % vec == 0 and pitched
+    assert info_f["vec"] == info_b["vec"] == (vec if pitched else 1)
+    assert info_f["shifted"] == info_b["shifted"] == (2 if pitched and not vectorised else 0)
     assert info_b["pack_rows"] == 1
     if vectorised:  # the same kernels as the contiguous call: the same bits
         ref, _ = H.run_cuda(inp, M, N, xd, "f32")
         for k in ("y", "dx", "dgamma", "dbeta"):
             assert np.array_equal(out[k], ref[k]), k
         assert out["dalpha"] == ref["dalpha"]
+
+
+def _placed_rows(src, M: int, N: int, off: int, ld: int, fill: float) -> tuple:
+    # M rows of N elements, `ld` apart, the first `off` elements past a 16-byte
+    # boundary, in a buffer filled with `fill`
+    buf = torch.full((M * ld + off + 64,), fill, dtype=src.dtype, device="cuda")
+    view = buf[off:off + M * ld].view(M, ld)[:, :N]
+    view.copy_(src.reshape(M, N))
+    return buf, view
+
+
+@pytest.mark.parametrize("xd", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [1, 3, 17, 100, 255, 520, 4099])
+@pytest.mark.parametrize("hx,hd,ho", [(0, 0, 0), (1, 1, 1), (0, 3, 1), (-1, 0, 2), (2, -1, -1)])
+def test_row_frame_rows(xd, N, hx, hd, ho):
+    # Strided rows whose pitches are whole 16-byte vectors, with tensors off
+    # 16-byte boundaries or a ragged N: each row shifted on its own. NaN
+    # between the rows of the inputs (the chunks at a row's ends read some of
+    # it; it must reach no result), 7 between the rows of the outputs (never
+    # written); elementwise results bit for bit those of the contiguous call,
+    # sums within the oracle's bounds.
+    import elementwise_reduction_b200 as dyt
+    size = 4 if xd == "f32" else 2
+    vec = 16 // size
+    hx, hd, ho = hx % vec, hd % vec, ho % vec
+    if not (hx or hd or ho or N % vec):
+        pytest.skip("aligned rows of whole vectors take the plain kernels")
+    M = 1201
+    base = -(-N // vec) * vec
+    inp = make(M, N, xd, "f32")
+    t = H.gpu_inputs(inp, xd, "f32")
+    _, x = _placed_rows(t["x"], M, N, hx, base + vec, float("nan"))
+    _, dy = _placed_rows(t["dy"], M, N, hd, base + 2 * vec, float("nan"))
+    zero = torch.zeros(M * N, dtype=t["x"].dtype, device="cuda")
+    ybuf, y = _placed_rows(zero, M, N, ho, base + 3 * vec, 7.0)
+    dxbuf, dx = _placed_rows(zero, M, N, ho, base, 7.0)
+    ymask = torch.ones_like(ybuf, dtype=torch.bool)
+    ymask[ho:ho + M * (base + 3 * vec)].view(M, -1)[:, :N] = False
+    dxmask = torch.ones_like(dxbuf, dtype=torch.bool)
+    dxmask[ho:ho + M * base].view(M, -1)[:, :N] = False
+    dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=y)
+    info_f = dyt.dyt_last_launch_info()
+    _, dalpha, dgamma, dbeta = dyt.backward(x, dy, t["alpha"], t["gamma"], dx=dx)
+    info_b = dyt.dyt_last_launch_info()
+    torch.cuda.synchronize()
+    assert (ybuf[ymask] == 7).all() and (dxbuf[dxmask] == 7).all()  # nothing outside the rows is written
+    assert info_f["shifted"] == info_b["shifted"] == 2 and info_f["shift"] == info_b["shift"] == ho
+    assert info_f["vec"] == info_b["vec"] == vec
+    out = {"y": H.to_numpy(y.contiguous(), xd), "dx": H.to_numpy(dx.contiguous(), xd),
+           "dgamma": H.to_numpy(dgamma, "f32"), "dbeta": H.to_numpy(dbeta, "f32"), "dalpha": float(dalpha.item())}
+    H.compare_all(inp, out, M, N, xd, "f32")
+    ref, _ = H.run_cuda(inp, M, N, xd, "f32")
+    assert np.array_equal(out["y"], ref["y"]) and np.array_equal(out["dx"], ref["dx"])
 
 
 def test_strided_in_place_and_autograd():
@@ -701,8 +758,11 @@ def test_unaligned_variant_full_size(name):
     inp = workloads.make_inputs(w)
     out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype, offset=w.offset, x_offset=w.x_offset,
                            pitch=w.pitch)
-    if w.pitch:
+    if w.pitch and (w.pitch * (4 if w.x_dtype == "f32" else 2)) % 16:
         assert info["fwd"]["vec"] == info["bwd"]["vec"] == 1
+    elif w.pitch:  # whole-vector pitches: the row frame
+        assert info["fwd"]["shifted"] == 2 and info["bwd"]["shifted"] == 2
+        assert info["fwd"]["shift"] == info["bwd"]["shift"] == w.offset
     else:
         assert info["fwd"]["shifted"] == 1 and info["bwd"]["shifted"] == 1
         assert info["fwd"]["shift"] == info["bwd"]["shift"] == w.offset

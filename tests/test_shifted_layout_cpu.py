@@ -25,6 +25,11 @@ def _cdiv(a, b):
     return -(-a // b)
 
 
+def _chunk_width(B, RL, ncc, NV):
+    # vector-columns per column chunk: equal chunks in whole warps
+    return B if RL > 1 else min(B, _cdiv(_cdiv(NV, ncc), 32) * 32)
+
+
 def replay(dyt, M, N, xd, hx, hd, ho, backward, sms=3):
     es = 4 if xd == 0 else 2
     vec = 16 // es
@@ -36,6 +41,7 @@ def replay(dyt, M, N, xd, hx, hd, ho, backward, sms=3):
     sh, total = ho, M * N + ho        # the matrix occupies positions [sh, total) of the layout
     Mp = _cdiv(total, Np)
     gq, grem = Mp // nrg, Mp % nrg
+    cw = _chunk_width(B, RL, ncc, NV)
     bases = {"x": 1 << 20, "dy": 2 << 20, "o": 3 << 20}  # 16-byte aligned regions, one per tensor
     lo = {"x": bases["x"] + hx * es, "dy": bases["dy"] + hd * es, "o": bases["o"] + ho * es}
     hi = {k: v + M * N * es for k, v in lo.items()}
@@ -54,8 +60,8 @@ def replay(dyt, M, N, xd, hx, hd, ho, backward, sms=3):
                 cc, rg = (0, item) if ncc == 1 else (item % ncc, item // ncc)
                 rb = rg * gq + min(rg, grem)
                 re = rb + gq + (1 if rg < grem else 0)
-                cv = cc * B + cvl
-                if not (live and cv < NV):
+                cv = cc * cw + cvl
+                if not (live and cvl < cw and cv < NV):
                     continue
                 c0 = cv * vec
                 first = rb + rl
@@ -150,3 +156,139 @@ def test_shifted_addressing_with_column_chunks(M, N, xd):
         for hx in (0, 1):
             for backward in (False, True):
                 replay(dyt, M, N, xd, hx, hx, ho, backward, sms=5)
+
+
+def _round_up(a, b):
+    return _cdiv(a, b) * b
+
+
+def replay_rowframe(dyt, M, N, xd, offs, lds, backward, sms=3):
+    """The row frame: strided rows whose pitches are whole 16-byte vectors,
+    each row laid out on its own from position sh (the output's offset) of a
+    row of ceil((N + sh) / vec) vectors. offs / lds: each tensor's offset past
+    a 16-byte boundary and its pitch, in elements."""
+    es = 4 if xd == 0 else 2
+    vec = 16 // es
+    ho = offs["o"]
+    p = dyt.dyt_plan_query(M, N, xd, 0, int(backward), 3, sms, 1, shift=ho)
+    if ho or N % vec:
+        assert p["shifted"] == 2 and p["shift"] == ho and p["pack_rows"] == 1
+    B, RL, ncc, nrg, grid = (p[k] for k in ("block", "row_lanes", "col_chunks", "row_groups", "grid"))
+    NV = _cdiv(N + ho, vec)           # vectors of a row's frame
+    assert ncc == (1 if RL > 1 else _cdiv(NV, B))
+    gq, grem = M // nrg, M % nrg
+    cw = _chunk_width(B, RL, ncc, NV)
+    ins = ["x", "dy"] if backward else ["x"]
+    bases = {"x": 1 << 24, "dy": 2 << 24, "o": 3 << 24}
+    lo = {k: bases[k] + offs[k] * es for k in bases}    # row 0 of each tensor
+    for k in bases:
+        assert lds[k] >= N and lds[k] * es % 16 == 0
+    frame = {}
+    for k in ins:  # where position 0 of row 0's frame falls: aligned chunk base, byte offset d
+        f = lo[k] - ho * es
+        frame[k] = (f - (f & 15), f & 15)
+        if offs[k] == ho:
+            assert frame[k][1] == 0  # same offset as the output: single chunks
+    assert (lo["o"] - ho * es) % 16 == 0
+    stored = set()
+    for blk in range(grid):
+        for tid in range(B):
+            rl, cvl, live = (tid // NV, tid % NV, tid // NV < RL) if RL > 1 else (0, tid, True)
+            for item in range(blk, nrg * ncc, grid):
+                cc, rg = (0, item) if ncc == 1 else (item % ncc, item // ncc)
+                rb = rg * gq + min(rg, grem)
+                re = rb + gq + (1 if rg < grem else 0)
+                cv = cc * cw + cvl
+                if not (live and cvl < cw and cv < NV):
+                    continue
+                c0 = cv * vec
+                first = rb + rl
+                n = 0 if first >= re else _cdiv(re - first, RL)
+                assert n <= 2048
+                mask = [ho <= c0 + e < N + ho for e in range(vec)]
+                assert any(mask)
+                cols = [min(max(c0 + e - ho, 0), N - 1) for e in range(vec)]
+                # the tensors' spans, first element to last: the copies may read
+                # the bytes between rows, never outside a span
+                span = {m: (lo[m], lo[m] + ((M - 1) * lds[m] + N) * es) for m in ins}
+
+                def chunk(k, m):
+                    return frame[m][0] + c0 * es + (first + k * RL) * lds[m] * es
+
+                def ok(k):
+                    return all(chunk(k, m) >= span[m][0] and chunk(k, m) + (32 if frame[m][1] else 16) <= span[m][1]
+                               for m in ins)
+
+                k_lo = 0
+                while k_lo < n and not ok(k_lo):
+                    k_lo += 1
+                k_hi = n
+                while k_hi > k_lo and not ok(k_hi - 1):
+                    k_hi -= 1
+                assert k_lo <= 1 and k_hi >= n - 1  # only the tensors' first and last rows are checked
+                for k in range(n):
+                    row = first + k * RL
+                    got = {}
+                    for m in ins:
+                        rlo = lo[m] + row * lds[m] * es
+                        slo, shi = span[m]
+                        a, d = chunk(k, m), frame[m][1]
+                        assert a % 16 == 0
+                        bytes_ = set()
+                        for ca in ([a, a + 16] if d else [a]):
+                            if k_lo <= k < k_hi:
+                                bytes_.update(range(ca, ca + 16))
+                            elif ca >= shi or ca + 16 <= slo:
+                                continue
+                            elif ca >= slo:
+                                bytes_.update(range(ca, ca + min(16, shi - ca)))
+                            else:
+                                assert (slo - ca) % es == 0
+                                bytes_.update(range(slo, min(shi, ca + 16)))
+                        assert all(slo <= b < shi for b in bytes_), ("read outside the tensor", m)
+                        got[m] = (a + d, rlo, bytes_)
+                    out_row = lo["o"] + row * lds["o"] * es
+                    for e in range(vec):
+                        if not mask[e]:
+                            continue  # the row's padding: neither stored nor summed
+                        col = c0 + e - ho
+                        assert (lo["o"] - ho * es) + row * lds["o"] * es + (c0 + e) * es == out_row + col * es
+                        assert (row, col) not in stored, "stored twice"
+                        stored.add((row, col))
+                        assert cols[e] == col
+                        for m in ins:
+                            start, rlo, bytes_ = got[m]
+                            for b in range(start + e * es, start + (e + 1) * es):
+                                assert b in bytes_, "an input byte was not copied"
+                                assert (b - rlo) // es == col
+                        assert c0 + e - ho == col  # partial-sum slot: the column itself
+    assert len(stored) == M * N
+
+
+RF_CASES = [(M, N) for N in (1, 3, 8, 17, 32, 100, 255) for M in (1, 3, 9)] + [(33, 17), (5, 520)]
+
+
+@pytest.mark.parametrize("xd", [0, 1])
+@pytest.mark.parametrize("M,N", RF_CASES)
+def test_row_frame_addressing_stays_inside_every_row(xd, M, N):
+    dyt = _lib()
+    vec = 4 if xd == 0 else 8
+    base = _round_up(N, vec)
+    lds = {"x": base + vec, "dy": base, "o": base + 2 * vec}
+    for backward in (False, True):
+        for ho in range(vec):
+            for hx in sorted({0, 1, vec - 1, ho}):
+                for hd in (sorted({0, ho, vec - 1}) if backward else [0]):
+                    replay_rowframe(dyt, M, N, xd, {"x": hx, "dy": hd, "o": ho}, lds, backward)
+
+
+@pytest.mark.parametrize("M,N,xd", [(3, 4104, 1), (2, 4099, 1), (4, 2051, 0)])
+def test_row_frame_addressing_with_column_chunks(M, N, xd):
+    dyt = _lib()
+    vec = 4 if xd == 0 else 8
+    base = _round_up(N, vec)
+    lds = {"x": base, "dy": base + vec, "o": base + vec}
+    for ho in (0, 1, vec - 1):
+        for hx in (0, 1):
+            for backward in (False, True):
+                replay_rowframe(dyt, M, N, xd, {"x": hx, "dy": hx, "o": ho}, lds, backward, sms=5)

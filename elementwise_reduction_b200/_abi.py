@@ -232,8 +232,9 @@ def dyt_plan_query(M, N, x_dtype, param_dtype, backward, layout, sm_count, ctas_
     layout: 0 = rows that are not whole 16-byte vectors (one-element kernels),
     1 = contiguous and 16-byte aligned, 2 = contiguous with the output `shift`
     elements past a 16-byte boundary (the shifted kernels), 3 = strided rows of
-    whole-vector pitches, the output `shift` elements past a boundary (the row
-    frame, unless shift is 0 and N a multiple of the vector)."""
+    whole-vector pitches, every tensor `shift` elements past a boundary (the
+    row frame, unless shift is 0 and N a multiple of the vector), 4 = as 3 with
+    the inputs at other offsets."""
     info = LaunchInfo()
     _check(lib.dyt_plan_query(M, N, x_dtype, param_dtype, int(backward), int(layout), int(shift), sm_count,
                               ctas_per_sm, ctypes.byref(info)), "dyt_plan_query")

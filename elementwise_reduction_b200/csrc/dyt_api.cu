@@ -128,6 +128,7 @@ struct Plan {
   bool shifted; // the shifted kernels: tensors not all 16-byte aligned, or strided rows of a ragged N
                 // (see dyt_async.cuh)
   bool rowframe;  // of those, the row frame: strided rows, each shifted on its own
+  bool wrap;      // the row frame with a wrapped vector-column (see make_plan)
   int shm;      // their mode: 0 = not shifted, else 1 | 2 (x's vectors cut out of two chunks) | 4 (dy's)
                 // | 8 (the row frame)
   int pack_rows;  // matrix rows per row of the packed layout: vec for a ragged N, else 1
@@ -159,20 +160,23 @@ size_t async_smem(bool backward, int block, size_t elem_bytes, bool shifted) {
 // shifted kernels, whose packed layout (packs of vec rows for a ragged N, else
 // of one row) starts the matrix at position sh, the output's offset past a
 // 16-byte boundary in elements. rowframe: the row frame, each matrix row laid
-// out on its own from position sh of a row of ceil((N + sh) / vec) vectors.
+// out on its own from position sh of a row of ceil((N + sh) / vec) vectors;
+// wrap (N a multiple of vec, sh > 0, every input at the output's offset): of
+// N / vec vectors instead, the first holding the row's last sh elements too.
 // The plan depends only on these arguments.
 Plan make_plan(int64_t M_rows, int64_t N_cols, int vec, bool backward, bool async, int sms, int ctas_per_sm,
-               bool ragged, bool shifted, bool rowframe, int sh, int64_t elem_bytes) {
+               bool ragged, bool shifted, bool rowframe, bool wrap, int sh, int64_t elem_bytes) {
   Plan p = {};
   p.vec = vec;
   p.async = async;
   p.packed = ragged || shifted;
   p.shifted = shifted || rowframe;
   p.rowframe = rowframe;
+  p.wrap = rowframe && wrap;
   p.pack_rows = ragged ? vec : 1;
   // the matrix's end in the (packed) layout; the row frame: a row's end in its frame
   const int64_t end = rowframe ? N_cols + sh : M_rows * N_cols + (shifted ? sh : 0);
-  const int64_t N = rowframe ? ceil_div(end, (int64_t)vec) * vec : (int64_t)p.pack_rows * N_cols;
+  const int64_t N = p.wrap ? N_cols : rowframe ? ceil_div(end, (int64_t)vec) * vec : (int64_t)p.pack_rows * N_cols;
   const int64_t M = p.packed ? ceil_div(end, N) : M_rows;
   const int64_t NV = N / vec;
   p.block = !async ? kScalarBlock : backward && NV <= kNarrowMaxNV ? kAsyncBlockNarrow : kAsyncBlock;
@@ -311,7 +315,7 @@ dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
     i.grid = p->grid;
     i.row_lanes = p->g.RL;
     i.pack_rows = p->pack_rows;
-    i.shifted = p->rowframe ? 2 : p->shifted ? 1 : 0;
+    i.shifted = p->wrap ? 3 : p->rowframe ? 2 : p->shifted ? 1 : 0;
     i.shift = p->g.sh;
     i.rows_per_step = p->g.RL * p->unroll * i.pack_rows;
     i.col_chunks = p->g.ncc;
@@ -360,18 +364,20 @@ dyt_status plan_for(int64_t M, int64_t N, bool aligned, bool pitched, bool adjac
   const PathChoice pc = choose_path(N, vec_of<T>(), aligned, pitched, adjacent);
   if (pc.async) {
     // One CTA per SM by construction (__launch_bounds__(B, 1), ring sized for it).
-    *out = make_plan(M, N, pc.vec, backward, true, sms, 1, pc.ragged, pc.shifted, pc.rowframe, sh,
+    const bool wrap = pc.rowframe && sh > 0 && N % pc.vec == 0 && win == 0;
+    *out = make_plan(M, N, pc.vec, backward, true, sms, 1, pc.ragged, pc.shifted, pc.rowframe, wrap, sh,
                      (int64_t)sizeof(T));
     if (out->too_big) return DYT_ERR_INVALID_VALUE;
     // dy alone off the output's offset runs the kernel that cuts both inputs
-    out->shm = !out->shifted ? 0 : (out->rowframe ? 8 : 0) | ((win & 4) ? 7 : 1 | (win & 2));
+    out->shm = !out->shifted ? 0
+                             : (out->rowframe ? 8 : 0) | (out->wrap ? 16 : 0) | ((win & 4) ? 7 : 1 | (win & 2));
     return prepare_smem(dev, main_kernel<T, P>(backward, true, out->packed, out->shm, out->block),
                         (int)out->smem);
   }
   int occ = 1;
   st = occupancy(dev, main_kernel<T, P>(backward, false, false, 0, kScalarBlock), kScalarBlock, &occ);
   if (st != DYT_OK) return st;
-  *out = make_plan(M, N, pc.vec, backward, false, sms, occ, false, false, false, 0, (int64_t)sizeof(T));
+  *out = make_plan(M, N, pc.vec, backward, false, sms, occ, false, false, false, false, 0, (int64_t)sizeof(T));
   if (out->too_big) return DYT_ERR_INVALID_VALUE;
   return DYT_OK;
 }
@@ -598,13 +604,14 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
     // per output offset) and the one-element plans may differ; cover them
     // all. The plans do not depend on P.
     constexpr int V = vec_of<T>();
-    for (int v = -3; v < 2 * V; ++v) {
+    for (int v = -3; v < 3 * V; ++v) {
       Plan p;
-      const dyt_status s = v == -3   ? plan_for<T, float>(M, N, true, true, true, 0, 0, true, &p)
-                           : v == -2 ? plan_for<T, float>(M, N, true, true, false, 0, 0, true, &p)
-                           : v == -1 ? plan_for<T, float>(M, N, false, false, false, 0, 0, true, &p)
-                           : v < V   ? plan_for<T, float>(M, N, false, false, true, v, 0, true, &p)
-                                     : plan_for<T, float>(M, N, false, true, false, v - V, 0, true, &p);
+      const dyt_status s = v == -3    ? plan_for<T, float>(M, N, true, true, true, 0, 0, true, &p)
+                           : v == -2  ? plan_for<T, float>(M, N, true, true, false, 0, 0, true, &p)
+                           : v == -1  ? plan_for<T, float>(M, N, false, false, false, 0, 0, true, &p)
+                           : v < V    ? plan_for<T, float>(M, N, false, false, true, v, 0, true, &p)
+                           : v < 2 * V ? plan_for<T, float>(M, N, false, true, false, v - V, 0, true, &p)
+                                       : plan_for<T, float>(M, N, false, true, false, v - 2 * V, 2, true, &p);
       if (s != DYT_OK) return s;
       if (p.ws_total > need) need = p.ws_total;
     }
@@ -783,7 +790,7 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
   if (st == DYT_OK && !valid_dtype(param_dtype)) st = DYT_ERR_UNSUPPORTED_DTYPE;
   if (st != DYT_OK) return st;
   const int v = 16 / (int)dsize(x_dtype);
-  if (layout < 0 || layout > 3 || (layout >= 2 && (shift < 0 || shift >= v))) return DYT_ERR_INVALID_VALUE;
+  if (layout < 0 || layout > 4 || (layout >= 2 && (shift < 0 || shift >= v))) return DYT_ERR_INVALID_VALUE;
   const int op = backward ? 2 : 1;
   if (M == 0 || N == 0) {
     *out = describe(op, nullptr, 0, 0);
@@ -791,13 +798,15 @@ dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype par
   }
   // layout 0: rows that are not whole 16-byte vectors; 1: contiguous and
   // 16-byte aligned; 2: contiguous, the output `shift` elements past a
-  // boundary; 3: strided rows of whole-vector pitches, the output `shift`
-  // elements past a boundary.
-  const PathChoice pc = choose_path(N, v, layout == 1 || (layout == 3 && shift == 0), layout == 1 || layout == 3,
+  // boundary; 3 / 4: strided rows of whole-vector pitches, the output `shift`
+  // elements past a boundary, every input at its offset (3) or not (4).
+  const bool strided = layout == 3 || layout == 4;
+  const PathChoice pc = choose_path(N, v, layout == 1 || (layout == 3 && shift == 0), layout == 1 || strided,
                                     layout == 1 || layout == 2);
+  const bool wrap = pc.rowframe && layout == 3 && shift > 0 && N % v == 0;
   // The 16-byte kernels always run one CTA per SM.
   Plan p = make_plan(M, N, pc.vec, backward != 0, pc.async, sm_count, pc.async ? 1 : ctas_per_sm, pc.ragged,
-                     pc.shifted, pc.rowframe, layout >= 2 ? shift : 0, (int64_t)dsize(x_dtype));
+                     pc.shifted, pc.rowframe, wrap, layout >= 2 ? shift : 0, (int64_t)dsize(x_dtype));
   if (p.too_big) return DYT_ERR_INVALID_VALUE;
   *out = describe(op, &p, backward ? 2 : 1, backward ? p.ws_total : 0);
   return DYT_OK;

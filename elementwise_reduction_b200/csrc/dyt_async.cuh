@@ -75,7 +75,11 @@ __device__ __forceinline__ void row_frame_columns(int64_t c, int64_t Nc, int64_t
 }
 
 // The elements of a 16-byte vector whose bit is set in m, one by one: the
-// vectors that straddle the start or the end of a packed matrix.
+// vectors that hold padding (a packed matrix's straddling vector, the shifted
+// layouts' partial vectors). Its masks are runs of set bits; storing a run as
+// aligned 8-, 4- and 2-byte pieces (a loop, or straight-line code) made the
+// kernels slower: the flat shifted backward on 16384 x 4096 bf16 one element
+// off 76.6 -> 85.0 us, the row frame's forward 63.8 -> 83.1 us.
 template <typename T, int VEC>
 __device__ __forceinline__ void store_mask(T *p, const uint4 &r, uint32_t m) {
 #pragma unroll
@@ -150,16 +154,42 @@ __device__ __forceinline__ void copy_chunk_checked(uint4 *slot, const char *a, u
 // (fast), checked ones elsewhere.
 // W: the kernel cuts windows out of this input (its offset may differ from
 // the output's); without W its vectors are single chunks (d = 0).
+// wb (row frame, wrapped vector-column only; W is then false): the second
+// chunk lies wb bytes after the first (the row's last elements).
 template <typename T, int B, bool W>
-__device__ __forceinline__ void copy_shifted(uint4 *slot, const T *src, const ShIn &s, bool fast) {
+__device__ __forceinline__ void copy_shifted(uint4 *slot, const T *src, const ShIn &s, bool fast,
+                                             uintptr_t wb = 0) {
   const char *a = reinterpret_cast<const char *>(src);
   if (fast) {
     cp_async16(slot, a);
     if (W && s.d) cp_async16(slot + B, a + 16);
+    if (!W && wb) cp_async16(slot + B, a + wb);
   } else {
     copy_chunk_checked<(int)sizeof(T)>(slot, a, s.lo, s.hi);
     if (W && s.d) copy_chunk_checked<(int)sizeof(T)>(slot + B, a + 16, s.lo, s.hi);
+    if (!W && wb) copy_chunk_checked<(int)sizeof(T)>(slot + B, a + wb, s.lo, s.hi);
   }
+}
+
+// The row frame's wrapped vector-column (SHM bit 4: N a multiple of VEC, every
+// tensor at the output's offset sh > 0): vector-column 0 of a row holds the
+// row's last sh elements at positions 0 .. sh - 1 (from the chunk N elements
+// on, the slot's second half) and its first VEC - sh at positions sh .. VEC - 1
+// (the first half), so a row spans N / VEC vectors as if it were aligned.
+// m: the bytes of positions 0 .. sh - 1.
+__device__ __forceinline__ uint4 wrap_bytes_mask(int sh, int es) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int nb = sh * es - 4 * i;  // bytes of this word below the cut
+    w[i] = nb >= 4 ? 0xFFFFFFFFu : nb <= 0 ? 0u : (1u << (8 * nb)) - 1u;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ uint4 read_wrapped(const uint4 *slot, int B, const uint4 &m) {
+  const uint4 a = slot[0], b = slot[B];
+  return make_uint4((a.x & ~m.x) | (b.x & m.x), (a.y & ~m.y) | (b.y & m.y), (a.z & ~m.z) | (b.z & m.z),
+                    (a.w & ~m.w) | (b.w & m.w));
 }
 
 // The input vector of a row from its slot: with W, bytes [d, d + 16) of its
@@ -320,14 +350,16 @@ __device__ __forceinline__ int last_vector_real(const Geom &g, int64_t first, in
 // past a tensor's ends handled one by one (checked copies, masked stores).
 // SHM bit 1: x's offset differs from y's, so its vectors are cut out of two
 // chunks. SHM bit 3: the row frame (RF) instead of the flat packed layout:
-// strided rows, each laid out on its own from position sh (see row_frame_*).
+// strided rows, each laid out on its own from position sh (see row_frame_*);
+// bit 4 (WR): with its wrapped vector-column (see read_wrapped).
 template <typename T, typename P, int VEC, int B, int S, bool PK, int SHM>
 __global__ void __launch_bounds__(B, 1)
     dyt_fwd_async_kernel(const T *__restrict__ x, const P *__restrict__ alpha_p, const P *__restrict__ gamma_p,
                          const P *__restrict__ beta_p, ParamTypes pt, T *y, Geom g) {
   using IO = VecIO<T, VEC>;
-  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0, RF = (SHM & 8) != 0;
+  constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0, RF = (SHM & 8) != 0, WR = (SHM & 16) != 0;
   constexpr bool FL = SH && !RF;  // the flat shifted layout
+  static_assert(!WR || (RF && !WX), "the wrapped column: row frame, inputs at the output's offset");
   static_assert(VEC * sizeof(T) == 16, "16-byte vectors");
   static_assert(PK == FL || (PK && !SH), "the flat shifted kernels use the packed layout, the row frame does not");
   constexpr int CH = SH ? 2 : 1;  // 16-byte chunks per slot
@@ -372,24 +404,31 @@ __global__ void __launch_bounds__(B, 1)
     // RF: the real elements of the thread's vectors are the same in every row
     const uint32_t rmask = RF ? shifted_mask<VEC>(g, c0) : 0xFFu;
     const bool rstore = !RF || rmask == (1u << VEC) - 1u;
+    // WR: vector-column 0 is the wrapped one; its second chunk lies N on
+    const bool wrap = WR && cv == 0;
+    const int64_t wn = wrap ? g.Nc : 0;
+    const uint4 wm = wrap_bytes_mask(WR ? g.sh : 0, (int)sizeof(T));
+    const uint32_t wlo = ~((1u << g.sh) - 1u) & ((1u << VEC) - 1u), whi = (1u << g.sh) - 1u;
     if constexpr (SH) {
       while (k_lo < n && !((RF || pos0 + k_lo * dpos >= g.sh) && shifted_lo_ok(ix, px + k_lo * sx))) ++k_lo;
       while (k_hi > k_lo &&
-             !((RF || pos0 + (k_hi - 1) * dpos + VEC <= g.total) && shifted_hi_ok(ix, px + (k_hi - 1) * sx)))
+             !((RF || pos0 + (k_hi - 1) * dpos + VEC <= g.total) && shifted_hi_ok(ix, px + (k_hi - 1) * sx + wn)))
         --k_hi;
     }
     // Rows first, parameters second: the parameter loads overlap the copies.
 #pragma unroll
     for (int k = 0; k < S - 1; ++k) {
       if (k < n) {
-        if constexpr (SH) copy_shifted<T, B, WX>(slot0 + k * CH * B, px + k * sx, ix, fast_row(k, k_lo, k_hi));
+        if constexpr (SH)
+          copy_shifted<T, B, WX>(slot0 + k * CH * B, px + k * sx, ix, fast_row(k, k_lo, k_hi), wn * sizeof(T));
         else if (PK) cp_async16_zfill(slot0 + k * B, px + k * sx, k == n - 1 ? last_bytes : 16u);
         else cp_async16(slot0 + k * B, px + k * sx);
       }
       cp_async_commit();
     }
     int64_t col[VEC];
-    if constexpr (RF) row_frame_columns<VEC>(c0 - g.sh, g.Nc, col);
+    if constexpr (WR) vector_columns<VEC, true>(c0 - g.sh, g.Nc, col);  // (c0 + e - sh) mod N
+    else if constexpr (RF) row_frame_columns<VEC>(c0 - g.sh, g.Nc, col);
     else vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
     float gam[VEC], bet[VEC], bth[VEC];
     fwd_params_at<T, VEC, P>(gamma_p, beta_p, pt, col, gam, bet, bth);
@@ -403,12 +442,17 @@ __global__ void __launch_bounds__(B, 1)
         constexpr bool CHK = decltype(chk)::value;
         const int64_t kn = k + S - 1;
         if (!CHK || kn < n)
-          copy_shifted<T, B, WX>(slot0 + s_wr * CH * B, px + kn * sx, ix, !CHK || fast_row((int)kn, k_lo, k_hi));
+          copy_shifted<T, B, WX>(slot0 + s_wr * CH * B, px + kn * sx, ix, !CHK || fast_row((int)kn, k_lo, k_hi),
+                                 wn * sizeof(T));
         cp_async_commit();
         cp_async_wait<S - 1>();
-        const typename IO::Raw ry =
-            fwd_vector<T, VEC>(read_shifted<B, WX>(slot0 + s_rd * CH * B, ix), alpha, gam, bet, bth);
-        if (!rstore) store_mask<T, VEC>(py, ry, rmask);  // RF: the row's padding is not stored
+        const uint4 v = WR && wrap ? read_wrapped(slot0 + s_rd * CH * B, B, wm)
+                                   : read_shifted<B, WX>(slot0 + s_rd * CH * B, ix);
+        const typename IO::Raw ry = fwd_vector<T, VEC>(v, alpha, gam, bet, bth);
+        if (WR && wrap) {  // the row's first VEC - sh elements, then its last sh
+          store_mask<T, VEC>(py, ry, wlo);
+          store_mask<T, VEC>(py + g.Nc, ry, whi);
+        } else if (!rstore) store_mask<T, VEC>(py, ry, rmask);  // RF: the row's padding is not stored
         else if (RF || !CHK || fast_row((int)k, k_lo, k_hi)) IO::store_raw(py, ry);
         else store_mask<T, VEC>(py, ry, shifted_mask<VEC>(g, pos0 + k * dpos));  // padding: not stored
         py += sy;
@@ -482,7 +526,7 @@ __global__ void __launch_bounds__(B, 1)
 
 // SHM != 0: as the forward's shifted kernels, x and dy each with their own
 // offset: bit 1 cuts x's vectors out of two chunks, bit 2 dy's; bit 3 the row
-// frame.
+// frame, bit 4 its wrapped vector-column.
 template <typename T, typename P, int VEC, int B, int S, bool PK, int SHM>
 __global__ void __launch_bounds__(B, 1)
     dyt_bwd_async_kernel(const T *__restrict__ x, const T *__restrict__ dy, const P *__restrict__ alpha_p,
@@ -490,7 +534,9 @@ __global__ void __launch_bounds__(B, 1)
                          double *__restrict__ part_db, double *__restrict__ part_da, Geom g) {
   using IO = VecIO<T, VEC>;
   constexpr bool SH = SHM != 0, WX = (SHM & 2) != 0, WD = (SHM & 4) != 0, RF = (SHM & 8) != 0;
+  constexpr bool WR = (SHM & 16) != 0;
   constexpr bool FL = SH && !RF;  // the flat shifted layout
+  static_assert(!WR || (RF && !WX && !WD), "the wrapped column: row frame, inputs at the output's offset");
   constexpr bool EXACT_G = ExactGamma<T>::value;
   constexpr int kRunBlocks = kGammaRunRows / S;  // unrolled blocks of S rows per binary32 dgamma run
   constexpr int CH = SH ? 2 : 1;                 // 16-byte chunks per slot
@@ -562,12 +608,19 @@ __global__ void __launch_bounds__(B, 1)
       // RF: the real elements of the thread's vectors are the same in every row
       const uint32_t rmask = RF ? shifted_mask<VEC>(g, c0) : 0xFFu;
       const bool rstore = !RF || rmask == (1u << VEC) - 1u;
+      // WR: vector-column 0 is the wrapped one; its second chunk lies N on
+      const bool wrap = WR && cv == 0;
+      const int64_t wn = wrap ? g.Nc : 0;
+      const uintptr_t wb = (uintptr_t)wn * sizeof(T);
+      const uint4 wm = wrap_bytes_mask(WR ? g.sh : 0, (int)sizeof(T));
+      const uint32_t wlo = ~((1u << g.sh) - 1u) & ((1u << VEC) - 1u), whi = (1u << g.sh) - 1u;
       if constexpr (SH) {
         while (k_lo < nn && !((RF || pos0 + k_lo * dpos >= g.sh) && shifted_lo_ok(ix, px + k_lo * sx) &&
                               shifted_lo_ok(id, pd + k_lo * sd)))
           ++k_lo;
-        while (k_hi > k_lo && !((RF || pos0 + (k_hi - 1) * dpos + VEC <= g.total) &&
-                                shifted_hi_ok(ix, px + (k_hi - 1) * sx) && shifted_hi_ok(id, pd + (k_hi - 1) * sd)))
+        while (k_hi > k_lo &&
+               !((RF || pos0 + (k_hi - 1) * dpos + VEC <= g.total) && shifted_hi_ok(ix, px + (k_hi - 1) * sx + wn) &&
+                 shifted_hi_ok(id, pd + (k_hi - 1) * sd + wn)))
           --k_hi;
       }
       // Rows first, parameters second: the gamma loads overlap the copies.
@@ -578,8 +631,8 @@ __global__ void __launch_bounds__(B, 1)
         if (k < nn) {
           if constexpr (SH) {
             const bool fast = fast_row(k, k_lo, k_hi);
-            copy_shifted<T, B, WX>(slot0 + (2 * k) * CH * B, px, ix, fast);
-            copy_shifted<T, B, WD>(slot0 + (2 * k + 1) * CH * B, pd, id, fast);
+            copy_shifted<T, B, WX>(slot0 + (2 * k) * CH * B, px, ix, fast, wb);
+            copy_shifted<T, B, WD>(slot0 + (2 * k + 1) * CH * B, pd, id, fast, wb);
           } else if (PK) {
             const uint32_t b = k == nn - 1 ? last_bytes : 16u;
             cp_async16_zfill(slot0 + (2 * k) * B, px, b);
@@ -594,7 +647,8 @@ __global__ void __launch_bounds__(B, 1)
         cp_async_commit();
       }
       int64_t col[VEC];
-      if constexpr (RF) row_frame_columns<VEC>(c0 - g.sh, g.Nc, col);
+      if constexpr (WR) vector_columns<VEC, true>(c0 - g.sh, g.Nc, col);  // (c0 + e - sh) mod N
+      else if constexpr (RF) row_frame_columns<VEC>(c0 - g.sh, g.Nc, col);
       else vector_columns<VEC, PK>(SH ? c0 - g.sh : c0, g.Nc, col);
       load_params<VEC, P>(gamma_p, pt.gamma, col, 4.0f, gam);  // 4 gamma (see bwd_vector)
       int run = 0;  // blocks in the current binary32 dgamma run
@@ -673,8 +727,8 @@ __global__ void __launch_bounds__(B, 1)
               const int sw = (j + S - 1) % S;
               if constexpr (SH) {
                 const bool fast = !CHK || fast_row(k + S - 1, k_lo, k_hi);
-                copy_shifted<T, B, WX>(slot0 + (2 * sw) * CH * B, px, ix, fast);
-                copy_shifted<T, B, WD>(slot0 + (2 * sw + 1) * CH * B, pd, id, fast);
+                copy_shifted<T, B, WX>(slot0 + (2 * sw) * CH * B, px, ix, fast, wb);
+                copy_shifted<T, B, WD>(slot0 + (2 * sw + 1) * CH * B, pd, id, fast, wb);
               } else if (PK) {
                 const uint32_t b = k + S - 1 == nn - 1 ? last_bytes : 16u;
                 cp_async16_zfill(slot0 + (2 * sw) * B, px, b);
@@ -689,15 +743,38 @@ __global__ void __launch_bounds__(B, 1)
             cp_async_commit();
             cp_async_wait<S - 1>();
             typename IO::Raw rx, rd;
-            if constexpr (SH) {
+            if constexpr (WR) {
+              if (wrap) {
+                rx = read_wrapped(slot0 + (2 * j) * CH * B, B, wm);
+                rd = read_wrapped(slot0 + (2 * j + 1) * CH * B, B, wm);
+              } else {
+                rx = *(slot0 + (2 * j) * CH * B);
+                rd = *(slot0 + (2 * j + 1) * CH * B);
+              }
+            } else if constexpr (SH) {
               rx = read_shifted<B, WX>(slot0 + (2 * j) * CH * B, ix);
               rd = read_shifted<B, WD>(slot0 + (2 * j + 1) * CH * B, id);
             } else {
               rx = *(const typename IO::Raw *)(slot0 + (2 * j) * B);
               rd = *(const typename IO::Raw *)(slot0 + (2 * j + 1) * B);
             }
-            if (!rstore) {  // RF: the row's padding is dropped
-              store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, rmask), rmask);
+            if constexpr (RF) {
+              // One computation for every thread, masked by the thread's own
+              // mask (the wrapped vector-column holds no padding), so that no
+              // warp runs it twice for its partial vectors: on 16384 x 4096
+              // bf16, pitch 4104, every tensor one element off, warp 0
+              // computing twice held the other warps at the item's barrier
+              // (ncu: barrier stalls 2.58 per issue against 0.07; 127 -> 98 us
+              // with one computation). Only the stores differ.
+              const typename IO::Raw o = bwd_vector<T, VEC, !WR, EXACT_G>(rx, rd, alpha, gam, acc, ca, rmask);
+              if (WR && wrap) {  // the row's first VEC - sh elements, then its last sh
+                store_mask<T, VEC>(pdx, o, wlo);
+                store_mask<T, VEC>(pdx + g.Nc, o, whi);
+              } else if (!rstore) {
+                store_mask<T, VEC>(pdx, o, rmask);  // the row's padding is dropped
+              } else {
+                IO::store_raw(pdx, o);
+              }
             } else if (FL && CHK && !fast_row(k, k_lo, k_hi)) {  // padding of the shifted layout: dropped
               const uint32_t m = shifted_mask<VEC>(g, pos0 + k * dpos);
               store_mask<T, VEC>(pdx, bwd_vector<T, VEC, true, EXACT_G>(rx, rd, alpha, gam, acc, ca, m), m);
@@ -741,7 +818,7 @@ __global__ void __launch_bounds__(B, 1)
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
           const int64_t q = c0 + e;
-          if constexpr (RF) {
+          if constexpr (RF && !WR) {
             if (q >= g.sh && q - g.sh < g.Nc) {
               pg[q - g.sh] = ag[e];
               pb[q - g.sh] = acc.b[e];
@@ -757,7 +834,7 @@ __global__ void __launch_bounds__(B, 1)
       __syncthreads();  // every thread's ring is drained: reuse it for the reduction
       if ((32 % g.NV) == 0) {
         // the chunk's columns start at 0 on the row-tiled path (one chunk)
-        lane_reduce_warps<VEC, B, RF ? 2 : SH ? 1 : 0>(ag, acc.b, red, g, ln, 0, pg, pb);
+        lane_reduce_warps<VEC, B, RF && !WR ? 2 : SH ? 1 : 0>(ag, acc.b, red, g, ln, 0, pg, pb);
       } else {  // dgamma and dbeta sums in one tree: 2 VEC values per thread
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
@@ -770,7 +847,7 @@ __global__ void __launch_bounds__(B, 1)
 #pragma unroll
           for (int e = 0; e < VEC; ++e) {
             const int64_t q = c0 + e;
-            if constexpr (RF) {
+            if constexpr (RF && !WR) {
               if (q >= g.sh && q - g.sh < g.Nc) {
                 pg[q - g.sh] = red[e * B + threadIdx.x];
                 pb[q - g.sh] = red[(VEC + e) * B + threadIdx.x];

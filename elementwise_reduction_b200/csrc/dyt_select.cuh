@@ -49,7 +49,7 @@ using BwdKernel = void (*)(const T *, const T *, const P *, const P *, ParamType
 // The forward kernel of a plan: the 16-byte kernels (aligned, packed or
 // shifted) or the one-element kernel. shm: the shifted kernels' mode (0 = not
 // shifted; else 1, | 2 when x's vectors are cut out of two chunks, | 8 for the
-// row frame).
+// row frame, | 16 for its wrapped vector-column).
 template <typename T, typename P>
 FwdKernel<T, P> fwd_kernel_of(bool async, bool packed, int shm);
 

@@ -21,6 +21,7 @@ FwdKernel<T, P> fwd_kernel_of(bool async, bool packed, int shm) {
     case 3: return dyt_fwd_async_kernel<T, P, V, B, S, true, 3>;
     case 9: return dyt_fwd_async_kernel<T, P, V, B, S, false, 9>;
     case 11: return dyt_fwd_async_kernel<T, P, V, B, S, false, 11>;
+    case 25: return dyt_fwd_async_kernel<T, P, V, B, S, false, 25>;
   }
   return packed ? dyt_fwd_async_kernel<T, P, V, B, S, true, 0> : dyt_fwd_async_kernel<T, P, V, B, S, false, 0>;
 }
@@ -35,6 +36,7 @@ BwdKernel<T, P> bwd_async_of(bool packed, int shm) {
     case 9: return dyt_bwd_async_kernel<T, P, V, B, S, false, 9>;
     case 11: return dyt_bwd_async_kernel<T, P, V, B, S, false, 11>;
     case 15: return dyt_bwd_async_kernel<T, P, V, B, S, false, 15>;
+    case 25: return dyt_bwd_async_kernel<T, P, V, B, S, false, 25>;
   }
   return packed ? dyt_bwd_async_kernel<T, P, V, B, S, true, 0> : dyt_bwd_async_kernel<T, P, V, B, S, false, 0>;
 }

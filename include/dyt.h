@@ -299,7 +299,11 @@ typedef struct dyt_launch_info {
   int shifted;       /* 1 = the flat shifted 16-byte kernels (adjacent rows, tensors not all
                         16-byte aligned); 2 = the row frame (strided rows whose pitches are
                         whole 16-byte vectors, tensors not all 16-byte aligned or N not a
-                        multiple of vec: each row shifted on its own); 0 otherwise */
+                        multiple of vec: each row shifted on its own); 3 = the row frame
+                        with a wrapped first vector-column (N a multiple of vec, every
+                        tensor shift elements off: the first vector of a row also holds
+                        its last shift elements, so a row spans N / vec vectors); 0
+                        otherwise */
   int shift;         /* shifted kernels: the output's offset past a 16-byte boundary, in
                         elements (0 .. vec - 1); 0 otherwise */
   int64_t workspace_bytes;
@@ -315,14 +319,15 @@ dyt_status dyt_last_launch_info(dyt_launch_info *out);
  * 1 = contiguous and 16-byte aligned (a ragged N gets the packed form,
  * out->pack_rows > 1), 2 = contiguous with the output `shift` elements past a
  * 16-byte boundary (the shifted kernels), 3 = strided rows (pitches not N)
- * whose pitches are whole 16-byte vectors, the output `shift` elements past a
- * 16-byte boundary (the row frame unless shift is 0 and N a multiple of vec;
- * `shift` is read for layouts 2 and 3 only).
+ * whose pitches are whole 16-byte vectors, every tensor `shift` elements past
+ * a 16-byte boundary (the row frame unless shift is 0 and N a multiple of
+ * vec), 4 = as 3 with the inputs at other offsets than the output (`shift`
+ * is read for layouts 2 to 4 only).
  * Host arithmetic only: touches no device, so the planning is testable
  * without a GPU. out->kernels is the number of kernels the call would launch
  * and out->workspace_bytes the workspace it needs.
  * Errors: as the shape checks of dyt_forward, or DYT_ERR_INVALID_VALUE for
- * out == NULL, sm_count / ctas_per_sm < 1, a layout outside 0..3 or a shift
+ * out == NULL, sm_count / ctas_per_sm < 1, a layout outside 0..4 or a shift
  * outside 0 .. 16 / element size - 1.
  */
 dyt_status dyt_plan_query(int64_t M, int64_t N, dyt_dtype x_dtype, dyt_dtype param_dtype,

@@ -125,7 +125,8 @@ def test_pointers_must_hold_whole_elements():
                                     (100003, 255, 0), (16384, 4096, 1), (32768, 8192, 1), (1, 1, 0),
                                     (3, 70000, 2), (10**7, 8, 1), (5, 513, 0), (7, 3, 1), (1, 17, 0),
                                     (100003, 4097, 1), (4099, 1001, 0)])
-@pytest.mark.parametrize("layout,shift", [(0, 0), (1, 0), (2, 0), (2, 1), (2, -1), (3, 0), (3, 1), (3, -1)])
+@pytest.mark.parametrize("layout,shift", [(0, 0), (1, 0), (2, 0), (2, 1), (2, -1), (3, 0), (3, 1), (3, -1),
+                                          (4, 0), (4, 1)])
 @pytest.mark.parametrize("sms,occ", [(148, 1), (148, 2), (7, 1)])
 def test_launch_plan_invariants(M, N, xd, layout, shift, sms, occ):
     dyt = _lib()
@@ -136,12 +137,15 @@ def test_launch_plan_invariants(M, N, xd, layout, shift, sms, occ):
     pk = p["pack_rows"]
     # strided rows of whole-vector pitches, off a boundary or of a ragged N:
     # the row frame
-    rf = layout == 3 and (sh != 0 or N % (16 // size) != 0)
+    rf = layout == 4 or (layout == 3 and (sh != 0 or N % (16 // size) != 0))
+    # every tensor at the output's offset sh > 0 and N a multiple of the
+    # vector: the first vector-column also holds each row's last sh elements
+    wrap = layout == 3 and sh != 0 and N % (16 // size) == 0
     # adjacent rows always take the 16-byte kernels (packed when N is ragged);
     # tensors off 16-byte boundaries the shifted ones; strided rows of
     # whole-vector pitches too
     assert bool(p["async_stages"]) == (layout != 0)
-    assert p["shifted"] == (2 if rf else 1 if layout == 2 else 0) and p["shift"] == sh
+    assert p["shifted"] == (3 if wrap else 2 if rf else 1 if layout == 2 else 0) and p["shift"] == sh
     if p["async_stages"]:    # per-thread copy ring: 16-byte vectors, one per thread
         assert vec == 16 // size
         # a ragged N on adjacent rows is streamed in packs of vec rows (exactly
@@ -152,7 +156,7 @@ def test_launch_plan_invariants(M, N, xd, layout, shift, sms, occ):
         assert vec == 1 and pk == 1
         ctas = sms * occ
     # pitch of a (packed) row; the row frame: a row's vectors from position sh
-    Np = -(-(N + sh) // vec) * vec if rf else pk * N
+    Np = N if wrap else -(-(N + sh) // vec) * vec if rf else pk * N
     Mp = -(-(M * N + sh) // Np) if layout == 2 else -(-M // pk)  # (packed) rows; shifted: the matrix from position sh
     nv = Np // vec
     B = p["block"]

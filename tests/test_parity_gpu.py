@@ -439,7 +439,7 @@ def _placed_rows(src, M: int, N: int, off: int, ld: int, fill: float) -> tuple:
 
 @pytest.mark.parametrize("xd", ["f32", "bf16"])
 @pytest.mark.parametrize("N", [1, 3, 17, 100, 255, 520, 4099])
-@pytest.mark.parametrize("hx,hd,ho", [(0, 0, 0), (1, 1, 1), (0, 3, 1), (-1, 0, 2), (2, -1, -1)])
+@pytest.mark.parametrize("hx,hd,ho", [(0, 0, 0), (1, 1, 1), (-3, -3, -3), (0, 3, 1), (-1, 0, 2), (2, -1, -1)])
 def test_row_frame_rows(xd, N, hx, hd, ho):
     # Strided rows whose pitches are whole 16-byte vectors, with tensors off
     # 16-byte boundaries or a ragged N: each row shifted on its own. NaN
@@ -472,7 +472,11 @@ def test_row_frame_rows(xd, N, hx, hd, ho):
     info_b = dyt.dyt_last_launch_info()
     torch.cuda.synchronize()
     assert (ybuf[ymask] == 7).all() and (dxbuf[dxmask] == 7).all()  # nothing outside the rows is written
-    assert info_f["shifted"] == info_b["shifted"] == 2 and info_f["shift"] == info_b["shift"] == ho
+    # every tensor at the output's offset sh > 0 and N a multiple of vec: the
+    # first vector-column also holds each row's last sh elements (3)
+    assert info_f["shifted"] == (3 if hx == ho and ho and N % vec == 0 else 2)
+    assert info_b["shifted"] == (3 if hx == hd == ho and ho and N % vec == 0 else 2)
+    assert info_f["shift"] == info_b["shift"] == ho
     assert info_f["vec"] == info_b["vec"] == vec
     out = {"y": H.to_numpy(y.contiguous(), xd), "dx": H.to_numpy(dx.contiguous(), xd),
            "dgamma": H.to_numpy(dgamma, "f32"), "dbeta": H.to_numpy(dbeta, "f32"), "dalpha": float(dalpha.item())}
@@ -760,8 +764,9 @@ def test_unaligned_variant_full_size(name):
                            pitch=w.pitch)
     if w.pitch and (w.pitch * (4 if w.x_dtype == "f32" else 2)) % 16:
         assert info["fwd"]["vec"] == info["bwd"]["vec"] == 1
-    elif w.pitch:  # whole-vector pitches: the row frame
-        assert info["fwd"]["shifted"] == 2 and info["bwd"]["shifted"] == 2
+    elif w.pitch:  # whole-vector pitches: the row frame (3: with the wrapped first vector-column)
+        wrapped = w.offset and w.x_off == w.offset and w.N % (4 if w.x_dtype == "f32" else 8) == 0
+        assert info["fwd"]["shifted"] == info["bwd"]["shifted"] == (3 if wrapped else 2)
         assert info["fwd"]["shift"] == info["bwd"]["shift"] == w.offset
     else:
         assert info["fwd"]["shifted"] == 1 and info["bwd"]["shifted"] == 1

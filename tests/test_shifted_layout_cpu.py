@@ -165,20 +165,26 @@ def _round_up(a, b):
 def replay_rowframe(dyt, M, N, xd, offs, lds, backward, sms=3):
     """The row frame: strided rows whose pitches are whole 16-byte vectors,
     each row laid out on its own from position sh (the output's offset) of a
-    row of ceil((N + sh) / vec) vectors. offs / lds: each tensor's offset past
-    a 16-byte boundary and its pitch, in elements."""
+    row of ceil((N + sh) / vec) vectors; with N a multiple of vec, sh > 0 and
+    every input at the output's offset, of N / vec vectors, the first one also
+    holding the row's last sh elements at its positions 0 .. sh - 1 (the
+    wrapped vector-column). offs / lds: each tensor's offset past a 16-byte
+    boundary and its pitch, in elements."""
     es = 4 if xd == 0 else 2
     vec = 16 // es
     ho = offs["o"]
-    p = dyt.dyt_plan_query(M, N, xd, 0, int(backward), 3, sms, 1, shift=ho)
+    ins = ["x", "dy"] if backward else ["x"]
+    layout = 3 if all(offs[m] == ho for m in ins) else 4
+    p = dyt.dyt_plan_query(M, N, xd, 0, int(backward), layout, sms, 1, shift=ho)
+    wrap = p["shifted"] == 3
+    assert wrap == (layout == 3 and ho > 0 and N % vec == 0)
     if ho or N % vec:
-        assert p["shifted"] == 2 and p["shift"] == ho and p["pack_rows"] == 1
+        assert p["shifted"] in (2, 3) and p["shift"] == ho and p["pack_rows"] == 1
     B, RL, ncc, nrg, grid = (p[k] for k in ("block", "row_lanes", "col_chunks", "row_groups", "grid"))
-    NV = _cdiv(N + ho, vec)           # vectors of a row's frame
+    NV = N // vec if wrap else _cdiv(N + ho, vec)  # vectors of a row's frame
     assert ncc == (1 if RL > 1 else _cdiv(NV, B))
     gq, grem = M // nrg, M % nrg
     cw = _chunk_width(B, RL, ncc, NV)
-    ins = ["x", "dy"] if backward else ["x"]
     bases = {"x": 1 << 24, "dy": 2 << 24, "o": 3 << 24}
     lo = {k: bases[k] + offs[k] * es for k in bases}    # row 0 of each tensor
     for k in bases:
@@ -205,9 +211,14 @@ def replay_rowframe(dyt, M, N, xd, offs, lds, backward, sms=3):
                 first = rb + rl
                 n = 0 if first >= re else _cdiv(re - first, RL)
                 assert n <= 2048
-                mask = [ho <= c0 + e < N + ho for e in range(vec)]
+                w = wrap and cv == 0
+                if w:  # positions 0 .. ho - 1: the row's last ho columns
+                    mask = [True] * vec
+                    cols = [(c0 + e - ho) % N for e in range(vec)]
+                else:
+                    mask = [ho <= c0 + e < N + ho for e in range(vec)]
+                    cols = [min(max(c0 + e - ho, 0), N - 1) for e in range(vec)]
                 assert any(mask)
-                cols = [min(max(c0 + e - ho, 0), N - 1) for e in range(vec)]
                 # the tensors' spans, first element to last: the copies may read
                 # the bytes between rows, never outside a span
                 span = {m: (lo[m], lo[m] + ((M - 1) * lds[m] + N) * es) for m in ins}
@@ -215,9 +226,12 @@ def replay_rowframe(dyt, M, N, xd, offs, lds, backward, sms=3):
                 def chunk(k, m):
                     return frame[m][0] + c0 * es + (first + k * RL) * lds[m] * es
 
+                def chunks(k, m):
+                    a = chunk(k, m)
+                    return [a] + ([a + 16] if frame[m][1] else []) + ([a + N * es] if w else [])
+
                 def ok(k):
-                    return all(chunk(k, m) >= span[m][0] and chunk(k, m) + (32 if frame[m][1] else 16) <= span[m][1]
-                               for m in ins)
+                    return all(chunks(k, m)[0] >= span[m][0] and chunks(k, m)[-1] + 16 <= span[m][1] for m in ins)
 
                 k_lo = 0
                 while k_lo < n and not ok(k_lo):
@@ -235,7 +249,8 @@ def replay_rowframe(dyt, M, N, xd, offs, lds, backward, sms=3):
                         a, d = chunk(k, m), frame[m][1]
                         assert a % 16 == 0
                         bytes_ = set()
-                        for ca in ([a, a + 16] if d else [a]):
+                        for ca in chunks(k, m):
+                            assert ca % 16 == 0
                             if k_lo <= k < k_hi:
                                 bytes_.update(range(ca, ca + 16))
                             elif ca >= shi or ca + 16 <= slo:
@@ -248,20 +263,25 @@ def replay_rowframe(dyt, M, N, xd, offs, lds, backward, sms=3):
                         assert all(slo <= b < shi for b in bytes_), ("read outside the tensor", m)
                         got[m] = (a + d, rlo, bytes_)
                     out_row = lo["o"] + row * lds["o"] * es
+                    out_frame = (lo["o"] - ho * es) + row * lds["o"] * es
                     for e in range(vec):
                         if not mask[e]:
                             continue  # the row's padding: neither stored nor summed
-                        col = c0 + e - ho
-                        assert (lo["o"] - ho * es) + row * lds["o"] * es + (c0 + e) * es == out_row + col * es
+                        col = cols[e]
+                        tail = w and e < ho  # stored N elements on, from the second chunk
+                        assert out_frame + (c0 + e + (N if tail else 0)) * es == out_row + col * es
                         assert (row, col) not in stored, "stored twice"
                         stored.add((row, col))
-                        assert cols[e] == col
+                        if not w:
+                            assert col == c0 + e - ho
                         for m in ins:
                             start, rlo, bytes_ = got[m]
-                            for b in range(start + e * es, start + (e + 1) * es):
+                            src = start + (N * es if tail else 0) + e * es
+                            for b in range(src, src + es):
                                 assert b in bytes_, "an input byte was not copied"
                                 assert (b - rlo) // es == col
-                        assert c0 + e - ho == col  # partial-sum slot: the column itself
+                        # partial-sum slot: (position - sh) mod N, the column itself
+                        assert (c0 + e - ho) % N == col
     assert len(stored) == M * N
 
 

@@ -565,6 +565,24 @@ def test_backward_in_cuda_graph_replays_and_with_garbage_workspace(M, N, xd):
     assert info["kernels"] == 2
 
 
+@pytest.mark.parametrize("xd", [0, 1, 2])
+def test_workspace_bytes_cover_every_vectorised_plan(xd):
+    # The size query must cover the plan of every layout a call can have:
+    # aligned, shifted (each output offset) and the row frame (wrapped or not).
+    from tests.test_abi_cpu import _lib
+    lib = _lib()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    vec = 4 if xd == 0 else 8
+    for M in (1, 3, 1000, 65537, 100003):
+        for N in (1, 3, 8, 17, 32, 100, 255, 256, 513, 4096, 4099, 8192):
+            need = lib.dyt_backward_workspace_bytes(M, N, xd, 0)
+            assert need > 0
+            for layout in (1, 2, 3, 4):
+                for shift in (range(vec) if layout >= 2 else [0]):
+                    p = lib.dyt_plan_query(M, N, xd, 0, 1, layout, sms, 1, shift=shift)
+                    assert p["workspace_bytes"] <= need, (M, N, layout, shift)
+
+
 def test_workspace_errors():
     import elementwise_reduction_b200 as dyt
     M, N = 100, 64

@@ -397,8 +397,8 @@ __global__ void __launch_bounds__(B, 1)
     const T *px = xb + first * g.ldx + c0;
     T *py = yb + first * g.ldo + c0;
     // SH: rows [k_lo, k_hi) copy whole chunks (and FL: store whole vectors);
-    // the others (at most a few at each end of the matrix) copy element by
-    // element.
+    // the others (at most a few at each end of the matrix; RF: the tensor's
+    // first and last rows) copy element by element.
     const int64_t pos0 = first * g.N + c0, dpos = (int64_t)g.RL * g.N;  // layout positions
     int k_lo = 0, k_hi = (int)n;  // n is at most kMaxRowsPerLane
     // RF: the real elements of the thread's vectors are the same in every row
@@ -601,8 +601,9 @@ __global__ void __launch_bounds__(B, 1)
       const T *px = xb + first * g.ldx + c0;  // the next rows to copy (advanced, not re-derived)
       const T *pd = db + first * g.ldd + c0;
       T *pdx = dxb + first * g.ldo + c0;
-      // SH: rows [k_lo, k_hi) copy and store whole vectors; the others (at
-      // most a few at each end of the matrix) go element by element.
+      // SH: rows [k_lo, k_hi) copy whole chunks (and FL: store whole
+      // vectors); the others (at most a few at each end of the matrix; RF:
+      // the tensors' first and last rows) copy element by element.
       const int64_t pos0 = first * g.N + c0, dpos = (int64_t)g.RL * g.N;  // layout positions
       int k_lo = 0, k_hi = nn;
       // RF: the real elements of the thread's vectors are the same in every row

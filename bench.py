@@ -144,9 +144,12 @@ def record_traffic(csv_path: str, workload: str, command: str) -> None:
     entry = {k: {"bytes_per_launch": v / len(launches[k]), "launches": len(launches[k]),
                  "source_hash": kernel_source_hash(), "command": command} for k, v in per.items()}
     if "dyt_bwd_kernel" in entry and "dyt_finalize_kernel" in entry:
+        # one backward call: its stage-1 launches (one per phase of a strided
+        # call whose pitches are not whole vectors, else one) and its finalize
+        calls = len(launches["dyt_finalize_kernel"])
         entry["dyt_backward"] = {
-            "bytes_per_launch": entry["dyt_bwd_kernel"]["bytes_per_launch"]
-            + entry["dyt_finalize_kernel"]["bytes_per_launch"],
+            "bytes_per_launch": (per["dyt_bwd_kernel"] + per["dyt_finalize_kernel"]) / calls,
+            "stage1_launches_per_call": len(launches["dyt_bwd_kernel"]) / calls,
             "source_hash": kernel_source_hash(), "command": command}
     d[workload] = entry
     with open(path, "w") as f:

@@ -106,11 +106,19 @@ def forward(x: torch.Tensor, alpha: torch.Tensor, gamma: torch.Tensor, beta: tor
     return y
 
 
-def workspace(x: torch.Tensor, gamma: torch.Tensor) -> torch.Tensor:
-    """A device workspace large enough for backward on x's shape and device."""
+def workspace(x: torch.Tensor, gamma: torch.Tensor, dy: torch.Tensor | None = None,
+              dx: torch.Tensor | None = None) -> torch.Tensor:
+    """A device workspace large enough for backward on x's shape and device;
+    given dy (and dx), also for the phases their row pitches call for."""
     M, N = _shape(x, gamma)
     with torch.cuda.device(x.device):
-        n = dyt_backward_workspace_bytes(M, N, _code(x, "x"), _code(gamma, "gamma"))
+        if dy is None:
+            n = dyt_backward_workspace_bytes(M, N, _code(x, "x"), _code(gamma, "gamma"))
+        else:
+            ldx, lddy = _rows(x, "x"), _rows(dy, "dy")
+            lddx = N if dx is None else _rows(dx, "dx")
+            n = _abi.dyt_backward_workspace_bytes_strided(M, N, ldx, lddy, lddx, _code(x, "x"),
+                                                          _code(gamma, "gamma"))
     return torch.empty(max(n, 16), dtype=torch.uint8, device=x.device)
 
 
@@ -142,7 +150,7 @@ def backward(x: torch.Tensor, dy: torch.Tensor, alpha: torch.Tensor, gamma: torc
         if t.dtype != like.dtype or t.numel() != like.numel():
             raise ValueError(f"{w} must match its parameter in size and dtype")
         _cuda_contig(t, w)
-    ws = workspace(x, gamma) if ws is None else ws
+    ws = workspace(x, gamma, dy, dx) if ws is None else ws
     with torch.cuda.device(x.device):
         st = dyt_backward_ex(x.data_ptr(), ldx, dy.data_ptr(), lddy, alpha.data_ptr(), gamma.data_ptr(),
                              None if beta is None else beta.data_ptr(), dx.data_ptr(), lddx, dgamma.data_ptr(),

@@ -40,6 +40,8 @@ lib.dyt_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp
 lib.dyt_forward.restype = _i32
 lib.dyt_backward_workspace_bytes.argtypes = [_i64, _i64, _i32, _i32]
 lib.dyt_backward_workspace_bytes.restype = _sz
+lib.dyt_backward_workspace_bytes_strided.argtypes = [_i64, _i64, _i64, _i64, _i64, _i32, _i32]
+lib.dyt_backward_workspace_bytes_strided.restype = _sz
 lib.dyt_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _sz, _vp]
 lib.dyt_backward.restype = _i32
 lib.dyt_forward_strided.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _vp]
@@ -131,6 +133,10 @@ def dyt_forward(x, alpha, gamma, beta, y, M, N, x_dtype, param_dtype, stream) ->
 
 def dyt_backward_workspace_bytes(M, N, x_dtype, param_dtype) -> int:
     return int(lib.dyt_backward_workspace_bytes(M, N, x_dtype, param_dtype))
+
+
+def dyt_backward_workspace_bytes_strided(M, N, ldx, lddy, lddx, x_dtype, param_dtype) -> int:
+    return int(lib.dyt_backward_workspace_bytes_strided(M, N, ldx, lddy, lddx, x_dtype, param_dtype))
 
 
 def dyt_backward(x, dy, alpha, gamma, beta, dx, dgamma, dbeta, dalpha, M, N, x_dtype, param_dtype, workspace,

@@ -303,6 +303,42 @@ dyt_status check_pitch(int64_t M, int64_t N, int64_t ld) {
 // A row pitch of whole 16-byte vectors.
 bool vec_pitch(int64_t ld, size_t elem) { return ((uint64_t)ld * elem) % 16 == 0; }
 
+// Rows ld elements apart: a row's offset past a 16-byte boundary repeats
+// every 16 / (lowest set bit of ld * elem mod 16) rows (1, 2, 4 or 8).
+int pitch_period(int64_t ld, size_t elem) {
+  const uint64_t r = ((uint64_t)ld * elem) & 15u;
+  return r == 0 ? 1 : (int)(16u / (unsigned)(r & (~r + 1u)));
+}
+
+// Phases of a strided call (not every pitch N) whose pitches are not all whole
+// 16-byte vectors: k = the longest period of its tensors' pitches. Rows j,
+// j + k, j + 2k, ... then form a matrix of pitch k * ld (whole vectors) for
+// every tensor, which the 16-byte kernels take (aligned, or the row frame);
+// the call runs its k phases one after another. 1: no phases (the pitches are
+// whole vectors, the rows are adjacent, or fewer than kPhaseMinRows rows per
+// phase, which the one-element kernels take in one launch).
+int phases_of(int64_t M, int64_t N, const int64_t *lds, int n, size_t elem) {
+  int k = 1;
+  bool adjacent = true;
+  for (int i = 0; i < n; ++i) {
+    k = std::max(k, pitch_period(lds[i], elem));
+    adjacent = adjacent && lds[i] == N;
+  }
+  if (adjacent || k == 1 || M < (int64_t)k * kPhaseMinRows) return 1;
+  return k;
+}
+
+// Rows of phase j of k: j, j + k, ... below M.
+int64_t phase_rows(int64_t M, int k, int j) { return (M - j + k - 1) / k; }
+
+// The backward runs phases only for k = 2: every phase leaves a full set of
+// binary64 partials (k times the finalize's reads) after a launch of its own.
+// Measured against the one-element kernels (us): 16384 x 4096 bf16, pitch
+// 4100 (2 phases) 154.6 -> 117.7; 100003 x 255 fp32, pitch 257 (4 phases)
+// 75.0 -> 87.6; 16384 x 4096 bf16, pitch 4097 (8 phases) 153.8 -> 231.9. The
+// forward gains at every k: 130.0 -> 61.0, 54.0 -> 50.5, 128.8 -> 96.5.
+int bwd_phases(int k) { return k == 2 ? 2 : 1; }
+
 dyt_launch_info describe(int op, const Plan *p, int kernels, size_t ws) {
   dyt_launch_info i = {};
   i.op = op;
@@ -500,6 +536,19 @@ dyt_status bwd_stage1(const void *x, int64_t ldx, const void *dy, int64_t lddy, 
 // in binary64 in a fixed order (rank by rank), each gradient rounded once.
 // Launched as a programmatic dependent: it may start while its predecessor in
 // the stream drains and waits (griddepcontrol.wait) for its results.
+// The workspace bytes stage 1 needs for these tensors (the plan only;
+// nothing is launched). The plans do not depend on the parameter type.
+dyt_status stage1_bytes(const void *x, int64_t ldx, const void *dy, int64_t lddy, const void *dx, int64_t lddx,
+                        int64_t M, int64_t N, dyt_dtype x_dtype, size_t *out) {
+  return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
+    using T = decltype(tx);
+    Plan p;
+    const dyt_status r = plan_for<T, float>(M, N, stage1_layout_args<T>(x, ldx, dy, lddy, dx, lddx, N), true, &p);
+    if (r == DYT_OK) *out = p.ws_total;
+    return r;
+  });
+}
+
 dyt_status bwd_finalize(const void *const *wss, const dyt_partials_layout *lay, int nranks, int64_t N, void *dgamma,
                         void *dbeta, void *dalpha, dyt_dtype ad, dyt_dtype gd, dyt_dtype bd, cudaStream_t s) {
   dyt::PartsSet ps = {};
@@ -570,25 +619,32 @@ dyt_status dyt_forward_ex(const void *x, int64_t ldx, const void *alpha, const v
       !elem_aligned(gamma, dsize(gamma_dtype)) || !elem_aligned(beta, dsize(beta_dtype)))
     return DYT_ERR_INVALID_VALUE;
   const dyt::ParamTypes pt = {(int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
+  const int64_t lds[2] = {ldx, ldy};
+  const int k = phases_of(M, N, lds, 2, es);  // 1 unless the pitches call for phases
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
     return with_ptype(alpha_dtype, gamma_dtype, beta_dtype, [&](auto tp) -> dyt_status {
     using P = typename decltype(tp)::type;
     Plan p;
-    dyt_status s = plan_for<T, P>(M, N, aligned16(x) && aligned16(y),
-                                  vec_pitch(ldx, sizeof(T)) && vec_pitch(ldy, sizeof(T)), ldx == N && ldy == N,
-                                  shift_of(y, sizeof(T)), same_offset(x, y) ? 0 : 2, false, &p);
-    if (s != DYT_OK) return s;
-    if (!p.packed) {
-      p.g.ldx = ldx;
-      p.g.ldo = ldy;
+    for (int j = 0; j < k; ++j) {  // phase j: rows j, j + k, ...
+      const T *xj = (const T *)x + j * ldx;
+      T *yj = (T *)y + j * ldy;
+      const int64_t lx = k * ldx, ly = k * ldy, Mj = phase_rows(M, k, j);
+      dyt_status s = plan_for<T, P>(Mj, N, aligned16(xj) && aligned16(yj),
+                                    vec_pitch(lx, sizeof(T)) && vec_pitch(ly, sizeof(T)), lx == N && ly == N,
+                                    shift_of(yj, sizeof(T)), same_offset(xj, yj) ? 0 : 2, false, &p);
+      if (s != DYT_OK) return s;
+      if (!p.packed) {
+        p.g.ldx = lx;
+        p.g.ldo = ly;
+      }
+      const P *pa = (const P *)alpha, *pg = (const P *)gamma, *pb = (const P *)beta;
+      PdlConfig lc(p.grid, p.block, p.smem, (cudaStream_t)stream);
+      const cudaError_t e = cudaLaunchKernelEx(&lc.cfg, fwd_kernel_of<T, P>(p.async, p.packed, p.shm), xj, pa, pg,
+                                               pb, pt, yj, p.g);
+      if (e != cudaSuccess) return cuda_fail(e);
     }
-    const P *pa = (const P *)alpha, *pg = (const P *)gamma, *pb = (const P *)beta;
-    PdlConfig lc(p.grid, p.block, p.smem, (cudaStream_t)stream);
-    const cudaError_t e = cudaLaunchKernelEx(&lc.cfg, fwd_kernel_of<T, P>(p.async, p.packed, p.shm),
-                                             (const T *)x, pa, pg, pb, pt, (T *)y, p.g);
-    if (e != cudaSuccess) return cuda_fail(e);
-    record(1, &p, 1, 0);
+    record(1, &p, k, 0);
     return DYT_OK;
     });
   });
@@ -618,6 +674,40 @@ size_t dyt_backward_workspace_bytes(int64_t M, int64_t N, dyt_dtype x_dtype, dyt
     return DYT_OK;
   });
   return st == DYT_OK ? need : 0;
+}
+
+size_t dyt_backward_workspace_bytes_strided(int64_t M, int64_t N, int64_t ldx, int64_t lddy, int64_t lddx,
+                                            dyt_dtype x_dtype, dyt_dtype param_dtype) {
+  const size_t plain = dyt_backward_workspace_bytes(M, N, x_dtype, param_dtype);
+  if (plain == 0 || check_pitch(M, N, ldx) != DYT_OK || check_pitch(M, N, lddy) != DYT_OK ||
+      check_pitch(M, N, lddx) != DYT_OK)
+    return plain;
+  const int64_t lds[3] = {ldx, lddy, lddx};
+  const int k = bwd_phases(phases_of(M, N, lds, 3, dsize(x_dtype)));
+  if (k == 1) return plain;
+  // Each phase's region: the largest plan its rows can take, whatever the
+  // tensors' offsets (aligned, or the row frame at any output offset, its
+  // inputs at that offset or not).
+  size_t need = 0;
+  const dyt_status st = with_xtype(x_dtype, [&](auto tx) -> dyt_status {
+    using T = decltype(tx);
+    constexpr int V = vec_of<T>();
+    for (int j = 0; j < k; ++j) {
+      const int64_t Mj = phase_rows(M, k, j);
+      size_t region = 0;
+      for (int v = -1; v < 2 * V; ++v) {
+        Plan p;
+        const dyt_status s = v < 0   ? plan_for<T, float>(Mj, N, true, true, false, 0, 0, true, &p)
+                             : v < V ? plan_for<T, float>(Mj, N, false, true, false, v, 0, true, &p)
+                                     : plan_for<T, float>(Mj, N, false, true, false, v - V, 2, true, &p);
+        if (s != DYT_OK) return s;
+        region = std::max(region, p.ws_total);
+      }
+      need += align16(region);
+    }
+    return DYT_OK;
+  });
+  return st == DYT_OK ? std::max(plain, need) : 0;
 }
 
 dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const void *gamma, const void *beta,
@@ -655,16 +745,43 @@ dyt_status dyt_backward_ex(const void *x, int64_t ldx, const void *dy, int64_t l
     if (st == DYT_OK) record(2, nullptr, 0, 0);
     return st;
   }
+  // Pitches that call for phases (see phases_of): one stage 1 per phase, each
+  // in its own workspace region, and one finalize over the phases' partials
+  // in phase order. When the regions do not fit in the workspace given, the
+  // call runs as one phase (the one-element kernels).
+  const size_t es = dsize(x_dtype);
+  const int64_t lds[3] = {ldx, lddy, lddx};
+  int k = bwd_phases(phases_of(M, N, lds, 3, es));
+  size_t off[dyt::kMaxRanks + 1] = {0};
+  static_assert(dyt::kMaxRanks >= 8, "the finalize takes up to 8 partial sets");
+  if (k > 1) {
+    if (!x || !dy || !dx || !elem_aligned(x, es) || !elem_aligned(dy, es) || !elem_aligned(dx, es))
+      return DYT_ERR_INVALID_VALUE;
+    for (int j = 0; j < k; ++j) {
+      size_t b = 0;
+      st = stage1_bytes((const char *)x + j * ldx * es, k * ldx, (const char *)dy + j * lddy * es, k * lddy,
+                        (const char *)dx + j * lddx * es, k * lddx, phase_rows(M, k, j), N, x_dtype, &b);
+      if (st != DYT_OK) return st;
+      off[j + 1] = off[j] + align16(b);
+    }
+    if (off[k] > workspace_bytes) k = 1;
+  }
   Plan p;
-  dyt_partials_layout lay;
-  st = bwd_stage1(x, ldx, dy, lddy, alpha, gamma, dx, lddx, M, N, x_dtype, alpha_dtype, gamma_dtype, workspace,
-                  workspace_bytes, (cudaStream_t)stream, &p, &lay);
-  if (st != DYT_OK) return st;
-  const void *wss[1] = {workspace};
-  st = bwd_finalize(wss, &lay, 1, N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype,
+  dyt_partials_layout lay[dyt::kMaxRanks];
+  const void *wss[dyt::kMaxRanks];
+  for (int j = 0; j < k; ++j) {
+    char *ws = (char *)workspace + off[j];
+    st = bwd_stage1((const char *)x + j * ldx * es, k * ldx, (const char *)dy + j * lddy * es, k * lddy, alpha,
+                    gamma, (char *)dx + j * lddx * es, k * lddx, phase_rows(M, k, j), N, x_dtype, alpha_dtype,
+                    gamma_dtype, ws, k == 1 ? workspace_bytes : off[j + 1] - off[j], (cudaStream_t)stream, &p,
+                    &lay[j]);
+    if (st != DYT_OK) return st;
+    wss[j] = ws;
+  }
+  st = bwd_finalize(wss, lay, k, N, dgamma, dbeta, dalpha, alpha_dtype, gamma_dtype, beta_dtype,
                     (cudaStream_t)stream);
   if (st != DYT_OK) return st;
-  record(2, &p, 2, p.ws_total);
+  record(2, &p, k + 1, k == 1 ? p.ws_total : off[k]);
   return DYT_OK;
 }
 

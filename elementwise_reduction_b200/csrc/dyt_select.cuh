@@ -31,6 +31,10 @@ constexpr int kNarrowMaxNV = 32;
 // a multiply-high by ceil(2^32 / RL), exact for counts below 2^32 / RL; a
 // count stays below 2049 RL, and 2049 RL^2 < 2^32 for every RL <= 1024.
 constexpr int kMaxRowsPerLane = 2048;
+// Strided rows whose pitches are not whole 16-byte vectors run as k phases
+// (rows j, j + k, ...) of whole-vector pitch only with at least this many rows
+// per phase; fewer go to the one-element kernels in one launch.
+constexpr int64_t kPhaseMinRows = 256;
 // Inputs read by one launch below which the L2 prefetch of the first rows is
 // skipped (bytes): smaller inputs are likely resident in L2 already.
 constexpr int64_t kPrefetchMinBytes = 1 << 20;

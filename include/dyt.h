@@ -157,12 +157,24 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
  * 16-byte chunks, so it reads the padding bytes that share a chunk with a
  * row's first or last elements (always between the tensor's first and last
  * elements); their values reach no result. The other kernels read no
- * padding. Pitches that are not whole 16-byte vectors take the one-element
- * kernels. y may alias x (dx may alias x or
+ * padding. Pitches that are not whole 16-byte vectors (pitch times element
+ * size a multiple of 8, 4 or 2 bytes: a row's offset past a boundary then
+ * repeats every k = 2, 4 or 8 rows) run as k phases, rows j, j + k, ... of
+ * pitch k * ld each through the kernels above, when every phase has at least
+ * 256 rows: the forward for every k, the backward for k = 2 when the
+ * workspace holds both phases' partials (dyt_backward_workspace_bytes_strided;
+ * the finalize then adds the phases' partials in phase order). Otherwise they
+ * take the one-element kernels.
+ * y may alias x (dx may alias x or
  * dy) only with equal pitches. A pitch below N, or (M - 1) * ld + N beyond
  * the int64 limit of byte offsets, gives DYT_ERR_INVALID_VALUE.
- * dyt_backward_workspace_bytes covers the strided call too.
+ * dyt_backward_workspace_bytes covers every strided call (one phase);
+ * dyt_backward_workspace_bytes_strided also covers the phases its pitches
+ * call for (and is at least dyt_backward_workspace_bytes). Both return 0 for
+ * invalid arguments or when no workspace is needed.
  */
+size_t dyt_backward_workspace_bytes_strided(int64_t M, int64_t N, int64_t ldx, int64_t lddy, int64_t lddx,
+                                            dyt_dtype x_dtype, dyt_dtype param_dtype);
 dyt_status dyt_forward_strided(const void *x, int64_t ldx, const void *alpha, const void *gamma,
                                const void *beta, void *y, int64_t ldy, int64_t M, int64_t N,
                                dyt_dtype x_dtype, dyt_dtype param_dtype, dyt_stream_t stream);

@@ -65,7 +65,9 @@ def test_traffic_csv_is_averaged_per_launch(tmp_path, monkeypatch):
     assert abs(d["dyt_bwd_kernel"]["bytes_per_launch"] - 12e6) < 1     # (8 + 4 + 10 + 2) MB / 2
     assert abs(d["dyt_finalize_kernel"]["bytes_per_launch"] - 42e3) < 1
     assert abs(d["dyt_fwd_kernel"]["bytes_per_launch"] - 1.024e6) < 1  # thousands separator
-    assert abs(d["dyt_backward"]["bytes_per_launch"] - 12.042e6) < 1
+    # one backward call: both stage-1 launches (two phases) and its one finalize
+    assert abs(d["dyt_backward"]["bytes_per_launch"] - 24.042e6) < 1
+    assert d["dyt_backward"]["stage1_launches_per_call"] == 2
     assert all(v["source_hash"] == bench.kernel_source_hash() for v in d.values())
     assert "at::" not in json.dumps(d)
 

@@ -386,6 +386,20 @@ def test_in_place_aliasing(M, N):
 
 # ---- row-strided matrices: each tensor with its own leading dimension -----------------------------
 
+def _phases(M: int, N: int, lds, size: int, backward: bool = False) -> int:
+    # The library's phase count for these row pitches: a row's offset past a
+    # 16-byte boundary repeats every 16 / (lowest set bit of pitch bytes mod 16)
+    # rows; strided calls whose pitches are not all whole vectors run that many
+    # phases of whole-vector pitch, when every phase has 256 rows or more (the
+    # backward only for 2 phases).
+    def period(ld):
+        r = (ld * size) % 16
+        return 1 if r == 0 else 16 // (r & -r)
+    k = max(period(ld) for ld in lds)
+    k = 1 if all(ld == N for ld in lds) or k == 1 or M < 256 * k else k
+    return (k if k == 2 else 1) if backward else k
+
+
 def _in_wider_rows(src: torch.Tensor, M: int, N: int, pitch: int, fill: float) -> tuple:
     buf = torch.full((M, pitch), fill, dtype=src.dtype, device="cuda")
     buf[:, :N] = src.view(M, N)
@@ -415,11 +429,18 @@ def test_strided_rows(N, pad, xd):
     size = 4 if xd == "f32" else 2
     vec = 16 // size
     # whole-vector pitches take the 16-byte kernels (aligned tensors and N a
-    # multiple of vec: the plain ones, else the row frame)
+    # multiple of vec: the plain ones, else the row frame); other pitches run
+    # as phases of whole-vector pitch through the same kernels
     pitched = all((p * size) % 16 == 0 for p in (N + pad, N + 2 * pad, N + 3 * pad, N + 4 * pad))
     vectorised = N % vec == 0 and pitched
-    assert info_f["vec"] == info_b["vec"] == (vec if pitched else 1)
-    assert info_f["shifted"] == info_b["shifted"] == (2 if pitched and not vectorised else 0)
+    k_f = _phases(M, N, (N + pad, N + 3 * pad), size)
+    k_b = _phases(M, N, (N + pad, N + 2 * pad, N + 4 * pad), size, backward=True)
+    whole_b = all((p * size) % 16 == 0 for p in (N + pad, N + 2 * pad, N + 4 * pad))
+    assert info_f["vec"] == vec
+    assert info_b["vec"] == (vec if whole_b or k_b > 1 else 1)
+    assert info_f["kernels"] == k_f and info_b["kernels"] == k_b + 1
+    if pitched:
+        assert info_f["shifted"] == info_b["shifted"] == (0 if vectorised else 2)
     assert info_b["pack_rows"] == 1
     if vectorised:  # the same kernels as the contiguous call: the same bits
         ref, _ = H.run_cuda(inp, M, N, xd, "f32")
@@ -483,6 +504,68 @@ def test_row_frame_rows(xd, N, hx, hd, ho):
     H.compare_all(inp, out, M, N, xd, "f32")
     ref, _ = H.run_cuda(inp, M, N, xd, "f32")
     assert np.array_equal(out["y"], ref["y"]) and np.array_equal(out["dx"], ref["dx"])
+
+
+@pytest.mark.parametrize("xd,N,lds,offs", [
+    ("bf16", 4096, (4100, 4100, 4100), (0, 0, 0)),      # 8200 bytes: 2 phases
+    ("bf16", 1000, (1004, 1004, 1012), (1, 1, 1)),      # 2 phases, every tensor one element off
+    ("bf16", 1000, (1002, 1006, 1010), (1, 1, 3)),      # 2004 / 2012 / 2020 bytes: 4 phases
+    ("bf16", 255, (257, 259, 261), (0, 5, 2)),          # odd pitches: 8 phases
+    ("f32", 100, (102, 102, 106), (0, 1, 2)),           # 408 / 424 bytes: 2 phases
+    ("f32", 17, (17, 21, 19), (3, 0, 1)),               # x adjacent, the others not: 4 phases
+    ("f16", 64, (66, 72, 68), (0, 0, 0)),               # 4 phases
+])
+def test_phased_rows(xd, N, lds, offs):
+    # Pitches that are not whole 16-byte vectors: rows j, j + k, ... run as k
+    # matrices of whole-vector pitch through the 16-byte kernels. NaN between
+    # the inputs' rows, 7 around the outputs (never written); elementwise
+    # results bit for bit those of the contiguous call, sums within the
+    # oracle's bounds; a workspace too small for the phases runs one phase.
+    import elementwise_reduction_b200 as dyt
+    size = 4 if xd == "f32" else 2
+    vec = 16 // size
+    M = 4001
+    ldx, lddy, ldo = lds
+    hx, hd, ho = offs
+    inp = make(M, N, xd, "f32")
+    t = H.gpu_inputs(inp, xd, "f32")
+    _, x = _placed_rows(t["x"], M, N, hx, ldx, float("nan"))
+    _, dy = _placed_rows(t["dy"], M, N, hd, lddy, float("nan"))
+    zero = torch.zeros(M * N, dtype=t["x"].dtype, device="cuda")
+    ybuf, y = _placed_rows(zero, M, N, ho, ldo, 7.0)
+    dxbuf, dx = _placed_rows(zero, M, N, ho, ldo, 7.0)
+    mask = torch.ones_like(ybuf, dtype=torch.bool)
+    mask[ho:ho + M * ldo].view(M, -1)[:, :N] = False
+    dyt.forward(x, t["alpha"], t["gamma"], t["beta"], out=y)
+    info_f = dyt.dyt_last_launch_info()
+    _, dalpha, dgamma, dbeta = dyt.backward(x, dy, t["alpha"], t["gamma"], dx=dx)
+    info_b = dyt.dyt_last_launch_info()
+    torch.cuda.synchronize()
+    assert (ybuf[mask] == 7).all() and (dxbuf[mask] == 7).all()  # nothing outside the rows is written
+    k_f, k_b = _phases(M, N, (ldx, ldo), size), _phases(M, N, (ldx, lddy, ldo), size, backward=True)
+    assert k_f > 1
+    assert info_f["kernels"] == k_f and info_b["kernels"] == k_b + 1
+    assert info_f["vec"] == vec and info_b["vec"] == (vec if k_b > 1 else 1)
+    out = {"y": H.to_numpy(y.contiguous(), xd), "dx": H.to_numpy(dx.contiguous(), xd),
+           "dgamma": H.to_numpy(dgamma, "f32"), "dbeta": H.to_numpy(dbeta, "f32"), "dalpha": float(dalpha.item())}
+    H.compare_all(inp, out, M, N, xd, "f32")
+    ref, _ = H.run_cuda(inp, M, N, xd, "f32")
+    assert np.array_equal(out["y"], ref["y"]) and np.array_equal(out["dx"], ref["dx"])
+    # The plain size query covers one phase (the one-element kernels); where
+    # that is less than the phases need, the same call runs as one phase.
+    small = dyt.workspace(x, t["gamma"])
+    fits = small.numel() >= dyt.workspace(x, t["gamma"], dy, dx).numel() or k_b == 1
+    dx2 = torch.empty_like(dx)
+    _, dalpha2, dgamma2, dbeta2 = dyt.backward(x, dy, t["alpha"], t["gamma"], dx=dx2, ws=small)
+    info_1 = dyt.dyt_last_launch_info()
+    torch.cuda.synchronize()
+    if fits:
+        assert info_1["kernels"] == k_b + 1 and info_1["vec"] == (vec if k_b > 1 else 1)
+    else:
+        assert info_1["kernels"] == 2 and info_1["vec"] == 1
+    out2 = {"y": out["y"], "dx": H.to_numpy(dx2.contiguous(), xd), "dgamma": H.to_numpy(dgamma2, "f32"),
+            "dbeta": H.to_numpy(dbeta2, "f32"), "dalpha": float(dalpha2.item())}
+    H.compare_all(inp, out2, M, N, xd, "f32")
 
 
 def test_strided_in_place_and_autograd():
@@ -781,7 +864,12 @@ def test_unaligned_variant_full_size(name):
     out, info = H.run_cuda(inp, w.M, w.N, w.x_dtype, w.p_dtype, offset=w.offset, x_offset=w.x_offset,
                            pitch=w.pitch)
     if w.pitch and (w.pitch * (4 if w.x_dtype == "f32" else 2)) % 16:
-        assert info["fwd"]["vec"] == info["bwd"]["vec"] == 1
+        # pitches off whole vectors: phases of whole-vector pitch
+        k = _phases(w.M, w.N, (w.pitch,), 4 if w.x_dtype == "f32" else 2)
+        k_b = _phases(w.M, w.N, (w.pitch,), 4 if w.x_dtype == "f32" else 2, backward=True)
+        assert k > 1 and info["fwd"]["vec"] == (4 if w.x_dtype == "f32" else 8)
+        assert info["bwd"]["vec"] == ((4 if w.x_dtype == "f32" else 8) if k_b > 1 else 1)
+        assert info["fwd"]["kernels"] == k and info["bwd"]["kernels"] == k_b + 1
     elif w.pitch:  # whole-vector pitches: the row frame (3: with the wrapped first vector-column)
         wrapped = w.offset and w.x_off == w.offset and w.N % (4 if w.x_dtype == "f32" else 8) == 0
         assert info["fwd"]["shifted"] == info["bwd"]["shifted"] == (3 if wrapped else 2)

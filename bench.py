@@ -494,7 +494,7 @@ def run_ours(args, w):
     inp = workloads.make_inputs(w)
     L2 = torch.cuda.get_device_properties(dev).L2_cache_size
     sets, (alpha, gamma, beta), set_bytes, nsets = _sets(w, inp, dev, L2)
-    ws = dyt.workspace(sets[0]["x"], gamma)
+    ws = dyt.workspace(sets[0]["x"], gamma, sets[0]["dy"], sets[0]["dx"])
     grads = torch.empty(2 * N + 1, dtype=torch.float32, device=dev)
     from elementwise_reduction_b200.dist import FusedGradientSum, allreduce_param_grads
 
@@ -612,7 +612,8 @@ def run_ours(args, w):
                                        "dx": _empty_like_matrix(x0, w, w.offset),
                                        "dg": torch.empty_like(gamma), "db": torch.empty_like(beta),
                                        "da": torch.empty_like(alpha)}
-        lanes.append({"dev": d, "ws": dyt.workspace(x0, gamma), "stream": stream if j == 0 else torch.cuda.Stream(dev),
+        lanes.append({"dev": d, "ws": dyt.workspace(x0, gamma, d["dy"], d["dx"]),
+                      "stream": stream if j == 0 else torch.cuda.Stream(dev),
                       "ex": exchange if j == 0 or exchange is None else make_exchange(x0, x0, x0)[0],
                       "grads": torch.empty(2 * N + 1, dtype=torch.float32, device=dev),
                       "hy": torch.empty_like(hx).pin_memory(), "hdx": torch.empty_like(hx).pin_memory(),
@@ -765,7 +766,7 @@ def call_latency(args, dev, calls=30):
               "dx": _empty_like_matrix(x, w, w.offset),
               "p": [_to_torch(inp[k], dt, dev) for k, dt in zip(("alpha", "gamma", "beta"), (ad, gd, bd))],
               "ws": None, "t": {"fwd": [], "bwd": []}}
-        st["ws"] = dyt.workspace(x, st["p"][1])
+        st["ws"] = dyt.workspace(x, st["p"][1], st["dy"], st["dx"])
         state[name] = st
     with torch.cuda.stream(stream):
         for i in range(calls + 2):  # the first two rounds are warm-up
@@ -815,7 +816,7 @@ def shape_table(args, dev, clock_index, cpu=True):
     for name, w in {**workloads.WORKLOADS, **workloads.VARIANTS}.items():
         inp = workloads.make_inputs(w)
         sets, (a, g, b), _, nsets = _sets(w, inp, dev, L2)
-        ws = dyt.workspace(sets[0]["x"], g)
+        ws = dyt.workspace(sets[0]["x"], g, sets[0]["dy"], sets[0]["dx"])
         stream = torch.cuda.Stream(dev)
         res = {}
         with torch.cuda.stream(stream):

@@ -310,26 +310,27 @@ int pitch_period(int64_t ld, size_t elem) {
   return r == 0 ? 1 : (int)(16u / (unsigned)(r & (~r + 1u)));
 }
 
+// Rows of phase j of k: j, j + k, ... below M.
+int64_t phase_rows(int64_t M, int k, int j) { return (M - j + k - 1) / k; }
+
 // Phases of a strided call (not every pitch N) whose pitches are not all whole
 // 16-byte vectors: k = the longest period of its tensors' pitches. Rows j,
 // j + k, j + 2k, ... then form a matrix of pitch k * ld (whole vectors) for
 // every tensor, which the 16-byte kernels take (aligned, or the row frame);
 // the call runs its k phases one after another. 1: no phases (the pitches are
-// whole vectors, the rows are adjacent, or fewer than kPhaseMinRows rows per
-// phase, which the one-element kernels take in one launch).
-int phases_of(int64_t M, int64_t N, const int64_t *lds, int n, size_t elem) {
+// whole vectors, the rows are adjacent, or a phase would move fewer than
+// min_bytes per tensor, which the one-element kernels take in one launch).
+int phases_of(int64_t M, int64_t N, const int64_t *lds, int n, size_t elem, int64_t min_bytes) {
   int k = 1;
   bool adjacent = true;
   for (int i = 0; i < n; ++i) {
     k = std::max(k, pitch_period(lds[i], elem));
     adjacent = adjacent && lds[i] == N;
   }
-  if (adjacent || k == 1 || M < (int64_t)k * kPhaseMinRows) return 1;
+  if (adjacent || k == 1 || M < k) return 1;
+  if (phase_rows(M, k, k - 1) * N * (int64_t)elem < min_bytes) return 1;  // the smallest phase
   return k;
 }
-
-// Rows of phase j of k: j, j + k, ... below M.
-int64_t phase_rows(int64_t M, int k, int j) { return (M - j + k - 1) / k; }
 
 // The backward runs phases only for k = 2: every phase leaves a full set of
 // binary64 partials (k times the finalize's reads) after a launch of its own.
@@ -620,7 +621,7 @@ dyt_status dyt_forward_ex(const void *x, int64_t ldx, const void *alpha, const v
     return DYT_ERR_INVALID_VALUE;
   const dyt::ParamTypes pt = {(int)alpha_dtype, (int)gamma_dtype, (int)beta_dtype};
   const int64_t lds[2] = {ldx, ldy};
-  const int k = phases_of(M, N, lds, 2, es);  // 1 unless the pitches call for phases
+  const int k = phases_of(M, N, lds, 2, es, kPhaseMinBytesFwd);  // 1 unless the pitches call for phases
   return with_xtype(x_dtype, [&](auto tx) -> dyt_status {
     using T = decltype(tx);
     return with_ptype(alpha_dtype, gamma_dtype, beta_dtype, [&](auto tp) -> dyt_status {
@@ -683,7 +684,7 @@ size_t dyt_backward_workspace_bytes_strided(int64_t M, int64_t N, int64_t ldx, i
       check_pitch(M, N, lddx) != DYT_OK)
     return plain;
   const int64_t lds[3] = {ldx, lddy, lddx};
-  const int k = bwd_phases(phases_of(M, N, lds, 3, dsize(x_dtype)));
+  const int k = bwd_phases(phases_of(M, N, lds, 3, dsize(x_dtype), kPhaseMinBytesBwd));
   if (k == 1) return plain;
   // Each phase's region: the largest plan its rows can take, whatever the
   // tensors' offsets (aligned, or the row frame at any output offset, its
@@ -751,7 +752,7 @@ dyt_status dyt_backward_ex(const void *x, int64_t ldx, const void *dy, int64_t l
   // call runs as one phase (the one-element kernels).
   const size_t es = dsize(x_dtype);
   const int64_t lds[3] = {ldx, lddy, lddx};
-  int k = bwd_phases(phases_of(M, N, lds, 3, es));
+  int k = bwd_phases(phases_of(M, N, lds, 3, es, kPhaseMinBytesBwd));
   size_t off[dyt::kMaxRanks + 1] = {0};
   static_assert(dyt::kMaxRanks >= 8, "the finalize takes up to 8 partial sets");
   if (k > 1) {

@@ -160,11 +160,11 @@ dyt_status dyt_backward(const void *x, const void *dy, const void *alpha, const 
  * padding. Pitches that are not whole 16-byte vectors (pitch times element
  * size a multiple of 8, 4 or 2 bytes: a row's offset past a boundary then
  * repeats every k = 2, 4 or 8 rows) run as k phases, rows j, j + k, ... of
- * pitch k * ld each through the kernels above, when every phase has at least
- * 256 rows: the forward for every k, the backward for k = 2 when the
- * workspace holds both phases' partials (dyt_backward_workspace_bytes_strided;
- * the finalize then adds the phases' partials in phase order). Otherwise they
- * take the one-element kernels.
+ * pitch k * ld each through the kernels above, when every phase moves at
+ * least 8 MiB per tensor (forward, any k) or 32 MiB per tensor (backward,
+ * k = 2, and the workspace holds both phases' partials:
+ * dyt_backward_workspace_bytes_strided; the finalize then adds the phases'
+ * partials in phase order). Otherwise they take the one-element kernels.
  * y may alias x (dx may alias x or
  * dy) only with equal pitches. A pitch below N, or (M - 1) * ld + N beyond
  * the int64 limit of byte offsets, gives DYT_ERR_INVALID_VALUE.

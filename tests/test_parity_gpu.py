@@ -390,14 +390,18 @@ def _phases(M: int, N: int, lds, size: int, backward: bool = False) -> int:
     # The library's phase count for these row pitches: a row's offset past a
     # 16-byte boundary repeats every 16 / (lowest set bit of pitch bytes mod 16)
     # rows; strided calls whose pitches are not all whole vectors run that many
-    # phases of whole-vector pitch, when every phase has 256 rows or more (the
-    # backward only for 2 phases).
+    # phases of whole-vector pitch, when every phase moves at least 8 MiB
+    # (forward) or 32 MiB (backward, 2 phases only) per tensor.
     def period(ld):
         r = (ld * size) % 16
         return 1 if r == 0 else 16 // (r & -r)
     k = max(period(ld) for ld in lds)
-    k = 1 if all(ld == N for ld in lds) or k == 1 or M < 256 * k else k
-    return (k if k == 2 else 1) if backward else k
+    if all(ld == N for ld in lds) or k == 1 or M < k:
+        return 1
+    smallest = (M - (k - 1) + k - 1) // k * N * size
+    if smallest < ((32 if backward else 8) << 20) or (backward and k != 2):
+        return 1
+    return k
 
 
 def _in_wider_rows(src: torch.Tensor, M: int, N: int, pitch: int, fill: float) -> tuple:
@@ -435,8 +439,9 @@ def test_strided_rows(N, pad, xd):
     vectorised = N % vec == 0 and pitched
     k_f = _phases(M, N, (N + pad, N + 3 * pad), size)
     k_b = _phases(M, N, (N + pad, N + 2 * pad, N + 4 * pad), size, backward=True)
+    whole_f = all((p * size) % 16 == 0 for p in (N + pad, N + 3 * pad))
     whole_b = all((p * size) % 16 == 0 for p in (N + pad, N + 2 * pad, N + 4 * pad))
-    assert info_f["vec"] == vec
+    assert info_f["vec"] == (vec if whole_f or k_f > 1 else 1)
     assert info_b["vec"] == (vec if whole_b or k_b > 1 else 1)
     assert info_f["kernels"] == k_f and info_b["kernels"] == k_b + 1
     if pitched:
@@ -506,16 +511,15 @@ def test_row_frame_rows(xd, N, hx, hd, ho):
     assert np.array_equal(out["y"], ref["y"]) and np.array_equal(out["dx"], ref["dx"])
 
 
-@pytest.mark.parametrize("xd,N,lds,offs", [
-    ("bf16", 4096, (4100, 4100, 4100), (0, 0, 0)),      # 8200 bytes: 2 phases
-    ("bf16", 1000, (1004, 1004, 1012), (1, 1, 1)),      # 2 phases, every tensor one element off
-    ("bf16", 1000, (1002, 1006, 1010), (1, 1, 3)),      # 2004 / 2012 / 2020 bytes: 4 phases
-    ("bf16", 255, (257, 259, 261), (0, 5, 2)),          # odd pitches: 8 phases
-    ("f32", 100, (102, 102, 106), (0, 1, 2)),           # 408 / 424 bytes: 2 phases
-    ("f32", 17, (17, 21, 19), (3, 0, 1)),               # x adjacent, the others not: 4 phases
-    ("f16", 64, (66, 72, 68), (0, 0, 0)),               # 4 phases
+@pytest.mark.parametrize("xd,M,N,lds,offs", [
+    ("bf16", 8200, 4096, (4100, 4100, 4100), (0, 0, 0)),   # 8200 bytes: 2 phases, forward and backward
+    ("bf16", 8200, 4096, (4100, 4100, 4108), (1, 1, 1)),   # 2 phases, every tensor one element off
+    ("f32", 4200, 2048, (2050, 2050, 2054), (0, 1, 2)),    # 8200 / 8216 bytes: 2 phases, forward only
+    ("bf16", 9000, 2048, (2050, 2054, 2058), (1, 1, 3)),   # 4 phases: the forward's
+    ("bf16", 33000, 1024, (1025, 1027, 1029), (0, 5, 2)),  # odd pitches: 8 phases, the forward's
+    ("f32", 4001, 17, (17, 21, 19), (3, 0, 1)),            # x adjacent, the others not: too small, one phase
 ])
-def test_phased_rows(xd, N, lds, offs):
+def test_phased_rows(xd, M, N, lds, offs):
     # Pitches that are not whole 16-byte vectors: rows j, j + k, ... run as k
     # matrices of whole-vector pitch through the 16-byte kernels. NaN between
     # the inputs' rows, 7 around the outputs (never written); elementwise
@@ -524,7 +528,6 @@ def test_phased_rows(xd, N, lds, offs):
     import elementwise_reduction_b200 as dyt
     size = 4 if xd == "f32" else 2
     vec = 16 // size
-    M = 4001
     ldx, lddy, ldo = lds
     hx, hd, ho = offs
     inp = make(M, N, xd, "f32")
@@ -543,9 +546,8 @@ def test_phased_rows(xd, N, lds, offs):
     torch.cuda.synchronize()
     assert (ybuf[mask] == 7).all() and (dxbuf[mask] == 7).all()  # nothing outside the rows is written
     k_f, k_b = _phases(M, N, (ldx, ldo), size), _phases(M, N, (ldx, lddy, ldo), size, backward=True)
-    assert k_f > 1
     assert info_f["kernels"] == k_f and info_b["kernels"] == k_b + 1
-    assert info_f["vec"] == vec and info_b["vec"] == (vec if k_b > 1 else 1)
+    assert info_f["vec"] == (vec if k_f > 1 else 1) and info_b["vec"] == (vec if k_b > 1 else 1)
     out = {"y": H.to_numpy(y.contiguous(), xd), "dx": H.to_numpy(dx.contiguous(), xd),
            "dgamma": H.to_numpy(dgamma, "f32"), "dbeta": H.to_numpy(dbeta, "f32"), "dalpha": float(dalpha.item())}
     H.compare_all(inp, out, M, N, xd, "f32")

@@ -312,3 +312,40 @@ def test_row_frame_addressing_with_column_chunks(M, N, xd):
         for hx in (0, 1):
             for backward in (False, True):
                 replay_rowframe(dyt, M, N, xd, {"x": hx, "dy": hx, "o": ho}, lds, backward, sms=5)
+
+
+def _period(ld, es):
+    r = (ld * es) % 16
+    return 1 if r == 0 else 16 // (r & -r)
+
+
+@pytest.mark.parametrize("xd,N,lds,offs", [
+    (1, 24, (26, 26, 26), (0, 0, 0)),     # 52 bytes: 4 phases
+    (1, 40, (44, 44, 52), (1, 1, 1)),     # 88 / 104 bytes: 2 phases, every tensor one element off
+    (1, 17, (19, 21, 23), (0, 3, 5)),     # odd pitches: 8 phases
+    (0, 10, (10, 14, 18), (0, 1, 2)),     # fp32, x adjacent: 4 phases
+    (0, 100, (102, 102, 106), (3, 3, 1)),  # 2 phases
+])
+def test_phase_plans_stay_inside_every_tensor(xd, N, lds, offs):
+    # A strided call whose pitches are not whole 16-byte vectors runs rows j,
+    # j + k, ... (k the longest pitch period) as k matrices of pitch k * ld.
+    # Each phase is an ordinary strided call at its own offsets: replay the
+    # library's plan for it and check that the phases cover every row once.
+    dyt = _lib()
+    es = 4 if xd == 0 else 2
+    k = max(_period(ld, es) for ld in lds)
+    assert k > 1
+    M = 3 * k + 1
+    ldx, ldd, ldo = lds
+    covered = []
+    for j in range(k):
+        Mj = (M - j + k - 1) // k
+        covered += [j + i * k for i in range(Mj)]
+        # phase j starts j rows in: its offset past a 16-byte boundary, in elements
+        sub_offs = {m: ((offs[i] + j * lds[i]) * es % 16) // es for i, m in enumerate(("x", "dy", "o"))}
+        sub_lds = {"x": k * ldx, "dy": k * ldd, "o": k * ldo}
+        for m in sub_lds:
+            assert sub_lds[m] * es % 16 == 0  # every phase's pitch is a whole number of vectors
+        for backward in (False, True):
+            replay_rowframe(dyt, Mj, N, xd, sub_offs, sub_lds, backward)
+    assert sorted(covered) == list(range(M))

@@ -96,6 +96,10 @@ def test_host_validation_without_a_device():
     assert dyt.dyt_forward_strided(0, 9, 0, 0, 0, 0, 9, 0, 4, 0, 0, None) == 0                  # empty
     assert dyt.dyt_backward_workspace_bytes(-1, 3, 0, 0) == 0
     assert dyt.dyt_backward_workspace_bytes(0, 3, 0, 0) == 0
+    from elementwise_reduction_b200 import _abi
+    assert _abi.dyt_backward_workspace_bytes_strided(-1, 3, 3, 3, 3, 0, 0) == 0
+    assert _abi.dyt_backward_workspace_bytes_strided(0, 3, 5, 5, 5, 0, 0) == 0   # empty: no workspace
+    assert _abi.dyt_backward_workspace_bytes_strided(4, 3, 5, 5, 5, 9, 0) == 0   # bad dtype
     for s in range(5):
         assert dyt.dyt_status_string(s).startswith("DYT_")
     assert dyt.dyt_status_string(99) == "DYT_ERR_UNKNOWN"
